@@ -1,0 +1,410 @@
+#!/usr/bin/env python
+"""Benchmark of the Prox sparse SwiGLU FFN decode path on B200.
+
+One step = the whole hot path (Stage 1 + Stage 2, every row of the path) over
+one batch of synthetic decode tokens: by default the 4096 x 12288 layer
+(Qwen3-8B shape, bf16 N(0, 0.02^2) weights with INT4 proxies), 512 Laplace
+tokens with 0.1% x20 outlier coordinates, processed at batch 1, thresholds
+calibrated on 512 vectors for 50% input keep and 70% channel sparsity.
+
+Timing: the 512 per-token calls are captured in one CUDA graph and replayed;
+the layer is held in 4 identical copies in HBM and token t reads copy t % 4,
+so every token streams its weights from HBM rather than from the 126 MB L2.
+CUDA events bracket the K timed steps (after W warm-up steps) with a barrier
+and a device synchronisation on both sides; the max over ranks is reported.
+Under torchrun each rank is an independent replica (no collective on the
+data path); value = all ranks' tokens / the slowest rank's time.
+
+Prints ONE JSON line (rank 0). --impl reference times the fp64 CPU oracle on
+the host cores on a bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "sparse SwiGLU FFN µs/token/layer @70% sparsity; achieved HBM GB/s vs peak"
+
+WORKLOADS = {
+    # name: d_model, d_ff, sigma, tokens, calibration vectors, outlier fraction
+    "qwen3-8b-ffn": dict(d=4096, f=12288, sigma=0.02, tokens=512, n_cal=512, outlier=0.001),
+    "tiny-ffn": dict(d=256, f=768, sigma=0.02, tokens=64, n_cal=256, outlier=0.0),
+    "large-ffn": dict(d=8192, f=28672, sigma=0.015, tokens=256, n_cal=256, outlier=0.0),
+}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="qwen3-8b-ffn")
+    ap.add_argument("--keep-x", type=float, default=0.5)
+    ap.add_argument("--keep-s", type=float, default=0.3)
+    ap.add_argument("--copies", type=int, default=4, help="rotating weight copies (L2 defeat)")
+    ap.add_argument("--no-dense", action="store_true", help="skip the dense cuBLAS reference")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
+    return 6650.0, "fallback 6.65 TB/s"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples while the timed region runs."""
+
+    def __init__(self, index: int):
+        self.index = index
+        self.samples = []
+        self.proc = None
+
+    def __enter__(self):
+        q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 7:
+                self.samples.append(parts)
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
+        sm = [num(s[0]) for s in self.samples if num(s[0]) is not None]
+        mx = [num(s[1]) for s in self.samples if num(s[1]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for s in self.samples for k in range(4)
+                          if s[3 + k].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the fp64 CPU oracle, timed on the host cores
+# ---------------------------------------------------------------------------
+
+def cpu_oracle_time(w, keep_x, keep_s, seconds):
+    """Time the oracle on a bounded token sample; returns (us/token, cores, sample)."""
+    import oracle
+    from free_ffn_activation_b200 import synth as S
+    L = S.make_layer(S.LayerSpec(w["d"], w["f"], sigma=w["sigma"], seed=0))
+    Por = oracle.make_proxy(L)
+    x_cal = S.make_tokens(min(w["n_cal"], 64), w["d"], stream="x_cal", outlier_frac=w["outlier"])
+    tau_x, tau_s = oracle.calibrate(x_cal, Por, keep_x, keep_s)
+    x = S.make_tokens(w["tokens"], w["d"], stream="x_eval", outlier_frac=w["outlier"])
+    cores = os.cpu_count() or 1
+    done, t_used, threads = 0, 0.0, 1
+    chunk = max(1, cores)
+    while done < w["tokens"] and t_used < seconds:
+        n = min(chunk, w["tokens"] - done)
+        t0 = time.perf_counter()
+        out = oracle.forward(x[done:done + n], tau_x, tau_s, L, Por, want=())
+        t_used += time.perf_counter() - t0
+        threads = out["threads"]
+        done += n
+    sample = (f"{done} of {w['tokens']} tokens of the {w['d']}x{w['f']} layer "
+              f"(thresholds from {x_cal.shape[0]} calibration vectors), all stages, fp64")
+    return t_used / done * 1e6, threads, sample
+
+
+def run_reference(args, w, rank, world):
+    if rank != 0:
+        return
+    us, cores, sample = cpu_oracle_time(w, args.keep_x, args.keep_s, args.cpu_seconds)
+    ms_step = us * w["tokens"] / 1e3
+    line = {
+        "impl": "reference", "metric": METRIC, "value": us, "unit": "us/token/layer",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "d_model": w["d"], "d_ff": w["f"], "batch": 1,
+                   "tokens_per_step": w["tokens"], "keep_x": args.keep_x, "keep_s": args.keep_s},
+        "cpu_baseline": {"value": us, "unit": "us/token/layer", "cores": cores,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": us, "unit": "us/token/layer", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args, w, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from free_ffn_activation_b200 import prox as P
+    from free_ffn_activation_b200 import synth as S
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    d, f, ntok = w["d"], w["f"], w["tokens"]
+    # each rank an independent replica with its own token stream
+    L = S.make_layer(S.LayerSpec(d, f, sigma=w["sigma"], seed=0))
+    x_np = S.make_tokens(ntok, d, seed=rank, stream="x_eval", outlier_frac=w["outlier"])
+    xc_np = S.make_tokens(w["n_cal"], d, seed=0, stream="x_cal", outlier_frac=w["outlier"])
+    base = P.ProxLayer.from_weights(L["w_up_cm"], L["w_gate_cm"], L["w_down"], device=dev)
+    tau_x, tau_s = P.calibrate(base, P.as_bf16(xc_np, dev), args.keep_x, args.keep_s)
+    R = max(1, args.copies)
+    layers = [base] + [P.ProxLayer(*(t.clone() for t in (
+        base.w_up_cm, base.w_gate_cm, base.w_down, base.q_up, base.q_gate, base.s_up, base.s_gate)))
+        for _ in range(R - 1)]
+    structs = [lay.cstruct() for lay in layers]
+    x = P.as_bf16(x_np, dev).contiguous()
+    y = torch.empty((ntok, d), dtype=torch.float32, device=dev)
+    ws = P.workspace(d, f, 1, dev)
+    wsb = ws.numel()
+
+    # realised keep ratios (untimed)
+    out = P.ffn_forward(base, x, tau_x, tau_s)
+    kx = out.mask_x.sum(dim=1).double().cpu().numpy()
+    ks = out.count_s.double().cpu().numpy()
+    touched = np.array([P.touched_bytes(d, f, int(a), int(b)) for a, b in zip(kx, ks)])
+    stage2_bytes = 3 * ks * d * 2
+
+    stream = torch.cuda.Stream(dev)
+    sp = stream.cuda_stream
+    xrow = d * 2
+    yrow = d * 4
+    xp, yp, wp = x.data_ptr(), y.data_ptr(), ws.data_ptr()
+    sample_every = 8
+    sampled = list(range(0, ntok, sample_every))
+    ev_a = {t: torch.cuda.Event(enable_timing=True, external=True) for t in sampled}
+    ev_b = {t: torch.cuda.Event(enable_timing=True, external=True) for t in sampled}
+
+    def one_step(record):
+        for t in range(ntok):
+            Ls = structs[t % R]
+            P.ffn_stage1_raw(Ls, xp + t * xrow, 1, tau_x, tau_s, yp + t * yrow, wp, wsb, sp)
+            if record and t in ev_a:
+                ev_a[t].record(stream)
+            P.ffn_stage2_raw(Ls, xp + t * xrow, 1, yp + t * yrow, wp, wsb, sp)
+            if record and t in ev_b:
+                ev_b[t].record(stream)
+
+    with torch.cuda.stream(stream):
+        one_step(False)
+    torch.cuda.synchronize(dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        one_step(True)
+    # parity spot-check of the graph's output against the direct call
+    g.replay()
+    torch.cuda.synchronize(dev)
+    assert torch.allclose(y[:8], out.y[:8], rtol=1e-4, atol=1e-5), "graph output differs"
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        g.replay()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    s2_ms = []
+    with ClockSampler(local_rank) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            with torch.cuda.stream(stream):
+                g.replay()
+            torch.cuda.current_stream(dev).wait_stream(stream)
+        e1.record(stream)
+        barrier()
+        # per-launch Stage-2 durations of the last replay's sampled tokens
+        s2_ms = [ev_a[t].elapsed_time(ev_b[t]) for t in sampled]
+    ms_total = e0.elapsed_time(e1)
+    if world > 1:
+        tt = torch.tensor([ms_total], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_total = float(tt.item())
+    ms_step = ms_total / args.steps
+    us_tok = ms_step * 1e3 / (ntok * world)
+    us_tok_rank = ms_step * 1e3 / ntok
+
+    peak, peak_src = load_peaks()
+    s2_us = statistics.mean(s2_ms) * 1e3
+    s2_bytes = float(np.mean(stage2_bytes[sampled]))
+    s2_gbs = s2_bytes / (s2_us * 1e-6) / 1e9
+    path_gbs = float(np.mean(touched)) / (us_tok_rank * 1e-6) / 1e9
+
+    # e2e through the public API with host buffers: pinned x in, y out
+    x_host = x.cpu().pin_memory()
+    y_host = torch.empty((ntok, d), dtype=torch.float32).pin_memory()
+    e2e_steps = max(1, min(args.steps, 5))
+
+    def e2e_step():
+        with torch.cuda.stream(stream):
+            x.copy_(x_host, non_blocking=True)
+            for t in range(ntok):
+                P.ffn_forward_raw(structs[t % R], xp + t * xrow, 1, tau_x, tau_s,
+                                  yp + t * yrow, wp, wsb, sp)
+            y_host.copy_(y, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    barrier()
+    f0 = torch.cuda.Event(enable_timing=True)
+    f1 = torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    f1.record(stream)
+    barrier()
+    e2e_ms = f0.elapsed_time(f1) / e2e_steps
+    if world > 1:
+        tt = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    e2e_us = e2e_ms * 1e3 / (ntok * world)
+
+    # dense bf16 reference on the same GPU, same protocol (cuBLAS GEMV)
+    dense = None
+    if not args.no_dense:
+        import torch.nn.functional as F
+        wd_t = [lay.w_down.t().contiguous() for lay in layers]
+        xs = x
+        yd = torch.empty((ntok, d), dtype=torch.bfloat16, device=dev)
+
+        def dense_step():
+            for t in range(ntok):
+                lay = layers[t % R]
+                xt = xs[t:t + 1]
+                u = F.linear(xt, lay.w_up_cm)
+                gg = F.linear(xt, lay.w_gate_cm)
+                yd[t:t + 1] = F.linear(F.silu(gg) * u, wd_t[t % R])
+
+        with torch.cuda.stream(stream):
+            dense_step()
+        torch.cuda.synchronize(dev)
+        gd = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gd, stream=stream):
+            dense_step()
+        for _ in range(args.warmup):
+            gd.replay()
+        barrier()
+        d0 = torch.cuda.Event(enable_timing=True)
+        d1 = torch.cuda.Event(enable_timing=True)
+        d0.record(stream)
+        for _ in range(args.steps):
+            with torch.cuda.stream(stream):
+                gd.replay()
+        d1.record(stream)
+        barrier()
+        dense_us = d0.elapsed_time(d1) / args.steps * 1e3 / ntok
+        dense_bytes = 3 * d * f * 2
+        dense = {"us_per_token": dense_us,
+                 "GBps": dense_bytes / (dense_us * 1e-6) / 1e9,
+                 "speedup_of_sparse": dense_us / us_tok_rank,
+                 "kind": "torch F.linear x3 + silu*mul (cuBLAS), bf16, same graph/L2 protocol"}
+        del gd
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        us_cpu, cores, sample = cpu_oracle_time(w, args.keep_x, args.keep_s, args.cpu_seconds)
+        cpu = {"value": us_cpu, "unit": "us/token/layer", "cores": cores, "kind": "oracle",
+               "sample": sample}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": us_tok, "unit": "us/token/layer", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": args.workload, "d_model": d, "d_ff": f, "batch": 1,
+                       "tokens_per_step": ntok, "keep_x": args.keep_x, "keep_s": args.keep_s,
+                       "tau_x": tau_x, "tau_s": tau_s,
+                       "l2": f"{R} rotating weight copies ({R * (3 * d * f * 2 + d * f + 8 * d) / 1e9:.2f} GB > L2)",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": {"bound": "hbm", "kernel": "k_stage2 (exact up/gate/down)",
+                         "achieved": s2_gbs, "peak": peak, "unit": "GB/s",
+                         "frac": s2_gbs / peak, "traffic": None, "peak_source": peak_src,
+                         "bytes_per_launch": s2_bytes, "us_per_launch": s2_us},
+            "path": {"touched_MB_per_token": float(np.mean(touched)) / 1e6,
+                     "GBps": path_gbs, "frac_of_peak": path_gbs / peak,
+                     "keep_x": float(np.mean(kx)) / d, "keep_s": float(np.mean(ks)) / f},
+            "dense_ref": dense,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_us, "unit": "us/token/layer",
+                    "h2d_bytes_per_step": ntok * d * 2, "d2h_bytes_per_step": ntok * d * 4},
+            "gpu_launches": 2 * ntok * args.steps,
+            "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    del g
+
+
+def main():
+    args = parse()
+    w = WORKLOADS[args.workload]
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, w, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_ours(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,418 @@
+// Stage 1 of the Prox sparse SwiGLU FFN on sm_100a: input mask, input-sparse
+// INT4 proxy GEMVs for up and gate, proxy state and the shared channel mask
+// (Prox deep-dive blog, section "Stage 1"; input-sparse projection Pi_in of
+// the translated arXiv page, section 2.2).
+//
+// Work split. The proxies are stored input-row-major ([d_model][d_ff/2]
+// nibbles), so a rejected input coordinate skips one whole contiguous row.
+// The d_ff channels are cut into column blocks of kCB = 256 channels (128
+// bytes of each proxy row); the kept rows are cut into n_r contiguous rank
+// ranges. CTA (c, r) streams the 128-byte segments of block c from the kept
+// rows of range r of BOTH proxies (one x read serves up and gate, as the
+// blog's "From formula to GPU" section describes for its split-N kernel) and
+// writes fp32 partial sums. The last CTA of a block to arrive (atomic ticket,
+// no waiting) sums the n_r partials in a fixed order, forms
+// s~ = u~ * SiLU(g~), thresholds it and compacts the kept channels into
+// ascending lists, so the result is deterministic.
+//
+// INT4 decode. A nibble n at bits 4p..4p+3 of a word, with every other bit
+// cleared, is the bit pattern of the subnormal float n * 2^(4p-149). XOR-ing
+// the nibble's top bit turns the stored two's complement code q into
+// n = q + 8 in the same single LOP3, so one logic op per weight yields an
+// exact float operand; the FMA multiplies it by x_i * scale_i pre-scaled by
+// 2^E (E chosen per CTA so products stay normal). At the end each channel's
+// sum is rescaled by the exact power of two 2^(149 - 4p - E) and the offset
+// 8 * sum(x_i * scale_i) is removed. Nibbles 5..7 of a word are first shifted
+// down by 12 bits (to positions 2..4). Subnormal operands need FMA without
+// flush-to-zero, which is the default without fast-math.
+#include "prox_internal.cuh"
+
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace prox {
+namespace {
+
+template <int B>
+struct S1 {
+    static constexpr int CPT = (B == 1) ? 32 : (B <= 4 ? 16 : 8);  // channels per thread
+    static constexpr int BYTES = CPT / 2;                            // bytes per row per thread
+    static constexpr int WORDS = BYTES / 4;
+    static constexpr int ACC = B * CPT;
+    static constexpr int TPRM = kCB / CPT;                           // threads per row per matrix
+    static constexpr int TPR = 2 * TPRM;                             // threads per row
+    static constexpr int RL = kS1Threads / TPR;                      // row lanes
+    static constexpr int U = 128 / BYTES;                            // rows in flight per thread
+};
+
+template <int WORDS>
+struct Vec;
+template <>
+struct Vec<4> {
+    uint32_t w[4];
+};
+template <>
+struct Vec<2> {
+    uint32_t w[2];
+};
+template <>
+struct Vec<1> {
+    uint32_t w[1];
+};
+
+__device__ __forceinline__ void ld_stream(Vec<4> &v, const uint8_t *p) {
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3])
+                 : "l"(p));
+}
+__device__ __forceinline__ void ld_stream(Vec<2> &v, const uint8_t *p) {
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
+                 : "=r"(v.w[0]), "=r"(v.w[1])
+                 : "l"(p));
+}
+__device__ __forceinline__ void ld_stream(Vec<1> &v, const uint8_t *p) {
+    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v.w[0]) : "l"(p));
+}
+
+// nibble position (in units of 4 bits) of local channel k of a word after
+// the decode above
+__host__ __device__ constexpr int nib_pos(int k) { return k < 5 ? k : k - 3; }
+
+__device__ __forceinline__ float nib_f(uint32_t w, int p) {
+    return __uint_as_float((w & (0xFu << (4 * p))) ^ (0x8u << (4 * p)));
+}
+
+// acc[t * CPT + wi * 8 + k] += xs[t] * code_k * 2^(4 pos(k) - 149)
+template <int B, int CPT>
+__device__ __forceinline__ void proc_word(uint32_t w, int wi, const float *xs, float *acc) {
+    const uint32_t v = w >> 12;
+    float2 d01 = make_float2(nib_f(w, 0), nib_f(w, 1));
+    float2 d23 = make_float2(nib_f(w, 2), nib_f(w, 3));
+    float2 d45 = make_float2(nib_f(w, 4), nib_f(v, 2));
+    float2 d67 = make_float2(nib_f(v, 3), nib_f(v, 4));
+#pragma unroll
+    for (int t = 0; t < B; ++t) {
+        const float2 xx = make_float2(xs[t], xs[t]);
+        float *a = acc + t * CPT + wi * 8;
+        float2 a01 = make_float2(a[0], a[1]);
+        float2 a23 = make_float2(a[2], a[3]);
+        float2 a45 = make_float2(a[4], a[5]);
+        float2 a67 = make_float2(a[6], a[7]);
+        a01 = __ffma2_rn(xx, d01, a01);
+        a23 = __ffma2_rn(xx, d23, a23);
+        a45 = __ffma2_rn(xx, d45, a45);
+        a67 = __ffma2_rn(xx, d67, a67);
+        a[0] = a01.x; a[1] = a01.y; a[2] = a23.x; a[3] = a23.y;
+        a[4] = a45.x; a[5] = a45.y; a[6] = a67.x; a[7] = a67.y;
+    }
+}
+
+// deterministic block-wide exclusive scan of one int per thread (256 threads)
+__device__ __forceinline__ int block_excl_scan(int v, int *warp_tot, int &total) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    int inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        int n = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += n;
+    }
+    if (lane == 31) warp_tot[wid] = inc;
+    __syncthreads();
+    int base = 0, tot = 0;
+#pragma unroll
+    for (int w = 0; w < kS1Threads / 32; ++w) {
+        if (w < wid) base += warp_tot[w];
+        tot += warp_tot[w];
+    }
+    __syncthreads();
+    total = tot;
+    return base + inc - v;
+}
+
+template <int B>
+__global__ void __launch_bounds__(kS1Threads, 2) k_stage1(const Stage1Args a) {
+    using T = S1<B>;
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int c = blockIdx.x % a.C;
+    const int r = blockIdx.x / a.C;
+    const int W = a.d / 32;  // mask words per token
+
+    // shared memory carve-up
+    float *red = reinterpret_cast<float *>(smem);                    // [RL][2][B][kCB]
+    uint32_t *tmask = reinterpret_cast<uint32_t *>(red + T::RL * 2 * B * kCB);  // [B][W]
+    uint32_t *umask = tmask + B * W;                                  // [W]
+    int *woff = reinterpret_cast<int *>(umask + W);                   // [W]
+    int *rowidx = woff + W;                                           // [unit_cap]
+    float *xs = reinterpret_cast<float *>(rowidx + a.unit_cap);       // [unit_cap][2][B]
+    __shared__ int s_warp[kS1Threads / 32];
+    __shared__ float s_red[kS1Threads / 32][4 * kMaxB];
+    __shared__ float s_S[2 * kMaxB];
+    __shared__ int s_E[kMaxB];
+    __shared__ int s_last;
+    __shared__ int s_cnt[kS1Threads / 32][kMaxB + 1];
+
+    // (1) Stage 2 accumulates y with atomics: clear it here.
+    if (a.y_zero) {
+        float4 *y4 = reinterpret_cast<float4 *>(a.y_zero);
+        const int n4 = a.nb * a.d / 4;
+        for (int k = blockIdx.x * kS1Threads + tid; k < n4; k += gridDim.x * kS1Threads)
+            y4[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+
+    // (2) input masks m_x = 1[|x_i| >= tau_x] per token, and their union
+    for (int wd = wid; wd < W; wd += kS1Threads / 32) {
+        uint32_t un = 0;
+#pragma unroll
+        for (int t = 0; t < B; ++t) {
+            uint32_t bits = 0;
+            if (t < a.nb) {
+                const uint16_t h = a.x[(size_t)t * a.d + wd * 32 + lane];
+                const bool keep = fabsf(__uint_as_float((uint32_t)h << 16)) >= a.tau_x;
+                bits = __ballot_sync(0xffffffffu, keep);
+                if (a.mask_x && blockIdx.x == 0)
+                    a.mask_x[(size_t)t * a.d + wd * 32 + lane] = keep ? 1 : 0;
+            }
+            if (lane == 0) tmask[t * W + wd] = bits;
+            un |= bits;
+        }
+        if (lane == 0) umask[wd] = un;
+    }
+    __syncthreads();
+
+    // (3) ranks of the kept (union) rows
+    int kx;
+    {
+        const int per = (W + kS1Threads - 1) / kS1Threads;
+        int loc = 0;
+        for (int k = 0; k < per; ++k) {
+            const int wd = tid * per + k;
+            if (wd < W) loc += __popc(umask[wd]);
+        }
+        int base = block_excl_scan(loc, s_warp, kx);
+        for (int k = 0; k < per; ++k) {
+            const int wd = tid * per + k;
+            if (wd < W) {
+                woff[wd] = base;
+                base += __popc(umask[wd]);
+            }
+        }
+    }
+    const int lo = (int)((long long)kx * r / a.n_r);
+    const int hi = (int)((long long)kx * (r + 1) / a.n_r);
+    const int n_units = hi - lo;
+    __syncthreads();
+
+    // (4) this CTA's units: row index and x_i * scale_i per matrix and token
+    for (int wd = wid; wd < W; wd += kS1Threads / 32) {
+        const uint32_t um = umask[wd];
+        if (!((um >> lane) & 1u)) continue;
+        const int rank = woff[wd] + __popc(um & ((1u << lane) - 1u));
+        if (rank < lo || rank >= hi) continue;
+        const int u = rank - lo;
+        const int i = wd * 32 + lane;
+        rowidx[u] = i;
+        const float su = a.s_up[i], sg = a.s_gate[i];
+#pragma unroll
+        for (int t = 0; t < B; ++t) {
+            float xv = 0.f;
+            if ((tmask[t * W + wd] >> lane) & 1u)
+                xv = __uint_as_float((uint32_t)a.x[(size_t)t * a.d + i] << 16);
+            xs[(u * 2 + 0) * B + t] = xv * su;
+            xs[(u * 2 + 1) * B + t] = xv * sg;
+        }
+    }
+    __syncthreads();
+
+    // (5) per token: S = sum of x_i * scale_i per matrix (offset removal) and
+    // the power-of-two pre-scale E from max |x_i * scale_i|
+    {
+        float v[4 * B];
+#pragma unroll
+        for (int k = 0; k < 4 * B; ++k) v[k] = 0.f;
+        for (int u = tid; u < n_units; u += kS1Threads) {
+#pragma unroll
+            for (int m = 0; m < 2; ++m)
+#pragma unroll
+                for (int t = 0; t < B; ++t) {
+                    const float q = xs[(u * 2 + m) * B + t];
+                    v[m * B + t] += q;
+                    v[2 * B + t] = fmaxf(v[2 * B + t], fabsf(q));
+                }
+        }
+#pragma unroll
+        for (int k = 0; k < 4 * B; ++k) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const float n = __shfl_xor_sync(0xffffffffu, v[k], o);
+                v[k] = (k < 2 * B) ? v[k] + n : fmaxf(v[k], n);
+            }
+            if (lane == 0) s_red[wid][k] = v[k];
+        }
+        __syncthreads();
+        if (tid < 3 * B) {
+            float acc = (tid < 2 * B) ? 0.f : 0.f;
+            for (int w = 0; w < kS1Threads / 32; ++w)
+                acc = (tid < 2 * B) ? acc + s_red[w][tid] : fmaxf(acc, s_red[w][tid]);
+            if (tid < 2 * B) {
+                s_S[tid] = acc;
+            } else {
+                const int t = tid - 2 * B;
+                s_E[t] = (acc > 0.f) ? 119 - ilogbf(acc) : 0;
+            }
+        }
+        __syncthreads();
+        for (int k = tid; k < n_units * 2 * B; k += kS1Threads)
+            xs[k] = ldexpf(xs[k], s_E[k % B]);
+        __syncthreads();
+    }
+
+    // (6) main loop: stream the 128-byte block segments of the kept rows
+    const int rl = tid / T::TPR;
+    const int m = (tid / T::TPRM) & 1;
+    const int chunk = tid % T::TPRM;
+    const uint8_t *qbase = (m ? a.q_gate : a.q_up) + (size_t)c * (kCB / 2) + chunk * T::BYTES;
+    const size_t rstride = (size_t)a.f / 2;
+    float acc[T::ACC];
+#pragma unroll
+    for (int k = 0; k < T::ACC; ++k) acc[k] = 0.f;
+
+    for (int u0 = rl; u0 < n_units; u0 += T::RL * T::U) {
+        Vec<T::WORDS> v[T::U];
+#pragma unroll
+        for (int k = 0; k < T::U; ++k) {
+            const int u = u0 + k * T::RL;
+            if (u < n_units) {
+                ld_stream(v[k], qbase + (size_t)rowidx[u] * rstride);
+            } else {
+#pragma unroll
+                for (int q = 0; q < T::WORDS; ++q) v[k].w[q] = 0x88888888u;  // code 0
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < T::U; ++k) {
+            const int u = u0 + k * T::RL;
+            float xv[B];
+#pragma unroll
+            for (int t = 0; t < B; ++t) xv[t] = (u < n_units) ? xs[(u * 2 + m) * B + t] : 0.f;
+#pragma unroll
+            for (int q = 0; q < T::WORDS; ++q) proc_word<B, T::CPT>(v[k].w[q], q, xv, acc);
+        }
+    }
+
+    // (7) reduce row lanes, undo the pre-scale and the +8 code offset, write
+    // this CTA's partial sums
+#pragma unroll
+    for (int t = 0; t < B; ++t)
+#pragma unroll
+        for (int k = 0; k < T::CPT; ++k)
+            red[((rl * 2 + m) * B + t) * kCB + chunk * T::CPT + k] = acc[t * T::CPT + k];
+    __syncthreads();
+    {
+        const int ch = tid;  // channel within the block
+        const int p = nib_pos(ch % 8);
+        float *part = a.partials + (((size_t)c * kS1MaxRowGroups + r) * 2) * B * kCB;
+#pragma unroll
+        for (int mm = 0; mm < 2; ++mm)
+#pragma unroll
+            for (int t = 0; t < B; ++t) {
+                float s = 0.f;
+                for (int q = 0; q < T::RL; ++q) s += red[((q * 2 + mm) * B + t) * kCB + ch];
+                const float val = ldexpf(s, 149 - 4 * p - s_E[t]) - 8.f * s_S[mm * B + t];
+                part[(mm * B + t) * kCB + ch] = val;
+            }
+    }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = (atomicInc(&a.arrive[c], (unsigned)(a.n_r - 1)) == (unsigned)(a.n_r - 1));
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+
+    // (8) last CTA of block c: s~ = u~ * SiLU(g~), m_s = 1[|s~| >= tau_s],
+    // ascending compaction per token and of the union
+    const int ch = tid;
+    const int j = c * kCB + ch;
+    uint32_t bits = 0;
+#pragma unroll
+    for (int t = 0; t < B; ++t) {
+        if (t >= a.nb) break;
+        float u = 0.f, g = 0.f;
+        for (int q = 0; q < a.n_r; ++q) {
+            const float *part = a.partials + (((size_t)c * kS1MaxRowGroups + q) * 2) * B * kCB;
+            u += __ldcg(part + (0 * B + t) * kCB + ch);
+            g += __ldcg(part + (1 * B + t) * kCB + ch);
+        }
+        const float st = u * (g / (1.f + expf(-g)));
+        if (a.s_out) a.s_out[(size_t)t * a.f + j] = st;
+        const bool keep = fabsf(st) >= a.tau_s;
+        if (a.mask_s) a.mask_s[(size_t)t * a.f + j] = keep ? 1 : 0;
+        bits |= (keep ? 1u : 0u) << t;
+    }
+    if (!a.build_lists) return;
+    // warp ballots and per-warp counts (token t in column t, union in column B)
+    uint32_t bal[kMaxB + 1];
+#pragma unroll
+    for (int t = 0; t <= B; ++t) {
+        const bool k = (t < B) ? ((bits >> t) & 1u) : (bits != 0u);
+        bal[t] = __ballot_sync(0xffffffffu, k);
+        if (lane == 0) s_cnt[wid][t] = __popc(bal[t]);
+    }
+    __syncthreads();
+    const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll
+    for (int t = 0; t <= B; ++t) {
+        int base = 0, tot = 0;
+        for (int w = 0; w < kS1Threads / 32; ++w) {
+            if (w < wid) base += s_cnt[w][t];
+            tot += s_cnt[w][t];
+        }
+        const bool k = (bal[t] >> lane) & 1u;
+        const int pos = base + __popc(bal[t] & lt);
+        if (t < B) {
+            if (k) a.tlist[(size_t)t * a.f + c * kCB + pos] = j;
+            if (tid == 0) a.tcount[c * B + t] = (t < a.nb) ? tot : 0;
+        } else {
+            if (k) a.ulist[(size_t)c * kCB + pos] = (uint32_t)j | (bits << 24);
+            if (tid == 0) a.ucount[c] = tot;
+        }
+    }
+}
+
+template <int B>
+cudaError_t launch1(const Stage1Args &a, const Stage1Plan &p, cudaStream_t s) {
+    auto k = k_stage1<B>;
+    static size_t configured = 0;  // dynamic smem limit already set for this kernel
+    if (p.smem > configured) {
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)p.smem);
+        if (e != cudaSuccess) return e;
+        configured = p.smem;
+    }
+    k<<<a.C * a.n_r, kS1Threads, p.smem, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_stage1(int B, const Stage1Args &a, const Stage1Plan &p, cudaStream_t s) {
+    switch (B) {
+        case 1: return launch1<1>(a, p, s);
+        case 2: return launch1<2>(a, p, s);
+        case 4: return launch1<4>(a, p, s);
+        case 8: return launch1<8>(a, p, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+// shared-memory bytes of one Stage-1 CTA for a plan (kept next to the kernel's
+// carve-up above)
+size_t stage1_smem_bytes(int d_model, int B, int unit_cap) {
+    const int tpr = 2 * (kCB / ((B == 1) ? 32 : (B <= 4 ? 16 : 8)));
+    const int rl = kS1Threads / tpr;
+    const int W = d_model / 32;
+    return (size_t)rl * 2 * B * kCB * 4 + (size_t)(B + 2) * W * 4 +
+           (size_t)unit_cap * (4 + 8 * B);
+}
+
+}  // namespace prox

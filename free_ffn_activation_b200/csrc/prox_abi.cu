@@ -1,0 +1,467 @@
+// Host side of the libprox C ABI (see include/prox.h): argument validation,
+// device checks, launch plans, workspace layout and kernel orchestration.
+// Nothing here computes any step of the method; every step runs in the
+// kernels of k_stage1.cu, k_stage2.cu and k_quantize.cu.
+#include "prox_internal.cuh"
+
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#define PROX_API extern "C" __attribute__((visibility("default")))
+
+namespace prox {
+
+size_t stage1_smem_bytes(int d_model, int B, int unit_cap);
+size_t stage2_smem_bytes(int d_model, int B, int nstage, int C);
+
+int max_tokens_per_pass(int d_model) {
+    if (d_model <= 4096) return 8;
+    if (d_model <= 8192) return 4;
+    return 0;
+}
+
+static int pow2_ceil(int v) {
+    int p = 1;
+    while (p < v) p <<= 1;
+    return p;
+}
+
+int tokens_per_pass(int d_model, int batch) {
+    const int mx = max_tokens_per_pass(d_model);
+    if (mx == 0) return 0;
+    int b = batch < 1 ? 1 : batch;
+    if (b > mx) b = mx;
+    return pow2_ceil(b);
+}
+
+Stage1Plan stage1_plan(int d, int f, int B, int num_sms) {
+    Stage1Plan p;
+    p.C = f / kCB;
+    const size_t red_and_masks = stage1_smem_bytes(d, B, 0);
+    const size_t per_unit = 4 + 8 * (size_t)B;
+    // two CTAs per SM: keep each under ~110 KB of shared memory
+    const size_t budget = 110 * 1024;
+    const size_t unit_budget = budget > red_and_masks ? budget - red_and_masks : per_unit;
+    int n_smem = (int)(((size_t)d * per_unit + unit_budget - 1) / unit_budget);
+    int n_bal = (2 * num_sms) / p.C;
+    int n_r = n_bal > n_smem ? n_bal : n_smem;
+    if (n_r < 1) n_r = 1;
+    if (n_r > kS1MaxRowGroups) n_r = kS1MaxRowGroups;
+    p.n_r = n_r;
+    p.unit_cap = (d + n_r - 1) / n_r;
+    p.smem = stage1_smem_bytes(d, B, p.unit_cap);
+    return p;
+}
+
+Stage2Plan stage2_plan(int d, int B) {
+    Stage2Plan p;
+    p.nchunk = pow2_ceil((d / 8 + kNCW * 32 - 1) / (kNCW * 32));
+    const size_t stage = (size_t)6 * d;
+    const size_t fixed = stage2_smem_bytes(d, B, 0, 1024);  // upper bound on C
+    int ns = (int)((kS2SmemBudget - fixed) / stage);
+    if (ns > 16) ns = 16;
+    p.nstage = ns;
+    p.smem = 0;
+    return p;
+}
+
+static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+WsLayout ws_layout(int d, int f, int B) {
+    (void)d;
+    const size_t C = (size_t)f / kCB;
+    WsLayout L;
+    size_t o = 0;
+    L.status = o;
+    o += 256;
+    L.arrive = o;
+    o = align_up(o + C * 4, 256);
+    L.ucount = o;
+    o = align_up(o + C * 4, 256);
+    L.tcount = o;
+    o = align_up(o + C * B * 4, 256);
+    L.ulist = o;
+    o = align_up(o + C * kCB * 4, 256);
+    L.tlist = o;
+    o = align_up(o + (size_t)B * f * 4, 256);
+    L.partials = o;
+    o = align_up(o + C * kS1MaxRowGroups * 2 * B * kCB * 4, 256);
+    L.total = o;
+    return L;
+}
+
+// ---------------------------------------------------------------------------
+// device checks
+// ---------------------------------------------------------------------------
+struct DevInfo {
+    int checked = 0;
+    int ok = 0;
+    int sms = 0;
+};
+static DevInfo g_dev[64];
+static std::mutex g_dev_mu;
+
+static prox_status current_device(int *sms) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return PROX_ECUDA;
+    if (dev < 0 || dev >= 64) return PROX_EDEVICE;
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DevInfo &di = g_dev[dev];
+    if (!di.checked) {
+        int major = 0, n = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return PROX_ECUDA;
+        di.ok = (major == 10);
+        di.sms = n;
+        di.checked = 1;
+    }
+    if (!di.ok) return PROX_EDEVICE;
+    *sms = di.sms;
+    return PROX_OK;
+}
+
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static bool shape_ok(int d, int f) {
+    return d >= 256 && f >= 256 && d % 256 == 0 && f % 256 == 0 && max_tokens_per_pass(d) > 0 &&
+           f <= 1024 * kCB;  // Stage-2 shared memory holds per-block scans of <= 1024 blocks
+}
+
+static prox_status check_layer(const prox_layer *L, bool need_exact) {
+    if (!L || !shape_ok(L->d_model, L->d_ff)) return PROX_EINVAL;
+    if (!L->q_up || !L->q_gate || !L->s_up || !L->s_gate) return PROX_EINVAL;
+    if (!aligned16(L->q_up) || !aligned16(L->q_gate) || !aligned16(L->s_up) ||
+        !aligned16(L->s_gate))
+        return PROX_EINVAL;
+    if (need_exact) {
+        if (!L->w_up_cm || !L->w_gate_cm || !L->w_down) return PROX_EINVAL;
+        if (!aligned16(L->w_up_cm) || !aligned16(L->w_gate_cm) || !aligned16(L->w_down))
+            return PROX_EINVAL;
+    }
+    return PROX_OK;
+}
+
+static bool tau_ok(float t) { return std::isfinite(t) && t >= 0.f; }
+
+// test hooks (set by prox_debug_set through the binding's test helpers only)
+static uint32_t g_spin_limit = kDefaultSpinLimit;
+static int g_debug_skip = -1;
+
+// One pass (nb <= tokens_per_pass tokens) of Stage 1: masks, kept-channel
+// lists in the workspace, s~ when s_out is given, and y cleared when given.
+static prox_status pass_stage1(const prox_layer *L, const uint16_t *x, int nb, float tau_x,
+                               float tau_s, float *y_clear, uint8_t *mask_x, uint8_t *mask_s,
+                               float *s_out, unsigned char *w, int sms, bool lists,
+                               cudaStream_t st) {
+    const int d = L->d_model, f = L->d_ff;
+    const int B = pow2_ceil(nb);
+    const WsLayout W = ws_layout(d, f, B);
+    const Stage1Plan p1 = stage1_plan(d, f, B, sms);
+    Stage1Args a{};
+    a.d = d;
+    a.f = f;
+    a.nb = nb;
+    a.C = p1.C;
+    a.n_r = p1.n_r;
+    a.unit_cap = p1.unit_cap;
+    a.x = x;
+    a.tau_x = tau_x;
+    a.tau_s = tau_s;
+    a.q_up = L->q_up;
+    a.q_gate = L->q_gate;
+    a.s_up = L->s_up;
+    a.s_gate = L->s_gate;
+    a.y_zero = y_clear;
+    a.mask_x = mask_x;
+    a.mask_s = mask_s;
+    a.s_out = s_out;
+    a.build_lists = lists ? 1 : 0;
+    a.partials = reinterpret_cast<float *>(w + W.partials);
+    a.arrive = reinterpret_cast<uint32_t *>(w + W.arrive);
+    a.ucount = reinterpret_cast<int32_t *>(w + W.ucount);
+    a.tcount = reinterpret_cast<int32_t *>(w + W.tcount);
+    a.ulist = reinterpret_cast<uint32_t *>(w + W.ulist);
+    a.tlist = reinterpret_cast<int32_t *>(w + W.tlist);
+    return launch_stage1(B, a, p1, st) == cudaSuccess ? PROX_OK : PROX_ECUDA;
+}
+
+// One pass of Stage 2, consuming the lists the preceding Stage 1 left in w.
+static prox_status pass_stage2(const prox_layer *L, const uint16_t *x, int nb, float *y,
+                               int32_t *idx_s, int32_t *count_s, unsigned char *w, int sms,
+                               cudaStream_t st) {
+    const int d = L->d_model, f = L->d_ff;
+    const int B = pow2_ceil(nb);
+    const WsLayout W = ws_layout(d, f, B);
+    const Stage2Plan p2 = stage2_plan(d, B);
+    const int C = f / kCB;
+    Stage2Args b{};
+    b.d = d;
+    b.f = f;
+    b.nb = nb;
+    b.C = C;
+    b.x = x;
+    b.w_up = L->w_up_cm;
+    b.w_gate = L->w_gate_cm;
+    b.w_down = L->w_down;
+    b.y = y;
+    b.idx_s = idx_s;
+    b.count_s = count_s;
+    b.ucount = reinterpret_cast<int32_t *>(w + W.ucount);
+    b.tcount = reinterpret_cast<int32_t *>(w + W.tcount);
+    b.ulist = reinterpret_cast<uint32_t *>(w + W.ulist);
+    b.tlist = reinterpret_cast<int32_t *>(w + W.tlist);
+    b.status = reinterpret_cast<uint32_t *>(w + W.status);
+    b.spin_limit = g_spin_limit;
+    b.debug_skip = g_debug_skip;
+    b.nstage = p2.nstage;
+    const size_t smem = stage2_smem_bytes(d, B, p2.nstage, C);
+    return launch_stage2(B, p2.nchunk, b, sms, smem, st) == cudaSuccess ? PROX_OK : PROX_ECUDA;
+}
+
+// Stage 1 [+ Stage 2] over `batch` tokens, in passes of at most B tokens
+static prox_status run_forward(const prox_layer *L, const uint16_t *x, int batch, float tau_x,
+                               float tau_s, float *y, uint8_t *mask_x, uint8_t *mask_s,
+                               int32_t *idx_s, int32_t *count_s, float *s_out, void *ws,
+                               size_t ws_bytes, cudaStream_t st, bool stage2) {
+    int sms = 0;
+    prox_status ps = current_device(&sms);
+    if (ps != PROX_OK) return ps;
+    const int d = L->d_model, f = L->d_ff;
+    const int Bmax = tokens_per_pass(d, batch);
+    if (ws_bytes < ws_layout(d, f, Bmax).total) return PROX_ENOMEM;
+    unsigned char *w = static_cast<unsigned char *>(ws);
+    for (int t0 = 0; t0 < batch; t0 += Bmax) {
+        const int nb = (batch - t0) < Bmax ? (batch - t0) : Bmax;
+        const uint16_t *xt = x + (size_t)t0 * d;
+        ps = pass_stage1(L, xt, nb, tau_x, tau_s, stage2 ? y + (size_t)t0 * d : nullptr,
+                         mask_x ? mask_x + (size_t)t0 * d : nullptr,
+                         mask_s ? mask_s + (size_t)t0 * f : nullptr,
+                         s_out ? s_out + (size_t)t0 * f : nullptr, w, sms, stage2, st);
+        if (ps != PROX_OK || !stage2) {
+            if (ps != PROX_OK) return ps;
+            continue;
+        }
+        ps = pass_stage2(L, xt, nb, y + (size_t)t0 * d, idx_s ? idx_s + (size_t)t0 * f : nullptr,
+                         count_s ? count_s + t0 : nullptr, w, sms, st);
+        if (ps != PROX_OK) return ps;
+    }
+    return PROX_OK;
+}
+
+}  // namespace prox
+
+using namespace prox;
+
+PROX_API prox_status prox_quantize_proxy(int d_model, int d_ff, const uint16_t *w_cm,
+                                         uint8_t *q_out, float *scale_out, void *stream) {
+    if (!w_cm || !q_out || !scale_out || !shape_ok(d_model, d_ff)) return PROX_EINVAL;
+    if (!aligned16(w_cm) || !aligned16(q_out) || !aligned16(scale_out)) return PROX_EINVAL;
+    int sms = 0;
+    prox_status ps = current_device(&sms);
+    if (ps != PROX_OK) return ps;
+    if (launch_quantize(d_model, d_ff, w_cm, q_out, scale_out, (cudaStream_t)stream) !=
+        cudaSuccess)
+        return PROX_ECUDA;
+    return PROX_OK;
+}
+
+PROX_API size_t prox_workspace_bytes(int d_model, int d_ff, int batch) {
+    if (!shape_ok(d_model, d_ff) || batch < 0) return 0;
+    return ws_layout(d_model, d_ff, tokens_per_pass(d_model, batch)).total;
+}
+
+PROX_API prox_status prox_ffn_forward(const prox_layer *layer, const uint16_t *x, int batch,
+                                      float tau_x, float tau_s, float *y, uint8_t *mask_x,
+                                      uint8_t *mask_s, int32_t *idx_s, int32_t *count_s,
+                                      void *ws, size_t ws_bytes, void *stream) {
+    prox_status ps = check_layer(layer, true);
+    if (ps != PROX_OK) return ps;
+    if (batch < 0 || !tau_ok(tau_x) || !tau_ok(tau_s)) return PROX_EINVAL;
+    if (batch == 0) return PROX_OK;
+    if (!x || !y || !ws || !aligned16(x) || !aligned16(y) || !aligned16(ws)) return PROX_EINVAL;
+    return run_forward(layer, x, batch, tau_x, tau_s, y, mask_x, mask_s, idx_s, count_s, nullptr,
+                       ws, ws_bytes, (cudaStream_t)stream, true);
+}
+
+PROX_API int prox_max_batch_per_pass(int d_model) { return max_tokens_per_pass(d_model); }
+
+PROX_API prox_status prox_ffn_stage1(const prox_layer *layer, const uint16_t *x, int batch,
+                                     float tau_x, float tau_s, float *y_clear, uint8_t *mask_x,
+                                     uint8_t *mask_s, void *ws, size_t ws_bytes, void *stream) {
+    prox_status ps = check_layer(layer, false);
+    if (ps != PROX_OK) return ps;
+    const int d = layer->d_model, f = layer->d_ff;
+    if (batch < 0 || batch > max_tokens_per_pass(d) || !tau_ok(tau_x) || !tau_ok(tau_s))
+        return PROX_EINVAL;
+    if (batch == 0) return PROX_OK;
+    if (!x || !ws || !aligned16(x) || !aligned16(ws) || (y_clear && !aligned16(y_clear)))
+        return PROX_EINVAL;
+    if (ws_bytes < ws_layout(d, f, tokens_per_pass(d, batch)).total) return PROX_ENOMEM;
+    int sms = 0;
+    ps = current_device(&sms);
+    if (ps != PROX_OK) return ps;
+    return pass_stage1(layer, x, batch, tau_x, tau_s, y_clear, mask_x, mask_s, nullptr,
+                       static_cast<unsigned char *>(ws), sms, true, (cudaStream_t)stream);
+}
+
+PROX_API prox_status prox_ffn_stage2(const prox_layer *layer, const uint16_t *x, int batch,
+                                     float *y, int32_t *idx_s, int32_t *count_s, void *ws,
+                                     size_t ws_bytes, void *stream) {
+    prox_status ps = check_layer(layer, true);
+    if (ps != PROX_OK) return ps;
+    const int d = layer->d_model, f = layer->d_ff;
+    if (batch < 0 || batch > max_tokens_per_pass(d)) return PROX_EINVAL;
+    if (batch == 0) return PROX_OK;
+    if (!x || !y || !ws || !aligned16(x) || !aligned16(y) || !aligned16(ws)) return PROX_EINVAL;
+    if (ws_bytes < ws_layout(d, f, tokens_per_pass(d, batch)).total) return PROX_ENOMEM;
+    int sms = 0;
+    ps = current_device(&sms);
+    if (ps != PROX_OK) return ps;
+    return pass_stage2(layer, x, batch, y, idx_s, count_s, static_cast<unsigned char *>(ws), sms,
+                       (cudaStream_t)stream);
+}
+
+PROX_API prox_status prox_proxy_state(const prox_layer *layer, const uint16_t *x, int batch,
+                                      float tau_x, float *s_out, uint8_t *mask_x, void *ws,
+                                      size_t ws_bytes, void *stream) {
+    prox_status ps = check_layer(layer, false);
+    if (ps != PROX_OK) return ps;
+    if (batch < 0 || !tau_ok(tau_x)) return PROX_EINVAL;
+    if (batch == 0) return PROX_OK;
+    if (!x || !s_out || !ws || !aligned16(x) || !aligned16(ws)) return PROX_EINVAL;
+    return run_forward(layer, x, batch, tau_x, 0.f, nullptr, mask_x, nullptr, nullptr, nullptr,
+                       s_out, ws, ws_bytes, (cudaStream_t)stream, false);
+}
+
+// calibration workspace: [forward ws for the widest pass][s~ n_cal x d_ff fp32]
+// [histogram 65536 u32][scratch 64 B][tau 2 x fp32]
+struct CalLayout {
+    size_t fwd, s, hist, scratch, tau, total;
+};
+static CalLayout cal_layout(int d, int f, int n_cal) {
+    CalLayout c;
+    size_t o = 0;
+    c.fwd = o;
+    o = align_up(o + prox_workspace_bytes(d, f, n_cal), 256);
+    c.s = o;
+    o = align_up(o + (size_t)n_cal * f * 4, 256);
+    c.hist = o;
+    o = align_up(o + 65536 * 4, 256);
+    c.scratch = o;
+    o += 64;
+    c.tau = o;
+    o += 64;
+    c.total = o;
+    return c;
+}
+
+PROX_API size_t prox_calibrate_workspace_bytes(int d_model, int d_ff, int n_cal) {
+    if (!shape_ok(d_model, d_ff) || n_cal < 1) return 0;
+    return cal_layout(d_model, d_ff, n_cal).total;
+}
+
+static long quantile_rank(long n, double keep) {
+    double r = std::floor((1.0 - keep) * (double)n);
+    long rank = (long)r;
+    if (rank < 0) rank = 0;
+    if (rank > n - 1) rank = n - 1;
+    return rank;
+}
+
+PROX_API prox_status prox_calibrate(const prox_layer *layer, const uint16_t *x_cal, int n_cal,
+                                    double keep_x, double keep_s, float *tau_x_out,
+                                    float *tau_s_out, void *ws, size_t ws_bytes, void *stream) {
+    prox_status ps = check_layer(layer, false);
+    if (ps != PROX_OK) return ps;
+    if (!x_cal || n_cal < 1 || !tau_x_out || !tau_s_out || !ws || !aligned16(x_cal) ||
+        !aligned16(ws))
+        return PROX_EINVAL;
+    if (!(keep_x >= 0.0 && keep_x <= 1.0) || !(keep_s >= 0.0 && keep_s <= 1.0)) return PROX_EINVAL;
+    const int d = layer->d_model, f = layer->d_ff;
+    const CalLayout c = cal_layout(d, f, n_cal);
+    if (ws_bytes < c.total) return PROX_ENOMEM;
+    int sms = 0;
+    ps = current_device(&sms);
+    if (ps != PROX_OK) return ps;
+    cudaStream_t st = (cudaStream_t)stream;
+    unsigned char *w = static_cast<unsigned char *>(ws);
+    uint32_t *hist = reinterpret_cast<uint32_t *>(w + c.hist);
+    uint32_t *scratch = reinterpret_cast<uint32_t *>(w + c.scratch);
+    float *tau = reinterpret_cast<float *>(w + c.tau);
+    const long nx = (long)n_cal * d;
+    if (launch_select_bf16_abs(x_cal, nx, quantile_rank(nx, keep_x), hist, scratch, tau, st) !=
+        cudaSuccess)
+        return PROX_ECUDA;
+    float tx = 0.f;
+    if (cudaMemcpyAsync(&tx, tau, sizeof(float), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+        return PROX_ECUDA;
+    float *s_all = reinterpret_cast<float *>(w + c.s);
+    ps = run_forward(layer, x_cal, n_cal, tx, 0.f, nullptr, nullptr, nullptr, nullptr, nullptr,
+                     s_all, w + c.fwd, c.s - c.fwd, st, false);
+    if (ps != PROX_OK) return ps;
+    const long ns = (long)n_cal * f;
+    if (launch_select_f32_abs(s_all, ns, quantile_rank(ns, keep_s), hist, scratch, tau + 1, st) !=
+        cudaSuccess)
+        return PROX_ECUDA;
+    float ts = 0.f;
+    if (cudaMemcpyAsync(&ts, tau + 1, sizeof(float), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+        return PROX_ECUDA;
+    *tau_x_out = tx;
+    *tau_s_out = ts;
+    return PROX_OK;
+}
+
+PROX_API prox_status prox_allocate(double e, double alpha, double s1_max, double s2_anchor,
+                                   double *s1_out, double *s2_out) {
+    if (!s1_out || !s2_out || !(alpha > 0.0) || !(e >= 0.0 && e <= 1.0) ||
+        !(s1_max >= 0.0 && s1_max <= 1.0) || !(s2_anchor >= 0.0 && s2_anchor <= 1.0))
+        return PROX_EINVAL;
+    double s2 = s2_anchor;
+    double s1 = 1.0 - 3.0 * (s2 - e) / (2.0 * alpha);
+    if (s1 > s1_max || s1 < 0.0) {
+        s1 = s1 > s1_max ? s1_max : 0.0;
+        s2 = e + 2.0 * alpha * (1.0 - s1) / 3.0;
+    }
+    *s1_out = s1;
+    *s2_out = s2;
+    return PROX_OK;
+}
+
+PROX_API prox_status prox_last_device_status(void *ws, size_t ws_bytes, void *stream,
+                                             uint32_t *flags_out) {
+    if (!ws || ws_bytes < 256) return PROX_EINVAL;
+    cudaStream_t st = (cudaStream_t)stream;
+    uint32_t v = 0;
+    if (cudaMemcpyAsync(&v, ws, sizeof v, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaMemsetAsync(ws, 0, sizeof v, st) != cudaSuccess || cudaStreamSynchronize(st) != cudaSuccess)
+        return PROX_ECUDA;
+    if (flags_out) *flags_out = v;
+    return v ? PROX_ETIMEOUT : PROX_OK;
+}
+
+PROX_API const char *prox_status_str(prox_status s) {
+    switch (s) {
+        case PROX_OK: return "ok";
+        case PROX_EINVAL: return "invalid argument";
+        case PROX_ENOMEM: return "workspace too small";
+        case PROX_ECUDA: return "CUDA error";
+        case PROX_ETIMEOUT: return "device-side wait timed out";
+        case PROX_EDEVICE: return "current device is not compute capability 10.x (B200)";
+    }
+    return "unknown status";
+}
+
+// Test hooks, not part of prox.h: shorten the bounded waits and make the
+// Stage-2 producer of CTA 0 skip one channel position, so that a test can
+// exercise the timeout path without faulting anything.
+PROX_API void prox_test_set_wait(uint32_t spin_limit, int skip_position) {
+    prox::g_spin_limit = spin_limit ? spin_limit : kDefaultSpinLimit;
+    prox::g_debug_skip = skip_position;
+}

@@ -1,0 +1,200 @@
+// Internal declarations of libprox: launch plans, workspace layout, kernel
+// argument blocks and the inline-PTX helpers (mbarriers with bounded waits,
+// bulk copies, vector reductions) the sm_100a kernels share.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+#include "prox.h"
+
+namespace prox {
+
+// ---------------------------------------------------------------------------
+// Fixed tiling constants
+// ---------------------------------------------------------------------------
+constexpr int kCB = 256;            // channels per Stage-1 column block
+constexpr int kS1Threads = 256;     // Stage-1 CTA size
+constexpr int kS1MaxRowGroups = 16; // upper bound of row groups per block
+constexpr int kNCW = 16;            // Stage-2 consumer warps
+constexpr int kS2Threads = kNCW * 32 + 32;  // + one producer warp
+constexpr int kMaxB = 8;            // tokens per pass (per-token masks)
+constexpr int kS1UnitBudget = 96 * 1024;    // smem bytes for Stage-1 unit lists
+constexpr int kS2SmemBudget = 224 * 1024;   // opt-in dynamic smem per CTA
+
+// status word bits (first word of the workspace)
+constexpr uint32_t kStTimeoutFull = 1u << 0;   // consumer waited for a stage
+constexpr uint32_t kStTimeoutEmpty = 1u << 1;  // producer waited for a free slot
+constexpr uint32_t kStTimeoutRed = 1u << 2;    // consumers waited for partials
+constexpr uint32_t kStTimeoutDrain = 1u << 3;  // producer waited for its copies
+
+// default poll budget of a bounded mbarrier wait (each poll is a try_wait,
+// which itself blocks for a hardware-defined interval)
+constexpr uint32_t kDefaultSpinLimit = 1u << 22;
+
+// ---------------------------------------------------------------------------
+// Host-side plans
+// ---------------------------------------------------------------------------
+struct Stage1Plan {
+    int C;          // column blocks = d_ff / kCB
+    int n_r;        // row groups per block; grid = C * n_r
+    int unit_cap;   // max units (kept rows) one CTA may own
+    size_t smem;    // dynamic shared memory bytes
+};
+
+struct Stage2Plan {
+    int nchunk;     // 16-byte chunks of a d_model row per consumer thread
+    int nstage;     // stages in the bulk-copy ring
+    size_t smem;    // dynamic shared memory bytes
+};
+
+// tokens per pass for a given d_model (register budget of Stage 2 and smem of
+// Stage 1); 0 if d_model is beyond what the kernels support
+int max_tokens_per_pass(int d_model);
+int tokens_per_pass(int d_model, int batch);   // 1, 2, 4 or 8
+Stage1Plan stage1_plan(int d_model, int d_ff, int B, int num_sms);
+Stage2Plan stage2_plan(int d_model, int B);
+
+// Workspace layout of one forward pass (B tokens). Offsets in bytes.
+struct WsLayout {
+    size_t status, arrive, ucount, tcount, ulist, tlist, partials, total;
+};
+WsLayout ws_layout(int d_model, int d_ff, int B);
+
+// ---------------------------------------------------------------------------
+// Kernel argument blocks
+// ---------------------------------------------------------------------------
+struct Stage1Args {
+    int d, f, nb;                // nb active tokens of this pass (<= B)
+    int C, n_r, unit_cap;
+    const uint16_t *x;           // [nb][d]
+    float tau_x, tau_s;
+    const uint8_t *q_up, *q_gate;
+    const float *s_up, *s_gate;
+    float *y_zero;               // [nb][d] zeroed here (Stage 2 accumulates), or null
+    uint8_t *mask_x;             // [nb][d] or null
+    uint8_t *mask_s;             // [nb][f] or null
+    float *s_out;                // [nb][f] or null
+    int build_lists;             // write ulist/tlist/counts for Stage 2
+    // workspace
+    float *partials;             // [C][kS1MaxRowGroups][2][B][kCB]
+    uint32_t *arrive;            // [C]
+    int32_t *ucount;             // [C]
+    int32_t *tcount;             // [C][B]
+    uint32_t *ulist;             // [C][kCB]  channel | token bits << 24
+    int32_t *tlist;              // [B][f]
+};
+
+struct Stage2Args {
+    int d, f, nb, C;
+    const uint16_t *x;           // [nb][d]
+    const uint16_t *w_up, *w_gate, *w_down;
+    float *y;                    // [nb][d], zeroed by Stage 1
+    int32_t *idx_s;              // [nb][f] or null
+    int32_t *count_s;            // [nb] or null
+    const int32_t *ucount, *tcount;
+    const uint32_t *ulist;
+    const int32_t *tlist;
+    uint32_t *status;
+    uint32_t spin_limit;
+    int debug_skip;              // test hook: producer never fills this
+                                 // channel position of CTA 0 (-1: off)
+    int nstage;
+};
+
+cudaError_t launch_stage1(int B, const Stage1Args &a, const Stage1Plan &p,
+                          cudaStream_t s);
+cudaError_t launch_stage2(int B, int nchunk, const Stage2Args &a, int grid,
+                          size_t smem, cudaStream_t s);
+cudaError_t launch_quantize(int d, int f, const uint16_t *w_cm, uint8_t *q,
+                            float *scale, cudaStream_t s);
+// exact order statistic of |values| (bf16 or fp32 bit patterns) on device;
+// writes the selected magnitude's fp32 value to *tau_dev
+cudaError_t launch_select_bf16_abs(const uint16_t *v, long n, long rank,
+                                   uint32_t *hist, uint32_t *scratch,
+                                   float *tau_dev, cudaStream_t s);
+cudaError_t launch_select_f32_abs(const float *v, long n, long rank,
+                                  uint32_t *hist, uint32_t *scratch,
+                                  float *tau_dev, cudaStream_t s);
+
+// ---------------------------------------------------------------------------
+// Device helpers
+// ---------------------------------------------------------------------------
+#ifdef __CUDACC__
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)),
+                 "r"(count)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_fence_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(
+                     smem_addr(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(
+                     smem_addr(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait: returns false (and leaves the barrier alone) after `limit`
+// unsuccessful polls.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t limit) {
+    for (uint32_t i = 0; i < limit; ++i)
+        if (mbar_try_wait(bar, parity))
+            return true;
+    return false;
+}
+
+// 1-D bulk copy global -> shared, completing on an mbarrier (TMA engine).
+// Both addresses 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes,
+                                         uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_addr(dst)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void red_add_v4(float *dst, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a), "f"(b),
+                 "f"(c), "f"(d)
+                 : "memory");
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+#endif  // __CUDACC__
+
+}  // namespace prox

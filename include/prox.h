@@ -1,0 +1,225 @@
+/*
+ * prox.h -- C ABI of the B200 (sm_100a) Prox two-stage sparse SwiGLU FFN.
+ *
+ * The method ("Prox: Training-Free FFN Activation Sparsity via Approximate
+ * Intermediate-Channel Salience in LLMs"; sections cited below are those of
+ * the Prox deep-dive blog post and of the translated arXiv HTML):
+ *
+ *   Stage 1 (blog, "Stage 1"): m_x = 1[|x| >= tau_x]; proxy branches
+ *     u~ = Pi_in(x, W~_up, m_x), h~ = SiLU(Pi_in(x, W~_gate, m_x)) with
+ *     symmetric per-row INT4 copies W~; s~ = u~ (.) h~; shared channel mask
+ *     m_s = 1[|s~| >= tau_s].
+ *   Stage 2 (blog, "Stage 2"): for the kept channels only, with the original
+ *     bf16 weights and the full x: u = Pi_out(x, W_up, m_s),
+ *     h = SiLU(Pi_out(x, W_gate, m_s)), s = u (.) h, y = Pi_in(s, W_down, m_s).
+ *   Pi_in / Pi_out are the input- and output-sparse projections of the arXiv
+ *   page, section 2.2; the SwiGLU FFN itself is its section 2.1.
+ *
+ * Conventions
+ *   - Every pointer named "device" is CUDA device memory owned by the caller;
+ *     the library never allocates, frees or keeps it. "host" pointers are
+ *     ordinary host memory.
+ *   - bf16 tensors are passed as uint16_t bit patterns.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream). Every
+ *     call except prox_calibrate and prox_last_device_status is asynchronous
+ *     on that stream and returns as soon as its kernels are enqueued.
+ *   - Argument errors are detected on the host and returned before anything
+ *     is launched. No C++ exception crosses this interface.
+ *   - Shapes: d_model and d_ff are multiples of 256 with 256 <= d_model <= 8192
+ *     and 256 <= d_ff <= 262144; batch >= 0. Anything else is PROX_EINVAL.
+ *   - The library runs on compute capability 10.0 devices (B200, sm_100a);
+ *     any other current device gives PROX_EDEVICE.
+ */
+#ifndef PROX_H
+#define PROX_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum prox_status {
+    PROX_OK = 0,
+    PROX_EINVAL = 1,   /* bad argument (null pointer, shape, threshold, ...)  */
+    PROX_ENOMEM = 2,   /* caller's workspace smaller than required           */
+    PROX_ECUDA = 3,    /* a CUDA runtime call or launch failed               */
+    PROX_ETIMEOUT = 4, /* a bounded device-side wait gave up (status word)   */
+    PROX_EDEVICE = 5   /* current device is not compute capability 10.x      */
+} prox_status;
+
+/*
+ * One FFN layer, all device pointers, caller-owned.
+ *   w_up_cm, w_gate_cm : bf16 [d_ff][d_model]; row j is output channel j
+ *                        (the pages' W_up[:, j]; nn.Linear weight layout).
+ *   w_down             : bf16 [d_ff][d_model]; row j is W_down[j, :] (the
+ *                        pages' orientation d_ff x d_model).
+ *   q_up, q_gate       : INT4 proxies, uint8 [d_model][d_ff/2] as written by
+ *                        prox_quantize_proxy.
+ *   s_up, s_gate       : fp32 [d_model] per-row proxy scales.
+ * Every pointer must be 16-byte aligned.
+ */
+typedef struct prox_layer {
+    int d_model;
+    int d_ff;
+    const uint16_t *w_up_cm;
+    const uint16_t *w_gate_cm;
+    const uint16_t *w_down;
+    const uint8_t *q_up;
+    const uint8_t *q_gate;
+    const float *s_up;
+    const float *s_gate;
+} prox_layer;
+
+/*
+ * prox_quantize_proxy -- symmetric per-row INT4 proxy copy of one projection
+ * (blog, "Stage 1": W~_up and W~_gate are symmetric per-row INT4 copies).
+ *
+ * Reading of "per-row": a row i of W in the pages' orientation
+ * W in R^{d_model x d_ff}, i.e. one scale per input coordinate, so that the
+ * input-sparse proxy product skips whole rows.
+ *   scale_i = max_j |W[i,j]| / 7                        (fp32, round to nearest)
+ *   q_ij    = clamp(round_half_even(W[i,j] / scale_i), -7, 7)  (fp32 division)
+ *   an all-zero row gives scale 0 and q 0.
+ * Output layout: q_out[i][m] (device, uint8 [d_model][d_ff/2]) holds channel 2m
+ * in its low nibble and 2m+1 in its high nibble, two's complement;
+ * scale_out (device, fp32 [d_model]).
+ *   w_cm : device, bf16 [d_ff][d_model] (channel-major, as in prox_layer).
+ * Errors: PROX_EINVAL on a null pointer or bad shape.
+ */
+prox_status prox_quantize_proxy(int d_model, int d_ff, const uint16_t *w_cm,
+                                uint8_t *q_out, float *scale_out, void *stream);
+
+/*
+ * prox_workspace_bytes -- bytes of device workspace prox_ffn_forward and
+ * prox_proxy_state need for this shape and batch. The workspace must be
+ * zero-filled once after allocation (cudaMemset to 0); the library leaves it
+ * ready for the next call at the end of every call. One workspace serves one
+ * stream at a time: calls that share it must not overlap on the device.
+ */
+size_t prox_workspace_bytes(int d_model, int d_ff, int batch);
+
+/*
+ * prox_ffn_forward -- Stage 1 then Stage 2 for `batch` tokens, each with its
+ * own masks; tau_x and tau_s are per-layer scalars shared by all tokens
+ * (blog, "Stage 1" and "Stage 2").
+ *   x       : device, bf16 [batch][d_model].
+ *   tau_x   : input threshold, finite and >= 0 (|x_i| >= tau_x is kept).
+ *   tau_s   : channel threshold, finite and >= 0 (|s~_j| >= tau_s is kept).
+ *   y       : device, fp32 [batch][d_model]; fully overwritten.
+ *   mask_x  : device, uint8 [batch][d_model] (1 = kept input) or NULL.
+ *   mask_s  : device, uint8 [batch][d_ff] (1 = kept channel) or NULL.
+ *   idx_s   : device, int32 [batch][d_ff]; row t starts with the kept channels
+ *             of token t in ascending order (the rest is left untouched) or NULL.
+ *   count_s : device, int32 [batch], kept-channel count per token, or NULL.
+ *   ws      : device workspace of at least prox_workspace_bytes(...) bytes.
+ * Arithmetic: proxy products accumulate in fp32 from exact INT4 codes; exact
+ * products read bf16 weights and accumulate in fp32; SiLU in fp32; y in fp32.
+ * Errors: PROX_EINVAL (null required pointer, shape, negative or non-finite
+ * threshold, misaligned pointer), PROX_ENOMEM (ws_bytes too small),
+ * PROX_ECUDA (launch failure). Device-side wait timeouts are reported through
+ * prox_last_device_status.
+ */
+prox_status prox_ffn_forward(const prox_layer *layer, const uint16_t *x, int batch,
+                             float tau_x, float tau_s, float *y, uint8_t *mask_x,
+                             uint8_t *mask_s, int32_t *idx_s, int32_t *count_s,
+                             void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * prox_max_batch_per_pass -- tokens one Stage-1/Stage-2 pass handles for this
+ * d_model (8 up to d_model 4096, 4 up to 8192, 0 beyond: unsupported).
+ * prox_ffn_forward splits larger batches into passes by itself.
+ */
+int prox_max_batch_per_pass(int d_model);
+
+/*
+ * prox_ffn_stage1 / prox_ffn_stage2 -- the two phases of prox_ffn_forward,
+ * callable separately (for instance to time or inspect Stage 1 alone).
+ * prox_ffn_forward(..) with batch <= prox_max_batch_per_pass(d_model) is
+ * exactly prox_ffn_stage1 followed by prox_ffn_stage2 on the same workspace.
+ *   prox_ffn_stage1: masks (as in prox_ffn_forward) plus the kept-channel
+ *     lists, left in `ws`; clears y_clear (device, fp32 [batch][d_model],
+ *     may be NULL when Stage 2 will not run).
+ *   prox_ffn_stage2: exact Stage 2 from the lists the immediately preceding
+ *     prox_ffn_stage1 call on the same `ws`, same x and batch, left there;
+ *     accumulates into y, which that Stage-1 call cleared; writes idx_s and
+ *     count_s (either may be NULL).
+ * Both require 0 <= batch <= prox_max_batch_per_pass(d_model) (else
+ * PROX_EINVAL); other arguments and errors as in prox_ffn_forward.
+ */
+prox_status prox_ffn_stage1(const prox_layer *layer, const uint16_t *x, int batch,
+                            float tau_x, float tau_s, float *y_clear, uint8_t *mask_x,
+                            uint8_t *mask_s, void *ws, size_t ws_bytes, void *stream);
+prox_status prox_ffn_stage2(const prox_layer *layer, const uint16_t *x, int batch, float *y,
+                            int32_t *idx_s, int32_t *count_s, void *ws, size_t ws_bytes,
+                            void *stream);
+
+/*
+ * prox_proxy_state -- Stage 1 alone: writes the proxy intermediate state
+ * s~ = u~ (.) SiLU(g~) (blog, "Stage 1") for every channel of every token.
+ *   s_out  : device, fp32 [batch][d_ff].
+ *   mask_x : device, uint8 [batch][d_model] or NULL.
+ * Other arguments as in prox_ffn_forward.
+ */
+prox_status prox_proxy_state(const prox_layer *layer, const uint16_t *x, int batch,
+                             float tau_x, float *s_out, uint8_t *mask_x, void *ws,
+                             size_t ws_bytes, void *stream);
+
+/*
+ * prox_calibrate_workspace_bytes -- device workspace prox_calibrate needs.
+ */
+size_t prox_calibrate_workspace_bytes(int d_model, int d_ff, int n_cal);
+
+/*
+ * prox_calibrate -- per-layer thresholds from calibration vectors (blog,
+ * "Stage 1": offline per-layer thresholds; "Evidence": thresholds taken from
+ * calibration activations, layer by layer).
+ * Reading: tau is the exact order statistic of the pooled magnitudes. With the
+ * n pooled values sorted ascending v[0..n-1] and
+ * rank = floor((1 - keep) * n) (IEEE double, clamped to [0, n-1]):
+ *   tau_x = v[rank] over |x| of all n_cal x d_model calibration coordinates;
+ *   tau_s = v[rank] over |s~| of all n_cal x d_ff channels, with s~ computed
+ *           by Stage 1 at the tau_x just found.
+ *   x_cal     : device, bf16 [n_cal][d_model]; n_cal >= 1.
+ *   keep_x, keep_s : kept fractions in [0, 1].
+ *   tau_x_out, tau_s_out : HOST pointers, written before the call returns.
+ *   ws        : device, >= prox_calibrate_workspace_bytes(...) bytes, zero-filled
+ *               once after allocation (left ready for reuse).
+ * The only call that synchronises `stream`.
+ */
+prox_status prox_calibrate(const prox_layer *layer, const uint16_t *x_cal, int n_cal,
+                           double keep_x, double keep_s, float *tau_x_out,
+                           float *tau_s_out, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * prox_allocate -- split a target effective sparsity between the stages
+ * (blog, "Compute budget"): C = 2 alpha (1 - s1) + 3 (1 - s2) and
+ * e = 1 - C/3 = s2 - 2 alpha (1 - s1) / 3.
+ * Reading of the allocation rule: anchor s2 at s2_anchor and solve for s1; if
+ * s1 falls outside [0, s1_max], clamp it and solve for s2. The blog's case
+ * e = 0.7, alpha = 1/3, s1_max = 0.7, anchor 0.7 gives s1 = 0.7, s2 ~= 0.7667.
+ * Host only; s1_out and s2_out are host pointers.
+ * Errors: PROX_EINVAL on null outputs, alpha <= 0, or e, s1_max, s2_anchor
+ * outside [0, 1].
+ */
+prox_status prox_allocate(double e, double alpha, double s1_max, double s2_anchor,
+                          double *s1_out, double *s2_out);
+
+/*
+ * prox_last_device_status -- reads and clears the device status word in a
+ * forward workspace (synchronises `stream`). Returns PROX_ETIMEOUT if a
+ * bounded device-side wait gave up since the last read, PROX_OK otherwise.
+ * *flags_out (host, may be NULL) receives the raw status bits.
+ */
+prox_status prox_last_device_status(void *ws, size_t ws_bytes, void *stream,
+                                    uint32_t *flags_out);
+
+/* Static English description of a status code. */
+const char *prox_status_str(prox_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PROX_H */

@@ -1,0 +1,121 @@
+"""The C-ABI library loads, exports every symbol include/*.h declares, and
+rejects bad arguments on the host before any CUDA call (runs without a GPU)."""
+import ctypes as C
+import glob
+import os
+import re
+
+import pytest
+
+from free_ffn_activation_b200 import prox as P
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"\b(prox_\w+)\s*\(", src):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+def test_headers_declare_the_boundary():
+    names = declared_functions()
+    for n in ("prox_quantize_proxy", "prox_calibrate", "prox_ffn_forward", "prox_workspace_bytes",
+              "prox_last_device_status", "prox_status_str", "prox_proxy_state", "prox_allocate"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = C.CDLL(P.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_only_abi_symbols_exported():
+    out = os.popen(f"nm -D --defined-only {P.LIB_PATH}").read()
+    exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    assert exported == set(declared_functions()), exported ^ set(declared_functions())
+
+
+def test_status_strings():
+    for s in range(6):
+        assert P.status_str(s)
+    assert "time" in P.status_str(P.PROX_ETIMEOUT)
+
+
+def test_workspace_sizes():
+    assert P.workspace_bytes(4096, 12288, 1) > 0
+    assert P.workspace_bytes(4096, 12288, 8) > P.workspace_bytes(4096, 12288, 1)
+    assert P.workspace_bytes(4096, 12288, 100) == P.workspace_bytes(4096, 12288, 8)
+    assert P.workspace_bytes(8192, 28672, 16) > 0
+    for d, f in ((255, 768), (256, 100), (0, 768), (16384, 768), (256, -256)):
+        assert P.workspace_bytes(d, f, 1) == 0
+    assert P.workspace_bytes(256, 768, -1) == 0
+    assert P.lib().prox_calibrate_workspace_bytes(256, 768, 0) == 0
+    assert P.lib().prox_calibrate_workspace_bytes(256, 768, 256) > 256 * 768 * 4
+
+
+def _fake_layer(d=256, f=768, **override):
+    base = 1 << 20
+    fields = dict(d_model=d, d_ff=f, w_up_cm=base, w_gate_cm=base * 2, w_down=base * 3,
+                  q_up=base * 4, q_gate=base * 5, s_up=base * 6, s_gate=base * 7)
+    fields.update(override)
+    return P._Layer(**fields)
+
+
+def _fwd(layer, x=1 << 24, batch=1, tau_x=0.5, tau_s=0.1, y=1 << 25, ws=1 << 26, ws_bytes=1 << 30):
+    return P.lib().prox_ffn_forward(C.byref(layer) if layer is not None else None, x, batch,
+                                    tau_x, tau_s, y, None, None, None, None, ws, ws_bytes, None)
+
+
+def test_forward_validation_before_launch():
+    L = _fake_layer()
+    assert _fwd(None) == P.PROX_EINVAL
+    assert _fwd(_fake_layer(d=300)) == P.PROX_EINVAL
+    assert _fwd(_fake_layer(f=700)) == P.PROX_EINVAL
+    assert _fwd(_fake_layer(w_down=None)) == P.PROX_EINVAL
+    assert _fwd(_fake_layer(q_gate=(1 << 20) + 4)) == P.PROX_EINVAL   # misaligned
+    assert _fwd(L, tau_x=float("nan")) == P.PROX_EINVAL
+    assert _fwd(L, tau_s=-1.0) == P.PROX_EINVAL
+    assert _fwd(L, tau_s=float("inf")) == P.PROX_EINVAL
+    assert _fwd(L, batch=-1) == P.PROX_EINVAL
+    assert _fwd(L, x=None) == P.PROX_EINVAL
+    assert _fwd(L, y=None) == P.PROX_EINVAL
+    assert _fwd(L, ws=None) == P.PROX_EINVAL
+    assert _fwd(L, batch=0) == P.PROX_OK            # nothing to do, nothing launched
+
+
+def test_other_entry_points_validate():
+    lib = P.lib()
+    assert lib.prox_quantize_proxy(256, 768, None, 1 << 20, 1 << 21, None) == P.PROX_EINVAL
+    assert lib.prox_quantize_proxy(250, 768, 1 << 20, 1 << 21, 1 << 22, None) == P.PROX_EINVAL
+    L = _fake_layer()
+    tx, ts = C.c_float(), C.c_float()
+    assert lib.prox_calibrate(C.byref(L), 1 << 20, 0, 0.5, 0.3, C.byref(tx), C.byref(ts),
+                              1 << 21, 1 << 30, None) == P.PROX_EINVAL
+    assert lib.prox_calibrate(C.byref(L), 1 << 20, 4, 1.5, 0.3, C.byref(tx), C.byref(ts),
+                              1 << 21, 1 << 30, None) == P.PROX_EINVAL
+    assert lib.prox_calibrate(C.byref(L), 1 << 20, 4, 0.5, 0.3, None, C.byref(ts),
+                              1 << 21, 1 << 30, None) == P.PROX_EINVAL
+    assert lib.prox_calibrate(C.byref(L), 1 << 20, 4, 0.5, 0.3, C.byref(tx), C.byref(ts),
+                              1 << 21, 16, None) == P.PROX_ENOMEM
+    assert lib.prox_proxy_state(C.byref(L), 1 << 20, 1, -0.5, 1 << 21, None, 1 << 22, 1 << 30,
+                                None) == P.PROX_EINVAL
+    assert lib.prox_last_device_status(None, 0, None, None) == P.PROX_EINVAL
+
+
+def test_budget_split_entry_point():
+    # blog "Compute budget": e = 0.7, alpha = 1/3, s1 capped at 0.7 -> s2 ~= 0.7667
+    s1, s2 = P.allocate(0.7)
+    assert s1 == pytest.approx(0.7) and abs(s2 - 0.7667) < 5e-5
+    import oracle
+    for e in (0.3, 0.45, 0.6, 0.7, 0.85):
+        assert P.allocate(e) == pytest.approx(oracle.allocate(e), abs=1e-15)
+    with pytest.raises(P.ProxError):
+        P.allocate(1.5)
+    with pytest.raises(P.ProxError):
+        P.allocate(0.5, alpha=0.0)
