@@ -152,6 +152,12 @@ __global__ void __launch_bounds__(kS1Threads, 2) k_stage1(const Stage1Args a) {
     __shared__ int s_last;
     __shared__ int s_cnt[kS1Threads / 32][kMaxB + 1];
 
+    // Programmatic dependent launch: x, y and the workspace may belong to the
+    // previous kernel in the stream; wait for it, then let the next kernel
+    // (Stage 2) start its own prologue.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
+
     // (1) Stage 2 accumulates y with atomics: clear it here.
     if (a.y_zero) {
         float4 *y4 = reinterpret_cast<float4 *>(a.y_zero);
@@ -160,23 +166,57 @@ __global__ void __launch_bounds__(kS1Threads, 2) k_stage1(const Stage1Args a) {
             y4[k] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
 
-    // (2) input masks m_x = 1[|x_i| >= tau_x] per token, and their union
-    for (int wd = wid; wd < W; wd += kS1Threads / 32) {
+    // (2) input masks m_x = 1[|x_i| >= tau_x] per token: each thread owns
+    // 16-byte chunks of 8 coordinates; all its loads are issued before any
+    // use. Chunk ci's 8 keep bits are byte ci of the token's mask words.
+    {
+        constexpr int MAXK = 4;  // chunks per thread per token (d_model <= 8192)
+        const int NC = a.d / 8;
+        uint4 xv[MAXK][B];
+#pragma unroll
+        for (int k = 0; k < MAXK; ++k)
+#pragma unroll
+            for (int t = 0; t < B; ++t) {
+                const int ci = tid + k * kS1Threads;
+                xv[k][t] = make_uint4(0, 0, 0, 0);
+                if (ci < NC && t < a.nb)
+                    xv[k][t] = *reinterpret_cast<const uint4 *>(a.x + (size_t)t * a.d + ci * 8);
+            }
+        uint8_t *tbytes = reinterpret_cast<uint8_t *>(tmask);
+#pragma unroll
+        for (int k = 0; k < MAXK; ++k) {
+            const int ci = tid + k * kS1Threads;
+            if (ci >= NC) break;
+#pragma unroll
+            for (int t = 0; t < B; ++t) {
+                const uint32_t w4[4] = {xv[k][t].x, xv[k][t].y, xv[k][t].z, xv[k][t].w};
+                uint32_t bits = 0;
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    bits |= (fabsf(bf16lo(w4[h])) >= a.tau_x ? 1u : 0u) << (2 * h);
+                    bits |= (fabsf(bf16hi(w4[h])) >= a.tau_x ? 1u : 0u) << (2 * h + 1);
+                }
+                if (t >= a.nb) bits = 0;
+                tbytes[t * NC + ci] = (uint8_t)bits;
+                if (a.mask_x && blockIdx.x == 0 && t < a.nb) {
+                    uint32_t lo = 0, hi = 0;
+#pragma unroll
+                    for (int b = 0; b < 4; ++b) {
+                        lo |= ((bits >> b) & 1u) << (8 * b);
+                        hi |= ((bits >> (b + 4)) & 1u) << (8 * b);
+                    }
+                    *reinterpret_cast<uint2 *>(a.mask_x + (size_t)t * a.d + ci * 8) =
+                        make_uint2(lo, hi);
+                }
+            }
+        }
+    }
+    __syncthreads();
+    for (int wd = tid; wd < W; wd += kS1Threads) {
         uint32_t un = 0;
 #pragma unroll
-        for (int t = 0; t < B; ++t) {
-            uint32_t bits = 0;
-            if (t < a.nb) {
-                const uint16_t h = a.x[(size_t)t * a.d + wd * 32 + lane];
-                const bool keep = fabsf(__uint_as_float((uint32_t)h << 16)) >= a.tau_x;
-                bits = __ballot_sync(0xffffffffu, keep);
-                if (a.mask_x && blockIdx.x == 0)
-                    a.mask_x[(size_t)t * a.d + wd * 32 + lane] = keep ? 1 : 0;
-            }
-            if (lane == 0) tmask[t * W + wd] = bits;
-            un |= bits;
-        }
-        if (lane == 0) umask[wd] = un;
+        for (int t = 0; t < B; ++t) un |= tmask[t * W + wd];
+        umask[wd] = un;
     }
     __syncthreads();
 
@@ -203,23 +243,47 @@ __global__ void __launch_bounds__(kS1Threads, 2) k_stage1(const Stage1Args a) {
     const int n_units = hi - lo;
     __syncthreads();
 
-    // (4) this CTA's units: row index and x_i * scale_i per matrix and token
+    // (4) this CTA's units: row index, then x_i * scale_i per matrix and token
     for (int wd = wid; wd < W; wd += kS1Threads / 32) {
         const uint32_t um = umask[wd];
         if (!((um >> lane) & 1u)) continue;
         const int rank = woff[wd] + __popc(um & ((1u << lane) - 1u));
         if (rank < lo || rank >= hi) continue;
-        const int u = rank - lo;
-        const int i = wd * 32 + lane;
-        rowidx[u] = i;
-        const float su = a.s_up[i], sg = a.s_gate[i];
+        rowidx[rank - lo] = wd * 32 + lane;
+    }
+    __syncthreads();
+    {
+        constexpr int G4 = 4;  // units per batch of loads
+        for (int u0 = tid; u0 < n_units; u0 += G4 * kS1Threads) {
+            float su[G4], sg[G4];
+            uint16_t xh[G4][B];
 #pragma unroll
-        for (int t = 0; t < B; ++t) {
-            float xv = 0.f;
-            if ((tmask[t * W + wd] >> lane) & 1u)
-                xv = __uint_as_float((uint32_t)a.x[(size_t)t * a.d + i] << 16);
-            xs[(u * 2 + 0) * B + t] = xv * su;
-            xs[(u * 2 + 1) * B + t] = xv * sg;
+            for (int k = 0; k < G4; ++k) {
+                const int u = u0 + k * kS1Threads;
+                su[k] = sg[k] = 0.f;
+                if (u < n_units) {
+                    const int i = rowidx[u];
+                    su[k] = a.s_up[i];
+                    sg[k] = a.s_gate[i];
+#pragma unroll
+                    for (int t = 0; t < B; ++t)
+                        xh[k][t] = (t < a.nb) ? a.x[(size_t)t * a.d + i] : (uint16_t)0;
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < G4; ++k) {
+                const int u = u0 + k * kS1Threads;
+                if (u >= n_units) break;
+                const int i = rowidx[u];
+#pragma unroll
+                for (int t = 0; t < B; ++t) {
+                    float xv = 0.f;
+                    if ((tmask[t * W + (i >> 5)] >> (i & 31)) & 1u)
+                        xv = __uint_as_float((uint32_t)xh[k][t] << 16);
+                    xs[(u * 2 + 0) * B + t] = xv * su[k];
+                    xs[(u * 2 + 1) * B + t] = xv * sg[k];
+                }
+            }
         }
     }
     __syncthreads();
@@ -389,8 +453,7 @@ cudaError_t launch1(const Stage1Args &a, const Stage1Plan &p, cudaStream_t s) {
         if (e != cudaSuccess) return e;
         configured = p.smem;
     }
-    k<<<a.C * a.n_r, kS1Threads, p.smem, s>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(k, dim3(a.C * a.n_r), dim3(kS1Threads), p.smem, s, a);
 }
 
 }  // namespace

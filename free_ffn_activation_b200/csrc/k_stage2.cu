@@ -24,10 +24,10 @@ namespace prox {
 
 // shared-memory carve-up, shared by the kernel and the host plan
 struct S2Smem {
-    size_t stages, xs, full, empty, redbar, meta, red, uscan, tscan, total;
+    size_t stages, xs, full, empty, redbar, meta, red, uscan, tscan, chan, total;
 };
 
-__host__ __device__ inline S2Smem s2_smem(int d, int B, int nstage, int C) {
+__host__ __device__ inline S2Smem s2_smem(int d, int B, int nstage, int C, int max_ch) {
     S2Smem s;
     size_t o = 0;
     s.stages = o;
@@ -50,6 +50,8 @@ __host__ __device__ inline S2Smem s2_smem(int d, int B, int nstage, int C) {
     o += (size_t)(C + 1) * 4;
     s.tscan = o;
     o += (size_t)B * (C + 1) * 4;
+    s.chan = o;
+    o += (size_t)max_ch * 4;
     s.total = (o + 127) & ~(size_t)127;
     return s;
 }
@@ -77,7 +79,7 @@ __global__ void __launch_bounds__(kS2Threads, 1) k_stage2(const Stage2Args a) {
     extern __shared__ __align__(128) unsigned char smem[];
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int d = a.d, C = a.C, NST = a.nstage;
-    const S2Smem L = s2_smem(d, B, NST, C);
+    const S2Smem L = s2_smem(d, B, NST, C, a.max_ch);
     uint16_t *stages = reinterpret_cast<uint16_t *>(smem + L.stages);
     uint16_t *xsm = reinterpret_cast<uint16_t *>(smem + L.xs);
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.full);
@@ -87,6 +89,7 @@ __global__ void __launch_bounds__(kS2Threads, 1) k_stage2(const Stage2Args a) {
     float *red = reinterpret_cast<float *>(smem + L.red);  // [2][kNCW][B][2]
     int *uscan = reinterpret_cast<int *>(smem + L.uscan);  // [C+1]
     int *tscan = reinterpret_cast<int *>(smem + L.tscan);  // [B][C+1]
+    uint32_t *chan = reinterpret_cast<uint32_t *>(smem + L.chan);  // [max_ch]
     const int nch16 = d / 8;  // 16-byte chunks per row
 
     if (tid == 0) {
@@ -98,15 +101,34 @@ __global__ void __launch_bounds__(kS2Threads, 1) k_stage2(const Stage2Args a) {
         mbar_init(&redbar[1], kNCW);
         mbar_fence_init();
     }
-    // exclusive scans of the per-block counts (warp 0)
+    // x (bf16) into shared memory; tokens beyond nb are zero. Stage 1, the
+    // kernel this one may overlap, only triggers this launch after its own
+    // griddepcontrol.wait, so x (written before Stage 1 ran) is complete.
+    for (int k = tid; k < B * nch16; k += kS2Threads) {
+        const int t = k / nch16, ci = k % nch16;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (t < a.nb) v = *reinterpret_cast<const uint4 *>(a.x + (size_t)t * d + ci * 8);
+        *reinterpret_cast<uint4 *>(xsm + (size_t)t * d + ci * 8) = v;
+    }
+    // Stage 1's lists are ready once it has completed
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    for (int k = tid; k < C * (B + 1); k += kS2Threads) {
+        if (k < C) {
+            uscan[k] = a.ucount[k];
+        } else {
+            const int c = (k - C) / B, t = (k - C) % B;
+            tscan[t * (C + 1) + c] = a.tcount[c * B + t];
+        }
+    }
+    __syncthreads();
+    // exclusive scans of the per-block counts, in place (warp 0)
     if (wid == 0) {
         for (int t = -1; t < B; ++t) {
             int carry = 0;
             int *dst = (t < 0) ? uscan : tscan + t * (C + 1);
             for (int c0 = 0; c0 < C; c0 += 32) {
                 const int c = c0 + lane;
-                int v = 0;
-                if (c < C) v = (t < 0) ? a.ucount[c] : a.tcount[c * B + t];
+                const int v = (c < C) ? dst[c] : 0;
                 int inc = v;
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
@@ -119,13 +141,6 @@ __global__ void __launch_bounds__(kS2Threads, 1) k_stage2(const Stage2Args a) {
             if (lane == 0) dst[C] = carry;
         }
     }
-    // x (bf16) into shared memory; tokens beyond nb are zero
-    for (int k = tid; k < B * nch16; k += kS2Threads) {
-        const int t = k / nch16, ci = k % nch16;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (t < a.nb) v = *reinterpret_cast<const uint4 *>(a.x + (size_t)t * d + ci * 8);
-        *reinterpret_cast<uint4 *>(xsm + (size_t)t * d + ci * 8) = v;
-    }
     __syncthreads();
 
     const long long U = uscan[C];
@@ -133,31 +148,27 @@ __global__ void __launch_bounds__(kS2Threads, 1) k_stage2(const Stage2Args a) {
     const int p0 = (int)(U * g / G), p1 = (int)(U * (g + 1) / G);
     const int n_ch = p1 - p0;
 
-    // per-token ascending kept-channel lists (blocks c = g, g + G, ...)
-    if (wid < kNCW) {
-        for (int c = g; c < C; c += G) {
-            for (int t = 0; t < a.nb; ++t) {
-                if (!a.idx_s) break;
-                const int n = a.tcount[c * B + t];
-                const int base = tscan[t * (C + 1) + c];
-                for (int k = tid; k < n; k += kNCW * 32)
-                    a.idx_s[(size_t)t * a.f + base + k] = a.tlist[(size_t)t * a.f + c * kCB + k];
-            }
+    // this CTA's share of the ascending kept-channel list, into shared memory
+    for (int n = tid; n < n_ch; n += kS2Threads) {
+        const int p = p0 + n;
+        int lo = 0, hi = C - 1;  // block cb with uscan[cb] <= p < uscan[cb + 1]
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (uscan[mid] <= p) lo = mid; else hi = mid - 1;
         }
-        if (g == 0 && a.count_s && tid < a.nb) a.count_s[tid] = tscan[tid * (C + 1) + C];
+        chan[n] = a.ulist[(size_t)lo * kCB + (p - uscan[lo])];
     }
+    __syncthreads();
+    asm volatile("griddepcontrol.launch_dependents;");
 
     if (wid == kNCW) {
         // ---------------- producer ----------------
         if (lane != 0) return;
         const uint32_t row_bytes = (uint32_t)d * 2;
-        int cb = 0;
         int issued = 0;
         bool ok = true;
         for (int n = 0; n < n_ch; ++n) {
-            const int p = p0 + n;
-            while (p >= uscan[cb + 1]) ++cb;
-            const uint32_t e = a.ulist[(size_t)cb * kCB + (p - uscan[cb])];
+            const uint32_t e = chan[n];
             const int s = n % NST, k = n / NST;
             if (k > 0 && !mbar_wait(&empty[s], (k - 1) & 1, a.spin_limit)) {
                 atomicOr(a.status, kStTimeoutEmpty);
@@ -279,6 +290,19 @@ __global__ void __launch_bounds__(kS2Threads, 1) k_stage2(const Stage2Args a) {
         if (lane == 0) mbar_arrive(&empty[s]);
     }
 
+    // per-token ascending kept-channel lists (blocks c = g, g + G, ...)
+    if (a.idx_s) {
+        for (int c = g; c < C; c += G) {
+            for (int t = 0; t < a.nb; ++t) {
+                const int n = a.tcount[c * B + t];
+                const int base = tscan[t * (C + 1) + c];
+                for (int k = tid; k < n; k += kNCW * 32)
+                    a.idx_s[(size_t)t * a.f + base + k] = a.tlist[(size_t)t * a.f + c * kCB + k];
+            }
+        }
+    }
+    if (g == 0 && a.count_s && tid < a.nb) a.count_s[tid] = tscan[tid * (C + 1) + C];
+
     if (n_ch == 0) return;
 #pragma unroll
     for (int t = 0; t < B; ++t) {
@@ -305,8 +329,7 @@ cudaError_t launch2(const Stage2Args &a, int grid, size_t smem, cudaStream_t s) 
         if (e != cudaSuccess) return e;
         configured = smem;
     }
-    k<<<grid, kS2Threads, smem, s>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(k, dim3(grid), dim3(kS2Threads), smem, s, a);
 }
 
 }  // namespace
@@ -323,8 +346,8 @@ cudaError_t launch_stage2(int B, int nchunk, const Stage2Args &a, int grid, size
     return cudaErrorInvalidValue;
 }
 
-size_t stage2_smem_bytes(int d_model, int B, int nstage, int C) {
-    return s2_smem(d_model, B, nstage, C).total;
+size_t stage2_smem_bytes(int d_model, int B, int nstage, int C, int max_ch) {
+    return s2_smem(d_model, B, nstage, C, max_ch).total;
 }
 
 }  // namespace prox

@@ -16,7 +16,7 @@
 namespace prox {
 
 size_t stage1_smem_bytes(int d_model, int B, int unit_cap);
-size_t stage2_smem_bytes(int d_model, int B, int nstage, int C);
+size_t stage2_smem_bytes(int d_model, int B, int nstage, int C, int max_ch);
 
 int max_tokens_per_pass(int d_model) {
     if (d_model <= 4096) return 8;
@@ -57,15 +57,15 @@ Stage1Plan stage1_plan(int d, int f, int B, int num_sms) {
     return p;
 }
 
-Stage2Plan stage2_plan(int d, int B) {
+Stage2Plan stage2_plan(int d, int B, int C, int max_ch) {
     Stage2Plan p;
     p.nchunk = pow2_ceil((d / 8 + kNCW * 32 - 1) / (kNCW * 32));
     const size_t stage = (size_t)6 * d;
-    const size_t fixed = stage2_smem_bytes(d, B, 0, 1024);  // upper bound on C
-    int ns = (int)((kS2SmemBudget - fixed) / stage);
+    const size_t fixed = stage2_smem_bytes(d, B, 0, C, max_ch);
+    int ns = fixed < (size_t)kS2SmemBudget ? (int)((kS2SmemBudget - fixed) / stage) : 0;
     if (ns > 16) ns = 16;
     p.nstage = ns;
-    p.smem = 0;
+    p.smem = stage2_smem_bytes(d, B, ns, C, max_ch);
     return p;
 }
 
@@ -125,6 +125,7 @@ static prox_status current_device(int *sms) {
     return PROX_OK;
 }
 
+// NULL counts as aligned: optional outputs are checked only when given
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 static bool shape_ok(int d, int f) {
@@ -197,8 +198,10 @@ static prox_status pass_stage2(const prox_layer *L, const uint16_t *x, int nb, f
     const int d = L->d_model, f = L->d_ff;
     const int B = pow2_ceil(nb);
     const WsLayout W = ws_layout(d, f, B);
-    const Stage2Plan p2 = stage2_plan(d, B);
     const int C = f / kCB;
+    const int max_ch = (f + sms - 1) / sms + 1;
+    const Stage2Plan p2 = stage2_plan(d, B, C, max_ch);
+    if (p2.nstage < 2) return PROX_EINVAL;
     Stage2Args b{};
     b.d = d;
     b.f = f;
@@ -219,8 +222,8 @@ static prox_status pass_stage2(const prox_layer *L, const uint16_t *x, int nb, f
     b.spin_limit = g_spin_limit;
     b.debug_skip = g_debug_skip;
     b.nstage = p2.nstage;
-    const size_t smem = stage2_smem_bytes(d, B, p2.nstage, C);
-    return launch_stage2(B, p2.nchunk, b, sms, smem, st) == cudaSuccess ? PROX_OK : PROX_ECUDA;
+    b.max_ch = max_ch;
+    return launch_stage2(B, p2.nchunk, b, sms, p2.smem, st) == cudaSuccess ? PROX_OK : PROX_ECUDA;
 }
 
 // Stage 1 [+ Stage 2] over `batch` tokens, in passes of at most B tokens
@@ -284,6 +287,8 @@ PROX_API prox_status prox_ffn_forward(const prox_layer *layer, const uint16_t *x
     if (batch < 0 || !tau_ok(tau_x) || !tau_ok(tau_s)) return PROX_EINVAL;
     if (batch == 0) return PROX_OK;
     if (!x || !y || !ws || !aligned16(x) || !aligned16(y) || !aligned16(ws)) return PROX_EINVAL;
+    if (!aligned16(mask_x) || !aligned16(mask_s) || !aligned16(idx_s) || !aligned16(count_s))
+        return PROX_EINVAL;
     return run_forward(layer, x, batch, tau_x, tau_s, y, mask_x, mask_s, idx_s, count_s, nullptr,
                        ws, ws_bytes, (cudaStream_t)stream, true);
 }
@@ -299,7 +304,8 @@ PROX_API prox_status prox_ffn_stage1(const prox_layer *layer, const uint16_t *x,
     if (batch < 0 || batch > max_tokens_per_pass(d) || !tau_ok(tau_x) || !tau_ok(tau_s))
         return PROX_EINVAL;
     if (batch == 0) return PROX_OK;
-    if (!x || !ws || !aligned16(x) || !aligned16(ws) || (y_clear && !aligned16(y_clear)))
+    if (!x || !ws || !aligned16(x) || !aligned16(ws) || !aligned16(y_clear) ||
+        !aligned16(mask_x) || !aligned16(mask_s))
         return PROX_EINVAL;
     if (ws_bytes < ws_layout(d, f, tokens_per_pass(d, batch)).total) return PROX_ENOMEM;
     int sms = 0;
@@ -317,7 +323,9 @@ PROX_API prox_status prox_ffn_stage2(const prox_layer *layer, const uint16_t *x,
     const int d = layer->d_model, f = layer->d_ff;
     if (batch < 0 || batch > max_tokens_per_pass(d)) return PROX_EINVAL;
     if (batch == 0) return PROX_OK;
-    if (!x || !y || !ws || !aligned16(x) || !aligned16(y) || !aligned16(ws)) return PROX_EINVAL;
+    if (!x || !y || !ws || !aligned16(x) || !aligned16(y) || !aligned16(ws) ||
+        !aligned16(idx_s) || !aligned16(count_s))
+        return PROX_EINVAL;
     if (ws_bytes < ws_layout(d, f, tokens_per_pass(d, batch)).total) return PROX_ENOMEM;
     int sms = 0;
     ps = current_device(&sms);
@@ -333,7 +341,9 @@ PROX_API prox_status prox_proxy_state(const prox_layer *layer, const uint16_t *x
     if (ps != PROX_OK) return ps;
     if (batch < 0 || !tau_ok(tau_x)) return PROX_EINVAL;
     if (batch == 0) return PROX_OK;
-    if (!x || !s_out || !ws || !aligned16(x) || !aligned16(ws)) return PROX_EINVAL;
+    if (!x || !s_out || !ws || !aligned16(x) || !aligned16(ws) || !aligned16(s_out) ||
+        !aligned16(mask_x))
+        return PROX_EINVAL;
     return run_forward(layer, x, batch, tau_x, 0.f, nullptr, mask_x, nullptr, nullptr, nullptr,
                        s_out, ws, ws_bytes, (cudaStream_t)stream, false);
 }

@@ -54,7 +54,7 @@ struct Stage2Plan {
 int max_tokens_per_pass(int d_model);
 int tokens_per_pass(int d_model, int batch);   // 1, 2, 4 or 8
 Stage1Plan stage1_plan(int d_model, int d_ff, int B, int num_sms);
-Stage2Plan stage2_plan(int d_model, int B);
+Stage2Plan stage2_plan(int d_model, int B, int C, int max_ch);
 
 // Workspace layout of one forward pass (B tokens). Offsets in bytes.
 struct WsLayout {
@@ -101,6 +101,7 @@ struct Stage2Args {
     int debug_skip;              // test hook: producer never fills this
                                  // channel position of CTA 0 (-1: off)
     int nstage;
+    int max_ch;                  // capacity of the per-CTA channel list
 };
 
 cudaError_t launch_stage1(int B, const Stage1Args &a, const Stage1Plan &p,
@@ -117,6 +118,25 @@ cudaError_t launch_select_bf16_abs(const uint16_t *v, long n, long rank,
 cudaError_t launch_select_f32_abs(const float *v, long n, long rank,
                                   uint32_t *hist, uint32_t *scratch,
                                   float *tau_dev, cudaStream_t s);
+
+// Launch with programmatic stream serialization (PDL): the kernel may start
+// while the previous kernel in the stream finishes; it must execute
+// griddepcontrol.wait before touching anything that kernel writes.
+template <typename Kern, typename Args>
+inline cudaError_t launch_pdl(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              const Args &args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args);
+}
 
 // ---------------------------------------------------------------------------
 // Device helpers

@@ -23,6 +23,8 @@
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream). Every
  *     call except prox_calibrate and prox_last_device_status is asynchronous
  *     on that stream and returns as soon as its kernels are enqueued.
+ *   - Every device pointer (inputs, outputs, workspace) must be 16-byte
+ *     aligned; optional outputs may be NULL.
  *   - Argument errors are detected on the host and returned before anything
  *     is launched. No C++ exception crosses this interface.
  *   - Shapes: d_model and d_ff are multiples of 256 with 256 <= d_model <= 8192

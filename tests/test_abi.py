@@ -87,6 +87,12 @@ def test_forward_validation_before_launch():
     assert _fwd(L, y=None) == P.PROX_EINVAL
     assert _fwd(L, ws=None) == P.PROX_EINVAL
     assert _fwd(L, batch=0) == P.PROX_OK            # nothing to do, nothing launched
+    lib = P.lib()
+    for k in range(4):   # optional outputs must be aligned when given
+        outs = [None] * 4
+        outs[k] = (1 << 27) + 8
+        assert lib.prox_ffn_forward(C.byref(L), 1 << 24, 1, 0.5, 0.1, 1 << 25, *outs,
+                                    1 << 26, 1 << 30, None) == P.PROX_EINVAL
 
 
 def test_other_entry_points_validate():
