@@ -216,24 +216,33 @@ def run_ours(args, w, rank, world, local_rank):
     xp, yp, wp = x.data_ptr(), y.data_ptr(), ws.data_ptr()
     sample_every = 8
     sampled = list(range(0, ntok, sample_every))
+    ev_s = {t: torch.cuda.Event(enable_timing=True, external=True) for t in sampled}
     ev_a = {t: torch.cuda.Event(enable_timing=True, external=True) for t in sampled}
     ev_b = {t: torch.cuda.Event(enable_timing=True, external=True) for t in sampled}
 
     def one_step(record):
+        # the public forward is Stage 1 then Stage 2; the split entry points
+        # let the instrumented copy put events between the two kernels
         for t in range(ntok):
             Ls = structs[t % R]
+            rec = record and t in ev_a
+            if rec:
+                ev_s[t].record(stream)
             P.ffn_stage1_raw(Ls, xp + t * xrow, 1, tau_x, tau_s, yp + t * yrow, wp, wsb, sp)
-            if record and t in ev_a:
+            if rec:
                 ev_a[t].record(stream)
             P.ffn_stage2_raw(Ls, xp + t * xrow, 1, yp + t * yrow, wp, wsb, sp)
-            if record and t in ev_b:
+            if rec:
                 ev_b[t].record(stream)
 
     with torch.cuda.stream(stream):
         one_step(False)
     torch.cuda.synchronize(dev)
-    g = torch.cuda.CUDAGraph()
+    g = torch.cuda.CUDAGraph()          # the timed step: no events inside
     with torch.cuda.graph(g, stream=stream):
+        one_step(False)
+    gi = torch.cuda.CUDAGraph()         # instrumented copy for per-kernel times
+    with torch.cuda.graph(gi, stream=stream):
         one_step(True)
     # parity spot-check of the graph's output against the direct call
     g.replay()
@@ -259,8 +268,15 @@ def run_ours(args, w, rank, world, local_rank):
             torch.cuda.current_stream(dev).wait_stream(stream)
         e1.record(stream)
         barrier()
-        # per-launch Stage-2 durations of the last replay's sampled tokens
-        s2_ms = [ev_a[t].elapsed_time(ev_b[t]) for t in sampled]
+        # per-kernel durations: events around each kernel of every 8th token,
+        # from instrumented replays run right after the timed ones
+        s1_ms, s2_ms = [], []
+        for _ in range(max(1, min(args.steps, 5))):
+            with torch.cuda.stream(stream):
+                gi.replay()
+            torch.cuda.synchronize(dev)
+            s1_ms += [ev_s[t].elapsed_time(ev_a[t]) for t in sampled]
+            s2_ms += [ev_a[t].elapsed_time(ev_b[t]) for t in sampled]
     ms_total = e0.elapsed_time(e1)
     if world > 1:
         tt = torch.tensor([ms_total], device=dev)
@@ -272,8 +288,11 @@ def run_ours(args, w, rank, world, local_rank):
 
     peak, peak_src = load_peaks()
     s2_us = statistics.mean(s2_ms) * 1e3
+    s1_us = statistics.mean(s1_ms) * 1e3
     s2_bytes = float(np.mean(stage2_bytes[sampled]))
     s2_gbs = s2_bytes / (s2_us * 1e-6) / 1e9
+    s1_bytes = float(np.mean((touched - stage2_bytes)[sampled]))
+    s1_gbs = s1_bytes / (s1_us * 1e-6) / 1e9
     path_gbs = float(np.mean(touched)) / (us_tok_rank * 1e-6) / 1e9
 
     # e2e through the public API with host buffers: pinned x in, y out
@@ -368,6 +387,8 @@ def run_ours(args, w, rank, world, local_rank):
                          "achieved": s2_gbs, "peak": peak, "unit": "GB/s",
                          "frac": s2_gbs / peak, "traffic": None, "peak_source": peak_src,
                          "bytes_per_launch": s2_bytes, "us_per_launch": s2_us},
+            "stage1": {"kernel": "k_stage1 (INT4 proxy + channel mask)", "us_per_launch": s1_us,
+                       "bytes_per_launch": s1_bytes, "GBps": s1_gbs, "frac": s1_gbs / peak},
             "path": {"touched_MB_per_token": float(np.mean(touched)) / 1e6,
                      "GBps": path_gbs, "frac_of_peak": path_gbs / peak,
                      "keep_x": float(np.mean(kx)) / d, "keep_s": float(np.mean(ks)) / f},
@@ -379,7 +400,7 @@ def run_ours(args, w, rank, world, local_rank):
             "clocks": clk.summary(),
         }
         print(json.dumps(line), flush=True)
-    del g
+    del g, gi
 
 
 def main():

@@ -42,7 +42,7 @@ struct S1 {
     static constexpr int TPRM = kCB / CPT;                           // threads per row per matrix
     static constexpr int TPR = 2 * TPRM;                             // threads per row
     static constexpr int RL = kS1Threads / TPR;                      // row lanes
-    static constexpr int U = 128 / BYTES;                            // rows in flight per thread
+    static constexpr int U = 64 / BYTES;                             // rows per load set (2 sets)
 };
 
 template <int WORDS>
@@ -170,7 +170,8 @@ __global__ void __launch_bounds__(kS1Threads, 2) k_stage1(const Stage1Args a) {
     // 16-byte chunks of 8 coordinates; all its loads are issued before any
     // use. Chunk ci's 8 keep bits are byte ci of the token's mask words.
     {
-        constexpr int MAXK = 4;  // chunks per thread per token (d_model <= 8192)
+        // chunks per thread per token: d_model <= 8192, and <= 4096 when B = 8
+        constexpr int MAXK = (B == 8) ? 2 : 4;
         const int NC = a.d / 8;
         uint4 xv[MAXK][B];
 #pragma unroll
@@ -252,6 +253,28 @@ __global__ void __launch_bounds__(kS1Threads, 2) k_stage1(const Stage1Args a) {
         rowidx[rank - lo] = wd * 32 + lane;
     }
     __syncthreads();
+
+    // main-loop geometry; the first set of proxy rows is requested now so that
+    // its latency overlaps the scale gather below
+    const int rl = tid / T::TPR;
+    const int m = (tid / T::TPRM) & 1;
+    const int chunk = tid % T::TPRM;
+    const uint8_t *qbase = (m ? a.q_gate : a.q_up) + (size_t)c * (kCB / 2) + chunk * T::BYTES;
+    const size_t rstride = (size_t)a.f / 2;
+    Vec<T::WORDS> va[T::U], vb[T::U];
+    auto load_set = [&](Vec<T::WORDS>(&v)[T::U], int u0) {
+#pragma unroll
+        for (int k = 0; k < T::U; ++k) {
+            const int u = u0 + k * T::RL;
+            if (u < n_units) {
+                ld_stream(v[k], qbase + (size_t)rowidx[u] * rstride);
+            } else {
+#pragma unroll
+                for (int q = 0; q < T::WORDS; ++q) v[k].w[q] = 0x88888888u;  // code 0
+            }
+        }
+    };
+    load_set(va, rl);
     {
         constexpr int G4 = 4;  // units per batch of loads
         for (int u0 = tid; u0 < n_units; u0 += G4 * kS1Threads) {
@@ -331,28 +354,12 @@ __global__ void __launch_bounds__(kS1Threads, 2) k_stage1(const Stage1Args a) {
         __syncthreads();
     }
 
-    // (6) main loop: stream the 128-byte block segments of the kept rows
-    const int rl = tid / T::TPR;
-    const int m = (tid / T::TPRM) & 1;
-    const int chunk = tid % T::TPRM;
-    const uint8_t *qbase = (m ? a.q_gate : a.q_up) + (size_t)c * (kCB / 2) + chunk * T::BYTES;
-    const size_t rstride = (size_t)a.f / 2;
+    // (6) main loop: stream the 128-byte block segments of the kept rows,
+    // two register sets in flight (load one while decoding the other)
     float acc[T::ACC];
 #pragma unroll
     for (int k = 0; k < T::ACC; ++k) acc[k] = 0.f;
-
-    for (int u0 = rl; u0 < n_units; u0 += T::RL * T::U) {
-        Vec<T::WORDS> v[T::U];
-#pragma unroll
-        for (int k = 0; k < T::U; ++k) {
-            const int u = u0 + k * T::RL;
-            if (u < n_units) {
-                ld_stream(v[k], qbase + (size_t)rowidx[u] * rstride);
-            } else {
-#pragma unroll
-                for (int q = 0; q < T::WORDS; ++q) v[k].w[q] = 0x88888888u;  // code 0
-            }
-        }
+    auto comp_set = [&](const Vec<T::WORDS>(&v)[T::U], int u0) {
 #pragma unroll
         for (int k = 0; k < T::U; ++k) {
             const int u = u0 + k * T::RL;
@@ -362,6 +369,13 @@ __global__ void __launch_bounds__(kS1Threads, 2) k_stage1(const Stage1Args a) {
 #pragma unroll
             for (int q = 0; q < T::WORDS; ++q) proc_word<B, T::CPT>(v[k].w[q], q, xv, acc);
         }
+    };
+    constexpr int STEP = T::RL * T::U;
+    for (int u0 = rl; u0 < n_units; u0 += 2 * STEP) {
+        load_set(vb, u0 + STEP);
+        comp_set(va, u0);
+        load_set(va, u0 + 2 * STEP);
+        comp_set(vb, u0 + STEP);
     }
 
     // (7) reduce row lanes, undo the pre-scale and the +8 code offset, write

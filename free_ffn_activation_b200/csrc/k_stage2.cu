@@ -7,14 +7,19 @@
 // One persistent CTA per SM takes an equal share of the kept channels (the
 // union over the pass's tokens, in ascending order). W_up and W_gate are
 // stored channel-major and W_down row-major, so a kept channel j is three
-// contiguous d_model-long bf16 rows. A producer lane moves them with 1-D bulk
-// copies (TMA) into a ring of shared-memory stages guarded by mbarriers;
-// 16 consumer warps each own a 1/16 slice of the d_model columns: they form
-// partial dot products x . W_up[j] and x . W_gate[j] on their slice, exchange
-// them through shared memory (an mbarrier, not a hardware barrier, so every
-// wait is bounded), compute s_j = u_j * SiLU(g_j) in fp32 and accumulate
-// s_j * W_down[j, slice] into registers. At the end each CTA adds its partial
-// y to global memory with 16-byte vector reductions.
+// contiguous d_model-long bf16 rows. Roles inside the CTA:
+//   * a producer lane moves each channel's three rows with 1-D bulk copies
+//     (TMA) into a ring of shared-memory stages (mbarrier "full");
+//   * 8 dot warps take whole channels round-robin: a warp forms x . W_up[j]
+//     and x . W_gate[j] over the full row, reduces across its lanes, computes
+//     s_j = u_j * SiLU(g_j) in fp32 and publishes it (mbarrier "sready");
+//   * the down warps own fixed column slices of y: for every channel, in
+//     order, they add s_j * W_down[j, slice] to register accumulators.
+// A stage is refilled once its dot warp and every down warp have released it
+// (mbarrier "empty"). Channels never wait on each other through a CTA-wide
+// barrier, so several channels are in flight at once, and every wait is
+// bounded. At the end each CTA adds its partial y to global memory with
+// 16-byte vector reductions.
 #include "prox_internal.cuh"
 
 #include <cuda_runtime.h>
@@ -22,9 +27,16 @@
 
 namespace prox {
 
+constexpr int kNDot = 8;
+
+// warps and shared x precision per tokens-per-pass
+__host__ __device__ constexpr int s2_ndown(int B) { return B <= 2 ? 8 : 16; }
+__host__ __device__ constexpr int s2_threads(int B) { return (kNDot + s2_ndown(B) + 1) * 32; }
+__host__ __device__ constexpr int s2_xbytes(int B) { return B <= 2 ? 4 : 2; }
+
 // shared-memory carve-up, shared by the kernel and the host plan
 struct S2Smem {
-    size_t stages, xs, full, empty, redbar, meta, red, uscan, tscan, chan, total;
+    size_t stages, xs, full, empty, sready, meta, svals, uscan, tscan, chan, total;
 };
 
 __host__ __device__ inline S2Smem s2_smem(int d, int B, int nstage, int C, int max_ch) {
@@ -33,19 +45,19 @@ __host__ __device__ inline S2Smem s2_smem(int d, int B, int nstage, int C, int m
     s.stages = o;
     o += (size_t)nstage * 3 * d * 2;
     s.xs = o;
-    o += (size_t)B * d * 2;
+    o += (size_t)B * d * s2_xbytes(B);
     o = (o + 15) & ~(size_t)15;
     s.full = o;
     o += (size_t)nstage * 8;
     s.empty = o;
     o += (size_t)nstage * 8;
-    s.redbar = o;
-    o += 2 * 8;
+    s.sready = o;
+    o += (size_t)nstage * 8;
     s.meta = o;
     o += (size_t)nstage * 4;
+    s.svals = o;
+    o += (size_t)nstage * B * 4;
     o = (o + 15) & ~(size_t)15;
-    s.red = o;
-    o += (size_t)2 * kNCW * 2 * B * 4;
     s.uscan = o;
     o += (size_t)(C + 1) * 4;
     s.tscan = o;
@@ -62,57 +74,64 @@ __device__ __forceinline__ uint4 lds128(const void *p) {
     return *reinterpret_cast<const uint4 *>(p);
 }
 
-// acc += x . w over 8 bf16 pairs
-__device__ __forceinline__ float dot8(const uint4 &x, const uint4 &w, float acc) {
-    const uint32_t xa[4] = {x.x, x.y, x.z, x.w};
-    const uint32_t wa[4] = {w.x, w.y, w.z, w.w};
+__device__ __forceinline__ void bf16x8_to_f2(const uint4 &w, float2 (&o)[4]) {
+    const uint32_t a[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        acc = fmaf(bf16lo(xa[q]), bf16lo(wa[q]), acc);
-        acc = fmaf(bf16hi(xa[q]), bf16hi(wa[q]), acc);
-    }
-    return acc;
+    for (int q = 0; q < 4; ++q) o[q] = make_float2(bf16lo(a[q]), bf16hi(a[q]));
 }
 
-template <int B, int NCH>
-__global__ void __launch_bounds__(kS2Threads, 1) k_stage2(const Stage2Args a) {
+template <int B, int NCHD>
+__global__ void __launch_bounds__(s2_threads(B), 1) k_stage2(const Stage2Args a) {
+    constexpr int NDOWN = s2_ndown(B);
+    constexpr bool XF32 = (B <= 2);
     extern __shared__ __align__(128) unsigned char smem[];
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int d = a.d, C = a.C, NST = a.nstage;
     const S2Smem L = s2_smem(d, B, NST, C, a.max_ch);
     uint16_t *stages = reinterpret_cast<uint16_t *>(smem + L.stages);
-    uint16_t *xsm = reinterpret_cast<uint16_t *>(smem + L.xs);
+    float *xf = reinterpret_cast<float *>(smem + L.xs);        // XF32: [B][2][d/2]
+    uint16_t *xh = reinterpret_cast<uint16_t *>(smem + L.xs);  // else: [B][d]
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.full);
     uint64_t *empty = reinterpret_cast<uint64_t *>(smem + L.empty);
-    uint64_t *redbar = reinterpret_cast<uint64_t *>(smem + L.redbar);
+    uint64_t *sready = reinterpret_cast<uint64_t *>(smem + L.sready);
     uint32_t *meta = reinterpret_cast<uint32_t *>(smem + L.meta);
-    float *red = reinterpret_cast<float *>(smem + L.red);  // [2][kNCW][B][2]
-    int *uscan = reinterpret_cast<int *>(smem + L.uscan);  // [C+1]
-    int *tscan = reinterpret_cast<int *>(smem + L.tscan);  // [B][C+1]
+    float *svals = reinterpret_cast<float *>(smem + L.svals);  // [NST][B]
+    int *uscan = reinterpret_cast<int *>(smem + L.uscan);      // [C+1]
+    int *tscan = reinterpret_cast<int *>(smem + L.tscan);      // [B][C+1]
     uint32_t *chan = reinterpret_cast<uint32_t *>(smem + L.chan);  // [max_ch]
     const int nch16 = d / 8;  // 16-byte chunks per row
 
     if (tid == 0) {
         for (int s = 0; s < NST; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kNCW);
+            mbar_init(&empty[s], 1 + NDOWN);
+            mbar_init(&sready[s], 1);
         }
-        mbar_init(&redbar[0], kNCW);
-        mbar_init(&redbar[1], kNCW);
         mbar_fence_init();
     }
-    // x (bf16) into shared memory; tokens beyond nb are zero. Stage 1, the
-    // kernel this one may overlap, only triggers this launch after its own
-    // griddepcontrol.wait, so x (written before Stage 1 ran) is complete.
-    for (int k = tid; k < B * nch16; k += kS2Threads) {
+    // x into shared memory (fp32, split in halves so that a lane's two
+    // 16-byte reads of a chunk fall in different bank groups; or bf16).
+    // Stage 1, the kernel this one may overlap, only triggers this launch
+    // after its own griddepcontrol.wait, so x (written before Stage 1 ran)
+    // is complete.
+    for (int k = tid; k < B * nch16; k += s2_threads(B)) {
         const int t = k / nch16, ci = k % nch16;
         uint4 v = make_uint4(0, 0, 0, 0);
         if (t < a.nb) v = *reinterpret_cast<const uint4 *>(a.x + (size_t)t * d + ci * 8);
-        *reinterpret_cast<uint4 *>(xsm + (size_t)t * d + ci * 8) = v;
+        if constexpr (XF32) {
+            float2 f[4];
+            bf16x8_to_f2(v, f);
+            float *base = xf + (size_t)t * d;
+            *reinterpret_cast<float4 *>(base + ci * 4) = make_float4(f[0].x, f[0].y, f[1].x, f[1].y);
+            *reinterpret_cast<float4 *>(base + d / 2 + ci * 4) =
+                make_float4(f[2].x, f[2].y, f[3].x, f[3].y);
+        } else {
+            *reinterpret_cast<uint4 *>(xh + (size_t)t * d + ci * 8) = v;
+        }
     }
     // Stage 1's lists are ready once it has completed
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    for (int k = tid; k < C * (B + 1); k += kS2Threads) {
+    for (int k = tid; k < C * (B + 1); k += s2_threads(B)) {
         if (k < C) {
             uscan[k] = a.ucount[k];
         } else {
@@ -149,7 +168,7 @@ __global__ void __launch_bounds__(kS2Threads, 1) k_stage2(const Stage2Args a) {
     const int n_ch = p1 - p0;
 
     // this CTA's share of the ascending kept-channel list, into shared memory
-    for (int n = tid; n < n_ch; n += kS2Threads) {
+    for (int n = tid; n < n_ch; n += s2_threads(B)) {
         const int p = p0 + n;
         int lo = 0, hi = C - 1;  // block cb with uscan[cb] <= p < uscan[cb + 1]
         while (lo < hi) {
@@ -161,18 +180,16 @@ __global__ void __launch_bounds__(kS2Threads, 1) k_stage2(const Stage2Args a) {
     __syncthreads();
     asm volatile("griddepcontrol.launch_dependents;");
 
-    if (wid == kNCW) {
+    if (wid == kNDot + NDOWN) {
         // ---------------- producer ----------------
         if (lane != 0) return;
         const uint32_t row_bytes = (uint32_t)d * 2;
         int issued = 0;
-        bool ok = true;
         for (int n = 0; n < n_ch; ++n) {
             const uint32_t e = chan[n];
             const int s = n % NST, k = n / NST;
             if (k > 0 && !mbar_wait(&empty[s], (k - 1) & 1, a.spin_limit)) {
                 atomicOr(a.status, kStTimeoutEmpty);
-                ok = false;
                 break;
             }
             meta[s] = e;
@@ -194,95 +211,117 @@ __global__ void __launch_bounds__(kS2Threads, 1) k_stage2(const Stage2Args a) {
                 break;
             }
         }
-        (void)ok;
         return;
     }
 
-    // ---------------- consumers ----------------
-    float yacc[B][NCH][8];
+    if (wid < kNDot) {
+        // ---------------- dot warps: u_j, g_j, s_j ----------------
+        for (int n = wid; n < n_ch; n += kNDot) {
+            const int s = n % NST, k = n / NST;
+            if (!mbar_wait(&full[s], k & 1, a.spin_limit)) {
+                if (lane == 0) atomicOr(a.status, kStTimeoutFull);
+                break;
+            }
+            const uint32_t bits = (B == 1) ? 1u : (meta[s] >> 24);
+            const uint16_t *up = stages + (size_t)s * 3 * d;
+            const uint16_t *gt = up + d;
+            float2 u2[B], g2[B];
+#pragma unroll
+            for (int t = 0; t < B; ++t) u2[t] = g2[t] = make_float2(0.f, 0.f);
+            for (int ci = lane; ci < nch16; ci += 32) {
+                float2 wu[4], wg[4];
+                bf16x8_to_f2(lds128(up + ci * 8), wu);
+                bf16x8_to_f2(lds128(gt + ci * 8), wg);
+#pragma unroll
+                for (int t = 0; t < B; ++t) {
+                    if (B > 1 && !((bits >> t) & 1u)) continue;
+                    float2 xv[4];
+                    if constexpr (XF32) {
+                        const float4 xa = *reinterpret_cast<const float4 *>(xf + (size_t)t * d + ci * 4);
+                        const float4 xb =
+                            *reinterpret_cast<const float4 *>(xf + (size_t)t * d + d / 2 + ci * 4);
+                        xv[0] = make_float2(xa.x, xa.y);
+                        xv[1] = make_float2(xa.z, xa.w);
+                        xv[2] = make_float2(xb.x, xb.y);
+                        xv[3] = make_float2(xb.z, xb.w);
+                    } else {
+                        bf16x8_to_f2(lds128(xh + (size_t)t * d + ci * 8), xv);
+                    }
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        u2[t] = __ffma2_rn(xv[q], wu[q], u2[t]);
+                        g2[t] = __ffma2_rn(xv[q], wg[q], g2[t]);
+                    }
+                }
+            }
+            float sv[B];
+#pragma unroll
+            for (int t = 0; t < B; ++t) {
+                float u = u2[t].x + u2[t].y, gg = g2[t].x + g2[t].y;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    u += __shfl_xor_sync(0xffffffffu, u, o);
+                    gg += __shfl_xor_sync(0xffffffffu, gg, o);
+                }
+                sv[t] = ((bits >> t) & 1u) ? u * (gg / (1.f + expf(-gg))) : 0.f;
+            }
+            __syncwarp();
+            if (lane == 0) {
+#pragma unroll
+                for (int t = 0; t < B; ++t) svals[s * B + t] = sv[t];
+                mbar_arrive(&sready[s]);
+                mbar_arrive(&empty[s]);  // done with the up/gate rows
+            }
+        }
+        // per-token ascending kept-channel lists (blocks c = g, g + G, ...)
+        if (a.idx_s) {
+            for (int c = g; c < C; c += G) {
+                for (int t = 0; t < a.nb; ++t) {
+                    const int nk = a.tcount[c * B + t];
+                    const int base = tscan[t * (C + 1) + c];
+                    for (int k = tid; k < nk; k += kNDot * 32)
+                        a.idx_s[(size_t)t * a.f + base + k] =
+                            a.tlist[(size_t)t * a.f + c * kCB + k];
+                }
+            }
+        }
+        if (g == 0 && a.count_s && tid < a.nb) a.count_s[tid] = tscan[tid * (C + 1) + C];
+        return;
+    }
+
+    // ---------------- down warps: y slice += s_j * W_down[j, slice] ----------
+    const int dt = tid - kNDot * 32;
+    float2 acc[B][NCHD][4];
 #pragma unroll
     for (int t = 0; t < B; ++t)
 #pragma unroll
-        for (int q = 0; q < NCH; ++q)
+        for (int m = 0; m < NCHD; ++m)
 #pragma unroll
-            for (int k = 0; k < 8; ++k) yacc[t][q][k] = 0.f;
+            for (int q = 0; q < 4; ++q) acc[t][m][q] = make_float2(0.f, 0.f);
 
     for (int n = 0; n < n_ch; ++n) {
-        const int s = n % NST, k = n / NST;
-        if (!mbar_wait(&full[s], k & 1, a.spin_limit)) {
-            if (lane == 0) atomicOr(a.status, kStTimeoutFull);
-            break;
-        }
-        const uint32_t bits = meta[s] >> 24;
-        const uint16_t *up = stages + (size_t)s * 3 * d;
-        const uint16_t *gt = up + d;
-        const uint16_t *dn = up + 2 * d;
-
-        float pu[B], pg[B];
-#pragma unroll
-        for (int t = 0; t < B; ++t) pu[t] = pg[t] = 0.f;
-#pragma unroll
-        for (int q = 0; q < NCH; ++q) {
-            const int ci = tid + q * kNCW * 32;
-            if (ci < nch16) {
-                const uint4 wu = lds128(up + ci * 8);
-                const uint4 wg = lds128(gt + ci * 8);
-#pragma unroll
-                for (int t = 0; t < B; ++t) {
-                    if (!((bits >> t) & 1u)) continue;
-                    const uint4 xv = lds128(xsm + (size_t)t * d + ci * 8);
-                    pu[t] = dot8(xv, wu, pu[t]);
-                    pg[t] = dot8(xv, wg, pg[t]);
-                }
-            }
-        }
-#pragma unroll
-        for (int t = 0; t < B; ++t) {
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                pu[t] += __shfl_xor_sync(0xffffffffu, pu[t], o);
-                pg[t] += __shfl_xor_sync(0xffffffffu, pg[t], o);
-            }
-        }
-        float *rb = red + (size_t)(n & 1) * kNCW * B * 2;
-        if (lane == 0) {
-#pragma unroll
-            for (int t = 0; t < B; ++t) {
-                rb[(wid * B + t) * 2 + 0] = pu[t];
-                rb[(wid * B + t) * 2 + 1] = pg[t];
-            }
-            mbar_arrive(&redbar[n & 1]);
-        }
-        if (!mbar_wait(&redbar[n & 1], (n >> 1) & 1, a.spin_limit)) {
+        const int s = n % NST, ph = (n / NST) & 1;
+        if (!mbar_wait(&full[s], ph, a.spin_limit) || !mbar_wait(&sready[s], ph, a.spin_limit)) {
             if (lane == 0) atomicOr(a.status, kStTimeoutRed);
             break;
         }
+        const uint32_t bits = (B == 1) ? 1u : (meta[s] >> 24);
         float sv[B];
 #pragma unroll
-        for (int t = 0; t < B; ++t) {
-            float u = 0.f, gg = 0.f;
-            if ((bits >> t) & 1u) {
+        for (int t = 0; t < B; ++t) sv[t] = svals[s * B + t];
+        const uint16_t *dn = stages + (size_t)s * 3 * d + 2 * d;
 #pragma unroll
-                for (int w = 0; w < kNCW; ++w) {
-                    u += rb[(w * B + t) * 2 + 0];
-                    gg += rb[(w * B + t) * 2 + 1];
-                }
-            }
-            sv[t] = ((bits >> t) & 1u) ? u * (gg / (1.f + expf(-gg))) : 0.f;
-        }
-#pragma unroll
-        for (int q = 0; q < NCH; ++q) {
-            const int ci = tid + q * kNCW * 32;
+        for (int m = 0; m < NCHD; ++m) {
+            const int ci = dt + m * NDOWN * 32;
             if (ci < nch16) {
-                const uint4 wd = lds128(dn + ci * 8);
-                const uint32_t wa[4] = {wd.x, wd.y, wd.z, wd.w};
+                float2 w[4];
+                bf16x8_to_f2(lds128(dn + ci * 8), w);
 #pragma unroll
                 for (int t = 0; t < B; ++t) {
+                    if (B > 1 && !((bits >> t) & 1u)) continue;
+                    const float2 ss = make_float2(sv[t], sv[t]);
 #pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                        yacc[t][q][2 * h] = fmaf(sv[t], bf16lo(wa[h]), yacc[t][q][2 * h]);
-                        yacc[t][q][2 * h + 1] = fmaf(sv[t], bf16hi(wa[h]), yacc[t][q][2 * h + 1]);
-                    }
+                    for (int q = 0; q < 4; ++q) acc[t][m][q] = __ffma2_rn(ss, w[q], acc[t][m][q]);
                 }
             }
         }
@@ -290,38 +329,25 @@ __global__ void __launch_bounds__(kS2Threads, 1) k_stage2(const Stage2Args a) {
         if (lane == 0) mbar_arrive(&empty[s]);
     }
 
-    // per-token ascending kept-channel lists (blocks c = g, g + G, ...)
-    if (a.idx_s) {
-        for (int c = g; c < C; c += G) {
-            for (int t = 0; t < a.nb; ++t) {
-                const int n = a.tcount[c * B + t];
-                const int base = tscan[t * (C + 1) + c];
-                for (int k = tid; k < n; k += kNCW * 32)
-                    a.idx_s[(size_t)t * a.f + base + k] = a.tlist[(size_t)t * a.f + c * kCB + k];
-            }
-        }
-    }
-    if (g == 0 && a.count_s && tid < a.nb) a.count_s[tid] = tscan[tid * (C + 1) + C];
-
     if (n_ch == 0) return;
 #pragma unroll
     for (int t = 0; t < B; ++t) {
         if (t >= a.nb) break;
 #pragma unroll
-        for (int q = 0; q < NCH; ++q) {
-            const int ci = tid + q * kNCW * 32;
+        for (int m = 0; m < NCHD; ++m) {
+            const int ci = dt + m * NDOWN * 32;
             if (ci < nch16) {
                 float *dst = a.y + (size_t)t * d + ci * 8;
-                red_add_v4(dst, yacc[t][q][0], yacc[t][q][1], yacc[t][q][2], yacc[t][q][3]);
-                red_add_v4(dst + 4, yacc[t][q][4], yacc[t][q][5], yacc[t][q][6], yacc[t][q][7]);
+                red_add_v4(dst, acc[t][m][0].x, acc[t][m][0].y, acc[t][m][1].x, acc[t][m][1].y);
+                red_add_v4(dst + 4, acc[t][m][2].x, acc[t][m][2].y, acc[t][m][3].x, acc[t][m][3].y);
             }
         }
     }
 }
 
-template <int B, int NCH>
+template <int B, int NCHD>
 cudaError_t launch2(const Stage2Args &a, int grid, size_t smem, cudaStream_t s) {
-    auto k = k_stage2<B, NCH>;
+    auto k = k_stage2<B, NCHD>;
     static size_t configured = 0;  // dynamic smem limit already set for this kernel
     if (smem > configured) {
         cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -329,16 +355,24 @@ cudaError_t launch2(const Stage2Args &a, int grid, size_t smem, cudaStream_t s) 
         if (e != cudaSuccess) return e;
         configured = smem;
     }
-    return launch_pdl(k, dim3(grid), dim3(kS2Threads), smem, s, a);
+    return launch_pdl(k, dim3(grid), dim3(s2_threads(B)), smem, s, a);
 }
 
 }  // namespace
 
-cudaError_t launch_stage2(int B, int nchunk, const Stage2Args &a, int grid, size_t smem,
+// chunks of 8 columns each down thread owns (a power of two)
+int stage2_nchd(int d_model, int B) {
+    const int per = (d_model / 8 + s2_ndown(B) * 32 - 1) / (s2_ndown(B) * 32);
+    int p = 1;
+    while (p < per) p <<= 1;
+    return p;
+}
+
+cudaError_t launch_stage2(int B, int nchd, const Stage2Args &a, int grid, size_t smem,
                           cudaStream_t s) {
 #define PROX_S2(BB, NN) \
-    if (B == BB && nchunk == NN) return launch2<BB, NN>(a, grid, smem, s);
-    PROX_S2(1, 1) PROX_S2(1, 2) PROX_S2(1, 4) PROX_S2(1, 8)
+    if (B == BB && nchd == NN) return launch2<BB, NN>(a, grid, smem, s);
+    PROX_S2(1, 1) PROX_S2(1, 2) PROX_S2(1, 4)
     PROX_S2(2, 1) PROX_S2(2, 2) PROX_S2(2, 4)
     PROX_S2(4, 1) PROX_S2(4, 2)
     PROX_S2(8, 1)

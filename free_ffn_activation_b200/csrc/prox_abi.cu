@@ -17,6 +17,7 @@ namespace prox {
 
 size_t stage1_smem_bytes(int d_model, int B, int unit_cap);
 size_t stage2_smem_bytes(int d_model, int B, int nstage, int C, int max_ch);
+int stage2_nchd(int d_model, int B);
 
 int max_tokens_per_pass(int d_model) {
     if (d_model <= 4096) return 8;
@@ -59,7 +60,7 @@ Stage1Plan stage1_plan(int d, int f, int B, int num_sms) {
 
 Stage2Plan stage2_plan(int d, int B, int C, int max_ch) {
     Stage2Plan p;
-    p.nchunk = pow2_ceil((d / 8 + kNCW * 32 - 1) / (kNCW * 32));
+    p.nchunk = stage2_nchd(d, B);
     const size_t stage = (size_t)6 * d;
     const size_t fixed = stage2_smem_bytes(d, B, 0, C, max_ch);
     int ns = fixed < (size_t)kS2SmemBudget ? (int)((kS2SmemBudget - fixed) / stage) : 0;

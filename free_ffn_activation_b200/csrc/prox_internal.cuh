@@ -17,8 +17,6 @@ namespace prox {
 constexpr int kCB = 256;            // channels per Stage-1 column block
 constexpr int kS1Threads = 256;     // Stage-1 CTA size
 constexpr int kS1MaxRowGroups = 16; // upper bound of row groups per block
-constexpr int kNCW = 16;            // Stage-2 consumer warps
-constexpr int kS2Threads = kNCW * 32 + 32;  // + one producer warp
 constexpr int kMaxB = 8;            // tokens per pass (per-token masks)
 constexpr int kS1UnitBudget = 96 * 1024;    // smem bytes for Stage-1 unit lists
 constexpr int kS2SmemBudget = 224 * 1024;   // opt-in dynamic smem per CTA
@@ -44,7 +42,7 @@ struct Stage1Plan {
 };
 
 struct Stage2Plan {
-    int nchunk;     // 16-byte chunks of a d_model row per consumer thread
+    int nchunk;     // 16-byte chunks of a d_model row per Stage-2 down thread
     int nstage;     // stages in the bulk-copy ring
     size_t smem;    // dynamic shared memory bytes
 };
