@@ -10,7 +10,8 @@
 // contiguous d_model-long bf16 rows. Roles inside the CTA:
 //   * a producer lane moves each channel's three rows with 1-D bulk copies
 //     (TMA) into a ring of shared-memory stages (mbarrier "full");
-//   * 8 dot warps take whole channels round-robin: a warp forms x . W_up[j]
+//   * 8 dot warps take whole channels (ring slot s belongs to warp s % 8): a
+//     warp forms x . W_up[j]
 //     and x . W_gate[j] over the full row, reduces across its lanes, computes
 //     s_j = u_j * SiLU(g_j) in fp32 and publishes it (mbarrier "sready");
 //   * the down warps own fixed column slices of y: for every channel, in
@@ -216,8 +217,12 @@ __global__ void __launch_bounds__(s2_threads(B), 1) k_stage2(const Stage2Args a)
 
     if (wid < kNDot) {
         // ---------------- dot warps: u_j, g_j, s_j ----------------
-        for (int n = wid; n < n_ch; n += kNDot) {
+        // Slot s always belongs to dot warp s % kNDot, so a warp waits on each
+        // of its slots' phases in order (a parity wait is only meaningful once
+        // the slot's previous phase has been observed by the same waiter).
+        for (int n = 0; n < n_ch; ++n) {
             const int s = n % NST, k = n / NST;
+            if (s % kNDot != wid) continue;
             if (!mbar_wait(&full[s], k & 1, a.spin_limit)) {
                 if (lane == 0) atomicOr(a.status, kStTimeoutFull);
                 break;

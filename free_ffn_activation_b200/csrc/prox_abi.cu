@@ -151,7 +151,7 @@ static prox_status check_layer(const prox_layer *L, bool need_exact) {
 static bool tau_ok(float t) { return std::isfinite(t) && t >= 0.f; }
 
 // test hooks (set by prox_debug_set through the binding's test helpers only)
-static uint32_t g_spin_limit = kDefaultSpinLimit;
+static uint32_t g_spin_limit = kDefaultWaitUs;
 static int g_debug_skip = -1;
 
 // One pass (nb <= tokens_per_pass tokens) of Stage 1: masks, kept-channel
@@ -473,6 +473,6 @@ PROX_API const char *prox_status_str(prox_status s) {
 // Stage-2 producer of CTA 0 skip one channel position, so that a test can
 // exercise the timeout path without faulting anything.
 PROX_API void prox_test_set_wait(uint32_t spin_limit, int skip_position) {
-    prox::g_spin_limit = spin_limit ? spin_limit : kDefaultSpinLimit;
+    prox::g_spin_limit = spin_limit ? spin_limit : kDefaultWaitUs;
     prox::g_debug_skip = skip_position;
 }

@@ -27,9 +27,8 @@ constexpr uint32_t kStTimeoutEmpty = 1u << 1;  // producer waited for a free slo
 constexpr uint32_t kStTimeoutRed = 1u << 2;    // consumers waited for partials
 constexpr uint32_t kStTimeoutDrain = 1u << 3;  // producer waited for its copies
 
-// default poll budget of a bounded mbarrier wait (each poll is a try_wait,
-// which itself blocks for a hardware-defined interval)
-constexpr uint32_t kDefaultSpinLimit = 1u << 22;
+// default wall-clock bound of a device-side wait, in microseconds
+constexpr uint32_t kDefaultWaitUs = 2000000u;
 
 // ---------------------------------------------------------------------------
 // Host-side plans
@@ -95,7 +94,7 @@ struct Stage2Args {
     const uint32_t *ulist;
     const int32_t *tlist;
     uint32_t *status;
-    uint32_t spin_limit;
+    uint32_t spin_limit;         // wall-clock bound of each wait, microseconds
     int debug_skip;              // test hook: producer never fills this
                                  // channel position of CTA 0 (-1: off)
     int nstage;
@@ -180,13 +179,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Bounded wait: returns false (and leaves the barrier alone) after `limit`
-// unsuccessful polls.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t limit) {
-    for (uint32_t i = 0; i < limit; ++i)
-        if (mbar_try_wait(bar, parity))
-            return true;
-    return false;
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Bounded wait on the phase of `bar` with the given parity: gives up and
+// returns false once `limit_us` microseconds of wall time have passed.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t limit_us) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    const uint64_t lim = (uint64_t)limit_us * 1000u;
+    while (!mbar_try_wait(bar, parity))
+        if (global_ns() - t0 > lim) return false;
+    return true;
 }
 
 // 1-D bulk copy global -> shared, completing on an mbarrier (TMA engine).

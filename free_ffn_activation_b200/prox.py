@@ -300,9 +300,9 @@ def last_device_status(ws: torch.Tensor) -> tuple[int, int]:
     return st, flags.value
 
 
-def test_set_wait(spin_limit: int = 0, skip_position: int = -1) -> None:
+def test_set_wait(wait_us: int = 0, skip_position: int = -1) -> None:
     """Test hook (prox_testing.h): shorter bounded waits / one unfilled stage."""
-    lib().prox_test_set_wait(int(spin_limit), int(skip_position))
+    lib().prox_test_set_wait(int(wait_us), int(skip_position))
 
 
 def touched_bytes(d_model: int, d_ff: int, k_x: int, k_s: int) -> int:
