@@ -8,8 +8,9 @@
 // i.e. per column i of the channel-major weight:
 //   scale_i = RN(max_j |W[i,j]| / 7),  q_ij = clamp(RN_even(RN(W[i,j] / scale_i)), -7, 7)
 // with IEEE fp32 division (__fdiv_rn) and round-half-even (__float2int_rn);
-// an all-zero row gives scale 0 and q 0. Packing: byte m of row i holds
-// channel 2m in the low nibble and 2m+1 in the high nibble, two's complement.
+// an all-zero row gives scale 0 and q 0. Packing (block-tiled, the layout
+// Stage 1 streams): byte m of granule q[c][i] holds channel 256c + 2m in the
+// low nibble and 256c + 2m + 1 in the high nibble, two's complement.
 //
 // Order statistic: the magnitude bit patterns of non-negative IEEE numbers
 // sort like unsigned integers, so the rank-k magnitude is found exactly by
@@ -66,7 +67,9 @@ __global__ void __launch_bounds__(256) k_pack(int d, int f, const uint16_t *__re
         }
         out[k / 8] |= (uint32_t)(v & 0xF) << (4 * (k % 8));
     }
-    *reinterpret_cast<uint4 *>(q + (size_t)(i0 + ii) * (f / 2) + (j0 + chunk * 32) / 2) =
+    // block-tiled output: q[c][i][0..127] holds channels [256c, 256c + 256) of row i
+    const int cblk = j0 / kCB, mbyte = (j0 % kCB + chunk * 32) / 2;
+    *reinterpret_cast<uint4 *>(q + ((size_t)cblk * d + i0 + ii) * (kCB / 2) + mbyte) =
         make_uint4(out[0], out[1], out[2], out[3]);
 }
 

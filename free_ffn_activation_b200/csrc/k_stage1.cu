@@ -3,32 +3,39 @@
 // (Prox deep-dive blog, section "Stage 1"; input-sparse projection Pi_in of
 // the translated arXiv page, section 2.2).
 //
-// Work split. The proxies are stored input-row-major ([d_model][d_ff/2]
-// nibbles), so a rejected input coordinate skips one whole contiguous row.
-// The d_ff channels are cut into column blocks of kCB = 256 channels (128
-// bytes of each proxy row); the kept rows are cut into n_r contiguous rank
-// ranges. CTA (c, r) streams the 128-byte segments of block c from the kept
-// rows of range r of BOTH proxies (one x read serves up and gate, as the
-// blog's "From formula to GPU" section describes for its split-N kernel) and
-// writes fp32 partial sums. The last CTA of a block to arrive (atomic ticket,
-// no waiting) sums the n_r partials in a fixed order, forms
-// s~ = u~ * SiLU(g~), thresholds it and compacts the kept channels into
-// ascending lists, so the result is deterministic.
+// Layout. The proxies are block-tiled: q[c][i][0..127] holds the 256 channels
+// [256c, 256c + 256) of input row i, two per byte. A rejected input
+// coordinate skips one 128-byte granule per block, and the kept rows of one
+// block are adjacent granules of one d_model * 128-byte region.
+//
+// Work split. Column block c (256 channels) is handled by a thread-block
+// cluster of n_r CTAs; CTA r of the cluster takes the r-th contiguous range
+// of the kept rows (ranks over the union of the pass's tokens) and streams
+// the granules of BOTH proxies (one read of x serves up and gate, the fused
+// split-N kernel of the blog's "From formula to GPU" section). Each thread
+// keeps a private ring of asynchronous copies (cp.async) several rows deep,
+// so about 64 KB per CTA is in flight without any barrier. The cluster's
+// partial sums meet in distributed shared memory: CTA 0 adds them in rank
+// order, forms s~ = u~ * SiLU(g~), thresholds it and compacts the kept
+// channels into ascending lists, so the result is deterministic.
 //
 // INT4 decode. A nibble n at bits 4p..4p+3 of a word, with every other bit
 // cleared, is the bit pattern of the subnormal float n * 2^(4p-149). XOR-ing
 // the nibble's top bit turns the stored two's complement code q into
 // n = q + 8 in the same single LOP3, so one logic op per weight yields an
 // exact float operand; the FMA multiplies it by x_i * scale_i pre-scaled by
-// 2^E (E chosen per CTA so products stay normal). At the end each channel's
-// sum is rescaled by the exact power of two 2^(149 - 4p - E) and the offset
+// 2^E (E chosen per CTA so sums stay normal). At the end each channel's sum
+// is rescaled by the exact power of two 2^(149 - 4p - E) and the offset
 // 8 * sum(x_i * scale_i) is removed. Nibbles 5..7 of a word are first shifted
 // down by 12 bits (to positions 2..4). Subnormal operands need FMA without
 // flush-to-zero, which is the default without fast-math.
 #include "prox_internal.cuh"
 
+#include <cooperative_groups.h>
 #include <cuda_runtime.h>
 #include <cstdint>
+
+namespace cg = cooperative_groups;
 
 namespace prox {
 namespace {
@@ -42,37 +49,8 @@ struct S1 {
     static constexpr int TPRM = kCB / CPT;                           // threads per row per matrix
     static constexpr int TPR = 2 * TPRM;                             // threads per row
     static constexpr int RL = kS1Threads / TPR;                      // row lanes
-    static constexpr int U = 64 / BYTES;                             // rows per load set (2 sets)
+    static constexpr int D = 256 / BYTES;                            // ring depth (rows)
 };
-
-template <int WORDS>
-struct Vec;
-template <>
-struct Vec<4> {
-    uint32_t w[4];
-};
-template <>
-struct Vec<2> {
-    uint32_t w[2];
-};
-template <>
-struct Vec<1> {
-    uint32_t w[1];
-};
-
-__device__ __forceinline__ void ld_stream(Vec<4> &v, const uint8_t *p) {
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3])
-                 : "l"(p));
-}
-__device__ __forceinline__ void ld_stream(Vec<2> &v, const uint8_t *p) {
-    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
-                 : "=r"(v.w[0]), "=r"(v.w[1])
-                 : "l"(p));
-}
-__device__ __forceinline__ void ld_stream(Vec<1> &v, const uint8_t *p) {
-    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v.w[0]) : "l"(p));
-}
 
 // nibble position (in units of 4 bits) of local channel k of a word after
 // the decode above
@@ -107,6 +85,24 @@ __device__ __forceinline__ void proc_word(uint32_t w, int wi, const float *xs, f
     }
 }
 
+// cp.async of BYTES (16, 8 or 4) from global to shared, L1 bypassed for 16
+template <int BYTES>
+__device__ __forceinline__ void cp_async(void *dst, const void *src) {
+    if constexpr (BYTES == 16) {
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src)
+                     : "memory");
+    } else {
+        asm volatile("cp.async.ca.shared.global [%0], [%1], %2;" ::"r"(smem_addr(dst)), "l"(src),
+                     "n"(BYTES)
+                     : "memory");
+    }
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // deterministic block-wide exclusive scan of one int per thread (256 threads)
 __device__ __forceinline__ int block_excl_scan(int v, int *warp_tot, int &total) {
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
@@ -129,27 +125,63 @@ __device__ __forceinline__ int block_excl_scan(int v, int *warp_tot, int &total)
     return base + inc - v;
 }
 
+}  // namespace
+
+// shared-memory carve-up of one Stage-1 CTA (kept next to the kernel)
+struct S1Smem {
+    size_t ring, tmask, umask, woff, rowidx, xs, part, total;
+};
+
+__host__ __device__ inline S1Smem s1_smem(int d, int B, int unit_cap) {
+    const int cpt = (B == 1) ? 32 : (B <= 4 ? 16 : 8);
+    const int rl = kS1Threads / (2 * (kCB / cpt));
+    const size_t ring = (size_t)kS1Threads * 256;                   // cp.async ring
+    const size_t red = (size_t)rl * 2 * B * (kCB + kCB / cpt) * 4;  // padded row-lane sums
+    const int W = d / 32;
+    S1Smem s;
+    size_t o = 0;
+    s.ring = o;  // the row-lane reduction reuses the ring once streaming is done
+    o += ring > red ? ring : red;
+    s.tmask = o;
+    o += (size_t)B * W * 4;
+    s.umask = o;
+    o += (size_t)W * 4;
+    s.woff = o;
+    o += (size_t)W * 4;
+    s.rowidx = o;
+    o += (size_t)unit_cap * 4;
+    s.xs = o;
+    o += (size_t)unit_cap * 2 * B * 4;
+    s.part = o;
+    o += (size_t)2 * B * kCB * 4;
+    s.total = o;
+    return s;
+}
+
+namespace {
+
 template <int B>
 __global__ void __launch_bounds__(kS1Threads, 2) k_stage1(const Stage1Args a) {
     using T = S1<B>;
     extern __shared__ __align__(16) unsigned char smem[];
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    const int c = blockIdx.x % a.C;
-    const int r = blockIdx.x / a.C;
-    const int W = a.d / 32;  // mask words per token
-
-    // shared memory carve-up
-    float *red = reinterpret_cast<float *>(smem);                    // [RL][2][B][kCB]
-    uint32_t *tmask = reinterpret_cast<uint32_t *>(red + T::RL * 2 * B * kCB);  // [B][W]
-    uint32_t *umask = tmask + B * W;                                  // [W]
-    int *woff = reinterpret_cast<int *>(umask + W);                   // [W]
-    int *rowidx = woff + W;                                           // [unit_cap]
-    float *xs = reinterpret_cast<float *>(rowidx + a.unit_cap);       // [unit_cap][2][B]
+    cg::cluster_group cluster = cg::this_cluster();
+    const int r = (int)cluster.block_rank();  // row group
+    const int c = blockIdx.x / a.n_r;          // column block
+    const int W = a.d / 32;                    // mask words per token
+    const S1Smem L = s1_smem(a.d, B, a.unit_cap);
+    unsigned char *ring = smem + L.ring;
+    float *red = reinterpret_cast<float *>(smem + L.ring);  // after streaming
+    uint32_t *tmask = reinterpret_cast<uint32_t *>(smem + L.tmask);  // [B][W]
+    uint32_t *umask = reinterpret_cast<uint32_t *>(smem + L.umask);  // [W]
+    int *woff = reinterpret_cast<int *>(smem + L.woff);              // [W]
+    int *rowidx = reinterpret_cast<int *>(smem + L.rowidx);          // [unit_cap]
+    float *xs = reinterpret_cast<float *>(smem + L.xs);              // [unit_cap][2][B]
+    float *part = reinterpret_cast<float *>(smem + L.part);          // [2][B][kCB]
     __shared__ int s_warp[kS1Threads / 32];
     __shared__ float s_red[kS1Threads / 32][4 * kMaxB];
     __shared__ float s_S[2 * kMaxB];
     __shared__ int s_E[kMaxB];
-    __shared__ int s_last;
     __shared__ int s_cnt[kS1Threads / 32][kMaxB + 1];
 
     // Programmatic dependent launch: x, y and the workspace may belong to the
@@ -244,7 +276,7 @@ __global__ void __launch_bounds__(kS1Threads, 2) k_stage1(const Stage1Args a) {
     const int n_units = hi - lo;
     __syncthreads();
 
-    // (4) this CTA's units: row index, then x_i * scale_i per matrix and token
+    // (4) this CTA's units (kept rows in its rank range)
     for (int wd = wid; wd < W; wd += kS1Threads / 32) {
         const uint32_t um = umask[wd];
         if (!((um >> lane) & 1u)) continue;
@@ -254,27 +286,27 @@ __global__ void __launch_bounds__(kS1Threads, 2) k_stage1(const Stage1Args a) {
     }
     __syncthreads();
 
-    // main-loop geometry; the first set of proxy rows is requested now so that
-    // its latency overlaps the scale gather below
+    // Each thread streams its rows u = rl, rl + RL, ... of one 16/8/4-byte
+    // column chunk of one proxy through a private ring of D shared-memory
+    // slots; the first D copies start now, so their latency overlaps the
+    // scale gather below.
     const int rl = tid / T::TPR;
     const int m = (tid / T::TPRM) & 1;
     const int chunk = tid % T::TPRM;
-    const uint8_t *qbase = (m ? a.q_gate : a.q_up) + (size_t)c * (kCB / 2) + chunk * T::BYTES;
-    const size_t rstride = (size_t)a.f / 2;
-    Vec<T::WORDS> va[T::U], vb[T::U];
-    auto load_set = [&](Vec<T::WORDS>(&v)[T::U], int u0) {
-#pragma unroll
-        for (int k = 0; k < T::U; ++k) {
-            const int u = u0 + k * T::RL;
-            if (u < n_units) {
-                ld_stream(v[k], qbase + (size_t)rowidx[u] * rstride);
-            } else {
-#pragma unroll
-                for (int q = 0; q < T::WORDS; ++q) v[k].w[q] = 0x88888888u;  // code 0
-            }
-        }
-    };
-    load_set(va, rl);
+    const uint8_t *qbase = (m ? a.q_gate : a.q_up) + (size_t)c * a.d * (kCB / 2) + chunk * T::BYTES;
+    unsigned char *myring = ring + (size_t)tid * 256;
+    const int n_rows = n_units > rl ? (n_units - rl + T::RL - 1) / T::RL : 0;
+#pragma unroll 1
+    for (int k = 0; k < T::D; ++k) {
+        if (k < n_rows)
+            cp_async<T::BYTES>(myring + k * T::BYTES,
+                               qbase + (size_t)rowidx[rl + k * T::RL] * (kCB / 2));
+        cp_commit();
+    }
+
+    // (5) x_i * scale_i per matrix and token for the units, then per token:
+    // S = sum of x_i * scale_i per matrix (offset removal) and the
+    // power-of-two pre-scale E from max |x_i * scale_i|
     {
         constexpr int G4 = 4;  // units per batch of loads
         for (int u0 = tid; u0 < n_units; u0 += G4 * kS1Threads) {
@@ -310,25 +342,22 @@ __global__ void __launch_bounds__(kS1Threads, 2) k_stage1(const Stage1Args a) {
         }
     }
     __syncthreads();
-
-    // (5) per token: S = sum of x_i * scale_i per matrix (offset removal) and
-    // the power-of-two pre-scale E from max |x_i * scale_i|
     {
-        float v[4 * B];
+        float v[3 * B];
 #pragma unroll
-        for (int k = 0; k < 4 * B; ++k) v[k] = 0.f;
+        for (int k = 0; k < 3 * B; ++k) v[k] = 0.f;
         for (int u = tid; u < n_units; u += kS1Threads) {
 #pragma unroll
-            for (int m = 0; m < 2; ++m)
+            for (int mm = 0; mm < 2; ++mm)
 #pragma unroll
                 for (int t = 0; t < B; ++t) {
-                    const float q = xs[(u * 2 + m) * B + t];
-                    v[m * B + t] += q;
+                    const float q = xs[(u * 2 + mm) * B + t];
+                    v[mm * B + t] += q;
                     v[2 * B + t] = fmaxf(v[2 * B + t], fabsf(q));
                 }
         }
 #pragma unroll
-        for (int k = 0; k < 4 * B; ++k) {
+        for (int k = 0; k < 3 * B; ++k) {
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
                 const float n = __shfl_xor_sync(0xffffffffu, v[k], o);
@@ -338,7 +367,7 @@ __global__ void __launch_bounds__(kS1Threads, 2) k_stage1(const Stage1Args a) {
         }
         __syncthreads();
         if (tid < 3 * B) {
-            float acc = (tid < 2 * B) ? 0.f : 0.f;
+            float acc = 0.f;
             for (int w = 0; w < kS1Threads / 32; ++w)
                 acc = (tid < 2 * B) ? acc + s_red[w][tid] : fmaxf(acc, s_red[w][tid]);
             if (tid < 2 * B) {
@@ -354,107 +383,117 @@ __global__ void __launch_bounds__(kS1Threads, 2) k_stage1(const Stage1Args a) {
         __syncthreads();
     }
 
-    // (6) main loop: stream the 128-byte block segments of the kept rows,
-    // two register sets in flight (load one while decoding the other)
+    // (6) main loop: consume the ring in order, refilling each slot with the
+    // row D positions later
     float acc[T::ACC];
 #pragma unroll
     for (int k = 0; k < T::ACC; ++k) acc[k] = 0.f;
-    auto comp_set = [&](const Vec<T::WORDS>(&v)[T::U], int u0) {
-#pragma unroll
-        for (int k = 0; k < T::U; ++k) {
-            const int u = u0 + k * T::RL;
-            float xv[B];
-#pragma unroll
-            for (int t = 0; t < B; ++t) xv[t] = (u < n_units) ? xs[(u * 2 + m) * B + t] : 0.f;
-#pragma unroll
-            for (int q = 0; q < T::WORDS; ++q) proc_word<B, T::CPT>(v[k].w[q], q, xv, acc);
+    for (int k = 0; k < n_rows; ++k) {
+        cp_wait<T::D - 1>();
+        const int u = rl + k * T::RL;
+        const int slot = k % T::D;
+        uint32_t w[T::WORDS];
+        if constexpr (T::WORDS == 4) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(myring + slot * 16);
+            w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+        } else if constexpr (T::WORDS == 2) {
+            const uint2 v = *reinterpret_cast<const uint2 *>(myring + slot * 8);
+            w[0] = v.x; w[1] = v.y;
+        } else {
+            w[0] = *reinterpret_cast<const uint32_t *>(myring + slot * 4);
         }
-    };
-    constexpr int STEP = T::RL * T::U;
-    for (int u0 = rl; u0 < n_units; u0 += 2 * STEP) {
-        load_set(vb, u0 + STEP);
-        comp_set(va, u0);
-        load_set(va, u0 + 2 * STEP);
-        comp_set(vb, u0 + STEP);
+        float xv[B];
+#pragma unroll
+        for (int t = 0; t < B; ++t) xv[t] = xs[(u * 2 + m) * B + t];
+#pragma unroll
+        for (int q = 0; q < T::WORDS; ++q) proc_word<B, T::CPT>(w[q], q, xv, acc);
+        // the slot's words have been consumed: refill it
+        const int kn = k + T::D;
+        if (kn < n_rows)
+            cp_async<T::BYTES>(myring + slot * T::BYTES,
+                               qbase + (size_t)rowidx[rl + kn * T::RL] * (kCB / 2));
+        cp_commit();
     }
+    cp_wait<0>();
+    __syncthreads();  // every thread is done with the ring before it becomes `red`
 
-    // (7) reduce row lanes, undo the pre-scale and the +8 code offset, write
-    // this CTA's partial sums
+    // (7) reduce row lanes (padded rows: conflict-free both ways), undo the
+    // pre-scale and the +8 code offset: this CTA's partial sums in `part`
+    constexpr int PAD = kCB + T::TPRM;  // one extra word per chunk row
 #pragma unroll
     for (int t = 0; t < B; ++t)
 #pragma unroll
         for (int k = 0; k < T::CPT; ++k)
-            red[((rl * 2 + m) * B + t) * kCB + chunk * T::CPT + k] = acc[t * T::CPT + k];
+            red[((rl * 2 + m) * B + t) * PAD + chunk * (T::CPT + 1) + k] = acc[t * T::CPT + k];
     __syncthreads();
     {
         const int ch = tid;  // channel within the block
         const int p = nib_pos(ch % 8);
-        float *part = a.partials + (((size_t)c * kS1MaxRowGroups + r) * 2) * B * kCB;
+        const int pos = (ch / T::CPT) * (T::CPT + 1) + ch % T::CPT;
 #pragma unroll
         for (int mm = 0; mm < 2; ++mm)
 #pragma unroll
             for (int t = 0; t < B; ++t) {
                 float s = 0.f;
-                for (int q = 0; q < T::RL; ++q) s += red[((q * 2 + mm) * B + t) * kCB + ch];
-                const float val = ldexpf(s, 149 - 4 * p - s_E[t]) - 8.f * s_S[mm * B + t];
-                part[(mm * B + t) * kCB + ch] = val;
+                for (int q = 0; q < T::RL; ++q) s += red[((q * 2 + mm) * B + t) * PAD + pos];
+                part[(mm * B + t) * kCB + ch] =
+                    ldexpf(s, 149 - 4 * p - s_E[t]) - 8.f * s_S[mm * B + t];
             }
     }
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) s_last = (atomicInc(&a.arrive[c], (unsigned)(a.n_r - 1)) == (unsigned)(a.n_r - 1));
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
+    cluster.sync();  // all partials of the block are in their CTAs' shared memory
 
-    // (8) last CTA of block c: s~ = u~ * SiLU(g~), m_s = 1[|s~| >= tau_s],
-    // ascending compaction per token and of the union
-    const int ch = tid;
-    const int j = c * kCB + ch;
-    uint32_t bits = 0;
+    if (r == 0) {
+        // (8) CTA 0 of the cluster: s~ = u~ * SiLU(g~), m_s = 1[|s~| >= tau_s],
+        // ascending compaction per token and of the union
+        const int ch = tid;
+        const int j = c * kCB + ch;
+        uint32_t bits = 0;
 #pragma unroll
-    for (int t = 0; t < B; ++t) {
-        if (t >= a.nb) break;
-        float u = 0.f, g = 0.f;
-        for (int q = 0; q < a.n_r; ++q) {
-            const float *part = a.partials + (((size_t)c * kS1MaxRowGroups + q) * 2) * B * kCB;
-            u += __ldcg(part + (0 * B + t) * kCB + ch);
-            g += __ldcg(part + (1 * B + t) * kCB + ch);
+        for (int t = 0; t < B; ++t) {
+            if (t >= a.nb) break;
+            float u = 0.f, g = 0.f;
+            for (int q = 0; q < a.n_r; ++q) {
+                const float *pq = cluster.map_shared_rank(part, q);
+                u += pq[(0 * B + t) * kCB + ch];
+                g += pq[(1 * B + t) * kCB + ch];
+            }
+            const float st = u * (g / (1.f + expf(-g)));
+            if (a.s_out) a.s_out[(size_t)t * a.f + j] = st;
+            const bool keep = fabsf(st) >= a.tau_s;
+            if (a.mask_s) a.mask_s[(size_t)t * a.f + j] = keep ? 1 : 0;
+            bits |= (keep ? 1u : 0u) << t;
         }
-        const float st = u * (g / (1.f + expf(-g)));
-        if (a.s_out) a.s_out[(size_t)t * a.f + j] = st;
-        const bool keep = fabsf(st) >= a.tau_s;
-        if (a.mask_s) a.mask_s[(size_t)t * a.f + j] = keep ? 1 : 0;
-        bits |= (keep ? 1u : 0u) << t;
-    }
-    if (!a.build_lists) return;
-    // warp ballots and per-warp counts (token t in column t, union in column B)
-    uint32_t bal[kMaxB + 1];
+        if (a.build_lists) {
+            // warp ballots and per-warp counts (token t in column t, union in column B)
+            uint32_t bal[kMaxB + 1];
 #pragma unroll
-    for (int t = 0; t <= B; ++t) {
-        const bool k = (t < B) ? ((bits >> t) & 1u) : (bits != 0u);
-        bal[t] = __ballot_sync(0xffffffffu, k);
-        if (lane == 0) s_cnt[wid][t] = __popc(bal[t]);
-    }
-    __syncthreads();
-    const uint32_t lt = (1u << lane) - 1u;
+            for (int t = 0; t <= B; ++t) {
+                const bool k = (t < B) ? ((bits >> t) & 1u) : (bits != 0u);
+                bal[t] = __ballot_sync(0xffffffffu, k);
+                if (lane == 0) s_cnt[wid][t] = __popc(bal[t]);
+            }
+            __syncthreads();
+            const uint32_t lt = (1u << lane) - 1u;
 #pragma unroll
-    for (int t = 0; t <= B; ++t) {
-        int base = 0, tot = 0;
-        for (int w = 0; w < kS1Threads / 32; ++w) {
-            if (w < wid) base += s_cnt[w][t];
-            tot += s_cnt[w][t];
-        }
-        const bool k = (bal[t] >> lane) & 1u;
-        const int pos = base + __popc(bal[t] & lt);
-        if (t < B) {
-            if (k) a.tlist[(size_t)t * a.f + c * kCB + pos] = j;
-            if (tid == 0) a.tcount[c * B + t] = (t < a.nb) ? tot : 0;
-        } else {
-            if (k) a.ulist[(size_t)c * kCB + pos] = (uint32_t)j | (bits << 24);
-            if (tid == 0) a.ucount[c] = tot;
+            for (int t = 0; t <= B; ++t) {
+                int base = 0, tot = 0;
+                for (int w = 0; w < kS1Threads / 32; ++w) {
+                    if (w < wid) base += s_cnt[w][t];
+                    tot += s_cnt[w][t];
+                }
+                const bool k = (bal[t] >> lane) & 1u;
+                const int pos = base + __popc(bal[t] & lt);
+                if (t < B) {
+                    if (k) a.tlist[(size_t)t * a.f + c * kCB + pos] = j;
+                    if (tid == 0) a.tcount[c * B + t] = (t < a.nb) ? tot : 0;
+                } else {
+                    if (k) a.ulist[(size_t)c * kCB + pos] = (uint32_t)j | (bits << 24);
+                    if (tid == 0) a.ucount[c] = tot;
+                }
+            }
         }
     }
+    cluster.sync();  // peers keep their shared memory until CTA 0 has read it
 }
 
 template <int B>
@@ -467,7 +506,21 @@ cudaError_t launch1(const Stage1Args &a, const Stage1Plan &p, cudaStream_t s) {
         if (e != cudaSuccess) return e;
         configured = p.smem;
     }
-    return launch_pdl(k, dim3(a.C * a.n_r), dim3(kS1Threads), p.smem, s, a);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.C * a.n_r);
+    cfg.blockDim = dim3(kS1Threads);
+    cfg.dynamicSmemBytes = p.smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = a.n_r;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, k, a);
 }
 
 }  // namespace
@@ -482,14 +535,8 @@ cudaError_t launch_stage1(int B, const Stage1Args &a, const Stage1Plan &p, cudaS
     }
 }
 
-// shared-memory bytes of one Stage-1 CTA for a plan (kept next to the kernel's
-// carve-up above)
 size_t stage1_smem_bytes(int d_model, int B, int unit_cap) {
-    const int tpr = 2 * (kCB / ((B == 1) ? 32 : (B <= 4 ? 16 : 8)));
-    const int rl = kS1Threads / tpr;
-    const int W = d_model / 32;
-    return (size_t)rl * 2 * B * kCB * 4 + (size_t)(B + 2) * W * 4 +
-           (size_t)unit_cap * (4 + 8 * B);
+    return s1_smem(d_model, B, unit_cap).total;
 }
 
 }  // namespace prox

@@ -42,13 +42,13 @@ int tokens_per_pass(int d_model, int batch) {
 Stage1Plan stage1_plan(int d, int f, int B, int num_sms) {
     Stage1Plan p;
     p.C = f / kCB;
-    const size_t red_and_masks = stage1_smem_bytes(d, B, 0);
+    const size_t fixed = stage1_smem_bytes(d, B, 0);
     const size_t per_unit = 4 + 8 * (size_t)B;
     // two CTAs per SM: keep each under ~110 KB of shared memory
     const size_t budget = 110 * 1024;
-    const size_t unit_budget = budget > red_and_masks ? budget - red_and_masks : per_unit;
-    int n_smem = (int)(((size_t)d * per_unit + unit_budget - 1) / unit_budget);
-    int n_bal = (2 * num_sms) / p.C;
+    const size_t unit_budget = budget > fixed + per_unit ? budget - fixed : per_unit;
+    const int n_smem = (int)(((size_t)d * per_unit + unit_budget - 1) / unit_budget);
+    const int n_bal = (2 * num_sms) / p.C;
     int n_r = n_bal > n_smem ? n_bal : n_smem;
     if (n_r < 1) n_r = 1;
     if (n_r > kS1MaxRowGroups) n_r = kS1MaxRowGroups;
@@ -79,8 +79,6 @@ WsLayout ws_layout(int d, int f, int B) {
     size_t o = 0;
     L.status = o;
     o += 256;
-    L.arrive = o;
-    o = align_up(o + C * 4, 256);
     L.ucount = o;
     o = align_up(o + C * 4, 256);
     L.tcount = o;
@@ -89,8 +87,6 @@ WsLayout ws_layout(int d, int f, int B) {
     o = align_up(o + C * kCB * 4, 256);
     L.tlist = o;
     o = align_up(o + (size_t)B * f * 4, 256);
-    L.partials = o;
-    o = align_up(o + C * kS1MaxRowGroups * 2 * B * kCB * 4, 256);
     L.total = o;
     return L;
 }
@@ -183,8 +179,6 @@ static prox_status pass_stage1(const prox_layer *L, const uint16_t *x, int nb, f
     a.mask_s = mask_s;
     a.s_out = s_out;
     a.build_lists = lists ? 1 : 0;
-    a.partials = reinterpret_cast<float *>(w + W.partials);
-    a.arrive = reinterpret_cast<uint32_t *>(w + W.arrive);
     a.ucount = reinterpret_cast<int32_t *>(w + W.ucount);
     a.tcount = reinterpret_cast<int32_t *>(w + W.tcount);
     a.ulist = reinterpret_cast<uint32_t *>(w + W.ulist);

@@ -16,9 +16,8 @@ namespace prox {
 // ---------------------------------------------------------------------------
 constexpr int kCB = 256;            // channels per Stage-1 column block
 constexpr int kS1Threads = 256;     // Stage-1 CTA size
-constexpr int kS1MaxRowGroups = 16; // upper bound of row groups per block
+constexpr int kS1MaxRowGroups = 8;  // row groups per block = cluster size (portable <= 8)
 constexpr int kMaxB = 8;            // tokens per pass (per-token masks)
-constexpr int kS1UnitBudget = 96 * 1024;    // smem bytes for Stage-1 unit lists
 constexpr int kS2SmemBudget = 224 * 1024;   // opt-in dynamic smem per CTA
 
 // status word bits (first word of the workspace)
@@ -55,7 +54,7 @@ Stage2Plan stage2_plan(int d_model, int B, int C, int max_ch);
 
 // Workspace layout of one forward pass (B tokens). Offsets in bytes.
 struct WsLayout {
-    size_t status, arrive, ucount, tcount, ulist, tlist, partials, total;
+    size_t status, ucount, tcount, ulist, tlist, total;
 };
 WsLayout ws_layout(int d_model, int d_ff, int B);
 
@@ -75,8 +74,6 @@ struct Stage1Args {
     float *s_out;                // [nb][f] or null
     int build_lists;             // write ulist/tlist/counts for Stage 2
     // workspace
-    float *partials;             // [C][kS1MaxRowGroups][2][B][kCB]
-    uint32_t *arrive;            // [C]
     int32_t *ucount;             // [C]
     int32_t *tcount;             // [C][B]
     uint32_t *ulist;             // [C][kCB]  channel | token bits << 24

@@ -127,7 +127,7 @@ class ProxLayer:
     w_up_cm: torch.Tensor      # bf16 [d_ff][d_model]
     w_gate_cm: torch.Tensor    # bf16 [d_ff][d_model]
     w_down: torch.Tensor       # bf16 [d_ff][d_model]
-    q_up: torch.Tensor         # uint8 [d_model][d_ff/2]
+    q_up: torch.Tensor         # uint8 [d_ff/256][d_model][128] (block-tiled)
     q_gate: torch.Tensor
     s_up: torch.Tensor         # fp32 [d_model]
     s_gate: torch.Tensor
@@ -143,8 +143,9 @@ class ProxLayer:
     def cstruct(self) -> _Layer:
         d, f = self.d_model, self.d_ff
         for name, dt, shp in (("w_up_cm", torch.bfloat16, (f, d)), ("w_gate_cm", torch.bfloat16, (f, d)),
-                              ("w_down", torch.bfloat16, (f, d)), ("q_up", torch.uint8, (d, f // 2)),
-                              ("q_gate", torch.uint8, (d, f // 2)), ("s_up", torch.float32, (d,)),
+                              ("w_down", torch.bfloat16, (f, d)),
+                              ("q_up", torch.uint8, (f // 256, d, 128)),
+                              ("q_gate", torch.uint8, (f // 256, d, 128)), ("s_up", torch.float32, (d,)),
                               ("s_gate", torch.float32, (d,))):
             _need(getattr(self, name), dt, shp, name)
         return _Layer(d, f, _ptr(self.w_up_cm), _ptr(self.w_gate_cm), _ptr(self.w_down),
@@ -161,10 +162,10 @@ class ProxLayer:
 
 def quantize_proxy(w_cm: torch.Tensor):
     """INT4 proxy of a channel-major bf16 weight [d_ff][d_model] ->
-    (q uint8 [d_model][d_ff/2], scale fp32 [d_model])."""
+    (q uint8 [d_ff/256][d_model][128] block-tiled, scale fp32 [d_model])."""
     f, d = w_cm.shape
     _need(w_cm, torch.bfloat16, (f, d), "w_cm")
-    q = torch.empty((d, f // 2), dtype=torch.uint8, device=w_cm.device)
+    q = torch.empty((f // 256, d, 128), dtype=torch.uint8, device=w_cm.device)
     s = torch.empty((d,), dtype=torch.float32, device=w_cm.device)
     _check(lib().prox_quantize_proxy(d, f, _ptr(w_cm), _ptr(q), _ptr(s), _stream(w_cm.device)),
            "prox_quantize_proxy")
@@ -305,6 +306,15 @@ def test_set_wait(wait_us: int = 0, skip_position: int = -1) -> None:
     lib().prox_test_set_wait(int(wait_us), int(skip_position))
 
 
+def untile_proxy(q):
+    """Block-tiled proxy [d_ff/256][d_model][128] -> row-major [d_model][d_ff/2]
+    (the same bytes reordered; numpy arrays or tensors)."""
+    C, d, _ = q.shape
+    if isinstance(q, torch.Tensor):
+        return q.permute(1, 0, 2).reshape(d, C * 128)
+    return q.transpose(1, 0, 2).reshape(d, C * 128)
+
+
 def touched_bytes(d_model: int, d_ff: int, k_x: int, k_s: int) -> int:
     """Weight bytes one token's forward reads: the kept rows of both INT4
     proxies with their scales, and three bf16 rows per kept channel."""
@@ -314,4 +324,4 @@ def touched_bytes(d_model: int, d_ff: int, k_x: int, k_s: int) -> int:
 __all__ = ["ProxLayer", "ProxError", "quantize_proxy", "workspace", "workspace_bytes",
            "ffn_forward", "ffn_forward_raw", "ffn_stage1_raw", "ffn_stage2_raw",
            "max_batch_per_pass", "proxy_state", "calibrate", "allocate",
-           "last_device_status", "touched_bytes", "as_bf16"]
+           "last_device_status", "touched_bytes", "untile_proxy", "as_bf16"]

@@ -57,8 +57,8 @@ typedef enum prox_status {
  *                        (the pages' W_up[:, j]; nn.Linear weight layout).
  *   w_down             : bf16 [d_ff][d_model]; row j is W_down[j, :] (the
  *                        pages' orientation d_ff x d_model).
- *   q_up, q_gate       : INT4 proxies, uint8 [d_model][d_ff/2] as written by
- *                        prox_quantize_proxy.
+ *   q_up, q_gate       : INT4 proxies, uint8 [d_ff/256][d_model][128] (block-
+ *                        tiled) as written by prox_quantize_proxy.
  *   s_up, s_gate       : fp32 [d_model] per-row proxy scales.
  * Every pointer must be 16-byte aligned.
  */
@@ -84,9 +84,12 @@ typedef struct prox_layer {
  *   scale_i = max_j |W[i,j]| / 7                        (fp32, round to nearest)
  *   q_ij    = clamp(round_half_even(W[i,j] / scale_i), -7, 7)  (fp32 division)
  *   an all-zero row gives scale 0 and q 0.
- * Output layout: q_out[i][m] (device, uint8 [d_model][d_ff/2]) holds channel 2m
- * in its low nibble and 2m+1 in its high nibble, two's complement;
- * scale_out (device, fp32 [d_model]).
+ * Output layout (block-tiled, the order the input-sparse proxy product
+ * streams): q_out is uint8 [d_ff/256][d_model][128]; the 128-byte granule
+ * q_out[c][i] holds the codes of row i for channels 256c .. 256c+255, byte m
+ * holding channel 256c+2m in its low nibble and 256c+2m+1 in its high
+ * nibble, two's complement. A rejected input coordinate i thus skips one
+ * contiguous granule per block. scale_out is fp32 [d_model].
  *   w_cm : device, bf16 [d_ff][d_model] (channel-major, as in prox_layer).
  * Errors: PROX_EINVAL on a null pointer or bad shape.
  */

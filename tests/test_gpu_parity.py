@@ -104,7 +104,7 @@ def check_forward(case, rows, out, tag=""):
 def test_quantize_bit_exact_c1(c1):
     for w, qk, sk in ((c1.layer.w_up_cm, "q_up", "s_up"), (c1.layer.w_gate_cm, "q_gate", "s_gate")):
         q, s = P.quantize_proxy(w)
-        assert np.array_equal(q.cpu().numpy(), c1.Por[qk])
+        assert np.array_equal(P.untile_proxy(q.cpu().numpy()), c1.Por[qk])
         assert np.array_equal(s.cpu().numpy().view(np.uint32), c1.Por[sk].view(np.uint32))
 
 
@@ -123,15 +123,15 @@ def test_quantize_hand_worked_rows(gpu):
     q, s = q.cpu().numpy(), s.cpu().numpy()
     for i, (_, sbits, packed) in enumerate(rows):
         assert int(s[i:i + 1].view(np.uint32)[0]) == sbits
-        assert bytes(q[i, :4]) == packed
-    assert not s[len(rows):].any() and not q[len(rows):].any()
+        assert bytes(q[0, i, :4]) == packed       # granule (block 0, row i)
+    assert not s[len(rows):].any() and not q[:, len(rows):].any()
 
 
 def test_quantize_bit_exact_c2(c2):
     q, s = P.quantize_proxy(c2.layer.w_up_cm)
-    assert np.array_equal(q.cpu().numpy(), c2.Por["q_up"])
+    assert np.array_equal(P.untile_proxy(q.cpu().numpy()), c2.Por["q_up"])
     assert np.array_equal(s.cpu().numpy().view(np.uint32), c2.Por["s_up"].view(np.uint32))
-    assert np.array_equal(c2.layer.q_gate.cpu().numpy(), c2.Por["q_gate"])
+    assert np.array_equal(P.untile_proxy(c2.layer.q_gate.cpu().numpy()), c2.Por["q_gate"])
 
 
 # ---------------------------------------------------------------------------
