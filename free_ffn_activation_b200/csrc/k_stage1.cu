@@ -294,12 +294,15 @@ __global__ void __launch_bounds__(kS1Threads, 2) k_stage1(const Stage1Args a) {
     const int m = (tid / T::TPRM) & 1;
     const int chunk = tid % T::TPRM;
     const uint8_t *qbase = (m ? a.q_gate : a.q_up) + (size_t)c * a.d * (kCB / 2) + chunk * T::BYTES;
-    unsigned char *myring = ring + (size_t)tid * 256;
+    // slot-major ring (ring[slot][thread]): a warp's accesses to one slot are
+    // consecutive words, free of bank conflicts
+    unsigned char *myring = ring + (size_t)tid * T::BYTES;
+    constexpr int SLOT = kS1Threads * T::BYTES;  // bytes between a thread's slots
     const int n_rows = n_units > rl ? (n_units - rl + T::RL - 1) / T::RL : 0;
 #pragma unroll 1
     for (int k = 0; k < T::D; ++k) {
         if (k < n_rows)
-            cp_async<T::BYTES>(myring + k * T::BYTES,
+            cp_async<T::BYTES>(myring + k * SLOT,
                                qbase + (size_t)rowidx[rl + k * T::RL] * (kCB / 2));
         cp_commit();
     }
@@ -394,13 +397,13 @@ __global__ void __launch_bounds__(kS1Threads, 2) k_stage1(const Stage1Args a) {
         const int slot = k % T::D;
         uint32_t w[T::WORDS];
         if constexpr (T::WORDS == 4) {
-            const uint4 v = *reinterpret_cast<const uint4 *>(myring + slot * 16);
+            const uint4 v = *reinterpret_cast<const uint4 *>(myring + slot * SLOT);
             w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
         } else if constexpr (T::WORDS == 2) {
-            const uint2 v = *reinterpret_cast<const uint2 *>(myring + slot * 8);
+            const uint2 v = *reinterpret_cast<const uint2 *>(myring + slot * SLOT);
             w[0] = v.x; w[1] = v.y;
         } else {
-            w[0] = *reinterpret_cast<const uint32_t *>(myring + slot * 4);
+            w[0] = *reinterpret_cast<const uint32_t *>(myring + slot * SLOT);
         }
         float xv[B];
 #pragma unroll
@@ -410,7 +413,7 @@ __global__ void __launch_bounds__(kS1Threads, 2) k_stage1(const Stage1Args a) {
         // the slot's words have been consumed: refill it
         const int kn = k + T::D;
         if (kn < n_rows)
-            cp_async<T::BYTES>(myring + slot * T::BYTES,
+            cp_async<T::BYTES>(myring + slot * SLOT,
                                qbase + (size_t)rowidx[rl + kn * T::RL] * (kCB / 2));
         cp_commit();
     }
