@@ -49,7 +49,8 @@ struct S1 {
     static constexpr int TPRM = kCB / CPT;                           // threads per row per matrix
     static constexpr int TPR = 2 * TPRM;                             // threads per row
     static constexpr int RL = kS1Threads / TPR;                      // row lanes
-    static constexpr int D = 256 / BYTES;                            // ring depth (rows)
+    static constexpr int RING = (B == 1) ? 256 : 128;                // ring bytes per thread
+    static constexpr int D = RING / BYTES;                           // ring depth (rows)
 };
 
 // nibble position (in units of 4 bits) of local channel k of a word after
@@ -60,28 +61,23 @@ __device__ __forceinline__ float nib_f(uint32_t w, int p) {
     return __uint_as_float((w & (0xFu << (4 * p))) ^ (0x8u << (4 * p)));
 }
 
-// acc[t * CPT + wi * 8 + k] += xs[t] * code_k * 2^(4 pos(k) - 149)
+// acc2 holds channel pairs: channel t * CPT + wi * 8 + k is component k % 2 of
+// acc2[(t * CPT + wi * 8 + k) / 2]; it gains xs[t] * code_k * 2^(4 pos(k) - 149)
 template <int B, int CPT>
-__device__ __forceinline__ void proc_word(uint32_t w, int wi, const float *xs, float *acc) {
+__device__ __forceinline__ void proc_word(uint32_t w, int wi, const float *xs, float2 *acc2) {
     const uint32_t v = w >> 12;
-    float2 d01 = make_float2(nib_f(w, 0), nib_f(w, 1));
-    float2 d23 = make_float2(nib_f(w, 2), nib_f(w, 3));
-    float2 d45 = make_float2(nib_f(w, 4), nib_f(v, 2));
-    float2 d67 = make_float2(nib_f(v, 3), nib_f(v, 4));
+    const float2 d01 = make_float2(nib_f(w, 0), nib_f(w, 1));
+    const float2 d23 = make_float2(nib_f(w, 2), nib_f(w, 3));
+    const float2 d45 = make_float2(nib_f(w, 4), nib_f(v, 2));
+    const float2 d67 = make_float2(nib_f(v, 3), nib_f(v, 4));
 #pragma unroll
     for (int t = 0; t < B; ++t) {
         const float2 xx = make_float2(xs[t], xs[t]);
-        float *a = acc + t * CPT + wi * 8;
-        float2 a01 = make_float2(a[0], a[1]);
-        float2 a23 = make_float2(a[2], a[3]);
-        float2 a45 = make_float2(a[4], a[5]);
-        float2 a67 = make_float2(a[6], a[7]);
-        a01 = __ffma2_rn(xx, d01, a01);
-        a23 = __ffma2_rn(xx, d23, a23);
-        a45 = __ffma2_rn(xx, d45, a45);
-        a67 = __ffma2_rn(xx, d67, a67);
-        a[0] = a01.x; a[1] = a01.y; a[2] = a23.x; a[3] = a23.y;
-        a[4] = a45.x; a[5] = a45.y; a[6] = a67.x; a[7] = a67.y;
+        float2 *a = acc2 + (t * CPT + wi * 8) / 2;
+        a[0] = __ffma2_rn(xx, d01, a[0]);
+        a[1] = __ffma2_rn(xx, d23, a[1]);
+        a[2] = __ffma2_rn(xx, d45, a[2]);
+        a[3] = __ffma2_rn(xx, d67, a[3]);
     }
 }
 
@@ -135,7 +131,7 @@ struct S1Smem {
 __host__ __device__ inline S1Smem s1_smem(int d, int B, int unit_cap) {
     const int cpt = (B == 1) ? 32 : (B <= 4 ? 16 : 8);
     const int rl = kS1Threads / (2 * (kCB / cpt));
-    const size_t ring = (size_t)kS1Threads * 256;                   // cp.async ring
+    const size_t ring = (size_t)kS1Threads * (B == 1 ? 256 : 128);  // cp.async ring
     const size_t red = (size_t)rl * 2 * B * (kCB + kCB / cpt) * 4;  // padded row-lane sums
     const int W = d / 32;
     S1Smem s;
@@ -161,7 +157,7 @@ __host__ __device__ inline S1Smem s1_smem(int d, int B, int unit_cap) {
 namespace {
 
 template <int B>
-__global__ void __launch_bounds__(kS1Threads, 2) k_stage1(const Stage1Args a) {
+__global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
     using T = S1<B>;
     extern __shared__ __align__(16) unsigned char smem[];
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
@@ -202,8 +198,8 @@ __global__ void __launch_bounds__(kS1Threads, 2) k_stage1(const Stage1Args a) {
     // 16-byte chunks of 8 coordinates; all its loads are issued before any
     // use. Chunk ci's 8 keep bits are byte ci of the token's mask words.
     {
-        // chunks per thread per token: d_model <= 8192, and <= 4096 when B = 8
-        constexpr int MAXK = (B == 8) ? 2 : 4;
+        // chunks per thread per token (d_model <= 8192)
+        constexpr int MAXK = (8192 / 8 + kS1Threads - 1) / kS1Threads;
         const int NC = a.d / 8;
         uint4 xv[MAXK][B];
 #pragma unroll
@@ -388,9 +384,9 @@ __global__ void __launch_bounds__(kS1Threads, 2) k_stage1(const Stage1Args a) {
 
     // (6) main loop: consume the ring in order, refilling each slot with the
     // row D positions later
-    float acc[T::ACC];
+    float2 acc2[T::ACC / 2];
 #pragma unroll
-    for (int k = 0; k < T::ACC; ++k) acc[k] = 0.f;
+    for (int k = 0; k < T::ACC / 2; ++k) acc2[k] = make_float2(0.f, 0.f);
     for (int k = 0; k < n_rows; ++k) {
         cp_wait<T::D - 1>();
         const int u = rl + k * T::RL;
@@ -409,7 +405,7 @@ __global__ void __launch_bounds__(kS1Threads, 2) k_stage1(const Stage1Args a) {
 #pragma unroll
         for (int t = 0; t < B; ++t) xv[t] = xs[(u * 2 + m) * B + t];
 #pragma unroll
-        for (int q = 0; q < T::WORDS; ++q) proc_word<B, T::CPT>(w[q], q, xv, acc);
+        for (int q = 0; q < T::WORDS; ++q) proc_word<B, T::CPT>(w[q], q, xv, acc2);
         // the slot's words have been consumed: refill it
         const int kn = k + T::D;
         if (kn < n_rows)
@@ -426,34 +422,35 @@ __global__ void __launch_bounds__(kS1Threads, 2) k_stage1(const Stage1Args a) {
 #pragma unroll
     for (int t = 0; t < B; ++t)
 #pragma unroll
-        for (int k = 0; k < T::CPT; ++k)
-            red[((rl * 2 + m) * B + t) * PAD + chunk * (T::CPT + 1) + k] = acc[t * T::CPT + k];
+        for (int k = 0; k < T::CPT; k += 2) {
+            float *dst = red + ((rl * 2 + m) * B + t) * PAD + chunk * (T::CPT + 1) + k;
+            dst[0] = acc2[(t * T::CPT + k) / 2].x;
+            dst[1] = acc2[(t * T::CPT + k) / 2].y;
+        }
     __syncthreads();
     {
-        const int ch = tid;  // channel within the block
+        // thread -> (matrix, channel within the block)
+        const int mm = tid / kCB, ch = tid % kCB;
         const int p = nib_pos(ch % 8);
         const int pos = (ch / T::CPT) * (T::CPT + 1) + ch % T::CPT;
 #pragma unroll
-        for (int mm = 0; mm < 2; ++mm)
-#pragma unroll
-            for (int t = 0; t < B; ++t) {
-                float s = 0.f;
-                for (int q = 0; q < T::RL; ++q) s += red[((q * 2 + mm) * B + t) * PAD + pos];
-                part[(mm * B + t) * kCB + ch] =
-                    ldexpf(s, 149 - 4 * p - s_E[t]) - 8.f * s_S[mm * B + t];
-            }
+        for (int t = 0; t < B; ++t) {
+            float s = 0.f;
+            for (int q = 0; q < T::RL; ++q) s += red[((q * 2 + mm) * B + t) * PAD + pos];
+            part[(mm * B + t) * kCB + ch] = ldexpf(s, 149 - 4 * p - s_E[t]) - 8.f * s_S[mm * B + t];
+        }
     }
     cluster.sync();  // all partials of the block are in their CTAs' shared memory
 
     if (r == 0) {
         // (8) CTA 0 of the cluster: s~ = u~ * SiLU(g~), m_s = 1[|s~| >= tau_s],
-        // ascending compaction per token and of the union
+        // ascending compaction per token and of the union (thread = channel)
         const int ch = tid;
         const int j = c * kCB + ch;
         uint32_t bits = 0;
 #pragma unroll
         for (int t = 0; t < B; ++t) {
-            if (t >= a.nb) break;
+            if (t >= a.nb || ch >= kCB) break;
             float u = 0.f, g = 0.f;
             for (int q = 0; q < a.n_r; ++q) {
                 const float *pq = cluster.map_shared_rank(part, q);
@@ -500,15 +497,60 @@ __global__ void __launch_bounds__(kS1Threads, 2) k_stage1(const Stage1Args a) {
 }
 
 template <int B>
-cudaError_t launch1(const Stage1Args &a, const Stage1Plan &p, cudaStream_t s) {
+cudaError_t launch1(Stage1Args a, const Stage1Plan &p0, cudaStream_t s) {
     auto k = k_stage1<B>;
-    static size_t configured = 0;  // dynamic smem limit already set for this kernel
-    if (p.smem > configured) {
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)p.smem);
-        if (e != cudaSuccess) return e;
-        configured = p.smem;
+    // Cluster size (row groups per block): every cluster of the grid must be
+    // resident at once, or the last clusters run as a second wave. Start from
+    // the plan's choice and shrink until the occupancy calculator agrees.
+    struct Cache {
+        int d = 0, C = 0, n_r = 0, cap = 0;
+        size_t smem = 0;
+    };
+    static Cache cache;
+    Stage1Plan p = p0;
+    if (cache.d == a.d && cache.C == a.C) {
+        p.n_r = cache.n_r;
+        p.unit_cap = cache.cap;
+        p.smem = cache.smem;
+    } else {
+        // fewest row groups whose rows fit in one CTA's shared memory
+        int n_min = 1;
+        while (n_min < kS1MaxRowGroups &&
+               s1_smem(a.d, B, (a.d + n_min - 1) / n_min).total > (size_t)kS2SmemBudget)
+            ++n_min;
+        if (p.n_r < n_min) p.n_r = n_min;
+        for (;;) {
+            p.unit_cap = (a.d + p.n_r - 1) / p.n_r;
+            p.smem = s1_smem(a.d, B, p.unit_cap).total;
+            cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)p.smem);
+            if (e != cudaSuccess) return e;
+            if (p.n_r <= n_min) break;
+            cudaLaunchConfig_t q = {};
+            q.gridDim = dim3(a.C * p.n_r);
+            q.blockDim = dim3(kS1Threads);
+            q.dynamicSmemBytes = p.smem;
+            cudaLaunchAttribute at[1];
+            at[0].id = cudaLaunchAttributeClusterDimension;
+            at[0].val.clusterDim.x = p.n_r;
+            at[0].val.clusterDim.y = 1;
+            at[0].val.clusterDim.z = 1;
+            q.attrs = at;
+            q.numAttrs = 1;
+            int active = 0;
+            e = cudaOccupancyMaxActiveClusters(&active, k, &q);
+            if (e != cudaSuccess) return e;
+            if (active >= a.C) break;
+            --p.n_r;
+        }
+        cache.d = a.d;
+        cache.C = a.C;
+        cache.n_r = p.n_r;
+        cache.cap = p.unit_cap;
+        cache.smem = p.smem;
     }
+    a.n_r = p.n_r;
+    a.unit_cap = p.unit_cap;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(a.C * a.n_r);
     cfg.blockDim = dim3(kS1Threads);

@@ -39,19 +39,19 @@ int tokens_per_pass(int d_model, int batch) {
     return pow2_ceil(b);
 }
 
+// Starting point of the Stage-1 launch plan: one CTA per SM, the row groups
+// of a column block form one thread-block cluster (<= 8, portable); the
+// launch shrinks the cluster if not every cluster could be resident at once.
 Stage1Plan stage1_plan(int d, int f, int B, int num_sms) {
     Stage1Plan p;
     p.C = f / kCB;
-    const size_t fixed = stage1_smem_bytes(d, B, 0);
-    const size_t per_unit = 4 + 8 * (size_t)B;
-    // two CTAs per SM: keep each under ~110 KB of shared memory
-    const size_t budget = 110 * 1024;
-    const size_t unit_budget = budget > fixed + per_unit ? budget - fixed : per_unit;
-    const int n_smem = (int)(((size_t)d * per_unit + unit_budget - 1) / unit_budget);
-    const int n_bal = (2 * num_sms) / p.C;
-    int n_r = n_bal > n_smem ? n_bal : n_smem;
+    int n_r = num_sms / p.C;
     if (n_r < 1) n_r = 1;
     if (n_r > kS1MaxRowGroups) n_r = kS1MaxRowGroups;
+    // enough row groups that one CTA's rows fit in shared memory
+    while (n_r < kS1MaxRowGroups &&
+           stage1_smem_bytes(d, B, (d + n_r - 1) / n_r) > (size_t)kS2SmemBudget)
+        ++n_r;
     p.n_r = n_r;
     p.unit_cap = (d + n_r - 1) / n_r;
     p.smem = stage1_smem_bytes(d, B, p.unit_cap);

@@ -15,7 +15,7 @@ namespace prox {
 // Fixed tiling constants
 // ---------------------------------------------------------------------------
 constexpr int kCB = 256;            // channels per Stage-1 column block
-constexpr int kS1Threads = 256;     // Stage-1 CTA size
+constexpr int kS1Threads = 512;     // Stage-1 CTA size (one CTA per SM)
 constexpr int kS1MaxRowGroups = 8;  // row groups per block = cluster size (portable <= 8)
 constexpr int kMaxB = 8;            // tokens per pass (per-token masks)
 constexpr int kS2SmemBudget = 224 * 1024;   // opt-in dynamic smem per CTA
@@ -164,14 +164,16 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                  : "memory");
 }
 
+// try_wait with a suspend-time hint: a waiting thread sleeps until the phase
+// completes (or about 0.5 ms pass) instead of spinning on the issue slots
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_addr(bar)), "r"(parity)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(500000u)
         : "memory");
     return ok != 0;
 }
