@@ -40,13 +40,15 @@ namespace cg = cooperative_groups;
 namespace prox {
 namespace {
 
-template <int B>
+template <int B, int NB>
 struct S1 {
+    static constexpr int CW = NB * kCB;                              // channels per CTA
     static constexpr int CPT = (B == 1) ? 32 : (B <= 4 ? 16 : 8);  // channels per thread
     static constexpr int BYTES = CPT / 2;                            // bytes per row per thread
     static constexpr int WORDS = BYTES / 4;
     static constexpr int ACC = B * CPT;
-    static constexpr int TPRM = kCB / CPT;                           // threads per row per matrix
+    static constexpr int TPRB = kCB / CPT;                           // threads per block per matrix
+    static constexpr int TPRM = CW / CPT;                            // threads per row per matrix
     static constexpr int TPR = 2 * TPRM;                             // threads per row
     static constexpr int RL = kS1Threads / TPR;                      // row lanes
     static constexpr int RING = (B == 1) ? 256 : 128;                // ring bytes per thread
@@ -128,11 +130,12 @@ struct S1Smem {
     size_t ring, tmask, umask, woff, rowidx, xs, part, total;
 };
 
-__host__ __device__ inline S1Smem s1_smem(int d, int B, int unit_cap) {
+__host__ __device__ inline S1Smem s1_smem(int d, int B, int NB, int unit_cap) {
+    const int cw = NB * kCB;
     const int cpt = (B == 1) ? 32 : (B <= 4 ? 16 : 8);
-    const int rl = kS1Threads / (2 * (kCB / cpt));
+    const int rl = kS1Threads / (2 * (cw / cpt));
     const size_t ring = (size_t)kS1Threads * (B == 1 ? 256 : 128);  // cp.async ring
-    const size_t red = (size_t)rl * 2 * B * (kCB + kCB / cpt) * 4;  // padded row-lane sums
+    const size_t red = (size_t)rl * 2 * B * (cw + cw / cpt) * 4;    // padded row-lane sums
     const int W = d / 32;
     S1Smem s;
     size_t o = 0;
@@ -149,23 +152,23 @@ __host__ __device__ inline S1Smem s1_smem(int d, int B, int unit_cap) {
     s.xs = o;
     o += (size_t)unit_cap * 2 * B * 4;
     s.part = o;
-    o += (size_t)2 * B * kCB * 4;
+    o += (size_t)2 * B * cw * 4;
     s.total = o;
     return s;
 }
 
 namespace {
 
-template <int B>
+template <int B, int NB>
 __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
-    using T = S1<B>;
+    using T = S1<B, NB>;
     extern __shared__ __align__(16) unsigned char smem[];
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     cg::cluster_group cluster = cg::this_cluster();
     const int r = (int)cluster.block_rank();  // row group
-    const int c = blockIdx.x / a.n_r;          // column block
+    const int c0 = (blockIdx.x / a.n_r) * NB;  // first column block of the group
     const int W = a.d / 32;                    // mask words per token
-    const S1Smem L = s1_smem(a.d, B, a.unit_cap);
+    const S1Smem L = s1_smem(a.d, B, NB, a.unit_cap);
     unsigned char *ring = smem + L.ring;
     float *red = reinterpret_cast<float *>(smem + L.ring);  // after streaming
     uint32_t *tmask = reinterpret_cast<uint32_t *>(smem + L.tmask);  // [B][W]
@@ -173,7 +176,7 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
     int *woff = reinterpret_cast<int *>(smem + L.woff);              // [W]
     int *rowidx = reinterpret_cast<int *>(smem + L.rowidx);          // [unit_cap]
     float *xs = reinterpret_cast<float *>(smem + L.xs);              // [unit_cap][2][B]
-    float *part = reinterpret_cast<float *>(smem + L.part);          // [2][B][kCB]
+    float *part = reinterpret_cast<float *>(smem + L.part);          // [2][B][CW]
     __shared__ int s_warp[kS1Threads / 32];
     __shared__ float s_red[kS1Threads / 32][4 * kMaxB];
     __shared__ float s_S[2 * kMaxB];
@@ -289,7 +292,9 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
     const int rl = tid / T::TPR;
     const int m = (tid / T::TPRM) & 1;
     const int chunk = tid % T::TPRM;
-    const uint8_t *qbase = (m ? a.q_gate : a.q_up) + (size_t)c * a.d * (kCB / 2) + chunk * T::BYTES;
+    const uint8_t *qbase = (m ? a.q_gate : a.q_up) +
+                           (size_t)(c0 + chunk / T::TPRB) * a.d * (kCB / 2) +
+                           (chunk % T::TPRB) * T::BYTES;
     // slot-major ring (ring[slot][thread]): a warp's accesses to one slot are
     // consecutive words, free of bank conflicts
     unsigned char *myring = ring + (size_t)tid * T::BYTES;
@@ -418,7 +423,7 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
 
     // (7) reduce row lanes (padded rows: conflict-free both ways), undo the
     // pre-scale and the +8 code offset: this CTA's partial sums in `part`
-    constexpr int PAD = kCB + T::TPRM;  // one extra word per chunk row
+    constexpr int PAD = T::CW + T::TPRM;  // one extra word per chunk row
 #pragma unroll
     for (int t = 0; t < B; ++t)
 #pragma unroll
@@ -428,16 +433,17 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
             dst[1] = acc2[(t * T::CPT + k) / 2].y;
         }
     __syncthreads();
-    {
-        // thread -> (matrix, channel within the block)
-        const int mm = tid / kCB, ch = tid % kCB;
+    for (int o = tid; o < 2 * T::CW; o += kS1Threads) {
+        // (matrix, channel within the CTA's columns)
+        const int mm = o / T::CW, ch = o % T::CW;
         const int p = nib_pos(ch % 8);
         const int pos = (ch / T::CPT) * (T::CPT + 1) + ch % T::CPT;
 #pragma unroll
         for (int t = 0; t < B; ++t) {
             float s = 0.f;
             for (int q = 0; q < T::RL; ++q) s += red[((q * 2 + mm) * B + t) * PAD + pos];
-            part[(mm * B + t) * kCB + ch] = ldexpf(s, 149 - 4 * p - s_E[t]) - 8.f * s_S[mm * B + t];
+            part[(mm * B + t) * T::CW + ch] =
+                ldexpf(s, 149 - 4 * p - s_E[t]) - 8.f * s_S[mm * B + t];
         }
     }
     cluster.sync();  // all partials of the block are in their CTAs' shared memory
@@ -445,17 +451,18 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
     if (r == 0) {
         // (8) CTA 0 of the cluster: s~ = u~ * SiLU(g~), m_s = 1[|s~| >= tau_s],
         // ascending compaction per token and of the union (thread = channel)
-        const int ch = tid;
-        const int j = c * kCB + ch;
+        const int ch = tid;                  // channel within the CTA's columns
+        const int j = c0 * kCB + ch;         // channel index
+        const int blk = wid / (kCB / 32);    // block of this warp's channels
         uint32_t bits = 0;
 #pragma unroll
         for (int t = 0; t < B; ++t) {
-            if (t >= a.nb || ch >= kCB) break;
+            if (t >= a.nb || ch >= T::CW) break;
             float u = 0.f, g = 0.f;
             for (int q = 0; q < a.n_r; ++q) {
                 const float *pq = cluster.map_shared_rank(part, q);
-                u += pq[(0 * B + t) * kCB + ch];
-                g += pq[(1 * B + t) * kCB + ch];
+                u += pq[(0 * B + t) * T::CW + ch];
+                g += pq[(1 * B + t) * T::CW + ch];
             }
             const float st = u * (g / (1.f + expf(-g)));
             if (a.s_out) a.s_out[(size_t)t * a.f + j] = st;
@@ -474,21 +481,26 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
             }
             __syncthreads();
             const uint32_t lt = (1u << lane) - 1u;
+            constexpr int WPB = kCB / 32;  // warps per 256-channel block
+            if (blk < NB) {
+                const int cb = c0 + blk;
 #pragma unroll
-            for (int t = 0; t <= B; ++t) {
-                int base = 0, tot = 0;
-                for (int w = 0; w < kS1Threads / 32; ++w) {
-                    if (w < wid) base += s_cnt[w][t];
-                    tot += s_cnt[w][t];
-                }
-                const bool k = (bal[t] >> lane) & 1u;
-                const int pos = base + __popc(bal[t] & lt);
-                if (t < B) {
-                    if (k) a.tlist[(size_t)t * a.f + c * kCB + pos] = j;
-                    if (tid == 0) a.tcount[c * B + t] = (t < a.nb) ? tot : 0;
-                } else {
-                    if (k) a.ulist[(size_t)c * kCB + pos] = (uint32_t)j | (bits << 24);
-                    if (tid == 0) a.ucount[c] = tot;
+                for (int t = 0; t <= B; ++t) {
+                    int base = 0, tot = 0;
+                    for (int w = blk * WPB; w < (blk + 1) * WPB; ++w) {
+                        if (w < wid) base += s_cnt[w][t];
+                        tot += s_cnt[w][t];
+                    }
+                    const bool k = (bal[t] >> lane) & 1u;
+                    const int pos = base + __popc(bal[t] & lt);
+                    const bool first = (wid == blk * WPB) && lane == 0;
+                    if (t < B) {
+                        if (k) a.tlist[(size_t)t * a.f + cb * kCB + pos] = j;
+                        if (first) a.tcount[cb * B + t] = (t < a.nb) ? tot : 0;
+                    } else {
+                        if (k) a.ulist[(size_t)cb * kCB + pos] = (uint32_t)j | (bits << 24);
+                        if (first) a.ucount[cb] = tot;
+                    }
                 }
             }
         }
@@ -496,9 +508,10 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
     cluster.sync();  // peers keep their shared memory until CTA 0 has read it
 }
 
-template <int B>
+template <int B, int NB>
 cudaError_t launch1(Stage1Args a, const Stage1Plan &p0, cudaStream_t s) {
-    auto k = k_stage1<B>;
+    auto k = k_stage1<B, NB>;
+    const int groups = a.C / NB;  // clusters
     // Cluster size (row groups per block): every cluster of the grid must be
     // resident at once, or the last clusters run as a second wave. Start from
     // the plan's choice and shrink until the occupancy calculator agrees.
@@ -516,18 +529,18 @@ cudaError_t launch1(Stage1Args a, const Stage1Plan &p0, cudaStream_t s) {
         // fewest row groups whose rows fit in one CTA's shared memory
         int n_min = 1;
         while (n_min < kS1MaxRowGroups &&
-               s1_smem(a.d, B, (a.d + n_min - 1) / n_min).total > (size_t)kS2SmemBudget)
+               s1_smem(a.d, B, NB, (a.d + n_min - 1) / n_min).total > (size_t)kS2SmemBudget)
             ++n_min;
         if (p.n_r < n_min) p.n_r = n_min;
         for (;;) {
             p.unit_cap = (a.d + p.n_r - 1) / p.n_r;
-            p.smem = s1_smem(a.d, B, p.unit_cap).total;
+            p.smem = s1_smem(a.d, B, NB, p.unit_cap).total;
             cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  (int)p.smem);
             if (e != cudaSuccess) return e;
             if (p.n_r <= n_min) break;
             cudaLaunchConfig_t q = {};
-            q.gridDim = dim3(a.C * p.n_r);
+            q.gridDim = dim3(groups * p.n_r);
             q.blockDim = dim3(kS1Threads);
             q.dynamicSmemBytes = p.smem;
             cudaLaunchAttribute at[1];
@@ -540,7 +553,7 @@ cudaError_t launch1(Stage1Args a, const Stage1Plan &p0, cudaStream_t s) {
             int active = 0;
             e = cudaOccupancyMaxActiveClusters(&active, k, &q);
             if (e != cudaSuccess) return e;
-            if (active >= a.C) break;
+            if (active >= groups) break;
             --p.n_r;
         }
         cache.d = a.d;
@@ -552,7 +565,7 @@ cudaError_t launch1(Stage1Args a, const Stage1Plan &p0, cudaStream_t s) {
     a.n_r = p.n_r;
     a.unit_cap = p.unit_cap;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(a.C * a.n_r);
+    cfg.gridDim = dim3(groups * a.n_r);
     cfg.blockDim = dim3(kS1Threads);
     cfg.dynamicSmemBytes = p.smem;
     cfg.stream = s;
@@ -571,17 +584,16 @@ cudaError_t launch1(Stage1Args a, const Stage1Plan &p0, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_stage1(int B, const Stage1Args &a, const Stage1Plan &p, cudaStream_t s) {
-    switch (B) {
-        case 1: return launch1<1>(a, p, s);
-        case 2: return launch1<2>(a, p, s);
-        case 4: return launch1<4>(a, p, s);
-        case 8: return launch1<8>(a, p, s);
-        default: return cudaErrorInvalidValue;
-    }
+#define PROX_S1(BB, NN) \
+    if (B == BB && p.nb_blocks == NN) return launch1<BB, NN>(a, p, s);
+    PROX_S1(1, 1) PROX_S1(1, 2) PROX_S1(2, 1) PROX_S1(2, 2)
+    PROX_S1(4, 1) PROX_S1(4, 2) PROX_S1(8, 1) PROX_S1(8, 2)
+#undef PROX_S1
+    return cudaErrorInvalidValue;
 }
 
-size_t stage1_smem_bytes(int d_model, int B, int unit_cap) {
-    return s1_smem(d_model, B, unit_cap).total;
+size_t stage1_smem_bytes(int d_model, int B, int NB, int unit_cap) {
+    return s1_smem(d_model, B, NB, unit_cap).total;
 }
 
 }  // namespace prox

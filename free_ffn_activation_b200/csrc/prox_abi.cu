@@ -15,7 +15,7 @@
 
 namespace prox {
 
-size_t stage1_smem_bytes(int d_model, int B, int unit_cap);
+size_t stage1_smem_bytes(int d_model, int B, int NB, int unit_cap);
 size_t stage2_smem_bytes(int d_model, int B, int nstage, int C, int max_ch);
 int stage2_nchd(int d_model, int B);
 
@@ -39,22 +39,33 @@ int tokens_per_pass(int d_model, int batch) {
     return pow2_ceil(b);
 }
 
-// Starting point of the Stage-1 launch plan: one CTA per SM, the row groups
-// of a column block form one thread-block cluster (<= 8, portable); the
+// Starting point of the Stage-1 launch plan: one CTA per SM; a CTA covers one
+// or two adjacent column blocks (whichever fills more SMs), and the row
+// groups of its columns form one thread-block cluster (<= 8, portable). The
 // launch shrinks the cluster if not every cluster could be resident at once.
 Stage1Plan stage1_plan(int d, int f, int B, int num_sms) {
     Stage1Plan p;
     p.C = f / kCB;
-    int n_r = num_sms / p.C;
-    if (n_r < 1) n_r = 1;
-    if (n_r > kS1MaxRowGroups) n_r = kS1MaxRowGroups;
+    int best = -1;
+    for (int nb = 1; nb <= 2; ++nb) {
+        if (p.C % nb) continue;
+        const int groups = p.C / nb;
+        int n_r = num_sms / groups;
+        if (n_r < 1) n_r = 1;
+        if (n_r > kS1MaxRowGroups) n_r = kS1MaxRowGroups;
+        const int ctas = groups * n_r;
+        if (ctas > best) {
+            best = ctas;
+            p.nb_blocks = nb;
+            p.n_r = n_r;
+        }
+    }
     // enough row groups that one CTA's rows fit in shared memory
-    while (n_r < kS1MaxRowGroups &&
-           stage1_smem_bytes(d, B, (d + n_r - 1) / n_r) > (size_t)kS2SmemBudget)
-        ++n_r;
-    p.n_r = n_r;
-    p.unit_cap = (d + n_r - 1) / n_r;
-    p.smem = stage1_smem_bytes(d, B, p.unit_cap);
+    while (p.n_r < kS1MaxRowGroups &&
+           stage1_smem_bytes(d, B, p.nb_blocks, (d + p.n_r - 1) / p.n_r) > (size_t)kS2SmemBudget)
+        ++p.n_r;
+    p.unit_cap = (d + p.n_r - 1) / p.n_r;
+    p.smem = stage1_smem_bytes(d, B, p.nb_blocks, p.unit_cap);
     return p;
 }
 

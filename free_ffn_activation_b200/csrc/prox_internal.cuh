@@ -34,7 +34,8 @@ constexpr uint32_t kDefaultWaitUs = 2000000u;
 // ---------------------------------------------------------------------------
 struct Stage1Plan {
     int C;          // column blocks = d_ff / kCB
-    int n_r;        // row groups per block; grid = C * n_r
+    int nb_blocks;  // column blocks per CTA (1 or 2)
+    int n_r;        // row groups = cluster size; grid = C / nb_blocks * n_r
     int unit_cap;   // max units (kept rows) one CTA may own
     size_t smem;    // dynamic shared memory bytes
 };
