@@ -20,10 +20,9 @@
 // channels into ascending lists, so the result is deterministic.
 //
 // INT4 decode. A nibble n at bits 4p..4p+3 of a word, with every other bit
-// cleared, is the bit pattern of the subnormal float n * 2^(4p-149). XOR-ing
-// the nibble's top bit turns the stored two's complement code q into
-// n = q + 8 in the same single LOP3, so one logic op per weight yields an
-// exact float operand; the FMA multiplies it by x_i * scale_i pre-scaled by
+// cleared, is the bit pattern of the subnormal float n * 2^(4p-149). One XOR
+// of the whole word with 0x88888888 turns every stored two's complement code q
+// into n = q + 8, then one AND per weight yields an exact float operand; the FMA multiplies it by x_i * scale_i pre-scaled by
 // 2^E (E chosen per CTA so sums stay normal). At the end each channel's sum
 // is rescaled by the exact power of two 2^(149 - 4p - E) and the offset
 // 8 * sum(x_i * scale_i) is removed. Nibbles 5..7 of a word are first shifted
@@ -59,14 +58,16 @@ struct S1 {
 // the decode above
 __host__ __device__ constexpr int nib_pos(int k) { return k < 5 ? k : k - 3; }
 
-__device__ __forceinline__ float nib_f(uint32_t w, int p) {
-    return __uint_as_float((w & (0xFu << (4 * p))) ^ (0x8u << (4 * p)));
+// nibble p of a word already XOR-ed with 0x88888888, as a subnormal float
+__device__ __forceinline__ float nib_f(uint32_t wx, int p) {
+    return __uint_as_float(wx & (0xFu << (4 * p)));
 }
 
 // acc2 holds channel pairs: channel t * CPT + wi * 8 + k is component k % 2 of
 // acc2[(t * CPT + wi * 8 + k) / 2]; it gains xs[t] * code_k * 2^(4 pos(k) - 149)
 template <int B, int CPT>
-__device__ __forceinline__ void proc_word(uint32_t w, int wi, const float *xs, float2 *acc2) {
+__device__ __forceinline__ void proc_word(uint32_t w0, int wi, const float *xs, float2 *acc2) {
+    const uint32_t w = w0 ^ 0x88888888u;  // every two's complement code q -> q + 8
     const uint32_t v = w >> 12;
     const float2 d01 = make_float2(nib_f(w, 0), nib_f(w, 1));
     const float2 d23 = make_float2(nib_f(w, 2), nib_f(w, 3));
@@ -127,7 +128,7 @@ __device__ __forceinline__ int block_excl_scan(int v, int *warp_tot, int &total)
 
 // shared-memory carve-up of one Stage-1 CTA (kept next to the kernel)
 struct S1Smem {
-    size_t ring, tmask, umask, woff, rowidx, xs, part, total;
+    size_t ring, tmask, rowidx, xs, part, total;
 };
 
 __host__ __device__ inline S1Smem s1_smem(int d, int B, int NB, int unit_cap) {
@@ -143,10 +144,6 @@ __host__ __device__ inline S1Smem s1_smem(int d, int B, int NB, int unit_cap) {
     o += ring > red ? ring : red;
     s.tmask = o;
     o += (size_t)B * W * 4;
-    s.umask = o;
-    o += (size_t)W * 4;
-    s.woff = o;
-    o += (size_t)W * 4;
     s.rowidx = o;
     o += (size_t)unit_cap * 4;
     s.xs = o;
@@ -172,14 +169,11 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
     unsigned char *ring = smem + L.ring;
     float *red = reinterpret_cast<float *>(smem + L.ring);  // after streaming
     uint32_t *tmask = reinterpret_cast<uint32_t *>(smem + L.tmask);  // [B][W]
-    uint32_t *umask = reinterpret_cast<uint32_t *>(smem + L.umask);  // [W]
-    int *woff = reinterpret_cast<int *>(smem + L.woff);              // [W]
     int *rowidx = reinterpret_cast<int *>(smem + L.rowidx);          // [unit_cap]
     float *xs = reinterpret_cast<float *>(smem + L.xs);              // [unit_cap][2][B]
     float *part = reinterpret_cast<float *>(smem + L.part);          // [2][B][CW]
     __shared__ int s_warp[kS1Threads / 32];
     __shared__ float s_red[kS1Threads / 32][4 * kMaxB];
-    __shared__ float s_S[2 * kMaxB];
     __shared__ int s_E[kMaxB];
     __shared__ int s_cnt[kS1Threads / 32][kMaxB + 1];
 
@@ -199,7 +193,9 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
 
     // (2) input masks m_x = 1[|x_i| >= tau_x] per token: each thread owns
     // 16-byte chunks of 8 coordinates; all its loads are issued before any
-    // use. Chunk ci's 8 keep bits are byte ci of the token's mask words.
+    // use. Chunk ci's 8 keep bits are byte ci of the token's mask words. The
+    // same pass finds max |x| per token, which fixes the power-of-two
+    // pre-scale 2^E (see the decode note above).
     {
         // chunks per thread per token (d_model <= 8192)
         constexpr int MAXK = (8192 / 8 + kS1Threads - 1) / kS1Threads;
@@ -215,6 +211,9 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
                     xv[k][t] = *reinterpret_cast<const uint4 *>(a.x + (size_t)t * a.d + ci * 8);
             }
         uint8_t *tbytes = reinterpret_cast<uint8_t *>(tmask);
+        float xmax[B];
+#pragma unroll
+        for (int t = 0; t < B; ++t) xmax[t] = 0.f;
 #pragma unroll
         for (int k = 0; k < MAXK; ++k) {
             const int ci = tid + k * kS1Threads;
@@ -225,8 +224,10 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
                 uint32_t bits = 0;
 #pragma unroll
                 for (int h = 0; h < 4; ++h) {
-                    bits |= (fabsf(bf16lo(w4[h])) >= a.tau_x ? 1u : 0u) << (2 * h);
-                    bits |= (fabsf(bf16hi(w4[h])) >= a.tau_x ? 1u : 0u) << (2 * h + 1);
+                    const float lo = fabsf(bf16lo(w4[h])), hi = fabsf(bf16hi(w4[h]));
+                    bits |= (lo >= a.tau_x ? 1u : 0u) << (2 * h);
+                    bits |= (hi >= a.tau_x ? 1u : 0u) << (2 * h + 1);
+                    xmax[t] = fmaxf(xmax[t], fmaxf(lo, hi));
                 }
                 if (t >= a.nb) bits = 0;
                 tbytes[t * NC + ci] = (uint8_t)bits;
@@ -242,46 +243,40 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
                 }
             }
         }
-    }
-    __syncthreads();
-    for (int wd = tid; wd < W; wd += kS1Threads) {
-        uint32_t un = 0;
 #pragma unroll
-        for (int t = 0; t < B; ++t) un |= tmask[t * W + wd];
-        umask[wd] = un;
+        for (int t = 0; t < B; ++t) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+                xmax[t] = fmaxf(xmax[t], __shfl_xor_sync(0xffffffffu, xmax[t], o));
+            if (lane == 0) s_red[wid][t] = xmax[t];
+        }
     }
     __syncthreads();
 
-    // (3) ranks of the kept (union) rows
-    int kx;
-    {
-        const int per = (W + kS1Threads - 1) / kS1Threads;
-        int loc = 0;
-        for (int k = 0; k < per; ++k) {
-            const int wd = tid * per + k;
-            if (wd < W) loc += __popc(umask[wd]);
-        }
-        int base = block_excl_scan(loc, s_warp, kx);
-        for (int k = 0; k < per; ++k) {
-            const int wd = tid * per + k;
-            if (wd < W) {
-                woff[wd] = base;
-                base += __popc(umask[wd]);
-            }
-        }
+    // (3) one thread per mask word: union mask, its population, ranks of the
+    // kept rows (one block-wide scan) and this CTA's share of them
+    if (tid < B) {
+        float mx = 0.f;
+        for (int w = 0; w < kS1Threads / 32; ++w) mx = fmaxf(mx, s_red[w][tid]);
+        // |x * 2^E| < 2^96: a row sum of (q + 8) * x_i * scale_i * 2^E over
+        // <= 8192 rows stays finite for scales below 2^15 and, for scales
+        // above 2^-70, partial sums of the subnormal-coded products stay normal
+        s_E[tid] = (mx > 0.f) ? 95 - ilogbf(mx) : 0;
     }
+    uint32_t um = 0;
+    if (tid < W) {
+#pragma unroll
+        for (int t = 0; t < B; ++t) um |= tmask[t * W + tid];
+    }
+    int kx;
+    const int woffs = block_excl_scan(__popc(um), s_warp, kx);  // syncs the CTA
     const int lo = (int)((long long)kx * r / a.n_r);
     const int hi = (int)((long long)kx * (r + 1) / a.n_r);
     const int n_units = hi - lo;
-    __syncthreads();
-
-    // (4) this CTA's units (kept rows in its rank range)
-    for (int wd = wid; wd < W; wd += kS1Threads / 32) {
-        const uint32_t um = umask[wd];
-        if (!((um >> lane) & 1u)) continue;
-        const int rank = woff[wd] + __popc(um & ((1u << lane) - 1u));
-        if (rank < lo || rank >= hi) continue;
-        rowidx[rank - lo] = wd * 32 + lane;
+    if (woffs < hi && woffs + __popc(um) > lo) {
+        int rank = woffs;
+        for (uint32_t b = um; b; b &= b - 1, ++rank)
+            if (rank >= lo && rank < hi) rowidx[rank - lo] = tid * 32 + (__ffs(b) - 1);
     }
     __syncthreads();
 
@@ -308,11 +303,17 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
         cp_commit();
     }
 
-    // (5) x_i * scale_i per matrix and token for the units, then per token:
-    // S = sum of x_i * scale_i per matrix (offset removal) and the
-    // power-of-two pre-scale E from max |x_i * scale_i|
+    // (4) x_i * scale_i * 2^E per matrix and token for the units (exact
+    // power-of-two scaling, split in two factors so each is a normal float)
     {
-        constexpr int G4 = 4;  // units per batch of loads
+        float pe1[B], pe2[B];
+#pragma unroll
+        for (int t = 0; t < B; ++t) {
+            const int e1 = s_E[t] / 2, e2 = s_E[t] - e1;
+            pe1[t] = __int_as_float((127 + e1) << 23);
+            pe2[t] = __int_as_float((127 + e2) << 23);
+        }
+        constexpr int G4 = 2;  // units per thread per batch of loads
         for (int u0 = tid; u0 < n_units; u0 += G4 * kS1Threads) {
             float su[G4], sg[G4];
             uint16_t xh[G4][B];
@@ -339,59 +340,23 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
                     float xv = 0.f;
                     if ((tmask[t * W + (i >> 5)] >> (i & 31)) & 1u)
                         xv = __uint_as_float((uint32_t)xh[k][t] << 16);
-                    xs[(u * 2 + 0) * B + t] = xv * su[k];
-                    xs[(u * 2 + 1) * B + t] = xv * sg[k];
+                    xs[(u * 2 + 0) * B + t] = (xv * su[k]) * pe1[t] * pe2[t];
+                    xs[(u * 2 + 1) * B + t] = (xv * sg[k]) * pe1[t] * pe2[t];
                 }
             }
         }
     }
     __syncthreads();
-    {
-        float v[3 * B];
-#pragma unroll
-        for (int k = 0; k < 3 * B; ++k) v[k] = 0.f;
-        for (int u = tid; u < n_units; u += kS1Threads) {
-#pragma unroll
-            for (int mm = 0; mm < 2; ++mm)
-#pragma unroll
-                for (int t = 0; t < B; ++t) {
-                    const float q = xs[(u * 2 + mm) * B + t];
-                    v[mm * B + t] += q;
-                    v[2 * B + t] = fmaxf(v[2 * B + t], fabsf(q));
-                }
-        }
-#pragma unroll
-        for (int k = 0; k < 3 * B; ++k) {
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const float n = __shfl_xor_sync(0xffffffffu, v[k], o);
-                v[k] = (k < 2 * B) ? v[k] + n : fmaxf(v[k], n);
-            }
-            if (lane == 0) s_red[wid][k] = v[k];
-        }
-        __syncthreads();
-        if (tid < 3 * B) {
-            float acc = 0.f;
-            for (int w = 0; w < kS1Threads / 32; ++w)
-                acc = (tid < 2 * B) ? acc + s_red[w][tid] : fmaxf(acc, s_red[w][tid]);
-            if (tid < 2 * B) {
-                s_S[tid] = acc;
-            } else {
-                const int t = tid - 2 * B;
-                s_E[t] = (acc > 0.f) ? 119 - ilogbf(acc) : 0;
-            }
-        }
-        __syncthreads();
-        for (int k = tid; k < n_units * 2 * B; k += kS1Threads)
-            xs[k] = ldexpf(xs[k], s_E[k % B]);
-        __syncthreads();
-    }
 
-    // (6) main loop: consume the ring in order, refilling each slot with the
-    // row D positions later
+    // (5) main loop: consume the ring in order, refilling each slot with the
+    // row D positions later; ssum collects this thread's sum of x_i * scale_i
+    // * 2^E for the +8 code offset
     float2 acc2[T::ACC / 2];
 #pragma unroll
     for (int k = 0; k < T::ACC / 2; ++k) acc2[k] = make_float2(0.f, 0.f);
+    float ssum[B];
+#pragma unroll
+    for (int t = 0; t < B; ++t) ssum[t] = 0.f;
     for (int k = 0; k < n_rows; ++k) {
         cp_wait<T::D - 1>();
         const int u = rl + k * T::RL;
@@ -408,7 +373,10 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
         }
         float xv[B];
 #pragma unroll
-        for (int t = 0; t < B; ++t) xv[t] = xs[(u * 2 + m) * B + t];
+        for (int t = 0; t < B; ++t) {
+            xv[t] = xs[(u * 2 + m) * B + t];
+            ssum[t] += xv[t];
+        }
 #pragma unroll
         for (int q = 0; q < T::WORDS; ++q) proc_word<B, T::CPT>(w[q], q, xv, acc2);
         // the slot's words have been consumed: refill it
@@ -421,50 +389,70 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
     cp_wait<0>();
     __syncthreads();  // every thread is done with the ring before it becomes `red`
 
-    // (7) reduce row lanes (padded rows: conflict-free both ways), undo the
-    // pre-scale and the +8 code offset: this CTA's partial sums in `part`
+    // (6) reduce row lanes (padded rows: conflict-free both ways), undo the
+    // pre-scale and the +8 code offset: this CTA's partial sums in `part`.
+    // The pad word after chunk 0's channels carries the row lane's offset sum.
     constexpr int PAD = T::CW + T::TPRM;  // one extra word per chunk row
 #pragma unroll
-    for (int t = 0; t < B; ++t)
+    for (int t = 0; t < B; ++t) {
+        float *row = red + ((rl * 2 + m) * B + t) * PAD;
 #pragma unroll
         for (int k = 0; k < T::CPT; k += 2) {
-            float *dst = red + ((rl * 2 + m) * B + t) * PAD + chunk * (T::CPT + 1) + k;
-            dst[0] = acc2[(t * T::CPT + k) / 2].x;
-            dst[1] = acc2[(t * T::CPT + k) / 2].y;
+            row[chunk * (T::CPT + 1) + k] = acc2[(t * T::CPT + k) / 2].x;
+            row[chunk * (T::CPT + 1) + k + 1] = acc2[(t * T::CPT + k) / 2].y;
         }
+        if (chunk == 0) row[T::CPT] = ssum[t];
+    }
     __syncthreads();
     for (int o = tid; o < 2 * T::CW; o += kS1Threads) {
         // (matrix, channel within the CTA's columns)
         const int mm = o / T::CW, ch = o % T::CW;
         const int p = nib_pos(ch % 8);
         const int pos = (ch / T::CPT) * (T::CPT + 1) + ch % T::CPT;
+        // 2^(149 - 4p) and 2^-E as products of normal floats
+        const float up1 = __int_as_float((127 + 75) << 23);
+        const float up2 = __int_as_float((127 + 74 - 4 * p) << 23);
 #pragma unroll
         for (int t = 0; t < B; ++t) {
-            float s = 0.f;
-            for (int q = 0; q < T::RL; ++q) s += red[((q * 2 + mm) * B + t) * PAD + pos];
+            float sacc = 0.f, soff = 0.f;
+            for (int q = 0; q < T::RL; ++q) {
+                const float *row = red + ((q * 2 + mm) * B + t) * PAD;
+                sacc += row[pos];
+                soff += row[T::CPT];
+            }
+            const int e1 = s_E[t] / 2, e2 = s_E[t] - e1;
+            const float v = (sacc * up1) * up2 - 8.f * soff;  // sum (q + 8 - 8) x s 2^E
             part[(mm * B + t) * T::CW + ch] =
-                ldexpf(s, 149 - 4 * p - s_E[t]) - 8.f * s_S[mm * B + t];
+                v * __int_as_float((127 - e1) << 23) * __int_as_float((127 - e2) << 23);
         }
     }
     cluster.sync();  // all partials of the block are in their CTAs' shared memory
 
     if (r == 0) {
-        // (8) CTA 0 of the cluster: s~ = u~ * SiLU(g~), m_s = 1[|s~| >= tau_s],
-        // ascending compaction per token and of the union (thread = channel)
+        // (7) CTA 0 of the cluster: gather the cluster's partials (in rank
+        // order), release the peers, then s~ = u~ * SiLU(g~),
+        // m_s = 1[|s~| >= tau_s] and the ascending compaction per token and of
+        // the union (thread = channel)
         const int ch = tid;                  // channel within the CTA's columns
         const int j = c0 * kCB + ch;         // channel index
         const int blk = wid / (kCB / 32);    // block of this warp's channels
+        float uu[B], gg[B];
+#pragma unroll
+        for (int t = 0; t < B; ++t) {
+            uu[t] = gg[t] = 0.f;
+            if (t >= a.nb || ch >= T::CW) continue;
+            for (int q = 0; q < a.n_r; ++q) {
+                const float *pq = cluster.map_shared_rank(part, q);
+                uu[t] += pq[(0 * B + t) * T::CW + ch];
+                gg[t] += pq[(1 * B + t) * T::CW + ch];
+            }
+        }
+        asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
         uint32_t bits = 0;
 #pragma unroll
         for (int t = 0; t < B; ++t) {
             if (t >= a.nb || ch >= T::CW) break;
-            float u = 0.f, g = 0.f;
-            for (int q = 0; q < a.n_r; ++q) {
-                const float *pq = cluster.map_shared_rank(part, q);
-                u += pq[(0 * B + t) * T::CW + ch];
-                g += pq[(1 * B + t) * T::CW + ch];
-            }
-            const float st = u * (g / (1.f + expf(-g)));
+            const float st = uu[t] * (gg[t] / (1.f + expf(-gg[t])));
             if (a.s_out) a.s_out[(size_t)t * a.f + j] = st;
             const bool keep = fabsf(st) >= a.tau_s;
             if (a.mask_s) a.mask_s[(size_t)t * a.f + j] = keep ? 1 : 0;
@@ -504,8 +492,12 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
                 }
             }
         }
+        asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+    } else {
+        // peers keep their shared memory until CTA 0 has gathered it
+        asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+        asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
     }
-    cluster.sync();  // peers keep their shared memory until CTA 0 has read it
 }
 
 template <int B, int NB>

@@ -36,8 +36,10 @@ __host__ __device__ constexpr int s2_threads(int B) { return (kNDot + s2_ndown(B
 __host__ __device__ constexpr int s2_xbytes(int B) { return B <= 2 ? 4 : 2; }
 
 // shared-memory carve-up, shared by the kernel and the host plan
+constexpr int kS2Prefetch = 4;  // channel-list blocks fetched with the counts
+
 struct S2Smem {
-    size_t stages, xs, full, empty, sready, meta, svals, uscan, tscan, chan, total;
+    size_t stages, xs, full, empty, sready, meta, svals, uscan, tscan, chan, chanpf, total;
 };
 
 __host__ __device__ inline S2Smem s2_smem(int d, int B, int nstage, int C, int max_ch) {
@@ -65,6 +67,8 @@ __host__ __device__ inline S2Smem s2_smem(int d, int B, int nstage, int C, int m
     o += (size_t)B * (C + 1) * 4;
     s.chan = o;
     o += (size_t)max_ch * 4;
+    s.chanpf = o;
+    o += (size_t)kS2Prefetch * kCB * 4;
     s.total = (o + 127) & ~(size_t)127;
     return s;
 }
@@ -100,6 +104,7 @@ __global__ void __launch_bounds__(s2_threads(B), 1) k_stage2(const Stage2Args a)
     int *uscan = reinterpret_cast<int *>(smem + L.uscan);      // [C+1]
     int *tscan = reinterpret_cast<int *>(smem + L.tscan);      // [B][C+1]
     uint32_t *chan = reinterpret_cast<uint32_t *>(smem + L.chan);  // [max_ch]
+    uint32_t *chanpf = reinterpret_cast<uint32_t *>(smem + L.chanpf);  // [kS2Prefetch][kCB]
     const int nch16 = d / 8;  // 16-byte chunks per row
 
     if (tid == 0) {
@@ -130,14 +135,44 @@ __global__ void __launch_bounds__(s2_threads(B), 1) k_stage2(const Stage2Args a)
             *reinterpret_cast<uint4 *>(xh + (size_t)t * d + ci * 8) = v;
         }
     }
-    // Stage 1's lists are ready once it has completed
+    // Stage 1's lists are ready once it has completed. One round trip brings
+    // the per-block counts and the list blocks this CTA most likely owns
+    // (those around block g * C / G).
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    for (int k = tid; k < C * (B + 1); k += s2_threads(B)) {
-        if (k < C) {
-            uscan[k] = a.ucount[k];
-        } else {
-            const int c = (k - C) / B, t = (k - C) % B;
-            tscan[t * (C + 1) + c] = a.tcount[c * B + t];
+    const int G = gridDim.x, g = blockIdx.x;
+    const int npf = C < kS2Prefetch ? C : kS2Prefetch;
+    int cpf = (int)((long long)g * C / G) - 1;
+    cpf = cpf < 0 ? 0 : (cpf > C - npf ? C - npf : cpf);
+    {
+        const int ncnt = C * (B + 1), total = ncnt + npf * kCB;
+        constexpr int NT = s2_threads(B);
+        for (int base = tid; base < total; base += 4 * NT) {
+            uint32_t v[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int k = base + q * NT;
+                v[q] = 0;
+                if (k < C) {
+                    v[q] = (uint32_t)a.ucount[k];
+                } else if (k < ncnt) {
+                    const int c = (k - C) / B, t = (k - C) % B;
+                    v[q] = (uint32_t)a.tcount[c * B + t];
+                } else if (k < total) {
+                    v[q] = a.ulist[(size_t)cpf * kCB + (k - ncnt)];
+                }
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int k = base + q * NT;
+                if (k < C) {
+                    uscan[k] = (int)v[q];
+                } else if (k < ncnt) {
+                    const int c = (k - C) / B, t = (k - C) % B;
+                    tscan[t * (C + 1) + c] = (int)v[q];
+                } else if (k < total) {
+                    chanpf[k - ncnt] = v[q];
+                }
+            }
         }
     }
     __syncthreads();
@@ -164,7 +199,6 @@ __global__ void __launch_bounds__(s2_threads(B), 1) k_stage2(const Stage2Args a)
     __syncthreads();
 
     const long long U = uscan[C];
-    const int G = gridDim.x, g = blockIdx.x;
     const int p0 = (int)(U * g / G), p1 = (int)(U * (g + 1) / G);
     const int n_ch = p1 - p0;
 
@@ -176,7 +210,9 @@ __global__ void __launch_bounds__(s2_threads(B), 1) k_stage2(const Stage2Args a)
             const int mid = (lo + hi + 1) >> 1;
             if (uscan[mid] <= p) lo = mid; else hi = mid - 1;
         }
-        chan[n] = a.ulist[(size_t)lo * kCB + (p - uscan[lo])];
+        const int off = p - uscan[lo];
+        chan[n] = (lo >= cpf && lo < cpf + npf) ? chanpf[(lo - cpf) * kCB + off]
+                                                : a.ulist[(size_t)lo * kCB + off];
     }
     __syncthreads();
     asm volatile("griddepcontrol.launch_dependents;");

@@ -54,7 +54,7 @@ Stage1Plan stage1_plan(int d, int f, int B, int num_sms) {
         if (n_r < 1) n_r = 1;
         if (n_r > kS1MaxRowGroups) n_r = kS1MaxRowGroups;
         const int ctas = groups * n_r;
-        if (ctas > best) {
+        if (ctas >= best) {  // on a tie, fewer and larger clusters
             best = ctas;
             p.nb_blocks = nb;
             p.n_r = n_r;
