@@ -12,9 +12,11 @@
 // cluster of n_r CTAs; CTA r of the cluster takes the r-th contiguous range
 // of the kept rows (ranks over the union of the pass's tokens) and streams
 // the granules of BOTH proxies (one read of x serves up and gate, the fused
-// split-N kernel of the blog's "From formula to GPU" section). Each thread
-// keeps a private ring of asynchronous copies (cp.async) several rows deep,
-// so about 64 KB per CTA is in flight without any barrier. The cluster's
+// split-N kernel of the blog's "From formula to GPU" section). Every warp
+// owns whole 128-byte granules of its rows and keeps a private ring of them
+// in shared memory, filled by 1-D bulk copies (TMA) and guarded by one
+// mbarrier per slot, so about 128 KB per CTA is in flight with no cross-warp
+// synchronisation. The cluster's
 // partial sums meet in distributed shared memory: CTA 0 adds them in rank
 // order, forms s~ = u~ * SiLU(g~), thresholds it and compacts the kept
 // channels into ascending lists, so the result is deterministic.
@@ -42,7 +44,8 @@ namespace {
 template <int B, int NB>
 struct S1 {
     static constexpr int CW = NB * kCB;                              // channels per CTA
-    static constexpr int CPT = (B == 1) ? 32 : (B <= 4 ? 16 : 8);  // channels per thread
+    // channels per thread; every warp covers whole rows of one row lane
+    static constexpr int CPT = (B == 1 && NB == 2) ? 32 : (B <= 4 ? 16 : 8);
     static constexpr int BYTES = CPT / 2;                            // bytes per row per thread
     static constexpr int WORDS = BYTES / 4;
     static constexpr int ACC = B * CPT;
@@ -50,8 +53,8 @@ struct S1 {
     static constexpr int TPRM = CW / CPT;                            // threads per row per matrix
     static constexpr int TPR = 2 * TPRM;                             // threads per row
     static constexpr int RL = kS1Threads / TPR;                      // row lanes
-    static constexpr int RING = (B == 1) ? 256 : 128;                // ring bytes per thread
-    static constexpr int D = RING / BYTES;                           // ring depth (rows)
+    static constexpr int D = 256 / BYTES;                            // ring depth (rows)
+    static constexpr int WBYTES = 32 * BYTES;                        // bytes of a row per warp
 };
 
 // nibble position (in units of 4 bits) of local channel k of a word after
@@ -84,24 +87,6 @@ __device__ __forceinline__ void proc_word(uint32_t w0, int wi, const float *xs, 
     }
 }
 
-// cp.async of BYTES (16, 8 or 4) from global to shared, L1 bypassed for 16
-template <int BYTES>
-__device__ __forceinline__ void cp_async(void *dst, const void *src) {
-    if constexpr (BYTES == 16) {
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src)
-                     : "memory");
-    } else {
-        asm volatile("cp.async.ca.shared.global [%0], [%1], %2;" ::"r"(smem_addr(dst)), "l"(src),
-                     "n"(BYTES)
-                     : "memory");
-    }
-}
-__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
 // deterministic block-wide exclusive scan of one int per thread (256 threads)
 __device__ __forceinline__ int block_excl_scan(int v, int *warp_tot, int &total) {
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
@@ -128,20 +113,22 @@ __device__ __forceinline__ int block_excl_scan(int v, int *warp_tot, int &total)
 
 // shared-memory carve-up of one Stage-1 CTA (kept next to the kernel)
 struct S1Smem {
-    size_t ring, tmask, rowidx, xs, part, total;
+    size_t ring, bars, tmask, rowidx, xs, part, total;
 };
 
 __host__ __device__ inline S1Smem s1_smem(int d, int B, int NB, int unit_cap) {
     const int cw = NB * kCB;
-    const int cpt = (B == 1) ? 32 : (B <= 4 ? 16 : 8);
+    const int cpt = (B == 1 && NB == 2) ? 32 : (B <= 4 ? 16 : 8);
     const int rl = kS1Threads / (2 * (cw / cpt));
-    const size_t ring = (size_t)kS1Threads * (B == 1 ? 256 : 128);  // cp.async ring
+    const size_t ring = (size_t)kS1Threads * 256;                   // per-warp granule rings
     const size_t red = (size_t)rl * 2 * B * (cw + cw / cpt) * 4;    // padded row-lane sums
     const int W = d / 32;
     S1Smem s;
     size_t o = 0;
     s.ring = o;  // the row-lane reduction reuses the ring once streaming is done
     o += ring > red ? ring : red;
+    s.bars = o;  // one mbarrier per (warp, ring slot)
+    o += (size_t)(kS1Threads / 32) * (256 / (cpt / 2)) * 8;
     s.tmask = o;
     o += (size_t)B * W * 4;
     s.rowidx = o;
@@ -167,6 +154,7 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
     const int W = a.d / 32;                    // mask words per token
     const S1Smem L = s1_smem(a.d, B, NB, a.unit_cap);
     unsigned char *ring = smem + L.ring;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bars);  // [warps][D]
     float *red = reinterpret_cast<float *>(smem + L.ring);  // after streaming
     uint32_t *tmask = reinterpret_cast<uint32_t *>(smem + L.tmask);  // [B][W]
     int *rowidx = reinterpret_cast<int *>(smem + L.rowidx);          // [unit_cap]
@@ -182,6 +170,9 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
     // (Stage 2) start its own prologue.
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;");
+
+    for (int k = tid; k < (kS1Threads / 32) * T::D; k += kS1Threads) mbar_init(&bars[k], 1);
+    mbar_fence_init();
 
     // (1) Stage 2 accumulates y with atomics: clear it here.
     if (a.y_zero) {
@@ -280,31 +271,31 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
     }
     __syncthreads();
 
-    // Each thread streams its rows u = rl, rl + RL, ... of one 16/8/4-byte
-    // column chunk of one proxy through a private ring of D shared-memory
-    // slots; the first D copies start now, so their latency overlaps the
-    // scale gather below.
+    // Each thread handles rows u = rl, rl + RL, ... of one 16/8/4-byte column
+    // chunk of one proxy; a warp's lanes cover whole 128-byte granules of
+    // those rows (GPW of them), which the first lane of each granule copies
+    // into the warp's ring slot with a 1-D bulk copy.
     const int rl = tid / T::TPR;
     const int m = (tid / T::TPRM) & 1;
     const int chunk = tid % T::TPRM;
-    const uint8_t *qbase = (m ? a.q_gate : a.q_up) +
-                           (size_t)(c0 + chunk / T::TPRB) * a.d * (kCB / 2) +
-                           (chunk % T::TPRB) * T::BYTES;
-    // slot-major ring (ring[slot][thread]): a warp's accesses to one slot are
-    // consecutive words, free of bank conflicts
-    unsigned char *myring = ring + (size_t)tid * T::BYTES;
-    constexpr int SLOT = kS1Threads * T::BYTES;  // bytes between a thread's slots
+    const uint8_t *gsrc = (m ? a.q_gate : a.q_up) +
+                          (size_t)(c0 + chunk / T::TPRB) * a.d * (kCB / 2);  // granule column
+    const bool issuer = (lane % T::TPRB) == 0;  // first lane of its granule
+    unsigned char *wring = ring + (size_t)wid * T::D * T::WBYTES;
+    uint64_t *wbars = bars + wid * T::D;
     const int n_rows = n_units > rl ? (n_units - rl + T::RL - 1) / T::RL : 0;
-#pragma unroll 1
-    for (int k = 0; k < T::D; ++k) {
-        if (k < n_rows)
-            cp_async<T::BYTES>(myring + k * SLOT,
-                               qbase + (size_t)rowidx[rl + k * T::RL] * (kCB / 2));
-        cp_commit();
-    }
+    auto issue_row = [&](int k) {  // bulk copies of row k of this warp into slot k % D
+        const int slot = k % T::D;
+        if (lane == 0) mbar_arrive_expect_tx(&wbars[slot], T::WBYTES);
+        if (issuer)
+            bulk_g2s(wring + slot * T::WBYTES + lane * T::BYTES,
+                     gsrc + (size_t)rowidx[rl + k * T::RL] * (kCB / 2), 128, &wbars[slot]);
+    };
 
     // (4) x_i * scale_i * 2^E per matrix and token for the units (exact
-    // power-of-two scaling, split in two factors so each is a normal float)
+    // power-of-two scaling, split in two factors so each is a normal float).
+    // The few gather loads are issued first; the ring fill goes out while
+    // they are in flight.
     {
         float pe1[B], pe2[B];
 #pragma unroll
@@ -314,7 +305,8 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
             pe2[t] = __int_as_float((127 + e2) << 23);
         }
         constexpr int G4 = 2;  // units per thread per batch of loads
-        for (int u0 = tid; u0 < n_units; u0 += G4 * kS1Threads) {
+        bool ring_filled = false;
+        for (int u0 = tid; u0 < n_units || !ring_filled; u0 += G4 * kS1Threads) {
             float su[G4], sg[G4];
             uint16_t xh[G4][B];
 #pragma unroll
@@ -329,6 +321,11 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
                     for (int t = 0; t < B; ++t)
                         xh[k][t] = (t < a.nb) ? a.x[(size_t)t * a.d + i] : (uint16_t)0;
                 }
+            }
+            if (!ring_filled) {
+                __syncwarp();
+                for (int k = 0; k < T::D && k < n_rows; ++k) issue_row(k);
+                ring_filled = true;
             }
 #pragma unroll
             for (int k = 0; k < G4; ++k) {
@@ -348,28 +345,34 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
     }
     __syncthreads();
 
-    // (5) main loop: consume the ring in order, refilling each slot with the
-    // row D positions later; ssum collects this thread's sum of x_i * scale_i
-    // * 2^E for the +8 code offset
+    // (5) main loop: consume the warp's ring in order, refilling each slot
+    // with the row D positions later; ssum collects this thread's sum of
+    // x_i * scale_i * 2^E for the +8 code offset
     float2 acc2[T::ACC / 2];
 #pragma unroll
     for (int k = 0; k < T::ACC / 2; ++k) acc2[k] = make_float2(0.f, 0.f);
     float ssum[B];
 #pragma unroll
     for (int t = 0; t < B; ++t) ssum[t] = 0.f;
+    int consumed = 0;
     for (int k = 0; k < n_rows; ++k) {
-        cp_wait<T::D - 1>();
-        const int u = rl + k * T::RL;
         const int slot = k % T::D;
+        // the decision to give up is warp-uniform (lanes share later shuffles)
+        if (!__all_sync(0xffffffffu, mbar_wait(&wbars[slot], (k / T::D) & 1, a.wait_us))) {
+            if (lane == 0) atomicOr(a.status, kStTimeoutRing);
+            break;
+        }
+        const int u = rl + k * T::RL;
+        const unsigned char *src = wring + slot * T::WBYTES + lane * T::BYTES;
         uint32_t w[T::WORDS];
         if constexpr (T::WORDS == 4) {
-            const uint4 v = *reinterpret_cast<const uint4 *>(myring + slot * SLOT);
+            const uint4 v = *reinterpret_cast<const uint4 *>(src);
             w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
         } else if constexpr (T::WORDS == 2) {
-            const uint2 v = *reinterpret_cast<const uint2 *>(myring + slot * SLOT);
+            const uint2 v = *reinterpret_cast<const uint2 *>(src);
             w[0] = v.x; w[1] = v.y;
         } else {
-            w[0] = *reinterpret_cast<const uint32_t *>(myring + slot * SLOT);
+            w[0] = *reinterpret_cast<const uint32_t *>(src);
         }
         float xv[B];
 #pragma unroll
@@ -379,15 +382,15 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
         }
 #pragma unroll
         for (int q = 0; q < T::WORDS; ++q) proc_word<B, T::CPT>(w[q], q, xv, acc2);
-        // the slot's words have been consumed: refill it
-        const int kn = k + T::D;
-        if (kn < n_rows)
-            cp_async<T::BYTES>(myring + slot * SLOT,
-                               qbase + (size_t)rowidx[rl + kn * T::RL] * (kCB / 2));
-        cp_commit();
+        consumed = k + 1;
+        // every lane has read the slot: refill it
+        __syncwarp();
+        if (k + T::D < n_rows) issue_row(k + T::D);
     }
-    cp_wait<0>();
-    __syncthreads();  // every thread is done with the ring before it becomes `red`
+    // never leave copies in flight (only after a timeout can any be pending)
+    for (int k = consumed; k < n_rows && k < consumed + T::D; ++k)
+        if (!mbar_wait(&wbars[k % T::D], (k / T::D) & 1, a.wait_us)) break;
+    __syncthreads();  // every warp is done with its ring before it becomes `red`
 
     // (6) reduce row lanes (padded rows: conflict-free both ways), undo the
     // pre-scale and the +8 code offset: this CTA's partial sums in `part`.

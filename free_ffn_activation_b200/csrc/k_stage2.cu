@@ -259,7 +259,8 @@ __global__ void __launch_bounds__(s2_threads(B), 1) k_stage2(const Stage2Args a)
         for (int n = 0; n < n_ch; ++n) {
             const int s = n % NST, k = n / NST;
             if (s % kNDot != wid) continue;
-            if (!mbar_wait(&full[s], k & 1, a.spin_limit)) {
+            // the decision to give up is warp-uniform (lanes share later shuffles)
+            if (!__all_sync(0xffffffffu, mbar_wait(&full[s], k & 1, a.spin_limit))) {
                 if (lane == 0) atomicOr(a.status, kStTimeoutFull);
                 break;
             }
@@ -342,7 +343,9 @@ __global__ void __launch_bounds__(s2_threads(B), 1) k_stage2(const Stage2Args a)
 
     for (int n = 0; n < n_ch; ++n) {
         const int s = n % NST, ph = (n / NST) & 1;
-        if (!mbar_wait(&full[s], ph, a.spin_limit) || !mbar_wait(&sready[s], ph, a.spin_limit)) {
+        const bool ok = mbar_wait(&full[s], ph, a.spin_limit) &&
+                        mbar_wait(&sready[s], ph, a.spin_limit);
+        if (!__all_sync(0xffffffffu, ok)) {  // warp-uniform decision
             if (lane == 0) atomicOr(a.status, kStTimeoutRed);
             break;
         }

@@ -190,6 +190,8 @@ static prox_status pass_stage1(const prox_layer *L, const uint16_t *x, int nb, f
     a.mask_s = mask_s;
     a.s_out = s_out;
     a.build_lists = lists ? 1 : 0;
+    a.wait_us = g_spin_limit;
+    a.status = reinterpret_cast<uint32_t *>(w + W.status);
     a.ucount = reinterpret_cast<int32_t *>(w + W.ucount);
     a.tcount = reinterpret_cast<int32_t *>(w + W.tcount);
     a.ulist = reinterpret_cast<uint32_t *>(w + W.ulist);

@@ -25,6 +25,7 @@ constexpr uint32_t kStTimeoutFull = 1u << 0;   // consumer waited for a stage
 constexpr uint32_t kStTimeoutEmpty = 1u << 1;  // producer waited for a free slot
 constexpr uint32_t kStTimeoutRed = 1u << 2;    // consumers waited for partials
 constexpr uint32_t kStTimeoutDrain = 1u << 3;  // producer waited for its copies
+constexpr uint32_t kStTimeoutRing = 1u << 4;   // Stage 1 waited for a ring slot
 
 // default wall-clock bound of a device-side wait, in microseconds
 constexpr uint32_t kDefaultWaitUs = 2000000u;
@@ -74,7 +75,9 @@ struct Stage1Args {
     uint8_t *mask_s;             // [nb][f] or null
     float *s_out;                // [nb][f] or null
     int build_lists;             // write ulist/tlist/counts for Stage 2
+    uint32_t wait_us;            // wall-clock bound of each wait, microseconds
     // workspace
+    uint32_t *status;
     int32_t *ucount;             // [C]
     int32_t *tcount;             // [C][B]
     uint32_t *ulist;             // [C][kCB]  channel | token bits << 24
