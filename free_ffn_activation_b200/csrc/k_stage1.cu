@@ -12,11 +12,9 @@
 // cluster of n_r CTAs; CTA r of the cluster takes the r-th contiguous range
 // of the kept rows (ranks over the union of the pass's tokens) and streams
 // the granules of BOTH proxies (one read of x serves up and gate, the fused
-// split-N kernel of the blog's "From formula to GPU" section). Every warp
-// owns whole 128-byte granules of its rows and keeps a private ring of them
-// in shared memory, filled by 1-D bulk copies (TMA) and guarded by one
-// mbarrier per slot, so about 128 KB per CTA is in flight with no cross-warp
-// synchronisation. The cluster's
+// split-N kernel of the blog's "From formula to GPU" section). Each thread
+// keeps two sets of rows of its 16/8/4-byte chunk in flight in registers
+// (load one set while decoding the other), about 64 KB per CTA. The cluster's
 // partial sums meet in distributed shared memory: CTA 0 adds them in rank
 // order, forms s~ = u~ * SiLU(g~), thresholds it and compacts the kept
 // channels into ascending lists, so the result is deterministic.
@@ -53,9 +51,28 @@ struct S1 {
     static constexpr int TPRM = CW / CPT;                            // threads per row per matrix
     static constexpr int TPR = 2 * TPRM;                             // threads per row
     static constexpr int RL = kS1Threads / TPR;                      // row lanes
-    static constexpr int D = 256 / BYTES;                            // ring depth (rows)
-    static constexpr int WBYTES = 32 * BYTES;                        // bytes of a row per warp
+    static constexpr int U = (B >= 4 ? 8 : 16) / WORDS;              // rows per load set
 };
+
+template <int WORDS>
+struct Vec {
+    uint32_t w[WORDS];
+};
+
+// streaming 16/8/4-byte load that does not allocate in L1
+__device__ __forceinline__ void ld_stream(Vec<4> &v, const uint8_t *p) {
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3])
+                 : "l"(p));
+}
+__device__ __forceinline__ void ld_stream(Vec<2> &v, const uint8_t *p) {
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
+                 : "=r"(v.w[0]), "=r"(v.w[1])
+                 : "l"(p));
+}
+__device__ __forceinline__ void ld_stream(Vec<1> &v, const uint8_t *p) {
+    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v.w[0]) : "l"(p));
+}
 
 // nibble position (in units of 4 bits) of local channel k of a word after
 // the decode above
@@ -113,22 +130,19 @@ __device__ __forceinline__ int block_excl_scan(int v, int *warp_tot, int &total)
 
 // shared-memory carve-up of one Stage-1 CTA (kept next to the kernel)
 struct S1Smem {
-    size_t ring, bars, tmask, rowidx, xs, part, total;
+    size_t red, tmask, rowidx, xs, part, total;
 };
 
 __host__ __device__ inline S1Smem s1_smem(int d, int B, int NB, int unit_cap) {
     const int cw = NB * kCB;
     const int cpt = (B == 1 && NB == 2) ? 32 : (B <= 4 ? 16 : 8);
     const int rl = kS1Threads / (2 * (cw / cpt));
-    const size_t ring = (size_t)kS1Threads * 256;                   // per-warp granule rings
     const size_t red = (size_t)rl * 2 * B * (cw + cw / cpt) * 4;    // padded row-lane sums
     const int W = d / 32;
     S1Smem s;
     size_t o = 0;
-    s.ring = o;  // the row-lane reduction reuses the ring once streaming is done
-    o += ring > red ? ring : red;
-    s.bars = o;  // one mbarrier per (warp, ring slot)
-    o += (size_t)(kS1Threads / 32) * (256 / (cpt / 2)) * 8;
+    s.red = o;
+    o += red;
     s.tmask = o;
     o += (size_t)B * W * 4;
     s.rowidx = o;
@@ -153,9 +167,7 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
     const int c0 = (blockIdx.x / a.n_r) * NB;  // first column block of the group
     const int W = a.d / 32;                    // mask words per token
     const S1Smem L = s1_smem(a.d, B, NB, a.unit_cap);
-    unsigned char *ring = smem + L.ring;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bars);  // [warps][D]
-    float *red = reinterpret_cast<float *>(smem + L.ring);  // after streaming
+    float *red = reinterpret_cast<float *>(smem + L.red);
     uint32_t *tmask = reinterpret_cast<uint32_t *>(smem + L.tmask);  // [B][W]
     int *rowidx = reinterpret_cast<int *>(smem + L.rowidx);          // [unit_cap]
     float *xs = reinterpret_cast<float *>(smem + L.xs);              // [unit_cap][2][B]
@@ -171,9 +183,6 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;");
 
-    for (int k = tid; k < (kS1Threads / 32) * T::D; k += kS1Threads) mbar_init(&bars[k], 1);
-    mbar_fence_init();
-
     // (1) Stage 2 accumulates y with atomics: clear it here.
     if (a.y_zero) {
         float4 *y4 = reinterpret_cast<float4 *>(a.y_zero);
@@ -188,8 +197,8 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
     // same pass finds max |x| per token, which fixes the power-of-two
     // pre-scale 2^E (see the decode note above).
     {
-        // chunks per thread per token (d_model <= 8192)
-        constexpr int MAXK = (8192 / 8 + kS1Threads - 1) / kS1Threads;
+        // chunks per thread per token (d_model <= 8192; <= 4096 when B = 8)
+        constexpr int MAXK = (B == 8 ? 4096 : 8192) / 8 / kS1Threads;
         const int NC = a.d / 8;
         uint4 xv[MAXK][B];
 #pragma unroll
@@ -271,31 +280,26 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
     }
     __syncthreads();
 
-    // Each thread handles rows u = rl, rl + RL, ... of one 16/8/4-byte column
-    // chunk of one proxy; a warp's lanes cover whole 128-byte granules of
-    // those rows (GPW of them), which the first lane of each granule copies
-    // into the warp's ring slot with a 1-D bulk copy.
+    // Each thread streams rows u = rl, rl + RL, ... (its k-th row is u =
+    // rl + k * RL) of one 16/8/4-byte chunk of one proxy's granules.
     const int rl = tid / T::TPR;
     const int m = (tid / T::TPRM) & 1;
     const int chunk = tid % T::TPRM;
     const uint8_t *gsrc = (m ? a.q_gate : a.q_up) +
-                          (size_t)(c0 + chunk / T::TPRB) * a.d * (kCB / 2);  // granule column
-    const bool issuer = (lane % T::TPRB) == 0;  // first lane of its granule
-    unsigned char *wring = ring + (size_t)wid * T::D * T::WBYTES;
-    uint64_t *wbars = bars + wid * T::D;
+                          (size_t)(c0 + chunk / T::TPRB) * a.d * (kCB / 2) +
+                          (chunk % T::TPRB) * T::BYTES;
     const int n_rows = n_units > rl ? (n_units - rl + T::RL - 1) / T::RL : 0;
-    auto issue_row = [&](int k) {  // bulk copies of row k of this warp into slot k % D
-        const int slot = k % T::D;
-        if (lane == 0) mbar_arrive_expect_tx(&wbars[slot], T::WBYTES);
-        if (issuer)
-            bulk_g2s(wring + slot * T::WBYTES + lane * T::BYTES,
-                     gsrc + (size_t)rowidx[rl + k * T::RL] * (kCB / 2), 128, &wbars[slot]);
+    Vec<T::WORDS> va[T::U], vb[T::U];
+    auto load_set = [&](Vec<T::WORDS>(&v)[T::U], int k0) {
+#pragma unroll
+        for (int j = 0; j < T::U; ++j)
+            if (k0 + j < n_rows)
+                ld_stream(v[j], gsrc + (size_t)rowidx[rl + (k0 + j) * T::RL] * (kCB / 2));
     };
 
     // (4) x_i * scale_i * 2^E per matrix and token for the units (exact
     // power-of-two scaling, split in two factors so each is a normal float).
-    // The few gather loads are issued first; the ring fill goes out while
-    // they are in flight.
+    // The few gather loads go out first, the first two row sets right after.
     {
         float pe1[B], pe2[B];
 #pragma unroll
@@ -305,8 +309,8 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
             pe2[t] = __int_as_float((127 + e2) << 23);
         }
         constexpr int G4 = 2;  // units per thread per batch of loads
-        bool ring_filled = false;
-        for (int u0 = tid; u0 < n_units || !ring_filled; u0 += G4 * kS1Threads) {
+        bool started = false;
+        for (int u0 = tid; u0 < n_units || !started; u0 += G4 * kS1Threads) {
             float su[G4], sg[G4];
             uint16_t xh[G4][B];
 #pragma unroll
@@ -322,10 +326,10 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
                         xh[k][t] = (t < a.nb) ? a.x[(size_t)t * a.d + i] : (uint16_t)0;
                 }
             }
-            if (!ring_filled) {
-                __syncwarp();
-                for (int k = 0; k < T::D && k < n_rows; ++k) issue_row(k);
-                ring_filled = true;
+            if (!started) {
+                load_set(va, 0);
+                load_set(vb, T::U);
+                started = true;
             }
 #pragma unroll
             for (int k = 0; k < G4; ++k) {
@@ -345,52 +349,36 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
     }
     __syncthreads();
 
-    // (5) main loop: consume the warp's ring in order, refilling each slot
-    // with the row D positions later; ssum collects this thread's sum of
-    // x_i * scale_i * 2^E for the +8 code offset
+    // (5) main loop: decode one register set while the other is in flight;
+    // ssum collects this thread's sum of x_i * scale_i * 2^E (+8 code offset)
     float2 acc2[T::ACC / 2];
 #pragma unroll
     for (int k = 0; k < T::ACC / 2; ++k) acc2[k] = make_float2(0.f, 0.f);
     float ssum[B];
 #pragma unroll
     for (int t = 0; t < B; ++t) ssum[t] = 0.f;
-    int consumed = 0;
-    for (int k = 0; k < n_rows; ++k) {
-        const int slot = k % T::D;
-        // the decision to give up is warp-uniform (lanes share later shuffles)
-        if (!__all_sync(0xffffffffu, mbar_wait(&wbars[slot], (k / T::D) & 1, a.wait_us))) {
-            if (lane == 0) atomicOr(a.status, kStTimeoutRing);
-            break;
-        }
-        const int u = rl + k * T::RL;
-        const unsigned char *src = wring + slot * T::WBYTES + lane * T::BYTES;
-        uint32_t w[T::WORDS];
-        if constexpr (T::WORDS == 4) {
-            const uint4 v = *reinterpret_cast<const uint4 *>(src);
-            w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
-        } else if constexpr (T::WORDS == 2) {
-            const uint2 v = *reinterpret_cast<const uint2 *>(src);
-            w[0] = v.x; w[1] = v.y;
-        } else {
-            w[0] = *reinterpret_cast<const uint32_t *>(src);
-        }
-        float xv[B];
+    auto comp_set = [&](const Vec<T::WORDS>(&v)[T::U], int k0) {
 #pragma unroll
-        for (int t = 0; t < B; ++t) {
-            xv[t] = xs[(u * 2 + m) * B + t];
-            ssum[t] += xv[t];
-        }
+        for (int j = 0; j < T::U; ++j) {
+            if (k0 + j >= n_rows) break;
+            const int u = rl + (k0 + j) * T::RL;
+            float xv[B];
 #pragma unroll
-        for (int q = 0; q < T::WORDS; ++q) proc_word<B, T::CPT>(w[q], q, xv, acc2);
-        consumed = k + 1;
-        // every lane has read the slot: refill it
-        __syncwarp();
-        if (k + T::D < n_rows) issue_row(k + T::D);
+            for (int t = 0; t < B; ++t) {
+                xv[t] = xs[(u * 2 + m) * B + t];
+                ssum[t] += xv[t];
+            }
+#pragma unroll
+            for (int q = 0; q < T::WORDS; ++q) proc_word<B, T::CPT>(v[j].w[q], q, xv, acc2);
+        }
+    };
+    for (int k0 = 0; k0 < n_rows; k0 += 2 * T::U) {
+        comp_set(va, k0);
+        load_set(va, k0 + 2 * T::U);
+        comp_set(vb, k0 + T::U);
+        load_set(vb, k0 + 3 * T::U);
     }
-    // never leave copies in flight (only after a timeout can any be pending)
-    for (int k = consumed; k < n_rows && k < consumed + T::D; ++k)
-        if (!mbar_wait(&wbars[k % T::D], (k / T::D) & 1, a.wait_us)) break;
-    __syncthreads();  // every warp is done with its ring before it becomes `red`
+    __syncthreads();
 
     // (6) reduce row lanes (padded rows: conflict-free both ways), undo the
     // pre-scale and the +8 code offset: this CTA's partial sums in `part`.
@@ -440,14 +428,25 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
         const int j = c0 * kCB + ch;         // channel index
         const int blk = wid / (kCB / 32);    // block of this warp's channels
         float uu[B], gg[B];
-#pragma unroll
+#pragma unroll(B > 2 ? 1 : B)
         for (int t = 0; t < B; ++t) {
             uu[t] = gg[t] = 0.f;
             if (t >= a.nb || ch >= T::CW) continue;
-            for (int q = 0; q < a.n_r; ++q) {
-                const float *pq = cluster.map_shared_rank(part, q);
-                uu[t] += pq[(0 * B + t) * T::CW + ch];
-                gg[t] += pq[(1 * B + t) * T::CW + ch];
+            // all remote loads first, then the sums in rank order
+            float pu[kS1MaxRowGroups], pg[kS1MaxRowGroups];
+#pragma unroll
+            for (int q = 0; q < kS1MaxRowGroups; ++q) {
+                pu[q] = pg[q] = 0.f;
+                if (q < a.n_r) {
+                    const float *pq = cluster.map_shared_rank(part, q);
+                    pu[q] = pq[(0 * B + t) * T::CW + ch];
+                    pg[q] = pq[(1 * B + t) * T::CW + ch];
+                }
+            }
+#pragma unroll
+            for (int q = 0; q < kS1MaxRowGroups; ++q) {
+                uu[t] += pu[q];
+                gg[t] += pg[q];
             }
         }
         asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
