@@ -39,11 +39,21 @@ namespace cg = cooperative_groups;
 namespace prox {
 namespace {
 
+// channels per thread: a warp covers whole rows of one row lane
+__host__ __device__ constexpr int s1_cpt(int B, int NB) {
+    return (B <= 2 && NB == 2) ? 32 : (B <= 4 ? 16 : 8);
+}
+// deepest per-thread ring (rows in flight) and the ring bytes it takes
+__host__ __device__ constexpr int s1_ring_bytes(int B) { return B <= 2 ? 384 : (B == 4 ? 256 : 128); }
+__host__ __device__ constexpr int s1_dmax(int B, int NB) {
+    return s1_ring_bytes(B) / (s1_cpt(B, NB) / 2) < 32 ? s1_ring_bytes(B) / (s1_cpt(B, NB) / 2)
+                                                          : 32;
+}
+
 template <int B, int NB>
 struct S1 {
     static constexpr int CW = NB * kCB;                              // channels per CTA
-    // channels per thread; every warp covers whole rows of one row lane
-    static constexpr int CPT = (B == 1 && NB == 2) ? 32 : (B <= 4 ? 16 : 8);
+    static constexpr int CPT = s1_cpt(B, NB);                        // channels per thread
     static constexpr int BYTES = CPT / 2;                            // bytes per row per thread
     static constexpr int WORDS = BYTES / 4;
     static constexpr int ACC = B * CPT;
@@ -51,27 +61,26 @@ struct S1 {
     static constexpr int TPRM = CW / CPT;                            // threads per row per matrix
     static constexpr int TPR = 2 * TPRM;                             // threads per row
     static constexpr int RL = kS1Threads / TPR;                      // row lanes
-    static constexpr int U = (B >= 4 ? 8 : 16) / WORDS;              // rows per load set
+    static constexpr int DMAX = s1_dmax(B, NB);                      // deepest ring (rows)
+    static constexpr int KMAX = (B == 8 ? 4096 : 8192) / 8 / kS1Threads;  // x chunks per thread
 };
 
-template <int WORDS>
-struct Vec {
-    uint32_t w[WORDS];
-};
-
-// streaming 16/8/4-byte load that does not allocate in L1
-__device__ __forceinline__ void ld_stream(Vec<4> &v, const uint8_t *p) {
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3])
-                 : "l"(p));
+// cp.async of BYTES (16, 8 or 4) from global to shared; 16-byte copies skip L1
+template <int BYTES>
+__device__ __forceinline__ void cp_async(void *dst, const void *src) {
+    if constexpr (BYTES == 16) {
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src)
+                     : "memory");
+    } else {
+        asm volatile("cp.async.ca.shared.global [%0], [%1], %2;" ::"r"(smem_addr(dst)), "l"(src),
+                     "n"(BYTES)
+                     : "memory");
+    }
 }
-__device__ __forceinline__ void ld_stream(Vec<2> &v, const uint8_t *p) {
-    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
-                 : "=r"(v.w[0]), "=r"(v.w[1])
-                 : "l"(p));
-}
-__device__ __forceinline__ void ld_stream(Vec<1> &v, const uint8_t *p) {
-    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v.w[0]) : "l"(p));
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // nibble position (in units of 4 bits) of local channel k of a word after
@@ -128,25 +137,26 @@ __device__ __forceinline__ int block_excl_scan(int v, int *warp_tot, int &total)
 
 }  // namespace
 
-// shared-memory carve-up of one Stage-1 CTA (kept next to the kernel)
+// shared-memory carve-up of one Stage-1 CTA (kept next to the kernel). The
+// copy ring (depth DMAX >> depth_sel rows per thread) and the row-lane
+// reduction area are used one after the other and share one region.
 struct S1Smem {
-    size_t red, tmask, rowidx, xs, part, total;
+    size_t ring, red, rowidx, xs, part, total;
 };
 
-__host__ __device__ inline S1Smem s1_smem(int d, int B, int NB, int unit_cap) {
+__host__ __device__ inline S1Smem s1_smem(int d, int B, int NB, int unit_cap, int depth_sel) {
     const int cw = NB * kCB;
-    const int cpt = (B == 1 && NB == 2) ? 32 : (B <= 4 ? 16 : 8);
+    const int cpt = s1_cpt(B, NB);
     const int rl = kS1Threads / (2 * (cw / cpt));
     const size_t red = (size_t)rl * 2 * B * (cw + cw / cpt) * 4;    // padded row-lane sums
-    const int W = d / 32;
+    const size_t ring = (size_t)kS1Threads * (s1_dmax(B, NB) >> depth_sel) * (cpt / 2);
+    (void)d;
     S1Smem s;
     size_t o = 0;
-    s.red = o;
-    o += red;
-    s.tmask = o;
-    o += (size_t)B * W * 4;
+    s.ring = s.red = o;
+    o += ring > red ? ring : red;
     s.rowidx = o;
-    o += (size_t)unit_cap * 4;
+    o += ((size_t)unit_cap * 4 + 15) / 16 * 16;
     s.xs = o;
     o += (size_t)unit_cap * 2 * B * 4;
     s.part = o;
@@ -157,6 +167,57 @@ __host__ __device__ inline S1Smem s1_smem(int d, int B, int NB, int unit_cap) {
 
 namespace {
 
+// (5) main loop: each thread streams rows u = rl, rl + RL, ... (its k-th row
+// is u = rl + k * RL) of one 16/8/4-byte chunk of one proxy's granules
+// through a private ring of D shared-memory slots, refilling each slot with
+// the row D positions later as soon as its words are decoded. ssum collects
+// the thread's sum of x_i * scale_i * 2^E (for the +8 code offset).
+template <int B, int NB, int D>
+__device__ __forceinline__ void s1_stream(const uint8_t *qbase, unsigned char *ring,
+                                          const int *rowidx, const float *xs, int rl, int m,
+                                          int n_rows, float2 *acc2, float *ssum) {
+    using T = S1<B, NB>;
+    // slot-major ring (ring[slot][thread]): a warp's accesses to one slot are
+    // consecutive words, free of bank conflicts
+    unsigned char *myring = ring + (size_t)threadIdx.x * T::BYTES;
+    constexpr int SLOT = kS1Threads * T::BYTES;  // bytes between a thread's slots
+#pragma unroll 1
+    for (int k = 0; k < D; ++k) {
+        if (k < n_rows)
+            cp_async<T::BYTES>(myring + k * SLOT, qbase + (size_t)rowidx[rl + k * T::RL] * (kCB / 2));
+        cp_commit();
+    }
+#pragma unroll 1
+    for (int k = 0; k < n_rows; ++k) {
+        cp_wait<D - 1>();
+        const int u = rl + k * T::RL;
+        const int slot = k % D;
+        uint32_t w[T::WORDS];
+        if constexpr (T::WORDS == 4) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(myring + slot * SLOT);
+            w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+        } else if constexpr (T::WORDS == 2) {
+            const uint2 v = *reinterpret_cast<const uint2 *>(myring + slot * SLOT);
+            w[0] = v.x; w[1] = v.y;
+        } else {
+            w[0] = *reinterpret_cast<const uint32_t *>(myring + slot * SLOT);
+        }
+        float xv[B];
+#pragma unroll
+        for (int t = 0; t < B; ++t) {
+            xv[t] = xs[(u * 2 + m) * B + t];
+            ssum[t] += xv[t];
+        }
+#pragma unroll
+        for (int q = 0; q < T::WORDS; ++q) proc_word<B, T::CPT>(w[q], q, xv, acc2);
+        const int kn = k + D;
+        if (kn < n_rows)
+            cp_async<T::BYTES>(myring + slot * SLOT, qbase + (size_t)rowidx[rl + kn * T::RL] * (kCB / 2));
+        cp_commit();
+    }
+    cp_wait<0>();
+}
+
 template <int B, int NB>
 __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
     using T = S1<B, NB>;
@@ -165,17 +226,27 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
     cg::cluster_group cluster = cg::this_cluster();
     const int r = (int)cluster.block_rank();  // row group
     const int c0 = (blockIdx.x / a.n_r) * NB;  // first column block of the group
-    const int W = a.d / 32;                    // mask words per token
-    const S1Smem L = s1_smem(a.d, B, NB, a.unit_cap);
+    const S1Smem L = s1_smem(a.d, B, NB, a.unit_cap, a.depth_sel);
+    unsigned char *ring = smem + L.ring;
     float *red = reinterpret_cast<float *>(smem + L.red);
-    uint32_t *tmask = reinterpret_cast<uint32_t *>(smem + L.tmask);  // [B][W]
     int *rowidx = reinterpret_cast<int *>(smem + L.rowidx);          // [unit_cap]
     float *xs = reinterpret_cast<float *>(smem + L.xs);              // [unit_cap][2][B]
     float *part = reinterpret_cast<float *>(smem + L.part);          // [2][B][CW]
     __shared__ int s_warp[kS1Threads / 32];
-    __shared__ float s_red[kS1Threads / 32][4 * kMaxB];
-    __shared__ int s_E[kMaxB];
+    __shared__ __align__(16) float s_red[kS1Threads / 32][kMaxB];
     __shared__ int s_cnt[kS1Threads / 32][kMaxB + 1];
+
+    // The proxy scales are layer weights: pull them into L2 while the
+    // previous kernel of the stream finishes (a prefetch only warms the
+    // coherent L2 and reads nothing into this CTA).
+    {
+        const int lines = a.d * 4 / 128;  // 128-byte lines per scale vector
+        const int g = blockIdx.x * kS1Threads + tid;
+        if (g < 2 * lines) {
+            const float *p = (g < lines ? a.s_up : a.s_gate) + (size_t)(g % lines) * 32;
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+        }
+    }
 
     // Programmatic dependent launch: x, y and the workspace may belong to the
     // previous kernel in the stream; wait for it, then let the next kernel
@@ -191,33 +262,45 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
             y4[k] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
 
-    // (2) input masks m_x = 1[|x_i| >= tau_x] per token: each thread owns
-    // 16-byte chunks of 8 coordinates; all its loads are issued before any
-    // use. Chunk ci's 8 keep bits are byte ci of the token's mask words. The
-    // same pass finds max |x| per token, which fixes the power-of-two
-    // pre-scale 2^E (see the decode note above).
-    {
-        // chunks per thread per token (d_model <= 8192; <= 4096 when B = 8)
-        constexpr int MAXK = (B == 8 ? 4096 : 8192) / 8 / kS1Threads;
-        const int NC = a.d / 8;
-        uint4 xv[MAXK][B];
+    // (2) input masks m_x = 1[|x_i| >= tau_x] per token. Thread tid owns the K
+    // adjacent 8-coordinate chunks [tid * K, tid * K + K) (K = 1, or 2 when
+    // d_model > 4096): it loads their x, s_up and s_gate with 16-byte loads
+    // (all issued before any use), finds their keep bits and max |x| per
+    // token (which fixes the power-of-two pre-scale 2^E, see the decode note
+    // above).
+    const int NC = a.d / 8;
+    const int K = (NC + kS1Threads - 1) / kS1Threads;
+    uint4 xv[T::KMAX][B];
+    float4 su[T::KMAX][2], sg[T::KMAX][2];
+    uint32_t kb[T::KMAX][B];  // keep bits of the chunk per token (8 used)
 #pragma unroll
-        for (int k = 0; k < MAXK; ++k)
+    for (int k = 0; k < T::KMAX; ++k) {
+        const int ci = tid * K + k;
+        const bool on = k < K && ci < NC;
 #pragma unroll
-            for (int t = 0; t < B; ++t) {
-                const int ci = tid + k * kS1Threads;
-                xv[k][t] = make_uint4(0, 0, 0, 0);
-                if (ci < NC && t < a.nb)
-                    xv[k][t] = *reinterpret_cast<const uint4 *>(a.x + (size_t)t * a.d + ci * 8);
+        for (int t = 0; t < B; ++t) {
+            xv[k][t] = make_uint4(0, 0, 0, 0);
+            if (on && t < a.nb) xv[k][t] = *reinterpret_cast<const uint4 *>(a.x + (size_t)t * a.d + ci * 8);
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            su[k][h] = sg[k][h] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (on) {
+                su[k][h] = *reinterpret_cast<const float4 *>(a.s_up + ci * 8 + 4 * h);
+                sg[k][h] = *reinterpret_cast<const float4 *>(a.s_gate + ci * 8 + 4 * h);
             }
-        uint8_t *tbytes = reinterpret_cast<uint8_t *>(tmask);
+        }
+    }
+    int cnt = 0;        // union-kept coordinates of this thread
+    uint32_t ub[T::KMAX];  // union keep bits per chunk
+    {
         float xmax[B];
 #pragma unroll
         for (int t = 0; t < B; ++t) xmax[t] = 0.f;
 #pragma unroll
-        for (int k = 0; k < MAXK; ++k) {
-            const int ci = tid + k * kS1Threads;
-            if (ci >= NC) break;
+        for (int k = 0; k < T::KMAX; ++k) {
+            const int ci = tid * K + k;
+            ub[k] = 0;
 #pragma unroll
             for (int t = 0; t < B; ++t) {
                 const uint32_t w4[4] = {xv[k][t].x, xv[k][t].y, xv[k][t].z, xv[k][t].w};
@@ -229,9 +312,10 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
                     bits |= (hi >= a.tau_x ? 1u : 0u) << (2 * h + 1);
                     xmax[t] = fmaxf(xmax[t], fmaxf(lo, hi));
                 }
-                if (t >= a.nb) bits = 0;
-                tbytes[t * NC + ci] = (uint8_t)bits;
-                if (a.mask_x && blockIdx.x == 0 && t < a.nb) {
+                if (t >= a.nb || k >= K || ci >= NC) bits = 0;
+                kb[k][t] = bits;
+                ub[k] |= bits;
+                if (a.mask_x && blockIdx.x == 0 && t < a.nb && k < K && ci < NC) {
                     uint32_t lo = 0, hi = 0;
 #pragma unroll
                     for (int b = 0; b < 4; ++b) {
@@ -242,6 +326,7 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
                         make_uint2(lo, hi);
                 }
             }
+            cnt += __popc(ub[k]);
         }
 #pragma unroll
         for (int t = 0; t < B; ++t) {
@@ -251,134 +336,84 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
             if (lane == 0) s_red[wid][t] = xmax[t];
         }
     }
-    __syncthreads();
 
-    // (3) one thread per mask word: union mask, its population, ranks of the
-    // kept rows (one block-wide scan) and this CTA's share of them
-    if (tid < B) {
-        float mx = 0.f;
-        for (int w = 0; w < kS1Threads / 32; ++w) mx = fmaxf(mx, s_red[w][tid]);
-        // |x * 2^E| < 2^96: a row sum of (q + 8) * x_i * scale_i * 2^E over
-        // <= 8192 rows stays finite for scales below 2^15 and, for scales
-        // above 2^-70, partial sums of the subnormal-coded products stay normal
-        s_E[tid] = (mx > 0.f) ? 95 - ilogbf(mx) : 0;
-    }
-    uint32_t um = 0;
-    if (tid < W) {
-#pragma unroll
-        for (int t = 0; t < B; ++t) um |= tmask[t * W + tid];
-    }
+    // (3) ranks of the union-kept rows (one block-wide scan, which also
+    // publishes the per-warp maxima) and this CTA's share [lo, hi) of them.
+    // Each thread writes the row index and x_i * scale_i * 2^E (per matrix and
+    // token; exact power-of-two scaling split in two normal-float factors) of
+    // its own kept coordinates that fall in the share: no gathers.
     int kx;
-    const int woffs = block_excl_scan(__popc(um), s_warp, kx);  // syncs the CTA
+    const int woffs = block_excl_scan(cnt, s_warp, kx);  // syncs the CTA
     const int lo = (int)((long long)kx * r / a.n_r);
     const int hi = (int)((long long)kx * (r + 1) / a.n_r);
     const int n_units = hi - lo;
-    if (woffs < hi && woffs + __popc(um) > lo) {
-        int rank = woffs;
-        for (uint32_t b = um; b; b &= b - 1, ++rank)
-            if (rank >= lo && rank < hi) rowidx[rank - lo] = tid * 32 + (__ffs(b) - 1);
-    }
-    __syncthreads();
-
-    // Each thread streams rows u = rl, rl + RL, ... (its k-th row is u =
-    // rl + k * RL) of one 16/8/4-byte chunk of one proxy's granules.
-    const int rl = tid / T::TPR;
-    const int m = (tid / T::TPRM) & 1;
-    const int chunk = tid % T::TPRM;
-    const uint8_t *gsrc = (m ? a.q_gate : a.q_up) +
-                          (size_t)(c0 + chunk / T::TPRB) * a.d * (kCB / 2) +
-                          (chunk % T::TPRB) * T::BYTES;
-    const int n_rows = n_units > rl ? (n_units - rl + T::RL - 1) / T::RL : 0;
-    Vec<T::WORDS> va[T::U], vb[T::U];
-    auto load_set = [&](Vec<T::WORDS>(&v)[T::U], int k0) {
+    int E[B];
 #pragma unroll
-        for (int j = 0; j < T::U; ++j)
-            if (k0 + j < n_rows)
-                ld_stream(v[j], gsrc + (size_t)rowidx[rl + (k0 + j) * T::RL] * (kCB / 2));
-    };
-
-    // (4) x_i * scale_i * 2^E per matrix and token for the units (exact
-    // power-of-two scaling, split in two factors so each is a normal float).
-    // The few gather loads go out first, the first two row sets right after.
-    {
+    for (int t = 0; t < B; ++t) {
+        float mx = 0.f;
+#pragma unroll
+        for (int w = 0; w < kS1Threads / 32; ++w) mx = fmaxf(mx, s_red[w][t]);
+        // |x * 2^E| < 2^96: a row sum of (q + 8) * x_i * scale_i * 2^E over
+        // <= 8192 rows stays finite for scales below 2^15 and, for scales
+        // above 2^-70, partial sums of the subnormal-coded products stay normal
+        E[t] = (mx > 0.f) ? 95 - ilogbf(mx) : 0;
+    }
+    if (woffs < hi && woffs + cnt > lo) {
         float pe1[B], pe2[B];
 #pragma unroll
         for (int t = 0; t < B; ++t) {
-            const int e1 = s_E[t] / 2, e2 = s_E[t] - e1;
+            const int e1 = E[t] / 2, e2 = E[t] - e1;
             pe1[t] = __int_as_float((127 + e1) << 23);
             pe2[t] = __int_as_float((127 + e2) << 23);
         }
-        constexpr int G4 = 2;  // units per thread per batch of loads
-        bool started = false;
-        for (int u0 = tid; u0 < n_units || !started; u0 += G4 * kS1Threads) {
-            float su[G4], sg[G4];
-            uint16_t xh[G4][B];
+        int rank = woffs;
 #pragma unroll
-            for (int k = 0; k < G4; ++k) {
-                const int u = u0 + k * kS1Threads;
-                su[k] = sg[k] = 0.f;
-                if (u < n_units) {
-                    const int i = rowidx[u];
-                    su[k] = a.s_up[i];
-                    sg[k] = a.s_gate[i];
+        for (int k = 0; k < T::KMAX; ++k) {
+            const float sus[8] = {su[k][0].x, su[k][0].y, su[k][0].z, su[k][0].w,
+                                  su[k][1].x, su[k][1].y, su[k][1].z, su[k][1].w};
+            const float sgs[8] = {sg[k][0].x, sg[k][0].y, sg[k][0].z, sg[k][0].w,
+                                  sg[k][1].x, sg[k][1].y, sg[k][1].z, sg[k][1].w};
 #pragma unroll
-                    for (int t = 0; t < B; ++t)
-                        xh[k][t] = (t < a.nb) ? a.x[(size_t)t * a.d + i] : (uint16_t)0;
+            for (int b = 0; b < 8; ++b) {
+                if (!((ub[k] >> b) & 1u)) continue;
+                if (rank >= lo && rank < hi) {
+                    const int u = rank - lo;
+                    rowidx[u] = (tid * K + k) * 8 + b;
+#pragma unroll
+                    for (int t = 0; t < B; ++t) {
+                        const uint32_t w = (b & 1) ? (&xv[k][t].x)[b / 2] & 0xFFFF0000u
+                                                   : (&xv[k][t].x)[b / 2] << 16;
+                        const float xx = ((kb[k][t] >> b) & 1u) ? __uint_as_float(w) : 0.f;
+                        xs[(u * 2 + 0) * B + t] = (xx * sus[b]) * pe1[t] * pe2[t];
+                        xs[(u * 2 + 1) * B + t] = (xx * sgs[b]) * pe1[t] * pe2[t];
+                    }
                 }
-            }
-            if (!started) {
-                load_set(va, 0);
-                load_set(vb, T::U);
-                started = true;
-            }
-#pragma unroll
-            for (int k = 0; k < G4; ++k) {
-                const int u = u0 + k * kS1Threads;
-                if (u >= n_units) break;
-                const int i = rowidx[u];
-#pragma unroll
-                for (int t = 0; t < B; ++t) {
-                    float xv = 0.f;
-                    if ((tmask[t * W + (i >> 5)] >> (i & 31)) & 1u)
-                        xv = __uint_as_float((uint32_t)xh[k][t] << 16);
-                    xs[(u * 2 + 0) * B + t] = (xv * su[k]) * pe1[t] * pe2[t];
-                    xs[(u * 2 + 1) * B + t] = (xv * sg[k]) * pe1[t] * pe2[t];
-                }
+                ++rank;
             }
         }
     }
     __syncthreads();
 
-    // (5) main loop: decode one register set while the other is in flight;
-    // ssum collects this thread's sum of x_i * scale_i * 2^E (+8 code offset)
+    const int rl = tid / T::TPR;
+    const int m = (tid / T::TPRM) & 1;
+    const int chunk = tid % T::TPRM;
+    const uint8_t *qbase = (m ? a.q_gate : a.q_up) +
+                           (size_t)(c0 + chunk / T::TPRB) * a.d * (kCB / 2) +
+                           (chunk % T::TPRB) * T::BYTES;
+    const int n_rows = n_units > rl ? (n_units - rl + T::RL - 1) / T::RL : 0;
     float2 acc2[T::ACC / 2];
 #pragma unroll
     for (int k = 0; k < T::ACC / 2; ++k) acc2[k] = make_float2(0.f, 0.f);
     float ssum[B];
 #pragma unroll
     for (int t = 0; t < B; ++t) ssum[t] = 0.f;
-    auto comp_set = [&](const Vec<T::WORDS>(&v)[T::U], int k0) {
-#pragma unroll
-        for (int j = 0; j < T::U; ++j) {
-            if (k0 + j >= n_rows) break;
-            const int u = rl + (k0 + j) * T::RL;
-            float xv[B];
-#pragma unroll
-            for (int t = 0; t < B; ++t) {
-                xv[t] = xs[(u * 2 + m) * B + t];
-                ssum[t] += xv[t];
-            }
-#pragma unroll
-            for (int q = 0; q < T::WORDS; ++q) proc_word<B, T::CPT>(v[j].w[q], q, xv, acc2);
-        }
-    };
-    for (int k0 = 0; k0 < n_rows; k0 += 2 * T::U) {
-        comp_set(va, k0);
-        load_set(va, k0 + 2 * T::U);
-        comp_set(vb, k0 + T::U);
-        load_set(vb, k0 + 3 * T::U);
-    }
-    __syncthreads();
+    if (a.depth_sel == 0)
+        s1_stream<B, NB, T::DMAX>(qbase, ring, rowidx, xs, rl, m, n_rows, acc2, ssum);
+    else if (a.depth_sel == 1)
+        s1_stream<B, NB, T::DMAX / 2>(qbase, ring, rowidx, xs, rl, m, n_rows, acc2, ssum);
+    else
+        s1_stream<B, NB, T::DMAX / 4>(qbase, ring, rowidx, xs, rl, m, n_rows, acc2, ssum);
+    __syncthreads();  // every thread is done with the ring before it becomes `red`
 
     // (6) reduce row lanes (padded rows: conflict-free both ways), undo the
     // pre-scale and the +8 code offset: this CTA's partial sums in `part`.
@@ -411,7 +446,7 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
                 sacc += row[pos];
                 soff += row[T::CPT];
             }
-            const int e1 = s_E[t] / 2, e2 = s_E[t] - e1;
+            const int e1 = E[t] / 2, e2 = E[t] - e1;
             const float v = (sacc * up1) * up2 - 8.f * soff;  // sum (q + 8 - 8) x s 2^E
             part[(mm * B + t) * T::CW + ch] =
                 v * __int_as_float((127 - e1) << 23) * __int_as_float((127 - e2) << 23);
@@ -502,6 +537,13 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
     }
 }
 
+// deepest ring that fits next to `unit_cap` rows (2 = the shallowest), or -1
+int s1_depth_sel(int d, int B, int NB, int unit_cap) {
+    for (int sel = 0; sel <= 2; ++sel)
+        if (s1_smem(d, B, NB, unit_cap, sel).total <= (size_t)kS2SmemBudget) return sel;
+    return -1;
+}
+
 template <int B, int NB>
 cudaError_t launch1(Stage1Args a, const Stage1Plan &p0, cudaStream_t s) {
     auto k = k_stage1<B, NB>;
@@ -510,7 +552,7 @@ cudaError_t launch1(Stage1Args a, const Stage1Plan &p0, cudaStream_t s) {
     // resident at once, or the last clusters run as a second wave. Start from
     // the plan's choice and shrink until the occupancy calculator agrees.
     struct Cache {
-        int d = 0, C = 0, n_r = 0, cap = 0;
+        int d = 0, C = 0, n_r = 0, cap = 0, sel = 0;
         size_t smem = 0;
     };
     static Cache cache;
@@ -518,17 +560,19 @@ cudaError_t launch1(Stage1Args a, const Stage1Plan &p0, cudaStream_t s) {
     if (cache.d == a.d && cache.C == a.C) {
         p.n_r = cache.n_r;
         p.unit_cap = cache.cap;
+        p.depth_sel = cache.sel;
         p.smem = cache.smem;
     } else {
         // fewest row groups whose rows fit in one CTA's shared memory
         int n_min = 1;
-        while (n_min < kS1MaxRowGroups &&
-               s1_smem(a.d, B, NB, (a.d + n_min - 1) / n_min).total > (size_t)kS2SmemBudget)
+        while (n_min < kS1MaxRowGroups && s1_depth_sel(a.d, B, NB, (a.d + n_min - 1) / n_min) < 0)
             ++n_min;
         if (p.n_r < n_min) p.n_r = n_min;
         for (;;) {
             p.unit_cap = (a.d + p.n_r - 1) / p.n_r;
-            p.smem = s1_smem(a.d, B, NB, p.unit_cap).total;
+            p.depth_sel = s1_depth_sel(a.d, B, NB, p.unit_cap);
+            if (p.depth_sel < 0) return cudaErrorInvalidConfiguration;
+            p.smem = s1_smem(a.d, B, NB, p.unit_cap, p.depth_sel).total;
             cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  (int)p.smem);
             if (e != cudaSuccess) return e;
@@ -554,10 +598,12 @@ cudaError_t launch1(Stage1Args a, const Stage1Plan &p0, cudaStream_t s) {
         cache.C = a.C;
         cache.n_r = p.n_r;
         cache.cap = p.unit_cap;
+        cache.sel = p.depth_sel;
         cache.smem = p.smem;
     }
     a.n_r = p.n_r;
     a.unit_cap = p.unit_cap;
+    a.depth_sel = p.depth_sel;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(groups * a.n_r);
     cfg.blockDim = dim3(kS1Threads);
@@ -587,7 +633,8 @@ cudaError_t launch_stage1(int B, const Stage1Args &a, const Stage1Plan &p, cudaS
 }
 
 size_t stage1_smem_bytes(int d_model, int B, int NB, int unit_cap) {
-    return s1_smem(d_model, B, NB, unit_cap).total;
+    const int sel = s1_depth_sel(d_model, B, NB, unit_cap);
+    return s1_smem(d_model, B, NB, unit_cap, sel < 0 ? 2 : sel).total;
 }
 
 }  // namespace prox

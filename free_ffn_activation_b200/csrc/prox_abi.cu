@@ -65,6 +65,7 @@ Stage1Plan stage1_plan(int d, int f, int B, int num_sms) {
            stage1_smem_bytes(d, B, p.nb_blocks, (d + p.n_r - 1) / p.n_r) > (size_t)kS2SmemBudget)
         ++p.n_r;
     p.unit_cap = (d + p.n_r - 1) / p.n_r;
+    p.depth_sel = 0;  // the launch picks the deepest ring that fits
     p.smem = stage1_smem_bytes(d, B, p.nb_blocks, p.unit_cap);
     return p;
 }

@@ -38,6 +38,7 @@ struct Stage1Plan {
     int nb_blocks;  // column blocks per CTA (1 or 2)
     int n_r;        // row groups = cluster size; grid = C / nb_blocks * n_r
     int unit_cap;   // max units (kept rows) one CTA may own
+    int depth_sel;  // Stage-1 copy ring depth: deepest >> depth_sel rows per thread
     size_t smem;    // dynamic shared memory bytes
 };
 
@@ -65,7 +66,7 @@ WsLayout ws_layout(int d_model, int d_ff, int B);
 // ---------------------------------------------------------------------------
 struct Stage1Args {
     int d, f, nb;                // nb active tokens of this pass (<= B)
-    int C, n_r, unit_cap;
+    int C, n_r, unit_cap, depth_sel;
     const uint16_t *x;           // [nb][d]
     float tau_x, tau_s;
     const uint8_t *q_up, *q_gate;
