@@ -44,7 +44,7 @@ __host__ __device__ constexpr int s1_cpt(int B, int NB) {
     return (B <= 2 && NB == 2) ? 32 : (B <= 4 ? 16 : 8);
 }
 // deepest per-thread ring (rows in flight) and the ring bytes it takes
-__host__ __device__ constexpr int s1_ring_bytes(int B) { return B <= 2 ? 384 : (B == 4 ? 256 : 128); }
+__host__ __device__ constexpr int s1_ring_bytes(int B) { return B <= 2 ? 256 : (B == 4 ? 256 : 128); }
 __host__ __device__ constexpr int s1_dmax(int B, int NB) {
     return s1_ring_bytes(B) / (s1_cpt(B, NB) / 2) < 32 ? s1_ring_bytes(B) / (s1_cpt(B, NB) / 2)
                                                           : 32;
@@ -65,15 +65,19 @@ struct S1 {
     static constexpr int KMAX = (B == 8 ? 4096 : 8192) / 8 / kS1Threads;  // x chunks per thread
 };
 
-// cp.async of BYTES (16, 8 or 4) from global to shared; 16-byte copies skip L1
+// cp.async of BYTES (16, 8 or 4) from global to shared under L2 policy pol;
+// 16-byte copies skip L1
 template <int BYTES>
-__device__ __forceinline__ void cp_async(void *dst, const void *src) {
+__device__ __forceinline__ void cp_async(void *dst, const void *src, uint64_t pol) {
     if constexpr (BYTES == 16) {
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src)
+        asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(
+                         smem_addr(dst)),
+                     "l"(src), "l"(pol)
                      : "memory");
     } else {
-        asm volatile("cp.async.ca.shared.global [%0], [%1], %2;" ::"r"(smem_addr(dst)), "l"(src),
-                     "n"(BYTES)
+        asm volatile("cp.async.ca.shared.global.L2::cache_hint [%0], [%1], %2, %3;" ::"r"(
+                         smem_addr(dst)),
+                     "l"(src), "n"(BYTES), "l"(pol)
                      : "memory");
     }
 }
@@ -181,10 +185,12 @@ __device__ __forceinline__ void s1_stream(const uint8_t *qbase, unsigned char *r
     // consecutive words, free of bank conflicts
     unsigned char *myring = ring + (size_t)threadIdx.x * T::BYTES;
     constexpr int SLOT = kS1Threads * T::BYTES;  // bytes between a thread's slots
+    const uint64_t pol = l2_evict_first();      // each granule is read once per pass
 #pragma unroll 1
     for (int k = 0; k < D; ++k) {
         if (k < n_rows)
-            cp_async<T::BYTES>(myring + k * SLOT, qbase + (size_t)rowidx[rl + k * T::RL] * (kCB / 2));
+            cp_async<T::BYTES>(myring + k * SLOT, qbase + (size_t)rowidx[rl + k * T::RL] * (kCB / 2),
+                               pol);
         cp_commit();
     }
 #pragma unroll 1
@@ -212,7 +218,8 @@ __device__ __forceinline__ void s1_stream(const uint8_t *qbase, unsigned char *r
         for (int q = 0; q < T::WORDS; ++q) proc_word<B, T::CPT>(w[q], q, xv, acc2);
         const int kn = k + D;
         if (kn < n_rows)
-            cp_async<T::BYTES>(myring + slot * SLOT, qbase + (size_t)rowidx[rl + kn * T::RL] * (kCB / 2));
+            cp_async<T::BYTES>(myring + slot * SLOT, qbase + (size_t)rowidx[rl + kn * T::RL] * (kCB / 2),
+                               pol);
         cp_commit();
     }
     cp_wait<0>();

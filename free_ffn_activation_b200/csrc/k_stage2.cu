@@ -176,25 +176,30 @@ __global__ void __launch_bounds__(s2_threads(B), 1) k_stage2(const Stage2Args a)
         }
     }
     __syncthreads();
-    // exclusive scans of the per-block counts, in place (warp 0)
-    if (wid == 0) {
-        for (int t = -1; t < B; ++t) {
-            int carry = 0;
-            int *dst = (t < 0) ? uscan : tscan + t * (C + 1);
-            for (int c0 = 0; c0 < C; c0 += 32) {
-                const int c = c0 + lane;
-                const int v = (c < C) ? dst[c] : 0;
-                int inc = v;
+    // exclusive scans of the per-block counts, in place: warp 0 scans the
+    // union counts, warp 1 + t those of token t. A lane owns the contiguous
+    // counts [lane * per, lane * per + per), so one shuffle scan suffices.
+    if (wid <= B) {
+        int *dst = (wid == 0) ? uscan : tscan + (wid - 1) * (C + 1);
+        const int per = (C + 31) / 32;
+        const int c0 = lane * per;
+        int loc = 0;
+        for (int k = 0; k < per; ++k)
+            if (c0 + k < C) loc += dst[c0 + k];
+        int inc = loc;
 #pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const int n = __shfl_up_sync(0xffffffffu, inc, o);
-                    if (lane >= o) inc += n;
-                }
-                if (c < C) dst[c] = carry + inc - v;
-                carry += __shfl_sync(0xffffffffu, inc, 31);
-            }
-            if (lane == 0) dst[C] = carry;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += n;
         }
+        int run = inc - loc;
+        for (int k = 0; k < per; ++k)
+            if (c0 + k < C) {
+                const int v = dst[c0 + k];
+                dst[c0 + k] = run;
+                run += v;
+            }
+        if (lane == 31) dst[C] = inc;
     }
     __syncthreads();
 
@@ -221,6 +226,7 @@ __global__ void __launch_bounds__(s2_threads(B), 1) k_stage2(const Stage2Args a)
         // ---------------- producer ----------------
         if (lane != 0) return;
         const uint32_t row_bytes = (uint32_t)d * 2;
+        const uint64_t pol = l2_evict_first();  // each weight row is read once per pass
         int issued = 0;
         for (int n = 0; n < n_ch; ++n) {
             const uint32_t e = chan[n];
@@ -235,9 +241,9 @@ __global__ void __launch_bounds__(s2_threads(B), 1) k_stage2(const Stage2Args a)
             const size_t j = e & 0xFFFFFFu;
             uint16_t *dst = stages + (size_t)s * 3 * d;
             mbar_arrive_expect_tx(&full[s], 3 * row_bytes);
-            bulk_g2s(dst, a.w_up + j * d, row_bytes, &full[s]);
-            bulk_g2s(dst + d, a.w_gate + j * d, row_bytes, &full[s]);
-            bulk_g2s(dst + 2 * d, a.w_down + j * d, row_bytes, &full[s]);
+            bulk_g2s_hint(dst, a.w_up + j * d, row_bytes, &full[s], pol);
+            bulk_g2s_hint(dst + d, a.w_gate + j * d, row_bytes, &full[s], pol);
+            bulk_g2s_hint(dst + 2 * d, a.w_down + j * d, row_bytes, &full[s], pol);
         }
         // never leave the CTA with copies in flight
         const int first = issued > NST ? issued - NST : 0;
