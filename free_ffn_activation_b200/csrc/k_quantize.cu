@@ -10,7 +10,8 @@
 // with IEEE fp32 division (__fdiv_rn) and round-half-even (__float2int_rn);
 // an all-zero row gives scale 0 and q 0. Packing (block-tiled, the layout
 // Stage 1 streams): byte m of granule q[c][i] holds channel 256c + 2m in the
-// low nibble and 256c + 2m + 1 in the high nibble, two's complement.
+// low nibble and 256c + 2m + 1 in the high nibble, each stored offset-binary
+// as q + 8 (1..15), which is the form Stage 1's decode consumes directly.
 //
 // Order statistic: the magnitude bit patterns of non-negative IEEE numbers
 // sort like unsigned integers, so the rank-k magnitude is found exactly by
@@ -65,7 +66,7 @@ __global__ void __launch_bounds__(256) k_pack(int d, int f, const uint16_t *__re
             v = __float2int_rn(__fdiv_rn(wv, s));
             v = v > 7 ? 7 : (v < -7 ? -7 : v);
         }
-        out[k / 8] |= (uint32_t)(v & 0xF) << (4 * (k % 8));
+        out[k / 8] |= (uint32_t)(v + 8) << (4 * (k % 8));
     }
     // block-tiled output: q[c][i][0..127] holds channels [256c, 256c + 256) of row i
     const int cblk = j0 / kCB, mbyte = (j0 % kCB + chunk * 32) / 2;

@@ -13,16 +13,18 @@
 // of the kept rows (ranks over the union of the pass's tokens) and streams
 // the granules of BOTH proxies (one read of x serves up and gate, the fused
 // split-N kernel of the blog's "From formula to GPU" section). Each thread
-// keeps two sets of rows of its 16/8/4-byte chunk in flight in registers
-// (load one set while decoding the other), about 64 KB per CTA. The cluster's
+// streams its 16/8/4-byte chunk of successive rows through a private ring of
+// cp.async shared-memory slots (12 rows deep when shared memory allows),
+// about 96 KB in flight per CTA: enough to cover the latency, and the decode
+// starts sooner than behind a deeper ring. The cluster's
 // partial sums meet in distributed shared memory: CTA 0 adds them in rank
 // order, forms s~ = u~ * SiLU(g~), thresholds it and compacts the kept
 // channels into ascending lists, so the result is deterministic.
 //
 // INT4 decode. A nibble n at bits 4p..4p+3 of a word, with every other bit
-// cleared, is the bit pattern of the subnormal float n * 2^(4p-149). One XOR
-// of the whole word with 0x88888888 turns every stored two's complement code q
-// into n = q + 8, then one AND per weight yields an exact float operand; the FMA multiplies it by x_i * scale_i pre-scaled by
+// cleared, is the bit pattern of the subnormal float n * 2^(4p-149). The codes
+// are stored offset-binary (n = q + 8), so one AND per weight yields an exact
+// float operand; the FMA multiplies it by x_i * scale_i pre-scaled by
 // 2^E (E chosen per CTA so sums stay normal). At the end each channel's sum
 // is rescaled by the exact power of two 2^(149 - 4p - E) and the offset
 // 8 * sum(x_i * scale_i) is removed. Nibbles 5..7 of a word are first shifted
@@ -44,7 +46,7 @@ __host__ __device__ constexpr int s1_cpt(int B, int NB) {
     return (B <= 2 && NB == 2) ? 32 : (B <= 4 ? 16 : 8);
 }
 // deepest per-thread ring (rows in flight) and the ring bytes it takes
-__host__ __device__ constexpr int s1_ring_bytes(int B) { return B <= 2 ? 256 : (B == 4 ? 256 : 128); }
+__host__ __device__ constexpr int s1_ring_bytes(int B) { return B <= 2 ? 192 : (B == 4 ? 256 : 128); }
 __host__ __device__ constexpr int s1_dmax(int B, int NB) {
     return s1_ring_bytes(B) / (s1_cpt(B, NB) / 2) < 32 ? s1_ring_bytes(B) / (s1_cpt(B, NB) / 2)
                                                           : 32;
@@ -91,7 +93,7 @@ __device__ __forceinline__ void cp_wait() {
 // the decode above
 __host__ __device__ constexpr int nib_pos(int k) { return k < 5 ? k : k - 3; }
 
-// nibble p of a word already XOR-ed with 0x88888888, as a subnormal float
+// nibble p of a word of offset-binary codes, as a subnormal float
 __device__ __forceinline__ float nib_f(uint32_t wx, int p) {
     return __uint_as_float(wx & (0xFu << (4 * p)));
 }
@@ -100,7 +102,7 @@ __device__ __forceinline__ float nib_f(uint32_t wx, int p) {
 // acc2[(t * CPT + wi * 8 + k) / 2]; it gains xs[t] * code_k * 2^(4 pos(k) - 149)
 template <int B, int CPT>
 __device__ __forceinline__ void proc_word(uint32_t w0, int wi, const float *xs, float2 *acc2) {
-    const uint32_t w = w0 ^ 0x88888888u;  // every two's complement code q -> q + 8
+    const uint32_t w = w0;  // nibbles hold q + 8
     const uint32_t v = w >> 12;
     const float2 d01 = make_float2(nib_f(w, 0), nib_f(w, 1));
     const float2 d23 = make_float2(nib_f(w, 2), nib_f(w, 3));

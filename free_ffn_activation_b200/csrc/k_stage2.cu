@@ -139,47 +139,78 @@ __global__ void __launch_bounds__(s2_threads(B), 1) k_stage2(const Stage2Args a)
     // the per-block counts and the list blocks this CTA most likely owns
     // (those around block g * C / G).
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    // (G is one CTA per SM, so every product below fits in 32 bits)
     const int G = gridDim.x, g = blockIdx.x;
     const int npf = C < kS2Prefetch ? C : kS2Prefetch;
-    int cpf = (int)((long long)g * C / G) - 1;
+    int cpf = g * C / G - 1;
     cpf = cpf < 0 ? 0 : (cpf > C - npf ? C - npf : cpf);
+    // per-token counts only when per-token lists or counts are requested
+    const bool tok = a.idx_s != nullptr || a.count_s != nullptr;
+    constexpr int NT = s2_threads(B);
+    // Warp 0 takes the union counts into registers (4 per lane covers
+    // C <= 128 column blocks; more go through shared memory), every thread a
+    // share of the likely list blocks and, when asked for, of the per-token
+    // counts: all loads of this round trip are issued before any is used.
+    constexpr int PER = 4;
+    const bool creg = C <= 32 * PER;
+    int cnt[PER];
+#pragma unroll
+    for (int k = 0; k < PER; ++k) cnt[k] = 0;
+    if (wid == 0 && creg) {
+#pragma unroll
+        for (int k = 0; k < PER; ++k)
+            if (lane * PER + k < C) cnt[k] = a.ucount[lane * PER + k];
+    }
     {
-        const int ncnt = C * (B + 1), total = ncnt + npf * kCB;
-        constexpr int NT = s2_threads(B);
+        const int nuc = creg ? 0 : C;          // union counts via shared memory
+        const int ntc = tok ? C * B : 0;       // per-token counts
+        const int total = nuc + ntc + npf * kCB;
         for (int base = tid; base < total; base += 4 * NT) {
             uint32_t v[4];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const int k = base + q * NT;
                 v[q] = 0;
-                if (k < C) {
-                    v[q] = (uint32_t)a.ucount[k];
-                } else if (k < ncnt) {
-                    const int c = (k - C) / B, t = (k - C) % B;
-                    v[q] = (uint32_t)a.tcount[c * B + t];
-                } else if (k < total) {
-                    v[q] = a.ulist[(size_t)cpf * kCB + (k - ncnt)];
-                }
+                if (k < nuc) v[q] = (uint32_t)a.ucount[k];
+                else if (k < nuc + ntc) v[q] = (uint32_t)a.tcount[k - nuc];
+                else if (k < total) v[q] = a.ulist[(size_t)cpf * kCB + (k - nuc - ntc)];
             }
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const int k = base + q * NT;
-                if (k < C) {
+                if (k < nuc) {
                     uscan[k] = (int)v[q];
-                } else if (k < ncnt) {
-                    const int c = (k - C) / B, t = (k - C) % B;
+                } else if (k < nuc + ntc) {
+                    const int c = (k - nuc) / B, t = (k - nuc) % B;
                     tscan[t * (C + 1) + c] = (int)v[q];
                 } else if (k < total) {
-                    chanpf[k - ncnt] = v[q];
+                    chanpf[k - nuc - ntc] = v[q];
                 }
             }
         }
     }
     __syncthreads();
-    // exclusive scans of the per-block counts, in place: warp 0 scans the
-    // union counts, warp 1 + t those of token t. A lane owns the contiguous
-    // counts [lane * per, lane * per + per), so one shuffle scan suffices.
-    if (wid <= B) {
+    // Exclusive scans of the per-block counts: warp 0 the union counts (in
+    // registers), warp 1 + t those of token t (in place). A lane owns
+    // contiguous counts, so one shuffle scan suffices.
+    if (wid == 0 && creg) {
+        int loc = 0;
+#pragma unroll
+        for (int k = 0; k < PER; ++k) loc += cnt[k];
+        int inc = loc;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += n;
+        }
+        int run = inc - loc;
+#pragma unroll
+        for (int k = 0; k < PER; ++k) {
+            if (lane * PER + k < C) uscan[lane * PER + k] = run;
+            run += cnt[k];
+        }
+        if (lane == 31) uscan[C] = inc;
+    } else if (wid == 0 || (tok && wid <= B)) {
         int *dst = (wid == 0) ? uscan : tscan + (wid - 1) * (C + 1);
         const int per = (C + 31) / 32;
         const int c0 = lane * per;
@@ -201,25 +232,26 @@ __global__ void __launch_bounds__(s2_threads(B), 1) k_stage2(const Stage2Args a)
             }
         if (lane == 31) dst[C] = inc;
     }
-    __syncthreads();
-
-    const long long U = uscan[C];
-    const int p0 = (int)(U * g / G), p1 = (int)(U * (g + 1) / G);
-    const int n_ch = p1 - p0;
-
-    // this CTA's share of the ascending kept-channel list, into shared memory
-    for (int n = tid; n < n_ch; n += s2_threads(B)) {
-        const int p = p0 + n;
-        int lo = 0, hi = C - 1;  // block cb with uscan[cb] <= p < uscan[cb + 1]
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (uscan[mid] <= p) lo = mid; else hi = mid - 1;
+    // warp 0: this CTA's share of the ascending kept-channel list
+    if (wid == 0) {
+        __syncwarp();
+        const unsigned U = (unsigned)uscan[C];  // <= 2^18 kept channels
+        const int p0 = (int)(U * g / G), p1 = (int)(U * (g + 1) / G);
+        for (int n = lane; n < p1 - p0; n += 32) {
+            const int p = p0 + n;
+            int lo = 0, hi = C - 1;  // block cb with uscan[cb] <= p < uscan[cb + 1]
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (uscan[mid] <= p) lo = mid; else hi = mid - 1;
+            }
+            const int off = p - uscan[lo];
+            chan[n] = (lo >= cpf && lo < cpf + npf) ? chanpf[(lo - cpf) * kCB + off]
+                                                    : a.ulist[(size_t)lo * kCB + off];
         }
-        const int off = p - uscan[lo];
-        chan[n] = (lo >= cpf && lo < cpf + npf) ? chanpf[(lo - cpf) * kCB + off]
-                                                : a.ulist[(size_t)lo * kCB + off];
     }
     __syncthreads();
+    const unsigned U = (unsigned)uscan[C];
+    const int n_ch = (int)(U * (g + 1) / G) - (int)(U * g / G);
     asm volatile("griddepcontrol.launch_dependents;");
 
     if (wid == kNDot + NDOWN) {

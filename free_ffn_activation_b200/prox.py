@@ -307,12 +307,14 @@ def test_set_wait(wait_us: int = 0, skip_position: int = -1) -> None:
 
 
 def untile_proxy(q):
-    """Block-tiled proxy [d_ff/256][d_model][128] -> row-major [d_model][d_ff/2]
-    (the same bytes reordered; numpy arrays or tensors)."""
+    """Block-tiled offset-binary proxy [d_ff/256][d_model][128] -> row-major
+    two's complement nibbles [d_model][d_ff/2] (numpy arrays or tensors):
+    the bytes reordered, and q + 8 turned back into q & 0xF by flipping bit 3
+    of each nibble."""
     C, d, _ = q.shape
     if isinstance(q, torch.Tensor):
-        return q.permute(1, 0, 2).reshape(d, C * 128)
-    return q.transpose(1, 0, 2).reshape(d, C * 128)
+        return q.permute(1, 0, 2).reshape(d, C * 128) ^ 0x88
+    return q.transpose(1, 0, 2).reshape(d, C * 128) ^ 0x88
 
 
 def touched_bytes(d_model: int, d_ff: int, k_x: int, k_s: int) -> int:

@@ -88,7 +88,8 @@ typedef struct prox_layer {
  * streams): q_out is uint8 [d_ff/256][d_model][128]; the 128-byte granule
  * q_out[c][i] holds the codes of row i for channels 256c .. 256c+255, byte m
  * holding channel 256c+2m in its low nibble and 256c+2m+1 in its high
- * nibble, two's complement. A rejected input coordinate i thus skips one
+ * nibble, each nibble holding q + 8 (offset binary, 1..15; 8 for q = 0).
+ * A rejected input coordinate i thus skips one
  * contiguous granule per block. scale_out is fp32 [d_model].
  *   w_cm : device, bf16 [d_ff][d_model] (channel-major, as in prox_layer).
  * Errors: PROX_EINVAL on a null pointer or bad shape.

@@ -121,10 +121,13 @@ def test_quantize_hand_worked_rows(gpu):
         W[i, :8] = vals
     q, s = P.quantize_proxy(to_dev_bf16(np.ascontiguousarray(S.to_bf16(W).T), gpu))
     q, s = q.cpu().numpy(), s.cpu().numpy()
+    # the device stores q + 8 block-tiled; the golden bytes are two's complement rows
+    assert bytes(q[0, 0, :4]) == bytes(b ^ 0x88 for b in rows[0][2])
+    qt = P.untile_proxy(q)
     for i, (_, sbits, packed) in enumerate(rows):
         assert int(s[i:i + 1].view(np.uint32)[0]) == sbits
-        assert bytes(q[0, i, :4]) == packed       # granule (block 0, row i)
-    assert not s[len(rows):].any() and not q[:, len(rows):].any()
+        assert bytes(qt[i, :4]) == packed
+    assert not s[len(rows):].any() and not qt[len(rows):].any()
 
 
 def test_quantize_bit_exact_c2(c2):
