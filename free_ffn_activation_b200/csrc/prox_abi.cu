@@ -302,6 +302,52 @@ PROX_API prox_status prox_ffn_forward(const prox_layer *layer, const uint16_t *x
                        ws, ws_bytes, (cudaStream_t)stream, true);
 }
 
+// Allocation-free forward: the workspace is one file-scope device array per
+// device, looked up once per device (see prox_ffn_forward_static in prox.h).
+namespace prox {
+constexpr size_t kStaticWsBytes = PROX_STATIC_WORKSPACE_BYTES;
+static __device__ __align__(256) unsigned char g_static_ws[kStaticWsBytes];
+static void *g_static_ptr[64];
+static std::mutex g_static_mu;
+
+static prox_status static_workspace(void **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return PROX_ECUDA;
+    if (dev < 0 || dev >= 64) return PROX_EDEVICE;
+    std::lock_guard<std::mutex> lk(g_static_mu);
+    if (!g_static_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_ws) != cudaSuccess || !p) return PROX_ECUDA;
+        g_static_ptr[dev] = p;
+    }
+    *out = g_static_ptr[dev];
+    return PROX_OK;
+}
+}  // namespace prox
+
+PROX_API prox_status prox_ffn_forward_static(const prox_layer *layer, const uint16_t *x,
+                                             int batch, float tau_x, float tau_s, float *y,
+                                             uint8_t *mask_x, uint8_t *mask_s, int32_t *idx_s,
+                                             int32_t *count_s, void *stream) {
+    prox_status ps = check_layer(layer, true);
+    if (ps != PROX_OK) return ps;
+    if (batch < 0 || !tau_ok(tau_x) || !tau_ok(tau_s)) return PROX_EINVAL;
+    if (batch == 0) return PROX_OK;
+    if (!x || !y || !aligned16(x) || !aligned16(y)) return PROX_EINVAL;
+    if (!aligned16(mask_x) || !aligned16(mask_s) || !aligned16(idx_s) || !aligned16(count_s))
+        return PROX_EINVAL;
+    const int d = layer->d_model, f = layer->d_ff;
+    if (ws_layout(d, f, tokens_per_pass(d, batch)).total > kStaticWsBytes) return PROX_ENOMEM;
+    int sms = 0;
+    ps = current_device(&sms);
+    if (ps != PROX_OK) return ps;
+    void *ws = nullptr;
+    ps = static_workspace(&ws);
+    if (ps != PROX_OK) return ps;
+    return run_forward(layer, x, batch, tau_x, tau_s, y, mask_x, mask_s, idx_s, count_s, nullptr,
+                       ws, kStaticWsBytes, (cudaStream_t)stream, true);
+}
+
 PROX_API int prox_max_batch_per_pass(int d_model) { return max_tokens_per_pass(d_model); }
 
 PROX_API prox_status prox_ffn_stage1(const prox_layer *layer, const uint16_t *x, int batch,

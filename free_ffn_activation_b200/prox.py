@@ -56,6 +56,8 @@ def lib() -> C.CDLL:
         L.prox_workspace_bytes.argtypes = [i, i, i]
         L.prox_workspace_bytes.restype = sz
         L.prox_ffn_forward.argtypes = [C.POINTER(_Layer), vp, i, f, f, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.prox_ffn_forward_static.argtypes = [C.POINTER(_Layer), vp, i, f, f, vp, vp, vp, vp,
+                                               vp, vp]
         L.prox_proxy_state.argtypes = [C.POINTER(_Layer), vp, i, f, vp, vp, vp, sz, vp]
         L.prox_calibrate_workspace_bytes.argtypes = [i, i, i]
         L.prox_calibrate_workspace_bytes.restype = sz
@@ -71,7 +73,8 @@ def lib() -> C.CDLL:
         L.prox_ffn_stage2.argtypes = [C.POINTER(_Layer), vp, i, vp, vp, vp, vp, sz, vp]
         L.prox_test_set_wait.argtypes = [C.c_uint32, i]
         L.prox_test_set_wait.restype = None
-        for name in ("prox_quantize_proxy", "prox_ffn_forward", "prox_proxy_state",
+        for name in ("prox_quantize_proxy", "prox_ffn_forward", "prox_ffn_forward_static",
+                     "prox_proxy_state",
                      "prox_ffn_stage1", "prox_ffn_stage2",
                      "prox_calibrate", "prox_allocate", "prox_last_device_status"):
             getattr(L, name).restype = C.c_int
@@ -224,6 +227,32 @@ def ffn_forward(layer: ProxLayer, x: torch.Tensor, tau_x: float, tau_s: float,
     return out
 
 
+def ffn_forward_static(layer: ProxLayer, x: torch.Tensor, tau_x: float, tau_s: float,
+                       *, want_masks: bool = True) -> ForwardOut:
+    """prox_ffn_forward_static: the forward on the library's static workspace."""
+    d, f = layer.d_model, layer.d_ff
+    if x.dim() == 1:
+        x = x.unsqueeze(0)
+    b = x.shape[0]
+    _need(x, torch.bfloat16, (b, d), "x")
+    dev = x.device
+    out = ForwardOut(
+        y=torch.empty((b, d), dtype=torch.float32, device=dev),
+        mask_x=torch.empty((b, d), dtype=torch.uint8, device=dev) if want_masks else None,
+        mask_s=torch.empty((b, f), dtype=torch.uint8, device=dev) if want_masks else None,
+        idx_s=torch.empty((b, f), dtype=torch.int32, device=dev) if want_masks else None,
+        count_s=torch.empty((b,), dtype=torch.int32, device=dev) if want_masks else None)
+    cl = layer.cstruct()
+    _check(lib().prox_ffn_forward_static(C.byref(cl), _ptr(x), b, float(tau_x), float(tau_s),
+                                         _ptr(out.y), _ptr(out.mask_x), _ptr(out.mask_s),
+                                         _ptr(out.idx_s), _ptr(out.count_s), _stream(dev)),
+           "prox_ffn_forward_static")
+    return out
+
+
+STATIC_WORKSPACE_BYTES = 2 << 20  # PROX_STATIC_WORKSPACE_BYTES
+
+
 def ffn_forward_raw(layer_struct: _Layer, x_ptr: int, batch: int, tau_x: float, tau_s: float,
                     y_ptr: int, ws_ptr: int, ws_bytes: int, stream: int, mask_x=None,
                     mask_s=None, idx_s=None, count_s=None) -> None:
@@ -324,6 +353,7 @@ def touched_bytes(d_model: int, d_ff: int, k_x: int, k_s: int) -> int:
 
 
 __all__ = ["ProxLayer", "ProxError", "quantize_proxy", "workspace", "workspace_bytes",
-           "ffn_forward", "ffn_forward_raw", "ffn_stage1_raw", "ffn_stage2_raw",
+           "ffn_forward", "ffn_forward_static", "STATIC_WORKSPACE_BYTES", "ffn_forward_raw",
+           "ffn_stage1_raw", "ffn_stage2_raw",
            "max_batch_per_pass", "proxy_state", "calibrate", "allocate",
            "last_device_status", "touched_bytes", "untile_proxy", "as_bf16"]

@@ -133,6 +133,39 @@ prox_status prox_ffn_forward(const prox_layer *layer, const uint16_t *x, int bat
                              void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * prox_ffn_forward_static -- prox_ffn_forward without a caller workspace: the
+ * library's own workspace is one file-scope device array of
+ * PROX_STATIC_WORKSPACE_BYTES (2 MiB) per device, so the call allocates
+ * nothing (no cudaMalloc/cudaFree, no allocating library). The Prox pages
+ * have no counterpart of this entry point; it is for callers that cannot
+ * allocate or hold device memory of their own, such as plain-C hosts with no
+ * device allocator, or serving loops that must not call cudaMalloc/cudaFree
+ * (both can synchronise the device) in steady state.
+ *   Arguments, arithmetic and results as in prox_ffn_forward, minus ws.
+ *   Limit: shapes with prox_workspace_bytes(d_model, d_ff, batch) above
+ *     PROX_STATIC_WORKSPACE_BYTES are rejected with PROX_ENOMEM (for example
+ *     d_model 4096 x d_ff 12288 fits at any batch; d_ff 262144 does not).
+ *   Setup: the first call on a device looks the array up
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     outside any stream capture. Later calls only launch kernels.
+ *   Sharing: every call on a device uses the same array, so calls must not
+ *     overlap on the device (one stream, or ordered by the caller); two
+ *     overlapping calls race on it.
+ *   Zero state: the array starts zero-filled (static device storage). The
+ *     only part that must be zero at a call's start is the status word, which
+ *     the kernels set only when a bounded wait gives up; such a timeout is not
+ *     reported here (use prox_ffn_forward with prox_last_device_status to
+ *     observe timeouts).
+ * Errors: as prox_ffn_forward; PROX_ENOMEM for a shape over the limit;
+ * PROX_ECUDA if the symbol lookup fails.
+ */
+#define PROX_STATIC_WORKSPACE_BYTES ((size_t)2 << 20)
+prox_status prox_ffn_forward_static(const prox_layer *layer, const uint16_t *x, int batch,
+                                    float tau_x, float tau_s, float *y, uint8_t *mask_x,
+                                    uint8_t *mask_s, int32_t *idx_s, int32_t *count_s,
+                                    void *stream);
+
+/*
  * prox_max_batch_per_pass -- tokens one Stage-1/Stage-2 pass handles for this
  * d_model (8 up to d_model 4096, 4 up to 8192, 0 beyond: unsupported).
  * prox_ffn_forward splits larger batches into passes by itself.
