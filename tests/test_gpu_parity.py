@@ -64,6 +64,15 @@ def c2(gpu):
     return Case(4096, 12288, 512, 512, outlier=0.001)
 
 
+@pytest.fixture(scope="module")
+def c4(gpu):
+    # large layer: d_model 8192, d_ff 28672, N(0, 0.015^2) weights, Laplace
+    # tokens; thresholds from 64 calibration vectors (the shape is what this
+    # case tests: 2-CTA clusters, two coordinate chunks per thread, a 3-stage
+    # Stage-2 ring, passes of 4 tokens)
+    return Case(8192, 28672, 32, 64, sigma=0.015)
+
+
 def check_forward(case, rows, out, tag=""):
     """Compare a device ForwardOut for tokens `rows` with the oracle."""
     x = case.x[rows]
@@ -213,6 +222,22 @@ def test_forward_c2_batched(c2, b):
     rows = list(range(10, 10 + b))
     out = P.ffn_forward(c2.layer, c2.xdev(rows), c2.tau_x, c2.tau_s)
     check_forward(c2, rows, out, f" c2 b={b}")
+
+
+def test_forward_c4_sampled_b1(c4):
+    ws = P.workspace(8192, 28672, 1)
+    rows = [0, 7, 31]
+    outs = [P.ffn_forward(c4.layer, c4.xdev([t]), c4.tau_x, c4.tau_s, ws) for t in rows]
+    merged = P.ForwardOut(*(torch.cat([getattr(o, k) for o in outs]) for k in
+                            ("y", "mask_x", "mask_s", "idx_s", "count_s")))
+    check_forward(c4, rows, merged, " c4 b=1")
+
+
+def test_forward_c4_batched_b16(c4):
+    # batch 16 runs as four passes of 4 tokens, each token with its own masks
+    rows = list(range(16))
+    out = P.ffn_forward(c4.layer, c4.xdev(rows), c4.tau_x, c4.tau_s)
+    check_forward(c4, rows, out, " c4 b=16")
 
 
 def test_zero_thresholds_dense(c1):
