@@ -61,9 +61,12 @@ def parse():
     return ap.parse_args()
 
 
-def stage2_traffic():
+def stage2_traffic(workload, batch):
     """DRAM bytes per launch of the Stage-2 kernel from the committed ncu summary,
-    if it was captured from the current kernel source (else None)."""
+    if it covers this workload and was captured from the current kernel source
+    (else None)."""
+    if workload != "qwen3-8b-ffn" or batch != 1:
+        return None
     import hashlib
     src = os.path.join(ROOT, "free_ffn_activation_b200", "csrc", "k_stage2.cu")
     summ = os.path.join(ROOT, "profiles", "k_stage2_qwen3-8b-ffn_b1.md")
@@ -425,7 +428,7 @@ def run_ours(args, w, rank, world, local_rank):
                        "parallelism": f"replicas x{world}"},
             "roofline": {"bound": "hbm", "kernel": "k_stage2 (exact up/gate/down)",
                          "achieved": s2_gbs, "peak": peak, "unit": "GB/s",
-                         "frac": s2_gbs / peak, "traffic": stage2_traffic(), "peak_source": peak_src,
+                         "frac": s2_gbs / peak, "traffic": stage2_traffic(args.workload, Bt), "peak_source": peak_src,
                          "bytes_per_launch": s2_bytes, "us_per_launch": s2_us},
             "stage1": {"kernel": "k_stage1 (INT4 proxy + channel mask)", "us_per_launch": s1_us,
                        "bytes_per_launch": s1_bytes, "GBps": s1_gbs, "frac": s1_gbs / peak},
