@@ -68,6 +68,8 @@ def _declare(L):
     L.oracle_calibrate.argtypes = [i, i, i, _u16p, _u8p, _f32p, _u8p, _f32p, d, d,
                                    C.POINTER(C.c_float), C.POINTER(C.c_float), i]
     L.oracle_calibrate.restype = None
+    L.oracle_rmsnorm_bf16.argtypes = [i, _f32p, d, _u16p]
+    L.oracle_rmsnorm_bf16.restype = None
     L.oracle_allocate.argtypes = [d, d, d, d, C.POINTER(C.c_double), C.POINTER(C.c_double)]
     L.oracle_allocate.restype = None
     L.oracle_effective_sparsity.argtypes = [d, d, d]
@@ -157,6 +159,15 @@ def calibrate(x_cal, proxy: dict, keep_x: float, keep_s: float, n_threads=0):
                            proxy["q_gate"], proxy["s_gate"], float(keep_x), float(keep_s),
                            C.byref(tx), C.byref(ts), int(n_threads))
     return tx.value, ts.value
+
+
+def rmsnorm_bf16(h, eps: float = 1e-6) -> np.ndarray:
+    """Stack pre-norm: bf16 bits of h / sqrt(mean(h^2) + eps) per row of h (fp32)."""
+    h = np.ascontiguousarray(np.atleast_2d(h), dtype=np.float32)
+    out = np.empty(h.shape, dtype=np.uint16)
+    for t in range(h.shape[0]):
+        lib().oracle_rmsnorm_bf16(h.shape[1], h[t], float(eps), out[t])
+    return out
 
 
 def allocate(e: float, alpha: float = 1.0 / 3.0, s1_max: float = 0.7,

@@ -340,3 +340,39 @@ double oracle_effective_sparsity(double s1, double s2, double alpha)
 {
     return s2 - 2.0 * alpha * (1.0 - s1) / 3.0;
 }
+
+/*
+ * Layer stack (the stacked-layer benchmark built on the Prox FFN; not on the
+ * Prox pages): pre-norm, h <- h + FFN(RMSNorm(h)), RMSNorm(h) = h /
+ * sqrt(mean(h^2) + eps) with unit gain, the FFN input rounded to bf16.
+ */
+
+/* nearest bf16 to v, ties to even, as a bit pattern (finite v in range) */
+static uint16_t bf16_round(double v)
+{
+    if (v == 0.0)
+        return (uint16_t)(signbit(v) ? 0x8000u : 0u);
+    int e;
+    frexp(fabs(v), &e);                 /* |v| in [2^(e-1), 2^e) */
+    int qexp = e - 8;                   /* 8 significant bits */
+    if (qexp < -133)
+        qexp = -133;                    /* bf16 subnormal spacing */
+    const double q = ldexp(1.0, qexp);
+    const double r = nearbyint(fabs(v) / q) * q;    /* default mode: ties to even */
+    const float f = (float)(signbit(v) ? -r : r);   /* exact: <= 8 significant bits */
+    uint32_t bits;
+    memcpy(&bits, &f, sizeof bits);
+    return (uint16_t)(bits >> 16);
+}
+
+/* one token: x = bf16(h / sqrt(mean(h^2) + eps)), h read exactly */
+void oracle_rmsnorm_bf16(int d, const float *h, double eps, uint16_t *x_out)
+{
+    double ss = 0.0;
+    for (int i = 0; i < d; ++i)
+        ss += (double)h[i] * (double)h[i];
+    const double rms = sqrt(ss / (double)d + eps);
+    for (int i = 0; i < d; ++i)
+        x_out[i] = bf16_round((double)h[i] / rms);
+}
+

@@ -35,6 +35,9 @@ MUTANTS = {
                   "double r = ceil((1.0 - keep) * (double)n);"),
     "budget_term": ("s2 = e + 2.0 * alpha * (1.0 - s1) / 3.0;",
                     "s2 = e + alpha * (1.0 - s1) / 3.0;"),
+    "rms_sum_not_mean": ("sqrt(ss / (double)d + eps)", "sqrt(ss + eps)"),
+    "rms_eps_dropped": ("sqrt(ss / (double)d + eps)", "sqrt(ss / (double)d)"),
+    "bf16_truncates": ("nearbyint(fabs(v) / q) * q", "floor(fabs(v) / q) * q"),
 }
 
 

@@ -329,3 +329,45 @@ def test_budget_split_matches_printed_value():
         assert 0.0 <= s1 <= 0.7 + 1e-12
         cost = 2 * (1 / 3) * (1 - s1) + 3 * (1 - s2)
         assert 1 - cost / 3 == pytest.approx(e, abs=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# Stack pre-norm (the stacked-layer benchmark on top of the Prox FFN; not on
+# the Prox pages): x = bf16(h / sqrt(mean(h^2) + eps)), unit gain
+# ---------------------------------------------------------------------------
+
+def _bf16_bits(v):
+    return int(np.array([v], np.float32).view(np.uint32)[0] >> 16)
+
+
+def test_rmsnorm_closed_forms():
+    # one nonzero coordinate: mean(h^2) = 1 for h = (2, 0, 0, 0), so x = h
+    x = oracle.rmsnorm_bf16(np.array([[2, 0, 0, 0]], np.float32), eps=0.0)
+    assert x.tolist() == [[_bf16_bits(2.0), 0, 0, 0]]
+    # a constant c with eps = 3 c^2: x = c / sqrt(4 c^2) = 1/2, any d and c
+    for c, d in [(3.0, 8), (0.125, 16), (-5.0, 4)]:
+        x = oracle.rmsnorm_bf16(np.full((1, d), c, np.float32), eps=3 * c * c)
+        assert (x == _bf16_bits(0.5 if c > 0 else -0.5)).all()
+    # alternating signs of one magnitude normalise to +-1 exactly
+    h = np.array([[7, -7, 7, -7, 7, -7]], np.float32)
+    assert oracle.rmsnorm_bf16(h, eps=0.0).tolist() == [[_bf16_bits(v) for v in (1, -1) * 3]]
+
+
+def test_rmsnorm_scale_invariance():
+    # with eps = 0 the norm is invariant under exact (power-of-two) scaling
+    rng = np.random.default_rng(3)
+    h = rng.standard_normal((4, 256)).astype(np.float32)
+    a = oracle.rmsnorm_bf16(h, eps=0.0)
+    for k in (0.25, 8.0, 1024.0):
+        assert np.array_equal(oracle.rmsnorm_bf16(h * np.float32(k), eps=0.0), a)
+
+
+def test_rmsnorm_ties_to_even_and_eps():
+    # eps chosen so that mean(h^2) + eps = 1 exactly: x is h rounded to bf16,
+    # and 1 + 2^-8, 1 + 3 * 2^-8 sit exactly halfway between bf16 neighbours
+    t0, t1 = 1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8
+    h = np.array([[t0, t1, -t0, 0.5]], np.float32)
+    eps = 1.0 - float(np.mean(h.astype(np.float64) ** 2))
+    x = oracle.rmsnorm_bf16(h, eps=eps)
+    assert x.tolist() == [[_bf16_bits(1.0), _bf16_bits(1.0 + 2.0 ** -6),
+                           _bf16_bits(-1.0), _bf16_bits(0.5)]]
