@@ -40,6 +40,10 @@ WORKLOADS = {
     "qwen3-8b-ffn": dict(d=4096, f=12288, sigma=0.02, tokens=512, n_cal=512, outlier=0.001),
     "tiny-ffn": dict(d=256, f=768, sigma=0.02, tokens=64, n_cal=256, outlier=0.0),
     "large-ffn": dict(d=8192, f=28672, sigma=0.015, tokens=256, n_cal=256, outlier=0.0),
+    # 36 pre-norm layers (RMSNorm eps 1e-6, unit gain, fp32 residual stream),
+    # each with its own weights and depth-sequentially calibrated thresholds
+    "qwen3-8b-stack36": dict(d=4096, f=12288, sigma=0.02, tokens=128, n_cal=128, outlier=0.0,
+                             layers=36),
 }
 
 
@@ -447,6 +451,181 @@ def run_ours(args, w, rank, world, local_rank):
     del g, gi
 
 
+def run_stack(args, w, rank, world, local_rank):
+    """A step is `tokens` decode tokens, each through all layers of the stack
+    (prox_ffn_block per layer: pre-norm, Prox FFN, residual add). The whole
+    stack is far larger than L2, so every layer streams from HBM."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from free_ffn_activation_b200 import prox as P
+    from free_ffn_activation_b200 import synth as S
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    d, f, ntok, nl = w["d"], w["f"], w["tokens"], w["layers"]
+    eps = 1e-6
+    layers = []
+    for ell in range(nl):
+        L = S.make_layer(S.LayerSpec(d, f, sigma=w["sigma"], seed=0, layer=ell))
+        layers.append(P.ProxLayer.from_weights(L["w_up_cm"], L["w_gate_cm"], L["w_down"],
+                                               device=dev))
+        del L
+    structs = [lay.cstruct() for lay in layers]
+    # thresholds, depth-sequentially: layer l's from the calibration vectors
+    # after layers 0..l-1 (each layer keeps 50% of inputs and 30% of channels)
+    h_cal = torch.from_numpy(S.bf16_to_f32(S.make_tokens(w["n_cal"], d, seed=0,
+                                                          stream="x_cal"))).to(dev)
+    taus = []
+    for lay in layers:
+        tx, ts = P.calibrate(lay, P.rmsnorm_bf16(h_cal, eps), args.keep_x, args.keep_s)
+        taus.append((tx, ts))
+        P.ffn_block(lay, h_cal, tx, ts, eps, h_out=h_cal, want_masks=False)
+    h0 = torch.from_numpy(S.bf16_to_f32(S.make_tokens(ntok, d, seed=rank,
+                                                       stream="x_eval"))).to(dev)
+    h = torch.empty_like(h0)
+    xbuf = torch.empty((ntok, d), dtype=torch.bfloat16, device=dev)
+    ws = P.workspace(d, f, 1, dev)
+    wsb, wp = ws.numel(), ws.data_ptr()
+    stream = torch.cuda.Stream(dev)
+    sp = stream.cuda_stream
+    hrow, xrow = d * 4, d * 2
+
+    def one_step():
+        h.copy_(h0)
+        for t in range(ntok):
+            hp, xp = h.data_ptr() + t * hrow, xbuf.data_ptr() + t * xrow
+            for ell in range(nl):
+                P.ffn_block_raw(structs[ell], hp, 1, taus[ell][0], taus[ell][1], eps, hp, xp,
+                                wp, wsb, sp)
+
+    with torch.cuda.stream(stream):
+        one_step()
+    torch.cuda.synchronize(dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        one_step()
+    for _ in range(args.warmup):
+        with torch.cuda.stream(stream):
+            g.replay()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            with torch.cuda.stream(stream):
+                g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+    ms_total = e0.elapsed_time(e1)
+    if world > 1:
+        tt = torch.tensor([ms_total], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_total = float(tt.item())
+    ms_step = ms_total / args.steps
+    us_tok = ms_step * 1e3 / ntok                     # all layers, per token (per rank)
+    # touched bytes: realised keep ratios of the last step's tokens, layer by layer
+    hh = h0.clone()
+    touched = 0.0
+    for ell, lay in enumerate(layers):
+        hh, _, out = P.ffn_block(lay, hh, taus[ell][0], taus[ell][1], eps)
+        kx = out.mask_x.sum(dim=1).double().mean().item()
+        ks = out.count_s.double().mean().item()
+        touched += P.touched_bytes(d, f, int(round(kx)), int(round(ks)))
+    peak, peak_src = load_peaks()
+    path_gbs = touched / (us_tok * 1e-6) / 1e9
+
+    # e2e: host h in, host h out, the public call per layer
+    h_host = h0.cpu().pin_memory()
+    out_host = torch.empty((ntok, d), dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        with torch.cuda.stream(stream):
+            h.copy_(h_host, non_blocking=True)
+            for t in range(ntok):
+                hp, xp = h.data_ptr() + t * hrow, xbuf.data_ptr() + t * xrow
+                for ell in range(nl):
+                    P.ffn_block_raw(structs[ell], hp, 1, taus[ell][0], taus[ell][1], eps, hp,
+                                    xp, wp, wsb, sp)
+            out_host.copy_(h, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    f0 = torch.cuda.Event(enable_timing=True)
+    f1 = torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    e2e_step()
+    f1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_us = f0.elapsed_time(f1) * 1e3 / ntok
+
+    dense = None
+    if not args.no_dense:
+        import torch.nn.functional as F
+        wd_t = [lay.w_down.t().contiguous() for lay in layers]
+        hd = torch.empty_like(h0)
+
+        def dense_step():
+            hd.copy_(h0)
+            for t in range(ntok):
+                ht = hd[t:t + 1]
+                for ell, lay in enumerate(layers):
+                    xt = (ht * torch.rsqrt(ht.pow(2).mean(dim=1, keepdim=True) + eps)).to(torch.bfloat16)
+                    u = F.linear(xt, lay.w_up_cm)
+                    gg = F.linear(xt, lay.w_gate_cm)
+                    ht.add_(F.linear(F.silu(gg) * u, wd_t[ell]).float())
+
+        with torch.cuda.stream(stream):
+            dense_step()
+        torch.cuda.synchronize(dev)
+        gd = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gd, stream=stream):
+            dense_step()
+        for _ in range(args.warmup):
+            with torch.cuda.stream(stream):
+                gd.replay()
+        torch.cuda.synchronize(dev)
+        d0 = torch.cuda.Event(enable_timing=True)
+        d1 = torch.cuda.Event(enable_timing=True)
+        d0.record(stream)
+        for _ in range(args.steps):
+            with torch.cuda.stream(stream):
+                gd.replay()
+        d1.record(stream)
+        torch.cuda.synchronize(dev)
+        dense_us = d0.elapsed_time(d1) / args.steps * 1e3 / ntok
+        dense = {"us_per_token": dense_us, "speedup_of_sparse": dense_us / us_tok,
+                 "kind": "torch RMSNorm + F.linear x3 + silu*mul (cuBLAS), bf16, same protocol"}
+        del gd
+
+    if rank == 0:
+        line = {
+            "metric": "sparse SwiGLU FFN stack µs/token (all layers) @70% sparsity",
+            "value": ms_step * 1e3 / (ntok * world),
+            "unit": "us/token", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_step, "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": args.workload, "layers": nl, "d_model": d, "d_ff": f,
+                       "batch": 1, "tokens_per_step": ntok, "keep_x": args.keep_x,
+                       "keep_s": args.keep_s, "rmsnorm_eps": eps,
+                       "l2": f"{nl} distinct layers ({nl * (3 * d * f * 2 + d * f + 8 * d) / 1e9:.1f} GB > L2)",
+                       "parallelism": f"replicas x{world}"},
+            "us_per_layer": us_tok / nl,
+            "path": {"touched_MB_per_token": touched / 1e6, "GBps": path_gbs,
+                     "frac_of_peak": path_gbs / peak, "peak_source": peak_src},
+            "dense_ref": dense,
+            "e2e": {"value": e2e_us, "unit": "us/token", "h2d_bytes_per_step": ntok * d * 4,
+                    "d2h_bytes_per_step": ntok * d * 4},
+            "gpu_launches": 3 * nl * ntok * args.steps,
+            "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     w = WORKLOADS[args.workload]
@@ -454,6 +633,11 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
+        if "layers" in w:
+            if rank == 0:
+                print(json.dumps({"impl": "reference", "unavailable":
+                                  "the layer stack has no CPU-oracle arm (single-layer workloads have one)"}))
+            return
         run_reference(args, w, rank, world)
         return
     if world > 1:
@@ -464,7 +648,10 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
-        run_ours(args, w, rank, world, local_rank)
+        if "layers" in w:
+            run_stack(args, w, rank, world, local_rank)
+        else:
+            run_ours(args, w, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist

@@ -263,12 +263,14 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;");
 
-    // (1) Stage 2 accumulates y with atomics: clear it here.
+    // (1) Stage 2 accumulates y with atomics: clear it here (or start it
+    // from y_init, the residual stream of a layer stack).
     if (a.y_zero) {
         float4 *y4 = reinterpret_cast<float4 *>(a.y_zero);
+        const float4 *i4 = reinterpret_cast<const float4 *>(a.y_init);
         const int n4 = a.nb * a.d / 4;
         for (int k = blockIdx.x * kS1Threads + tid; k < n4; k += gridDim.x * kS1Threads)
-            y4[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+            y4[k] = i4 ? i4[k] : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 
     // (2) input masks m_x = 1[|x_i| >= tau_x] per token. Thread tid owns the K

@@ -167,7 +167,7 @@ static int g_debug_skip = -1;
 static prox_status pass_stage1(const prox_layer *L, const uint16_t *x, int nb, float tau_x,
                                float tau_s, float *y_clear, uint8_t *mask_x, uint8_t *mask_s,
                                float *s_out, unsigned char *w, int sms, bool lists,
-                               cudaStream_t st) {
+                               const float *y_init, cudaStream_t st) {
     const int d = L->d_model, f = L->d_ff;
     const int B = pow2_ceil(nb);
     const WsLayout W = ws_layout(d, f, B);
@@ -187,6 +187,7 @@ static prox_status pass_stage1(const prox_layer *L, const uint16_t *x, int nb, f
     a.s_up = L->s_up;
     a.s_gate = L->s_gate;
     a.y_zero = y_clear;
+    a.y_init = y_clear ? y_init : nullptr;
     a.mask_x = mask_x;
     a.mask_s = mask_s;
     a.s_out = s_out;
@@ -239,7 +240,8 @@ static prox_status pass_stage2(const prox_layer *L, const uint16_t *x, int nb, f
 static prox_status run_forward(const prox_layer *L, const uint16_t *x, int batch, float tau_x,
                                float tau_s, float *y, uint8_t *mask_x, uint8_t *mask_s,
                                int32_t *idx_s, int32_t *count_s, float *s_out, void *ws,
-                               size_t ws_bytes, cudaStream_t st, bool stage2) {
+                               size_t ws_bytes, cudaStream_t st, bool stage2,
+                               const float *y_init = nullptr) {
     int sms = 0;
     prox_status ps = current_device(&sms);
     if (ps != PROX_OK) return ps;
@@ -253,7 +255,8 @@ static prox_status run_forward(const prox_layer *L, const uint16_t *x, int batch
         ps = pass_stage1(L, xt, nb, tau_x, tau_s, stage2 ? y + (size_t)t0 * d : nullptr,
                          mask_x ? mask_x + (size_t)t0 * d : nullptr,
                          mask_s ? mask_s + (size_t)t0 * f : nullptr,
-                         s_out ? s_out + (size_t)t0 * f : nullptr, w, sms, stage2, st);
+                         s_out ? s_out + (size_t)t0 * f : nullptr, w, sms, stage2,
+                         y_init ? y_init + (size_t)t0 * d : nullptr, st);
         if (ps != PROX_OK || !stage2) {
             if (ps != PROX_OK) return ps;
             continue;
@@ -348,6 +351,46 @@ PROX_API prox_status prox_ffn_forward_static(const prox_layer *layer, const uint
                        ws, kStaticWsBytes, (cudaStream_t)stream, true);
 }
 
+static bool eps_ok(float e) { return std::isfinite(e) && e >= 0.f; }
+
+PROX_API prox_status prox_rmsnorm_bf16(int d_model, int batch, const float *h, float eps,
+                                       uint16_t *x_out, void *stream) {
+    if (d_model < 256 || d_model % 256 != 0 || batch < 0 || !eps_ok(eps)) return PROX_EINVAL;
+    if (batch == 0) return PROX_OK;
+    if (!h || !x_out || !aligned16(h) || !aligned16(x_out)) return PROX_EINVAL;
+    int sms = 0;
+    prox_status ps = current_device(&sms);
+    if (ps != PROX_OK) return ps;
+    return launch_rmsnorm(d_model, batch, h, eps, x_out, (cudaStream_t)stream) == cudaSuccess
+               ? PROX_OK
+               : PROX_ECUDA;
+}
+
+PROX_API prox_status prox_ffn_block(const prox_layer *layer, const float *h_in, int batch,
+                                    float tau_x, float tau_s, float eps, float *h_out,
+                                    uint16_t *x_out, uint8_t *mask_x, uint8_t *mask_s,
+                                    int32_t *idx_s, int32_t *count_s, void *ws, size_t ws_bytes,
+                                    void *stream) {
+    prox_status ps = check_layer(layer, true);
+    if (ps != PROX_OK) return ps;
+    if (batch < 0 || !tau_ok(tau_x) || !tau_ok(tau_s) || !eps_ok(eps)) return PROX_EINVAL;
+    if (batch == 0) return PROX_OK;
+    if (!h_in || !h_out || !x_out || !ws || !aligned16(h_in) || !aligned16(h_out) ||
+        !aligned16(x_out) || !aligned16(ws))
+        return PROX_EINVAL;
+    if (!aligned16(mask_x) || !aligned16(mask_s) || !aligned16(idx_s) || !aligned16(count_s))
+        return PROX_EINVAL;
+    const int d = layer->d_model;
+    if (ws_bytes < ws_layout(d, layer->d_ff, tokens_per_pass(d, batch)).total) return PROX_ENOMEM;
+    int sms = 0;
+    ps = current_device(&sms);
+    if (ps != PROX_OK) return ps;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (launch_rmsnorm(d, batch, h_in, eps, x_out, st) != cudaSuccess) return PROX_ECUDA;
+    return run_forward(layer, x_out, batch, tau_x, tau_s, h_out, mask_x, mask_s, idx_s, count_s,
+                       nullptr, ws, ws_bytes, st, true, h_in);
+}
+
 PROX_API int prox_max_batch_per_pass(int d_model) { return max_tokens_per_pass(d_model); }
 
 PROX_API prox_status prox_ffn_stage1(const prox_layer *layer, const uint16_t *x, int batch,
@@ -367,7 +410,7 @@ PROX_API prox_status prox_ffn_stage1(const prox_layer *layer, const uint16_t *x,
     ps = current_device(&sms);
     if (ps != PROX_OK) return ps;
     return pass_stage1(layer, x, batch, tau_x, tau_s, y_clear, mask_x, mask_s, nullptr,
-                       static_cast<unsigned char *>(ws), sms, true, (cudaStream_t)stream);
+                       static_cast<unsigned char *>(ws), sms, true, nullptr, (cudaStream_t)stream);
 }
 
 PROX_API prox_status prox_ffn_stage2(const prox_layer *layer, const uint16_t *x, int batch,

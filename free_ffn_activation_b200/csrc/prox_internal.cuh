@@ -72,6 +72,7 @@ struct Stage1Args {
     const uint8_t *q_up, *q_gate;
     const float *s_up, *s_gate;
     float *y_zero;               // [nb][d] zeroed here (Stage 2 accumulates), or null
+    const float *y_init;         // [nb][d] copied into y_zero instead of zeros, or null
     uint8_t *mask_x;             // [nb][d] or null
     uint8_t *mask_s;             // [nb][f] or null
     float *s_out;                // [nb][f] or null
@@ -107,6 +108,8 @@ cudaError_t launch_stage1(int B, const Stage1Args &a, const Stage1Plan &p,
                           cudaStream_t s);
 cudaError_t launch_stage2(int B, int nchunk, const Stage2Args &a, int grid,
                           size_t smem, cudaStream_t s);
+cudaError_t launch_rmsnorm(int d, int nb, const float *h, float eps, uint16_t *x,
+                           cudaStream_t s);
 cudaError_t launch_quantize(int d, int f, const uint16_t *w_cm, uint8_t *q,
                             float *scale, cudaStream_t s);
 // exact order statistic of |values| (bf16 or fp32 bit patterns) on device;

@@ -58,6 +58,9 @@ def lib() -> C.CDLL:
         L.prox_ffn_forward.argtypes = [C.POINTER(_Layer), vp, i, f, f, vp, vp, vp, vp, vp, vp, sz, vp]
         L.prox_ffn_forward_static.argtypes = [C.POINTER(_Layer), vp, i, f, f, vp, vp, vp, vp,
                                                vp, vp]
+        L.prox_rmsnorm_bf16.argtypes = [i, i, vp, f, vp, vp]
+        L.prox_ffn_block.argtypes = [C.POINTER(_Layer), vp, i, f, f, f, vp, vp, vp, vp, vp, vp,
+                                     vp, sz, vp]
         L.prox_proxy_state.argtypes = [C.POINTER(_Layer), vp, i, f, vp, vp, vp, sz, vp]
         L.prox_calibrate_workspace_bytes.argtypes = [i, i, i]
         L.prox_calibrate_workspace_bytes.restype = sz
@@ -74,6 +77,7 @@ def lib() -> C.CDLL:
         L.prox_test_set_wait.argtypes = [C.c_uint32, i]
         L.prox_test_set_wait.restype = None
         for name in ("prox_quantize_proxy", "prox_ffn_forward", "prox_ffn_forward_static",
+                     "prox_rmsnorm_bf16", "prox_ffn_block",
                      "prox_proxy_state",
                      "prox_ffn_stage1", "prox_ffn_stage2",
                      "prox_calibrate", "prox_allocate", "prox_last_device_status"):
@@ -253,6 +257,59 @@ def ffn_forward_static(layer: ProxLayer, x: torch.Tensor, tau_x: float, tau_s: f
 STATIC_WORKSPACE_BYTES = 2 << 20  # PROX_STATIC_WORKSPACE_BYTES
 
 
+def rmsnorm_bf16(h: torch.Tensor, eps: float = 1e-6) -> torch.Tensor:
+    """prox_rmsnorm_bf16: bf16 h / sqrt(mean(h^2) + eps) per row of fp32 h."""
+    if h.dim() == 1:
+        h = h.unsqueeze(0)
+    b, d = h.shape
+    _need(h, torch.float32, (b, d), "h")
+    x = torch.empty((b, d), dtype=torch.bfloat16, device=h.device)
+    _check(lib().prox_rmsnorm_bf16(d, b, _ptr(h), float(eps), _ptr(x), _stream(h.device)),
+           "prox_rmsnorm_bf16")
+    return x
+
+
+def ffn_block(layer: ProxLayer, h_in: torch.Tensor, tau_x: float, tau_s: float,
+              eps: float = 1e-6, h_out: torch.Tensor | None = None,
+              ws: torch.Tensor | None = None, *, want_masks: bool = True):
+    """prox_ffn_block: one pre-norm stack layer, h_out = h_in + FFN(RMSNorm(h_in)).
+    Returns (h_out, x, ForwardOut with y=None and the masks)."""
+    d, f = layer.d_model, layer.d_ff
+    if h_in.dim() == 1:
+        h_in = h_in.unsqueeze(0)
+    b = h_in.shape[0]
+    _need(h_in, torch.float32, (b, d), "h_in")
+    dev = h_in.device
+    if h_out is None:
+        h_out = torch.empty_like(h_in)
+    if ws is None:
+        ws = workspace(d, f, b, dev)
+    x = torch.empty((b, d), dtype=torch.bfloat16, device=dev)
+    out = ForwardOut(
+        y=None,
+        mask_x=torch.empty((b, d), dtype=torch.uint8, device=dev) if want_masks else None,
+        mask_s=torch.empty((b, f), dtype=torch.uint8, device=dev) if want_masks else None,
+        idx_s=torch.empty((b, f), dtype=torch.int32, device=dev) if want_masks else None,
+        count_s=torch.empty((b,), dtype=torch.int32, device=dev) if want_masks else None)
+    cl = layer.cstruct()
+    _check(lib().prox_ffn_block(C.byref(cl), _ptr(h_in), b, float(tau_x), float(tau_s),
+                                float(eps), _ptr(h_out), _ptr(x), _ptr(out.mask_x),
+                                _ptr(out.mask_s), _ptr(out.idx_s), _ptr(out.count_s), _ptr(ws),
+                                ws.numel(), _stream(dev)),
+           "prox_ffn_block")
+    return h_out, x, out
+
+
+def ffn_block_raw(layer_struct: _Layer, h_in_ptr: int, batch: int, tau_x: float, tau_s: float,
+                  eps: float, h_out_ptr: int, x_ptr: int, ws_ptr: int, ws_bytes: int,
+                  stream: int) -> None:
+    """prox_ffn_block with raw device pointers (no masks)."""
+    _check(lib().prox_ffn_block(C.byref(layer_struct), h_in_ptr, batch, float(tau_x),
+                                float(tau_s), float(eps), h_out_ptr, x_ptr, None, None, None,
+                                None, ws_ptr, ws_bytes, stream),
+           "prox_ffn_block")
+
+
 def ffn_forward_raw(layer_struct: _Layer, x_ptr: int, batch: int, tau_x: float, tau_s: float,
                     y_ptr: int, ws_ptr: int, ws_bytes: int, stream: int, mask_x=None,
                     mask_s=None, idx_s=None, count_s=None) -> None:
@@ -354,6 +411,6 @@ def touched_bytes(d_model: int, d_ff: int, k_x: int, k_s: int) -> int:
 
 __all__ = ["ProxLayer", "ProxError", "quantize_proxy", "workspace", "workspace_bytes",
            "ffn_forward", "ffn_forward_static", "STATIC_WORKSPACE_BYTES", "ffn_forward_raw",
-           "ffn_stage1_raw", "ffn_stage2_raw",
+           "ffn_stage1_raw", "ffn_stage2_raw", "rmsnorm_bf16", "ffn_block", "ffn_block_raw",
            "max_batch_per_pass", "proxy_state", "calibrate", "allocate",
            "last_device_status", "touched_bytes", "untile_proxy", "as_bf16"]

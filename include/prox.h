@@ -166,6 +166,32 @@ prox_status prox_ffn_forward_static(const prox_layer *layer, const uint16_t *x, 
                                     void *stream);
 
 /*
+ * Layer stacks. The Prox pages define one FFN; a stack of FFN layers (as in
+ * the stacked-layer benchmark) runs them pre-norm on an fp32 residual stream:
+ *   x = bf16(RMSNorm(h)),  RMSNorm(h) = h / sqrt(mean(h^2) + eps) (unit gain),
+ *   h <- h + FFN(x)        with FFN the Prox forward above.
+ *
+ * prox_rmsnorm_bf16 -- x_out = bf16 (round to nearest even) of
+ *   h / sqrt(mean(h^2) + eps) per token, fp32 sum of squares in a fixed order.
+ *   h : device, fp32 [batch][d_model];  x_out : device, bf16 [batch][d_model].
+ *   Errors: PROX_EINVAL (null or misaligned pointer, bad shape, eps < 0 or
+ *   not finite), PROX_EDEVICE, PROX_ECUDA.
+ *
+ * prox_ffn_block -- one layer of the stack: x_out = RMSNorm(h_in) as above,
+ *   then h_out = h_in + FFN(x_out) with the Prox forward (Stage 2 adds its
+ *   products onto a copy of h_in, so y is never stored). h_out may be h_in
+ *   (in place). x_out (device, bf16 [batch][d_model]) is required: it is the
+ *   FFN's input. Other arguments, workspace and errors as in
+ *   prox_ffn_forward.
+ */
+prox_status prox_rmsnorm_bf16(int d_model, int batch, const float *h, float eps,
+                              uint16_t *x_out, void *stream);
+prox_status prox_ffn_block(const prox_layer *layer, const float *h_in, int batch,
+                           float tau_x, float tau_s, float eps, float *h_out, uint16_t *x_out,
+                           uint8_t *mask_x, uint8_t *mask_s, int32_t *idx_s, int32_t *count_s,
+                           void *ws, size_t ws_bytes, void *stream);
+
+/*
  * prox_max_batch_per_pass -- tokens one Stage-1/Stage-2 pass handles for this
  * d_model (8 up to d_model 4096, 4 up to 8192, 0 beyond: unsupported).
  * prox_ffn_forward splits larger batches into passes by itself.

@@ -125,3 +125,30 @@ def test_budget_split_entry_point():
         P.allocate(1.5)
     with pytest.raises(P.ProxError):
         P.allocate(0.5, alpha=0.0)
+
+
+def test_stack_entry_points_validate_before_launch():
+    lib = P.lib()
+    base = 1 << 20
+    L = P._Layer(d_model=256, d_ff=768, w_up_cm=base, w_gate_cm=base * 2, w_down=base * 3,
+                 q_up=base * 4, q_gate=base * 5, s_up=base * 6, s_gate=base * 7)
+    # rmsnorm: bad shape, negative or non-finite eps, null or misaligned pointers
+    assert lib.prox_rmsnorm_bf16(250, 1, base, 1e-6, base * 2, None) == P.PROX_EINVAL
+    assert lib.prox_rmsnorm_bf16(256, 1, base, -1.0, base * 2, None) == P.PROX_EINVAL
+    assert lib.prox_rmsnorm_bf16(256, 1, base, float("nan"), base * 2, None) == P.PROX_EINVAL
+    assert lib.prox_rmsnorm_bf16(256, 1, None, 1e-6, base * 2, None) == P.PROX_EINVAL
+    assert lib.prox_rmsnorm_bf16(256, 1, base + 4, 1e-6, base * 2, None) == P.PROX_EINVAL
+    assert lib.prox_rmsnorm_bf16(256, 0, None, 1e-6, None, None) == P.PROX_OK
+    # block: x_out is required, eps checked, workspace size checked
+    ws = P.lib().prox_workspace_bytes(256, 768, 1)
+    args = lambda **k: dict(dict(h_in=base * 8, tau_x=0.5, tau_s=0.1, eps=1e-6, h_out=base * 9,
+                                 x_out=base * 10, ws=base * 11, wsb=ws), **k)
+    def call(a):
+        return lib.prox_ffn_block(C.byref(L), a["h_in"], 1, a["tau_x"], a["tau_s"], a["eps"],
+                                  a["h_out"], a["x_out"], None, None, None, None, a["ws"],
+                                  a["wsb"], None)
+    assert call(args(x_out=None)) == P.PROX_EINVAL
+    assert call(args(eps=-1e-6)) == P.PROX_EINVAL
+    assert call(args(h_in=None)) == P.PROX_EINVAL
+    assert call(args(tau_s=float("inf"))) == P.PROX_EINVAL
+    assert call(args(wsb=ws - 1)) == P.PROX_ENOMEM
