@@ -56,6 +56,9 @@ def parse():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="qwen3-8b-ffn")
     ap.add_argument("--keep-x", type=float, default=0.5)
     ap.add_argument("--keep-s", type=float, default=0.3)
+    ap.add_argument("--effective-sparsity", type=float, default=None,
+                    help="target effective sparsity e: keep ratios from the budget split "
+                         "(prox_allocate, alpha 1/3, s1 <= 0.7) instead of --keep-x/--keep-s")
     ap.add_argument("--batch", type=int, default=1,
                     help="tokens per forward call (each token keeps its own masks)")
     ap.add_argument("--copies", type=int, default=4, help="rotating weight copies (L2 defeat)")
@@ -436,6 +439,10 @@ def run_ours(args, w, rank, world, local_rank):
                          "bytes_per_launch": s2_bytes, "us_per_launch": s2_us},
             "stage1": {"kernel": "k_stage1 (INT4 proxy + channel mask)", "us_per_launch": s1_us,
                        "bytes_per_launch": s1_bytes, "GBps": s1_gbs, "frac": s1_gbs / peak},
+            "effective_sparsity": None if args.effective_sparsity is None else {
+                "target": args.effective_sparsity,
+                "realised": (1.0 - ks_tok / f) - 2.0 / 3.0 * (kx_tok / d) / 3.0,
+                "s1": 1.0 - args.keep_x, "s2": 1.0 - args.keep_s},
             "path": {"touched_MB_per_call": float(np.mean(touched)) / 1e6,
                      "GBps": path_gbs, "frac_of_peak": path_gbs / peak,
                      "keep_x": kx_tok / d, "keep_s": ks_tok / f,
@@ -628,6 +635,11 @@ def run_stack(args, w, rank, world, local_rank):
 
 def main():
     args = parse()
+    if args.effective_sparsity is not None:
+        # the pages' compute budget: e = s2 - 2 alpha (1 - s1) / 3 with alpha = 1/3
+        from free_ffn_activation_b200 import prox as P
+        s1, s2 = P.allocate(args.effective_sparsity)
+        args.keep_x, args.keep_s = 1.0 - s1, 1.0 - s2
     w = WORKLOADS[args.workload]
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

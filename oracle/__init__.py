@@ -52,21 +52,21 @@ def _declare(L):
     L.oracle_quantize_proxy.restype = None
     L.oracle_stage1_token.argtypes = [i, i, _u16p, f, _u8p, _f32p, _u8p, _f32p, f,
                                       _Opt(_u8p), _Opt(_f64p), _Opt(_f64p), _Opt(_f64p),
-                                      _Opt(_u8p)]
+                                      _Opt(_u8p), i]
     L.oracle_stage1_token.restype = None
     L.oracle_stage2_token.argtypes = [i, i, _u16p, _u16p, _u16p, _u16p, _u8p,
-                                      _Opt(_f64p), _f64p]
+                                      _Opt(_f64p), _f64p, i]
     L.oracle_stage2_token.restype = None
     L.oracle_forward.argtypes = [i, i, i, _u16p, f, f, _u16p, _u16p, _u16p, _u8p, _f32p,
                                  _u8p, _f32p, _Opt(_u8p), _Opt(_u8p), _Opt(_u8p),
-                                 _Opt(_f64p), _Opt(_f64p), _f64p, i]
+                                 _Opt(_f64p), _Opt(_f64p), _f64p, i, i]
     L.oracle_forward.restype = C.c_int
     L.oracle_quantile_rank.argtypes = [C.c_long, d]
     L.oracle_quantile_rank.restype = C.c_long
     L.oracle_order_statistic.argtypes = [_f64p, C.c_long, d]
     L.oracle_order_statistic.restype = C.c_float
     L.oracle_calibrate.argtypes = [i, i, i, _u16p, _u8p, _f32p, _u8p, _f32p, d, d,
-                                   C.POINTER(C.c_float), C.POINTER(C.c_float), i]
+                                   C.POINTER(C.c_float), C.POINTER(C.c_float), i, i]
     L.oracle_calibrate.restype = None
     L.oracle_rmsnorm_bf16.argtypes = [i, _f32p, d, _u16p]
     L.oracle_rmsnorm_bf16.restype = None
@@ -90,7 +90,10 @@ def quantize_proxy(w_cm: np.ndarray):
     return q, s
 
 
-def stage1(x, tau_x, q_up, s_up, q_gate, s_gate, tau_s):
+ACT_SWIGLU, ACT_GEGLU = 0, 1   # gate activation: SiLU (SwiGLU) or GELU (GeGLU)
+
+
+def stage1(x, tau_x, q_up, s_up, q_gate, s_gate, tau_s, act=ACT_SWIGLU):
     """Stage 1 for one token. Returns dict mask_x, u, g, s (fp64), mask_s."""
     d_model = x.shape[-1]
     d_ff = q_up.shape[1] * 2
@@ -98,22 +101,23 @@ def stage1(x, tau_x, q_up, s_up, q_gate, s_gate, tau_s):
                s=np.zeros(d_ff), mask_s=np.zeros(d_ff, np.uint8))
     lib().oracle_stage1_token(d_model, d_ff, _u16(x), float(tau_x), q_up, s_up, q_gate,
                               s_gate, float(tau_s), out["mask_x"], out["u"], out["g"],
-                              out["s"], out["mask_s"])
+                              out["s"], out["mask_s"], int(act))
     return out
 
 
-def stage2(x, w_up_cm, w_gate_cm, w_down, mask_s):
+def stage2(x, w_up_cm, w_gate_cm, w_down, mask_s, act=ACT_SWIGLU):
     """Stage 2 for one token given its channel mask. Returns (s_exact, y)."""
     d_ff, d_model = w_up_cm.shape
     s = np.zeros(d_ff)
     y = np.zeros(d_model)
     lib().oracle_stage2_token(d_model, d_ff, _u16(x), _u16(w_up_cm), _u16(w_gate_cm),
-                              _u16(w_down), np.ascontiguousarray(mask_s, np.uint8), s, y)
+                              _u16(w_down), np.ascontiguousarray(mask_s, np.uint8), s, y,
+                              int(act))
     return s, y
 
 
 def forward(x, tau_x, tau_s, layer: dict, proxy: dict, mask_s_in=None, n_threads=0,
-            want=("mask_x", "mask_s", "s_proxy", "s_exact")):
+            want=("mask_x", "mask_s", "s_proxy", "s_exact"), act=ACT_SWIGLU):
     """Forward over a batch x [b][d_model]. ``layer`` holds w_up_cm, w_gate_cm,
     w_down; ``proxy`` holds q_up, s_up, q_gate, s_gate. With ``mask_s_in``
     [b][d_ff] Stage 2 uses that mask instead of the oracle's own.
@@ -136,7 +140,7 @@ def forward(x, tau_x, tau_s, layer: dict, proxy: dict, mask_s_in=None, n_threads
         d_model, d_ff, b, x, float(tau_x), float(tau_s), _u16(layer["w_up_cm"]),
         _u16(layer["w_gate_cm"]), _u16(layer["w_down"]), proxy["q_up"], proxy["s_up"],
         proxy["q_gate"], proxy["s_gate"], ms_in, out.get("mask_x"), out.get("mask_s"),
-        out.get("s_proxy"), out.get("s_exact"), out["y"], int(n_threads))
+        out.get("s_proxy"), out.get("s_exact"), out["y"], int(n_threads), int(act))
     return out
 
 
@@ -149,7 +153,7 @@ def order_statistic(v: np.ndarray, keep: float) -> float:
     return float(np.float32(lib().oracle_order_statistic(v, v.size, float(keep))))
 
 
-def calibrate(x_cal, proxy: dict, keep_x: float, keep_s: float, n_threads=0):
+def calibrate(x_cal, proxy: dict, keep_x: float, keep_s: float, n_threads=0, act=ACT_SWIGLU):
     """Thresholds (tau_x, tau_s) as fp32 values (returned as Python floats)."""
     x_cal = _u16(np.atleast_2d(x_cal))
     n, d_model = x_cal.shape
@@ -157,7 +161,7 @@ def calibrate(x_cal, proxy: dict, keep_x: float, keep_s: float, n_threads=0):
     tx, ts = C.c_float(), C.c_float()
     lib().oracle_calibrate(d_model, d_ff, n, x_cal, proxy["q_up"], proxy["s_up"],
                            proxy["q_gate"], proxy["s_gate"], float(keep_x), float(keep_s),
-                           C.byref(tx), C.byref(ts), int(n_threads))
+                           C.byref(tx), C.byref(ts), int(n_threads), int(act))
     return tx.value, ts.value
 
 

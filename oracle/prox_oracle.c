@@ -58,6 +58,20 @@ static double silu(double z)
     return z / (1.0 + exp(-z));
 }
 
+/* GELU(z) = z * Phi(z) = z (1 + erf(z / sqrt 2)) / 2, the gate activation of
+ * the GeGLU-style models the pages also evaluate [blog "Evidence"]. Reading
+ * adopted: the exact (erf) GELU; the pages do not name a variant. */
+static double gelu(double z)
+{
+    return 0.5 * z * (1.0 + erf(z / sqrt(2.0)));
+}
+
+/* act 0: SwiGLU (SiLU gate), act 1: GeGLU (GELU gate) */
+static double activation(double z, int act)
+{
+    return act == 1 ? gelu(z) : silu(z);
+}
+
 /* ------------------------------------------------------------------------
  * Offline: symmetric per-row INT4 proxy copy of one projection
  * [blog "Stage 1": W~_up and W~_gate are symmetric per-row INT4 copies].
@@ -126,7 +140,7 @@ void oracle_stage1_token(int d_model, int d_ff, const uint16_t *x, float tau_x,
                          const uint8_t *q_up, const float *s_up,
                          const uint8_t *q_gate, const float *s_gate,
                          float tau_s, uint8_t *mask_x, double *u_proxy,
-                         double *g_proxy, double *s_proxy, uint8_t *mask_s)
+                         double *g_proxy, double *s_proxy, uint8_t *mask_s, int act)
 {
     uint8_t *mx = (uint8_t *)malloc((size_t)d_model);
     for (int i = 0; i < d_model; ++i)
@@ -147,7 +161,7 @@ void oracle_stage1_token(int d_model, int d_ff, const uint16_t *x, float tau_x,
         }
     }
     for (int j = 0; j < d_ff; ++j) {
-        double s = u[j] * silu(g[j]);
+        double s = u[j] * activation(g[j], act);
         if (u_proxy) u_proxy[j] = u[j];
         if (g_proxy) g_proxy[j] = g[j];
         if (s_proxy) s_proxy[j] = s;
@@ -169,7 +183,7 @@ void oracle_stage1_token(int d_model, int d_ff, const uint16_t *x, float tau_x,
 void oracle_stage2_token(int d_model, int d_ff, const uint16_t *x,
                          const uint16_t *w_up_cm, const uint16_t *w_gate_cm,
                          const uint16_t *w_down, const uint8_t *mask_s,
-                         double *s_exact, double *y)
+                         double *s_exact, double *y, int act)
 {
     for (int k = 0; k < d_model; ++k)
         y[k] = 0.0;
@@ -182,7 +196,7 @@ void oracle_stage2_token(int d_model, int d_ff, const uint16_t *x,
                 u += xi * bf16_value(w_up_cm[(size_t)j * d_model + i]);
                 g += xi * bf16_value(w_gate_cm[(size_t)j * d_model + i]);
             }
-            s = u * silu(g);
+            s = u * activation(g, act);
             for (int k = 0; k < d_model; ++k)
                 y[k] += s * bf16_value(w_down[(size_t)j * d_model + k]);
         }
@@ -207,7 +221,7 @@ int oracle_forward(int d_model, int d_ff, int batch, const uint16_t *x,
                    const float *s_up, const uint8_t *q_gate,
                    const float *s_gate, const uint8_t *mask_s_in,
                    uint8_t *mask_x, uint8_t *mask_s, double *s_proxy,
-                   double *s_exact, double *y, int n_threads)
+                   double *s_exact, double *y, int n_threads, int act)
 {
     int used = 1;
 #ifdef _OPENMP
@@ -230,12 +244,12 @@ int oracle_forward(int d_model, int d_ff, int batch, const uint16_t *x,
                                 s_gate, tau_s,
                                 mask_x ? mask_x + (size_t)t * d_model : NULL,
                                 NULL, NULL,
-                                s_proxy ? s_proxy + (size_t)t * d_ff : NULL, ms);
+                                s_proxy ? s_proxy + (size_t)t * d_ff : NULL, ms, act);
             const uint8_t *use = mask_s_in ? mask_s_in + (size_t)t * d_ff : ms;
             oracle_stage2_token(d_model, d_ff, xt, w_up_cm, w_gate_cm, w_down,
                                 use,
                                 s_exact ? s_exact + (size_t)t * d_ff : NULL,
-                                y + (size_t)t * d_model);
+                                y + (size_t)t * d_model, act);
             if (!mask_s)
                 free(ms);
         }
@@ -287,7 +301,7 @@ void oracle_calibrate(int d_model, int d_ff, int n_cal, const uint16_t *x_cal,
                       const uint8_t *q_up, const float *s_up,
                       const uint8_t *q_gate, const float *s_gate,
                       double keep_x, double keep_s, float *tau_x_out,
-                      float *tau_s_out, int n_threads)
+                      float *tau_s_out, int n_threads, int act)
 {
     long nx = (long)n_cal * d_model;
     double *ax = (double *)malloc(sizeof(double) * (size_t)nx);
@@ -308,7 +322,7 @@ void oracle_calibrate(int d_model, int d_ff, int n_cal, const uint16_t *x_cal,
     for (int t = 0; t < n_cal; ++t)
         oracle_stage1_token(d_model, d_ff, x_cal + (size_t)t * d_model, tau_x,
                             q_up, s_up, q_gate, s_gate, 0.0f, NULL, NULL, NULL,
-                            sv + (size_t)t * d_ff, NULL);
+                            sv + (size_t)t * d_ff, NULL, act);
     *tau_s_out = oracle_order_statistic(sv, ns, keep_s);
     *tau_x_out = tau_x;
     free(sv);

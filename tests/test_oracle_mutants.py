@@ -30,7 +30,12 @@ MUTANTS = {
                         "y[k] += s * bf16_value(w_down[(size_t)(k % d_ff) * d_model + (j % d_model)]);"),
     "round_truncates": ("v = (int)nearbyintf(r);", "v = (int)r;"),
     "scale_over_8": ("float s = amax / 7.0f;", "float s = amax / 8.0f;"),
-    "up_gate_swapped": ("s = u * silu(g);\n            for", "s = g * silu(u);\n            for"),
+    "up_gate_swapped": ("s = u * activation(g, act);\n            for",
+                        "s = g * activation(u, act);\n            for"),
+    "gelu_half_dropped": ("return 0.5 * z * (1.0 + erf(z / sqrt(2.0)));",
+                          "return z * (1.0 + erf(z / sqrt(2.0)));"),
+    "gelu_scale": ("return 0.5 * z * (1.0 + erf(z / sqrt(2.0)));",
+                   "return 0.5 * z * (1.0 + erf(z));"),
     "rank_ceil": ("double r = floor((1.0 - keep) * (double)n);",
                   "double r = ceil((1.0 - keep) * (double)n);"),
     "budget_term": ("s2 = e + 2.0 * alpha * (1.0 - s1) / 3.0;",

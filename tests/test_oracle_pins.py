@@ -371,3 +371,45 @@ def test_rmsnorm_ties_to_even_and_eps():
     x = oracle.rmsnorm_bf16(h, eps=eps)
     assert x.tolist() == [[_bf16_bits(1.0), _bf16_bits(1.0 + 2.0 ** -6),
                            _bf16_bits(-1.0), _bf16_bits(0.5)]]
+
+
+# ---------------------------------------------------------------------------
+# GeGLU variant (blog, "Evidence": GeGLU-style models): the gate activation is
+# GELU(z) = z Phi(z); reading adopted: the exact (erf) GELU
+# ---------------------------------------------------------------------------
+
+def dense_geglu(x, L):
+    """Textbook dense GeGLU FFN(x) = (x W_up (.) GELU(x W_gate)) W_down with
+    GELU(z) = z Phi(z), Phi the standard normal CDF from scipy."""
+    from scipy.stats import norm
+    xd = f64(x)
+    u = xd @ f64(L["w_up_cm"]).T
+    g = xd @ f64(L["w_gate_cm"]).T
+    return (u * g * norm.cdf(g)) @ f64(L["w_down"])
+
+
+def test_zero_thresholds_give_dense_geglu():
+    L = small_layer(32, 64, seed=5)
+    P = oracle.make_proxy(L)
+    x = S.make_tokens(4, 32, seed=5)
+    out = oracle.forward(x, 0.0, 0.0, L, P, act=oracle.ACT_GEGLU)
+    assert rel(out["y"], dense_geglu(x, L)) < 1e-12
+    # and the SwiGLU output differs (the activation is really switched)
+    assert rel(out["y"], dense_swiglu(x, L)) > 1e-3
+
+
+def test_geglu_proxy_state_identity():
+    # GELU(z) - GELU(-z) = z exactly in the reals (Phi(z) + Phi(-z) = 1): the
+    # proxy state s~ = u~ GELU(g~) of a layer and of the same layer with the
+    # gate negated differ by u~ g~ channel by channel
+    L = small_layer(32, 64, seed=6)
+    Lneg = dict(L)
+    Lneg["w_gate_cm"] = L["w_gate_cm"] ^ np.uint16(0x8000)   # exact negation of bf16
+    P, Pn = oracle.make_proxy(L), oracle.make_proxy(Lneg)
+    x = S.make_tokens(1, 32, seed=6)[0]
+    a = oracle.stage1(x, 0.0, P["q_up"], P["s_up"], P["q_gate"], P["s_gate"], 0.0,
+                      act=oracle.ACT_GEGLU)
+    b = oracle.stage1(x, 0.0, Pn["q_up"], Pn["s_up"], Pn["q_gate"], Pn["s_gate"], 0.0,
+                      act=oracle.ACT_GEGLU)
+    assert np.allclose(b["g"], -a["g"], rtol=0, atol=0)
+    assert np.allclose(a["s"] - b["s"], a["u"] * a["g"], rtol=1e-12, atol=1e-15)
