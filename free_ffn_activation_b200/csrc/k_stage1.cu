@@ -500,7 +500,7 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
 #pragma unroll
         for (int t = 0; t < B; ++t) {
             if (t >= a.nb || ch >= T::CW) break;
-            const float st = uu[t] * (gg[t] / (1.f + expf(-gg[t])));
+            const float st = uu[t] * gate_act(gg[t], a.act);
             if (a.s_out) a.s_out[(size_t)t * a.f + j] = st;
             const bool keep = fabsf(st) >= a.tau_s;
             if (a.mask_s) a.mask_s[(size_t)t * a.f + j] = keep ? 1 : 0;

@@ -343,7 +343,7 @@ __global__ void __launch_bounds__(s2_threads(B), 1) k_stage2(const Stage2Args a)
                     u += __shfl_xor_sync(0xffffffffu, u, o);
                     gg += __shfl_xor_sync(0xffffffffu, gg, o);
                 }
-                sv[t] = ((bits >> t) & 1u) ? u * (gg / (1.f + expf(-gg))) : 0.f;
+                sv[t] = ((bits >> t) & 1u) ? u * gate_act(gg, a.act) : 0.f;
             }
             __syncwarp();
             if (lane == 0) {

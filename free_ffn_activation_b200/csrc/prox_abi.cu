@@ -144,6 +144,7 @@ static bool shape_ok(int d, int f) {
 
 static prox_status check_layer(const prox_layer *L, bool need_exact) {
     if (!L || !shape_ok(L->d_model, L->d_ff)) return PROX_EINVAL;
+    if (L->activation != PROX_ACT_SWIGLU && L->activation != PROX_ACT_GEGLU) return PROX_EINVAL;
     if (!L->q_up || !L->q_gate || !L->s_up || !L->s_gate) return PROX_EINVAL;
     if (!aligned16(L->q_up) || !aligned16(L->q_gate) || !aligned16(L->s_up) ||
         !aligned16(L->s_gate))
@@ -192,6 +193,7 @@ static prox_status pass_stage1(const prox_layer *L, const uint16_t *x, int nb, f
     a.mask_s = mask_s;
     a.s_out = s_out;
     a.build_lists = lists ? 1 : 0;
+    a.act = L->activation;
     a.wait_us = g_spin_limit;
     a.status = reinterpret_cast<uint32_t *>(w + W.status);
     a.ucount = reinterpret_cast<int32_t *>(w + W.ucount);
@@ -223,6 +225,7 @@ static prox_status pass_stage2(const prox_layer *L, const uint16_t *x, int nb, f
     b.w_down = L->w_down;
     b.y = y;
     b.idx_s = idx_s;
+    b.act = L->activation;
     b.count_s = count_s;
     b.ucount = reinterpret_cast<int32_t *>(w + W.ucount);
     b.tcount = reinterpret_cast<int32_t *>(w + W.tcount);

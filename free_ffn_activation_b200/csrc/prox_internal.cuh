@@ -77,6 +77,7 @@ struct Stage1Args {
     uint8_t *mask_s;             // [nb][f] or null
     float *s_out;                // [nb][f] or null
     int build_lists;             // write ulist/tlist/counts for Stage 2
+    int act;                     // gate activation (PROX_ACT_*)
     uint32_t wait_us;            // wall-clock bound of each wait, microseconds
     // workspace
     uint32_t *status;
@@ -93,6 +94,7 @@ struct Stage2Args {
     float *y;                    // [nb][d], zeroed by Stage 1
     int32_t *idx_s;              // [nb][f] or null
     int32_t *count_s;            // [nb] or null
+    int act;                     // gate activation (PROX_ACT_*)
     const int32_t *ucount, *tcount;
     const uint32_t *ulist;
     const int32_t *tlist;
@@ -236,6 +238,13 @@ __device__ __forceinline__ void red_add_v4(float *dst, float a, float b, float c
     asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a), "f"(b),
                  "f"(c), "f"(d)
                  : "memory");
+}
+
+// gate activation of s = u * act(g): SiLU(g) = g / (1 + e^-g) for SwiGLU,
+// GELU(g) = g (1 + erf(g / sqrt 2)) / 2 for GeGLU (CUDA's expf and erff)
+__device__ __forceinline__ float gate_act(float g, int act) {
+    return act == PROX_ACT_GEGLU ? 0.5f * g * (1.f + erff(g * 0.70710678118654752f))
+                                 : g / (1.f + expf(-g));
 }
 
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }

@@ -37,7 +37,10 @@ class _Layer(C.Structure):
     _fields_ = [("d_model", C.c_int), ("d_ff", C.c_int),
                 ("w_up_cm", C.c_void_p), ("w_gate_cm", C.c_void_p), ("w_down", C.c_void_p),
                 ("q_up", C.c_void_p), ("q_gate", C.c_void_p),
-                ("s_up", C.c_void_p), ("s_gate", C.c_void_p)]
+                ("s_up", C.c_void_p), ("s_gate", C.c_void_p), ("activation", C.c_int)]
+
+
+ACT_SWIGLU, ACT_GEGLU = 0, 1   # PROX_ACT_SWIGLU, PROX_ACT_GEGLU
 
 
 _lib = None
@@ -138,6 +141,7 @@ class ProxLayer:
     q_gate: torch.Tensor
     s_up: torch.Tensor         # fp32 [d_model]
     s_gate: torch.Tensor
+    activation: int = 0        # ACT_SWIGLU (SiLU gate) or ACT_GEGLU (GELU gate)
 
     @property
     def d_model(self) -> int:
@@ -156,15 +160,17 @@ class ProxLayer:
                               ("s_gate", torch.float32, (d,))):
             _need(getattr(self, name), dt, shp, name)
         return _Layer(d, f, _ptr(self.w_up_cm), _ptr(self.w_gate_cm), _ptr(self.w_down),
-                      _ptr(self.q_up), _ptr(self.q_gate), _ptr(self.s_up), _ptr(self.s_gate))
+                      _ptr(self.q_up), _ptr(self.q_gate), _ptr(self.s_up), _ptr(self.s_gate),
+                      int(self.activation))
 
     @staticmethod
-    def from_weights(w_up_cm, w_gate_cm, w_down, device="cuda") -> "ProxLayer":
+    def from_weights(w_up_cm, w_gate_cm, w_down, device="cuda",
+                     activation: int = ACT_SWIGLU) -> "ProxLayer":
         """Upload bf16 weights and build their INT4 proxies on the device."""
         up, gate, down = (as_bf16(w, device).contiguous() for w in (w_up_cm, w_gate_cm, w_down))
         q_up, s_up = quantize_proxy(up)
         q_gate, s_gate = quantize_proxy(gate)
-        return ProxLayer(up, gate, down, q_up, q_gate, s_up, s_gate)
+        return ProxLayer(up, gate, down, q_up, q_gate, s_up, s_gate, int(activation))
 
 
 def quantize_proxy(w_cm: torch.Tensor):

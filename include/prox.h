@@ -72,7 +72,14 @@ typedef struct prox_layer {
     const uint8_t *q_gate;
     const float *s_up;
     const float *s_gate;
+    /* gate activation: PROX_ACT_SWIGLU (SiLU, the pages' SwiGLU FFN) or
+       PROX_ACT_GEGLU (GELU(z) = z Phi(z), exact erf form: the GeGLU-style
+       models of the blog's "Evidence" section); anything else is PROX_EINVAL */
+    int activation;
 } prox_layer;
+
+#define PROX_ACT_SWIGLU 0
+#define PROX_ACT_GEGLU 1
 
 /*
  * prox_quantize_proxy -- symmetric per-row INT4 proxy copy of one projection

@@ -152,3 +152,14 @@ def test_stack_entry_points_validate_before_launch():
     assert call(args(h_in=None)) == P.PROX_EINVAL
     assert call(args(tau_s=float("inf"))) == P.PROX_EINVAL
     assert call(args(wsb=ws - 1)) == P.PROX_ENOMEM
+
+
+def test_unknown_activation_rejected():
+    base = 1 << 20
+    L = P._Layer(d_model=256, d_ff=768, w_up_cm=base, w_gate_cm=base * 2, w_down=base * 3,
+                 q_up=base * 4, q_gate=base * 5, s_up=base * 6, s_gate=base * 7, activation=2)
+    st = P.lib().prox_ffn_forward(C.byref(L), 1 << 24, 1, 0.5, 0.1, 1 << 25, None, None, None,
+                                  None, 1 << 26, 1 << 30, None)
+    assert st == P.PROX_EINVAL
+    L.activation = P.ACT_GEGLU
+    assert P.lib().prox_quantize_proxy(250, 768, base, base, base, None) == P.PROX_EINVAL

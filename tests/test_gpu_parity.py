@@ -33,17 +33,18 @@ class Case:
     """One layer with its oracle proxies, device layer and thresholds."""
 
     def __init__(self, d, f, n_tok, n_cal, sigma=0.02, seed=0, outlier=0.0, layer=0,
-                 keep_x=0.5, keep_s=0.3, dev="cuda"):
+                 keep_x=0.5, keep_s=0.3, dev="cuda", act=oracle.ACT_SWIGLU):
         self.spec = S.LayerSpec(d, f, sigma=sigma, seed=seed, layer=layer)
         self.L = S.make_layer(self.spec)
         self.Por = oracle.make_proxy(self.L)
         self.dev = dev
+        self.act = act
         self.layer = P.ProxLayer.from_weights(self.L["w_up_cm"], self.L["w_gate_cm"],
-                                              self.L["w_down"], device=dev)
+                                              self.L["w_down"], device=dev, activation=act)
         self.x = S.make_tokens(n_tok, d, seed=seed, stream="x_eval", outlier_frac=outlier)
         self.x_cal = S.make_tokens(n_cal, d, seed=seed, stream="x_cal", outlier_frac=outlier)
         self.keep_x, self.keep_s = keep_x, keep_s
-        self.tau_x, self.tau_s = oracle.calibrate(self.x_cal, self.Por, keep_x, keep_s)
+        self.tau_x, self.tau_s = oracle.calibrate(self.x_cal, self.Por, keep_x, keep_s, act=act)
 
     def xdev(self, rows=None):
         x = self.x if rows is None else self.x[rows]
@@ -73,10 +74,16 @@ def c4(gpu):
     return Case(8192, 28672, 32, 64, sigma=0.015)
 
 
+@pytest.fixture(scope="module")
+def c1g(gpu):
+    # the tiny layer with a GeGLU gate (GELU instead of SiLU)
+    return Case(256, 768, 64, 256, act=oracle.ACT_GEGLU)
+
+
 def check_forward(case, rows, out, tag=""):
     """Compare a device ForwardOut for tokens `rows` with the oracle."""
     x = case.x[rows]
-    ref = oracle.forward(x, case.tau_x, case.tau_s, case.L, case.Por)
+    ref = oracle.forward(x, case.tau_x, case.tau_s, case.L, case.Por, act=case.act)
     mx = out.mask_x.cpu().numpy()
     ms = out.mask_s.cpu().numpy()
     idx = out.idx_s.cpu().numpy()
@@ -94,7 +101,7 @@ def check_forward(case, rows, out, tag=""):
         assert cnt[t] == kept.size
         assert np.array_equal(idx[t, :cnt[t]], kept), f"{tag} idx_s token {t}"
     y_ref = oracle.forward(x, case.tau_x, case.tau_s, case.L, case.Por, mask_s_in=ms,
-                           want=())["y"]
+                           want=(), act=case.act)["y"]
     y = out.y.cpu().numpy().astype(np.float64)
     num = np.linalg.norm(y - y_ref, axis=1)
     den = np.maximum(np.linalg.norm(y_ref, axis=1), 1e-30)
@@ -154,7 +161,8 @@ def _proxy_check(case, rows):
     s_gpu, mx = P.proxy_state(case.layer, case.xdev(rows), case.tau_x)
     s_gpu = s_gpu.cpu().numpy().astype(np.float64)
     ref = np.stack([oracle.stage1(case.x[t], case.tau_x, case.Por["q_up"], case.Por["s_up"],
-                                  case.Por["q_gate"], case.Por["s_gate"], case.tau_s)["s"]
+                                  case.Por["q_gate"], case.Por["s_gate"], case.tau_s,
+                                  act=case.act)["s"]
                     for t in rows])
     assert np.array_equal(mx.cpu().numpy(),
                           (np.abs(S.bf16_to_f32(case.x[rows])) >= np.float32(case.tau_x)).astype(np.uint8))
@@ -179,6 +187,23 @@ def test_calibrate_c1(c1):
     tx, ts = P.calibrate(c1.layer, to_dev_bf16(c1.x_cal, "cuda"), c1.keep_x, c1.keep_s)
     assert np.float32(tx) == np.float32(c1.tau_x)
     assert abs(ts - c1.tau_s) <= 1e-5 * c1.tau_s, (ts, c1.tau_s)
+
+
+def test_geglu_proxy_state_c1(c1g):
+    _proxy_check(c1g, list(range(16)))
+
+
+def test_geglu_calibrate_c1(c1g):
+    tx, ts = P.calibrate(c1g.layer, to_dev_bf16(c1g.x_cal, "cuda"), c1g.keep_x, c1g.keep_s)
+    assert np.float32(tx) == np.float32(c1g.tau_x)
+    assert abs(ts - c1g.tau_s) <= 1e-5 * c1g.tau_s, (ts, c1g.tau_s)
+
+
+@pytest.mark.parametrize("b", [1, 5, 64])
+def test_geglu_forward_c1(c1g, b):
+    rows = list(range(b))
+    out = P.ffn_forward(c1g.layer, c1g.xdev(rows), c1g.tau_x, c1g.tau_s)
+    check_forward(c1g, rows, out, f" c1 GeGLU b={b}")
 
 
 def test_calibrate_c2(c2):
