@@ -150,7 +150,8 @@ struct S1Smem {
     size_t ring, red, rowidx, xs, part, total;
 };
 
-__host__ __device__ inline S1Smem s1_smem(int d, int B, int NB, int unit_cap, int depth_sel) {
+__host__ __device__ inline S1Smem s1_smem(int d, int B, int NB, int unit_cap, int depth_sel,
+                                         int n_r = kS1MaxRowGroups) {
     const int cw = NB * kCB;
     const int cpt = s1_cpt(B, NB);
     const int rl = kS1Threads / (2 * (cw / cpt));
@@ -166,7 +167,7 @@ __host__ __device__ inline S1Smem s1_smem(int d, int B, int NB, int unit_cap, in
     s.xs = o;
     o += (size_t)unit_cap * 2 * B * 4;
     s.part = o;
-    o += (size_t)2 * B * cw * 4;
+    o += (size_t)(B <= 2 ? n_r : 1) * 2 * B * cw * 4;  // B <= 2: every rank's partials
     s.total = o;
     return s;
 }
@@ -240,10 +241,16 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
     float *red = reinterpret_cast<float *>(smem + L.red);
     int *rowidx = reinterpret_cast<int *>(smem + L.rowidx);          // [unit_cap]
     float *xs = reinterpret_cast<float *>(smem + L.xs);              // [unit_cap][2][B]
-    float *part = reinterpret_cast<float *>(smem + L.part);          // [2][B][CW]
+    float *part = reinterpret_cast<float *>(smem + L.part);          // [n_r or 1][2][B][CW]
+    constexpr bool kPush = (B <= 2);
+    // B <= 2: each rank stores its partials straight into slot r of CTA 0's array
+    float *dst_part = kPush ? cluster.map_shared_rank(part, 0) + (size_t)r * 2 * B * T::CW : part;
     __shared__ int s_warp[kS1Threads / 32];
     __shared__ __align__(16) float s_red[kS1Threads / 32][kMaxB];
     __shared__ int s_cnt[kS1Threads / 32][kMaxB + 1];
+    // every CTA of the cluster has started once this phase completes: only
+    // then may ranks store into CTA 0's shared memory (waited for before (6))
+    if (kPush) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 
     // The proxy scales are layer weights: pull them into L2 while the
     // previous kernel of the stream finishes (a prefetch only warms the
@@ -425,6 +432,7 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
     else
         s1_stream<B, NB, T::DMAX / 4>(qbase, ring, rowidx, xs, rl, m, n_rows, acc2, ssum);
     __syncthreads();  // every thread is done with the ring before it becomes `red`
+    if (kPush) asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
 
     // (6) reduce row lanes (padded rows: conflict-free both ways), undo the
     // pre-scale and the +8 code offset: this CTA's partial sums in `part`.
@@ -459,7 +467,7 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
             }
             const int e1 = E[t] / 2, e2 = E[t] - e1;
             const float v = (sacc * up1) * up2 - 8.f * soff;  // sum (q + 8 - 8) x s 2^E
-            part[(mm * B + t) * T::CW + ch] =
+            dst_part[(mm * B + t) * T::CW + ch] =
                 v * __int_as_float((127 - e1) << 23) * __int_as_float((127 - e2) << 23);
         }
     }
@@ -484,7 +492,8 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
             for (int q = 0; q < kS1MaxRowGroups; ++q) {
                 pu[q] = pg[q] = 0.f;
                 if (q < a.n_r) {
-                    const float *pq = cluster.map_shared_rank(part, q);
+                    const float *pq = kPush ? part + (size_t)q * 2 * B * T::CW
+                                            : cluster.map_shared_rank(part, q);
                     pu[q] = pq[(0 * B + t) * T::CW + ch];
                     pg[q] = pq[(1 * B + t) * T::CW + ch];
                 }
@@ -495,7 +504,7 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
                 gg[t] += pg[q];
             }
         }
-        asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+        if (!kPush) asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
         uint32_t bits = 0;
 #pragma unroll
         for (int t = 0; t < B; ++t) {
@@ -540,8 +549,8 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
                 }
             }
         }
-        asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-    } else {
+        if (!kPush) asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+    } else if (!kPush) {
         // peers keep their shared memory until CTA 0 has gathered it
         asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
         asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
