@@ -68,6 +68,12 @@ def _declare(L):
     L.oracle_calibrate.argtypes = [i, i, i, _u16p, _u8p, _f32p, _u8p, _f32p, d, d,
                                    C.POINTER(C.c_float), C.POINTER(C.c_float), i, i]
     L.oracle_calibrate.restype = None
+    L.oracle_hist_quantile.argtypes = [_f32p, C.c_long, d, C.c_long, i]
+    L.oracle_hist_quantile.restype = C.c_float
+    L.oracle_calibrate_hist.argtypes = [i, i, i, _u16p, _u8p, _f32p, _u8p, _f32p, d, d,
+                                        C.c_long, i, C.POINTER(C.c_float),
+                                        C.POINTER(C.c_float), i, i]
+    L.oracle_calibrate_hist.restype = None
     L.oracle_rmsnorm_bf16.argtypes = [i, _f32p, d, _u16p]
     L.oracle_rmsnorm_bf16.restype = None
     L.oracle_allocate.argtypes = [d, d, d, d, C.POINTER(C.c_double), C.POINTER(C.c_double)]
@@ -162,6 +168,31 @@ def calibrate(x_cal, proxy: dict, keep_x: float, keep_s: float, n_threads=0, act
     lib().oracle_calibrate(d_model, d_ff, n, x_cal, proxy["q_up"], proxy["s_up"],
                            proxy["q_gate"], proxy["s_gate"], float(keep_x), float(keep_s),
                            C.byref(tx), C.byref(ts), int(n_threads), int(act))
+    return tx.value, ts.value
+
+
+HIST_SAMPLES, HIST_BINS = 200_000, 4096   # the pages' per-layer calibration budget
+
+
+def hist_quantile(v, keep: float, max_samples: int = HIST_SAMPLES,
+                  bins: int = HIST_BINS) -> float:
+    """Histogram threshold of |v| (fp32 values, pooled order) for `keep`."""
+    v = np.ascontiguousarray(v, dtype=np.float32).ravel()
+    return float(lib().oracle_hist_quantile(v, v.size, float(keep), int(max_samples), int(bins)))
+
+
+def calibrate_hist(x_cal, proxy: dict, keep_x: float, keep_s: float,
+                   max_samples: int = HIST_SAMPLES, bins: int = HIST_BINS, n_threads=0, act=0):
+    """Histogram thresholds (tau_x, tau_s): each from at most max_samples pooled
+    magnitudes and a histogram of `bins` bins (see oracle_hist_quantile)."""
+    x_cal = _u16(np.atleast_2d(x_cal))
+    n, d_model = x_cal.shape
+    d_ff = proxy["q_up"].shape[1] * 2
+    tx, ts = C.c_float(), C.c_float()
+    lib().oracle_calibrate_hist(d_model, d_ff, n, x_cal, proxy["q_up"], proxy["s_up"],
+                                proxy["q_gate"], proxy["s_gate"], float(keep_x), float(keep_s),
+                                int(max_samples), int(bins), C.byref(tx), C.byref(ts),
+                                int(n_threads), int(act))
     return tx.value, ts.value
 
 

@@ -297,6 +297,57 @@ float oracle_order_statistic(const double *v, long n, double keep)
     return tau;
 }
 
+/* ------------------------------------------------------------------------
+ * Histogram quantile [blog "Evidence": per layer at most 200,000 activation
+ * samples and a 4,096-bin histogram]. The pages fix no more than that; the
+ * readings adopted here make every step plain fp32 arithmetic:
+ *   samples: every k-th pooled magnitude, k = ceil(n / max_samples), in
+ *            pooled order (|v[0]|, |v[k]|, |v[2k]|, ...);
+ *   bins:    `bins` equal bins of width w = m / bins over [0, m], m the largest
+ *            sample; sample s falls in bin trunc(fp32(s / w)), and m itself
+ *            (and anything rounding to bins) in the top bin;
+ *   tau:     fp32(b * w), the lower edge of the bin b holding the sample of
+ *            rank floor((1 - keep) * n_s) in ascending order (the rank rule of
+ *            the exact order statistic), so tau <= that sample < tau + w.
+ * v holds fp32 values (the magnitudes are taken here).
+ * ---------------------------------------------------------------------- */
+float oracle_hist_quantile(const float *v, long n, double keep, long max_samples, int bins)
+{
+    long k = (n + max_samples - 1) / max_samples;
+    if (k < 1)
+        k = 1;
+    long ns = (n + k - 1) / k;
+    float m = 0.0f;
+    for (long i = 0; i < ns; ++i) {
+        float a = fabsf(v[i * k]);
+        if (a > m)
+            m = a;
+    }
+    if (m == 0.0f)
+        return 0.0f;
+    const float w = m / (float)bins;
+    long *hist = (long *)calloc((size_t)bins, sizeof(long));
+    for (long i = 0; i < ns; ++i) {
+        float q = fabsf(v[i * k]) / w;
+        long b = (long)q;                 /* q >= 0: truncation */
+        if (b > bins - 1)
+            b = bins - 1;
+        hist[b] += 1;
+    }
+    long rank = oracle_quantile_rank(ns, keep);
+    long cum = 0;
+    int sel = bins - 1;
+    for (int b = 0; b < bins; ++b) {
+        if (rank < cum + hist[b]) {
+            sel = b;
+            break;
+        }
+        cum += hist[b];
+    }
+    free(hist);
+    return (float)sel * w;
+}
+
 void oracle_calibrate(int d_model, int d_ff, int n_cal, const uint16_t *x_cal,
                       const uint8_t *q_up, const float *s_up,
                       const uint8_t *q_gate, const float *s_gate,
@@ -325,6 +376,44 @@ void oracle_calibrate(int d_model, int d_ff, int n_cal, const uint16_t *x_cal,
                             sv + (size_t)t * d_ff, NULL, act);
     *tau_s_out = oracle_order_statistic(sv, ns, keep_s);
     *tau_x_out = tau_x;
+    free(sv);
+}
+
+/* Histogram calibration [blog "Evidence"]: as oracle_calibrate, with each
+ * threshold the histogram quantile above of the pooled fp32 magnitudes (s~
+ * rounded to fp32, pooled token by token, channel by channel). */
+void oracle_calibrate_hist(int d_model, int d_ff, int n_cal, const uint16_t *x_cal,
+                           const uint8_t *q_up, const float *s_up,
+                           const uint8_t *q_gate, const float *s_gate,
+                           double keep_x, double keep_s, long max_samples, int bins,
+                           float *tau_x_out, float *tau_s_out, int n_threads, int act)
+{
+    long nx = (long)n_cal * d_model;
+    float *ax = (float *)malloc(sizeof(float) * (size_t)nx);
+    for (long k = 0; k < nx; ++k)
+        ax[k] = bf16_value_f(x_cal[k]);
+    float tau_x = oracle_hist_quantile(ax, nx, keep_x, max_samples, bins);
+    free(ax);
+
+    long ns = (long)n_cal * d_ff;
+    double *sv = (double *)malloc(sizeof(double) * (size_t)ns);
+#ifdef _OPENMP
+    if (n_threads <= 0)
+        n_threads = omp_get_max_threads();
+#pragma omp parallel for num_threads(n_threads) schedule(dynamic, 1)
+#else
+    (void)n_threads;
+#endif
+    for (int t = 0; t < n_cal; ++t)
+        oracle_stage1_token(d_model, d_ff, x_cal + (size_t)t * d_model, tau_x,
+                            q_up, s_up, q_gate, s_gate, 0.0f, NULL, NULL, NULL,
+                            sv + (size_t)t * d_ff, NULL, act);
+    float *sf = (float *)malloc(sizeof(float) * (size_t)ns);
+    for (long k = 0; k < ns; ++k)
+        sf[k] = (float)sv[k];
+    *tau_s_out = oracle_hist_quantile(sf, ns, keep_s, max_samples, bins);
+    *tau_x_out = tau_x;
+    free(sf);
     free(sv);
 }
 

@@ -413,3 +413,43 @@ def test_geglu_proxy_state_identity():
                       act=oracle.ACT_GEGLU)
     assert np.allclose(b["g"], -a["g"], rtol=0, atol=0)
     assert np.allclose(a["s"] - b["s"], a["u"] * a["g"], rtol=1e-12, atol=1e-15)
+
+
+# ---------------------------------------------------------------------------
+# Histogram calibration (blog, "Evidence": at most 200,000 samples and a
+# 4,096-bin histogram per layer; readings: every k-th sample, equal bins over
+# [0, max], tau = the lower edge of the bin holding the rank-floor sample)
+# ---------------------------------------------------------------------------
+
+def test_hist_quantile_hand_worked():
+    # 0..15 in 4 bins of width 3.75: counts 4, 4, 4, 4 (15 itself in the top
+    # bin); keep 0.5 -> rank 8 -> third bin -> tau = 2 * 3.75
+    v = np.arange(16, dtype=np.float32)
+    assert oracle.hist_quantile(v, 0.5, bins=4) == 7.5
+    # keep 1.0 -> rank 0 -> first bin -> 0; keep 0.0 -> rank 15 (clamped) -> top bin
+    assert oracle.hist_quantile(v, 1.0, bins=4) == 0.0
+    assert oracle.hist_quantile(v, 0.0, bins=4) == 11.25
+    # signs do not matter, and an all-zero input gives 0
+    assert oracle.hist_quantile(-v, 0.5, bins=4) == 7.5
+    assert oracle.hist_quantile(np.zeros(8, np.float32), 0.5) == 0.0
+
+
+def test_hist_quantile_subsamples_every_kth():
+    # 10 values, at most 4 samples -> every 3rd: 0, 1, 2, 3 (the 100s are
+    # skipped); 3 bins of width 1 -> counts 1, 1, 2; rank floor(0.5 * 4) = 2
+    v = np.array([0, 100, 100, 1, 100, 100, 2, 100, 100, 3], np.float32)
+    assert oracle.hist_quantile(v, 0.5, max_samples=4, bins=3) == 2.0
+    # without the budget the 100s dominate
+    assert oracle.hist_quantile(v, 0.5, max_samples=1000, bins=3) > 50.0
+
+
+def test_hist_quantile_brackets_the_order_statistic():
+    # with every value sampled, the histogram threshold is the lower edge of
+    # the bin that holds the exact rank-floor((1-keep) n) value
+    rng = np.random.default_rng(7)
+    for n, keep in [(5000, 0.5), (20001, 0.3), (777, 0.9)]:
+        v = rng.laplace(size=n).astype(np.float32)
+        th = oracle.hist_quantile(v, keep)
+        tx = oracle.order_statistic(v.astype(np.float64), keep)
+        w = np.float32(np.abs(v).max()) / np.float32(4096)
+        assert th <= tx < th + w * 1.0001, (n, keep, th, tx, w)
