@@ -133,6 +133,53 @@ __global__ void __launch_bounds__(1024) k_select(const uint32_t *hist, int nbins
 }
 
 __global__ void k_tau_bf16(const uint32_t *sel, float *tau) { *tau = __uint_as_float(sel[0] << 16); }
+
+// Histogram quantile (every k-th of n values, `bins` equal bins over [0, m],
+// m the largest sample; tau = the lower edge of the bin holding the rank-r
+// sample): fp32 magnitude of value i, for bf16 or fp32 inputs
+template <typename V>
+__device__ __forceinline__ float mag(const V *v, long i);
+template <>
+__device__ __forceinline__ float mag<uint16_t>(const uint16_t *v, long i) {
+    return __uint_as_float((uint32_t)(v[i] & 0x7FFFu) << 16);
+}
+template <>
+__device__ __forceinline__ float mag<float>(const float *v, long i) {
+    return fabsf(v[i]);
+}
+
+// scratch[2] = bit pattern of the largest sample (non-negative floats order
+// like their bit patterns)
+template <typename V>
+__global__ void k_sub_max(const V *__restrict__ v, long ns, long k, uint32_t *scratch) {
+    uint32_t m = 0;
+    for (long s = blockIdx.x * (long)blockDim.x + threadIdx.x; s < ns;
+         s += (long)gridDim.x * blockDim.x)
+        m = max(m, __float_as_uint(mag(v, s * k)));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((threadIdx.x & 31) == 0) atomicMax(&scratch[2], m);
+}
+
+template <typename V>
+__global__ void k_sub_hist(const V *__restrict__ v, long ns, long k, int bins,
+                           const uint32_t *scratch, uint32_t *hist) {
+    const float m = __uint_as_float(scratch[2]);
+    if (m == 0.f) return;
+    const float w = __fdiv_rn(m, (float)bins);
+    for (long s = blockIdx.x * (long)blockDim.x + threadIdx.x; s < ns;
+         s += (long)gridDim.x * blockDim.x) {
+        const float q = __fdiv_rn(mag(v, s * k), w);
+        int b = (int)q;  // q >= 0: truncation
+        if (b > bins - 1) b = bins - 1;
+        atomicAdd(&hist[b], 1u);
+    }
+}
+
+__global__ void k_tau_hist(const uint32_t *scratch, int bins, float *tau) {
+    const float m = __uint_as_float(scratch[2]);
+    *tau = (m == 0.f) ? 0.f : (float)scratch[0] * __fdiv_rn(m, (float)bins);
+}
 __global__ void k_tau_f32(const uint32_t *sel, float *tau) {
     *tau = __uint_as_float((sel[0] << 15) | sel[1]);
 }
@@ -146,6 +193,34 @@ cudaError_t launch_quantize(int d, int f, const uint16_t *w_cm, uint8_t *q, floa
     if (e != cudaSuccess) return e;
     k_pack<<<dim3(d / kQRows, f / kQChan), 256, 0, s>>>(d, f, w_cm, scale, q);
     return cudaGetLastError();
+}
+
+// Histogram threshold of |v| (bf16 bit patterns or fp32): ns = ceil(n / k)
+// samples v[0], v[k], ...; rank counts within the samples; bins a multiple of
+// 1024, at most 65536. scratch: >= 16 bytes; hist: `bins` words.
+template <typename V>
+cudaError_t launch_hist_quantile(const V *v, long n, long k, long rank, int bins, uint32_t *hist,
+                                 uint32_t *scratch, float *tau_dev, cudaStream_t s) {
+    const long ns = (n + k - 1) / k;
+    cudaError_t e = cudaMemsetAsync(hist, 0, (size_t)bins * sizeof(uint32_t), s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(scratch, 0, 3 * sizeof(uint32_t), s);
+    if (e != cudaSuccess) return e;
+    k_sub_max<V><<<1184, 256, 0, s>>>(v, ns, k, scratch);
+    k_sub_hist<V><<<1184, 256, 0, s>>>(v, ns, k, bins, scratch, hist);
+    k_select<<<1, 1024, 0, s>>>(hist, bins, rank, nullptr, scratch, 0);
+    k_tau_hist<<<1, 1, 0, s>>>(scratch, bins, tau_dev);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_hist_quantile_bf16(const uint16_t *v, long n, long k, long rank, int bins,
+                                      uint32_t *hist, uint32_t *scratch, float *tau_dev,
+                                      cudaStream_t s) {
+    return launch_hist_quantile(v, n, k, rank, bins, hist, scratch, tau_dev, s);
+}
+cudaError_t launch_hist_quantile_f32(const float *v, long n, long k, long rank, int bins,
+                                     uint32_t *hist, uint32_t *scratch, float *tau_dev,
+                                     cudaStream_t s) {
+    return launch_hist_quantile(v, n, k, rank, bins, hist, scratch, tau_dev, s);
 }
 
 // scratch: >= 16 bytes (two selected bins) + 8 bytes (rank); hist: 65536 words

@@ -529,6 +529,57 @@ PROX_API prox_status prox_calibrate(const prox_layer *layer, const uint16_t *x_c
     return PROX_OK;
 }
 
+PROX_API prox_status prox_calibrate_histogram(const prox_layer *layer, const uint16_t *x_cal,
+                                              int n_cal, double keep_x, double keep_s,
+                                              long max_samples, int bins, float *tau_x_out,
+                                              float *tau_s_out, void *ws, size_t ws_bytes,
+                                              void *stream) {
+    prox_status ps = check_layer(layer, false);
+    if (ps != PROX_OK) return ps;
+    if (!x_cal || n_cal < 1 || !tau_x_out || !tau_s_out || !ws || !aligned16(x_cal) ||
+        !aligned16(ws))
+        return PROX_EINVAL;
+    if (!(keep_x >= 0.0 && keep_x <= 1.0) || !(keep_s >= 0.0 && keep_s <= 1.0)) return PROX_EINVAL;
+    if (max_samples < 1 || bins < 1024 || bins > 65536 || bins % 1024 != 0) return PROX_EINVAL;
+    const int d = layer->d_model, f = layer->d_ff;
+    const CalLayout c = cal_layout(d, f, n_cal);
+    if (ws_bytes < c.total) return PROX_ENOMEM;
+    int sms = 0;
+    ps = current_device(&sms);
+    if (ps != PROX_OK) return ps;
+    cudaStream_t st = (cudaStream_t)stream;
+    unsigned char *w = static_cast<unsigned char *>(ws);
+    uint32_t *hist = reinterpret_cast<uint32_t *>(w + c.hist);
+    uint32_t *scratch = reinterpret_cast<uint32_t *>(w + c.scratch);
+    float *tau = reinterpret_cast<float *>(w + c.tau);
+    // every k-th of n pooled values, k = ceil(n / max_samples); the rank counts samples
+    auto stride = [&](long n) { return (n + max_samples - 1) / max_samples; };
+    auto samples = [&](long n) { return (n + stride(n) - 1) / stride(n); };
+    const long nx = (long)n_cal * d;
+    if (launch_hist_quantile_bf16(x_cal, nx, stride(nx), quantile_rank(samples(nx), keep_x), bins,
+                                  hist, scratch, tau, st) != cudaSuccess)
+        return PROX_ECUDA;
+    float tx = 0.f;
+    if (cudaMemcpyAsync(&tx, tau, sizeof(float), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+        return PROX_ECUDA;
+    float *s_all = reinterpret_cast<float *>(w + c.s);
+    ps = run_forward(layer, x_cal, n_cal, tx, 0.f, nullptr, nullptr, nullptr, nullptr, nullptr,
+                     s_all, w + c.fwd, c.s - c.fwd, st, false);
+    if (ps != PROX_OK) return ps;
+    const long ns = (long)n_cal * f;
+    if (launch_hist_quantile_f32(s_all, ns, stride(ns), quantile_rank(samples(ns), keep_s), bins,
+                                 hist, scratch, tau + 1, st) != cudaSuccess)
+        return PROX_ECUDA;
+    float ts = 0.f;
+    if (cudaMemcpyAsync(&ts, tau + 1, sizeof(float), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+        return PROX_ECUDA;
+    *tau_x_out = tx;
+    *tau_s_out = ts;
+    return PROX_OK;
+}
+
 PROX_API prox_status prox_allocate(double e, double alpha, double s1_max, double s2_anchor,
                                    double *s1_out, double *s2_out) {
     if (!s1_out || !s2_out || !(alpha > 0.0) || !(e >= 0.0 && e <= 1.0) ||

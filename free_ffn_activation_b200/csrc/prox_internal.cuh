@@ -112,6 +112,13 @@ cudaError_t launch_stage2(int B, int nchunk, const Stage2Args &a, int grid,
                           size_t smem, cudaStream_t s);
 cudaError_t launch_rmsnorm(int d, int nb, const float *h, float eps, uint16_t *x,
                            cudaStream_t s);
+// histogram threshold of |v| over every k-th of n values (see k_quantize.cu)
+cudaError_t launch_hist_quantile_bf16(const uint16_t *v, long n, long k, long rank, int bins,
+                                      uint32_t *hist, uint32_t *scratch, float *tau_dev,
+                                      cudaStream_t s);
+cudaError_t launch_hist_quantile_f32(const float *v, long n, long k, long rank, int bins,
+                                     uint32_t *hist, uint32_t *scratch, float *tau_dev,
+                                     cudaStream_t s);
 cudaError_t launch_quantize(int d, int f, const uint16_t *w_cm, uint8_t *q,
                             float *scale, cudaStream_t s);
 // exact order statistic of |values| (bf16 or fp32 bit patterns) on device;

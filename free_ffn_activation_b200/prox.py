@@ -69,6 +69,9 @@ def lib() -> C.CDLL:
         L.prox_calibrate_workspace_bytes.restype = sz
         L.prox_calibrate.argtypes = [C.POINTER(_Layer), vp, i, d, d, C.POINTER(C.c_float),
                                      C.POINTER(C.c_float), vp, sz, vp]
+        L.prox_calibrate_histogram.argtypes = [C.POINTER(_Layer), vp, i, d, d, C.c_long, i,
+                                               C.POINTER(C.c_float), C.POINTER(C.c_float), vp,
+                                               sz, vp]
         L.prox_allocate.argtypes = [d, d, d, d, C.POINTER(C.c_double), C.POINTER(C.c_double)]
         L.prox_last_device_status.argtypes = [vp, sz, vp, C.POINTER(C.c_uint32)]
         L.prox_status_str.argtypes = [i]
@@ -80,7 +83,7 @@ def lib() -> C.CDLL:
         L.prox_test_set_wait.argtypes = [C.c_uint32, i]
         L.prox_test_set_wait.restype = None
         for name in ("prox_quantize_proxy", "prox_ffn_forward", "prox_ffn_forward_static",
-                     "prox_rmsnorm_bf16", "prox_ffn_block",
+                     "prox_rmsnorm_bf16", "prox_ffn_block", "prox_calibrate_histogram",
                      "prox_proxy_state",
                      "prox_ffn_stage1", "prox_ffn_stage2",
                      "prox_calibrate", "prox_allocate", "prox_last_device_status"):
@@ -378,6 +381,28 @@ def calibrate(layer: ProxLayer, x_cal: torch.Tensor, keep_x: float, keep_s: floa
     return tx.value, ts.value
 
 
+HIST_SAMPLES, HIST_BINS = 200_000, 4096   # the pages' per-layer calibration budget
+
+
+def calibrate_histogram(layer: ProxLayer, x_cal: torch.Tensor, keep_x: float, keep_s: float,
+                        max_samples: int = HIST_SAMPLES, bins: int = HIST_BINS):
+    """Histogram thresholds (tau_x, tau_s): see prox_calibrate_histogram."""
+    n, d = x_cal.shape
+    _need(x_cal, torch.bfloat16, (n, layer.d_model), "x_cal")
+    nbytes = int(lib().prox_calibrate_workspace_bytes(layer.d_model, layer.d_ff, n))
+    if nbytes == 0:
+        raise ProxError(PROX_EINVAL, "prox_calibrate_workspace_bytes")
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device=x_cal.device)
+    tx, ts = C.c_float(), C.c_float()
+    cl = layer.cstruct()
+    _check(lib().prox_calibrate_histogram(C.byref(cl), _ptr(x_cal), n, float(keep_x),
+                                          float(keep_s), int(max_samples), int(bins),
+                                          C.byref(tx), C.byref(ts), _ptr(ws), nbytes,
+                                          _stream(x_cal.device)),
+           "prox_calibrate_histogram")
+    return tx.value, ts.value
+
+
 def allocate(e: float, alpha: float = 1.0 / 3.0, s1_max: float = 0.7, s2_anchor: float = 0.7):
     """(s1, s2) for a target effective sparsity e (host only)."""
     s1, s2 = C.c_double(), C.c_double()
@@ -418,5 +443,6 @@ def touched_bytes(d_model: int, d_ff: int, k_x: int, k_s: int) -> int:
 __all__ = ["ProxLayer", "ProxError", "quantize_proxy", "workspace", "workspace_bytes",
            "ffn_forward", "ffn_forward_static", "STATIC_WORKSPACE_BYTES", "ffn_forward_raw",
            "ffn_stage1_raw", "ffn_stage2_raw", "rmsnorm_bf16", "ffn_block", "ffn_block_raw",
+           "calibrate_histogram",
            "max_batch_per_pass", "proxy_state", "calibrate", "allocate",
            "last_device_status", "touched_bytes", "untile_proxy", "as_bf16"]

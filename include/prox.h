@@ -265,6 +265,27 @@ prox_status prox_calibrate(const prox_layer *layer, const uint16_t *x_cal, int n
                            float *tau_s_out, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * prox_calibrate_histogram -- prox_calibrate with the pages' bounded
+ * calibration (blog, "Evidence": at most 200,000 activation samples and a
+ * 4,096-bin histogram per layer) instead of the exact order statistic:
+ *   samples: every k-th pooled magnitude, k = ceil(n / max_samples), in pooled
+ *            order (x_cal row by row; s~ token by token, channel by channel);
+ *   bins:    `bins` equal bins of width w = m / bins over [0, m], m the
+ *            largest sample; a sample s falls in bin trunc(fp32(s / w)), m in
+ *            the top bin;
+ *   tau:     fp32(b * w), the lower edge of the bin holding the sample of rank
+ *            floor((1 - keep) * n_samples), so at least the asked-for share of
+ *            samples is kept.
+ *   max_samples >= 1; bins a multiple of 1024 in [1024, 65536] (the pages:
+ *   200000 and 4096). Workspace as prox_calibrate. Synchronises `stream`.
+ * Errors: as prox_calibrate; PROX_EINVAL for max_samples or bins outside range.
+ */
+prox_status prox_calibrate_histogram(const prox_layer *layer, const uint16_t *x_cal, int n_cal,
+                                     double keep_x, double keep_s, long max_samples, int bins,
+                                     float *tau_x_out, float *tau_s_out, void *ws,
+                                     size_t ws_bytes, void *stream);
+
+/*
  * prox_allocate -- split a target effective sparsity between the stages
  * (blog, "Compute budget"): C = 2 alpha (1 - s1) + 3 (1 - s2) and
  * e = 1 - C/3 = s2 - 2 alpha (1 - s1) / 3.

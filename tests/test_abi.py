@@ -163,3 +163,17 @@ def test_unknown_activation_rejected():
     assert st == P.PROX_EINVAL
     L.activation = P.ACT_GEGLU
     assert P.lib().prox_quantize_proxy(250, 768, base, base, base, None) == P.PROX_EINVAL
+
+
+def test_calibrate_histogram_validates():
+    base = 1 << 20
+    L = P._Layer(d_model=256, d_ff=768, w_up_cm=base, w_gate_cm=base * 2, w_down=base * 3,
+                 q_up=base * 4, q_gate=base * 5, s_up=base * 6, s_gate=base * 7)
+    tx, ts = C.c_float(), C.c_float()
+    wsb = P.lib().prox_calibrate_workspace_bytes(256, 768, 4)
+    call = lambda ms, bins, wb=wsb: P.lib().prox_calibrate_histogram(
+        C.byref(L), base * 8, 4, 0.5, 0.3, ms, bins, C.byref(tx), C.byref(ts), base * 9, wb, None)
+    assert call(0, 4096) == P.PROX_EINVAL          # no samples
+    assert call(200000, 4000) == P.PROX_EINVAL     # bins not a multiple of 1024
+    assert call(200000, 131072) == P.PROX_EINVAL   # too many bins
+    assert call(200000, 4096, wsb - 1) == P.PROX_ENOMEM

@@ -189,6 +189,38 @@ def test_calibrate_c1(c1):
     assert abs(ts - c1.tau_s) <= 1e-5 * c1.tau_s, (ts, c1.tau_s)
 
 
+def _check_hist_calibration(case):
+    # the device's histogram thresholds equal the oracle's histogram quantile
+    # of the same pooled values bit for bit (|x| exactly, s~ as the device
+    # computed it), and stay within one bin of the oracle's own calibration
+    tx, ts = P.calibrate_histogram(case.layer, to_dev_bf16(case.x_cal, "cuda"),
+                                   case.keep_x, case.keep_s)
+    ax = S.bf16_to_f32(case.x_cal)
+    assert np.float32(tx) == np.float32(oracle.hist_quantile(ax, case.keep_x))
+    s_dev, _ = P.proxy_state(case.layer, to_dev_bf16(case.x_cal, "cuda"), tx)
+    s_dev = s_dev.cpu().numpy()
+    assert np.float32(ts) == np.float32(oracle.hist_quantile(s_dev, case.keep_s))
+    otx, ots = oracle.calibrate_hist(case.x_cal, case.Por, case.keep_x, case.keep_s, act=case.act)
+    w = np.float32(np.abs(s_dev).max()) / np.float32(oracle.HIST_BINS)
+    assert otx == tx and abs(ots - ts) <= 1.0001 * w
+    # against the exact order statistic: the asked-for share is kept, up to
+    # the sampling error of the bounded sample (about 1e-3 at 200k samples)
+    kept_x = (np.abs(ax) >= np.float32(tx)).mean()
+    kept_s = (np.abs(s_dev) >= np.float32(ts)).mean()
+    print(f"[hist calibration] tau_x {tx:.6g} (exact {case.tau_x:.6g}) kept {kept_x:.4f}; "
+          f"tau_s {ts:.6g} (exact {case.tau_s:.6g}) kept {kept_s:.4f}")
+    assert kept_x >= case.keep_x - 3e-3 and kept_s >= case.keep_s - 3e-3
+
+
+def test_calibrate_histogram_c1(c1):
+    _check_hist_calibration(c1)
+
+
+def test_calibrate_histogram_c2(c2):
+    # 512 x 12288 s~ values: 6.3 M pooled, sampled every 32nd (196,608 samples)
+    _check_hist_calibration(c2)
+
+
 def test_geglu_proxy_state_c1(c1g):
     _proxy_check(c1g, list(range(16)))
 
