@@ -93,6 +93,17 @@ def stage2_traffic(workload, batch):
         return None
 
 
+def max_over_ranks(x, world, dev):
+    """Largest x over the ranks: the job's time is its slowest rank's."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -326,10 +337,7 @@ def run_ours(args, w, rank, world, local_rank):
             s1_ms += [ev_s[t].elapsed_time(ev_a[t]) for t in sampled]
             s2_ms += [ev_a[t].elapsed_time(ev_b[t]) for t in sampled]
     ms_total = e0.elapsed_time(e1)
-    if world > 1:
-        tt = torch.tensor([ms_total], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_total = float(tt.item())
+    ms_total = max_over_ranks(ms_total, world, dev)
     ms_step = ms_total / args.steps
     us_tok = ms_step * 1e3 / (ntok * world)
     us_tok_rank = ms_step * 1e3 / ntok
@@ -368,10 +376,7 @@ def run_ours(args, w, rank, world, local_rank):
     f1.record(stream)
     barrier()
     e2e_ms = f0.elapsed_time(f1) / e2e_steps
-    if world > 1:
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms = max_over_ranks(e2e_ms, world, dev)
     e2e_us = e2e_ms * 1e3 / (ntok * world)
 
     # dense bf16 reference on the same GPU, same protocol (cuBLAS GEMV)
@@ -529,10 +534,7 @@ def run_stack(args, w, rank, world, local_rank):
         e1.record(stream)
         torch.cuda.synchronize(dev)
     ms_total = e0.elapsed_time(e1)
-    if world > 1:
-        tt = torch.tensor([ms_total], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_total = float(tt.item())
+    ms_total = max_over_ranks(ms_total, world, dev)
     ms_step = ms_total / args.steps
     us_tok = ms_step * 1e3 / ntok                     # all layers, per token (per rank)
     # touched bytes: realised keep ratios of the last step's tokens, layer by layer

@@ -1,0 +1,73 @@
+"""Host-side logic of the benchmark's multi-process launch (no GPU).
+
+The path does not shard (replicas only): N ranks run independent replicas, the
+job's time is the slowest rank's (max over ranks), and the reference arm runs
+on rank 0 alone. These run as world-size-2 gloo processes on the CPU."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, port, out_dir):
+    sys.path.insert(0, ROOT)
+    import bench
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=2)
+    try:
+        v = bench.max_over_ranks(1.5 + rank, 2, "cpu")
+    finally:
+        dist.destroy_process_group()
+    with open(os.path.join(out_dir, f"r{rank}.txt"), "w") as f:
+        f.write(repr(v))
+
+
+def test_max_over_ranks_gloo(tmp_path):
+    mp.spawn(_rank_main, args=(_free_port(), str(tmp_path)), nprocs=2, join=True)
+    got = [float(open(tmp_path / f"r{r}.txt").read()) for r in range(2)]
+    assert got == [2.5, 2.5]
+
+
+def test_max_over_ranks_single_process():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(3.25, 1, "cpu") == 3.25
+
+
+def _run_reference(rank, world):
+    env = dict(os.environ, RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank),
+               MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
+    return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                           "--workload", "tiny-ffn", "--gpus", str(world), "--steps", "1",
+                           "--warmup", "1", "--cpu-seconds", "0.5"],
+                          env=env, capture_output=True, text=True, timeout=600)
+
+
+def test_reference_arm_rank0_prints_one_line():
+    r = _run_reference(0, 2)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["higher_is_better"] is False
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_reference_arm_other_ranks_exit_quietly():
+    r = _run_reference(1, 2)
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert not [l for l in r.stdout.splitlines() if l.startswith("{")]
