@@ -52,27 +52,28 @@ def _declare(L):
     L.oracle_quantize_proxy.restype = None
     L.oracle_stage1_token.argtypes = [i, i, _u16p, f, _u8p, _f32p, _u8p, _f32p, f,
                                       _Opt(_u8p), _Opt(_f64p), _Opt(_f64p), _Opt(_f64p),
-                                      _Opt(_u8p), i]
+                                      _Opt(_u8p), i, _Opt(_u16p), _Opt(_u16p)]
     L.oracle_stage1_token.restype = None
     L.oracle_stage2_token.argtypes = [i, i, _u16p, _u16p, _u16p, _u16p, _u8p,
                                       _Opt(_f64p), _f64p, i]
     L.oracle_stage2_token.restype = None
     L.oracle_forward.argtypes = [i, i, i, _u16p, f, f, _u16p, _u16p, _u16p, _u8p, _f32p,
                                  _u8p, _f32p, _Opt(_u8p), _Opt(_u8p), _Opt(_u8p),
-                                 _Opt(_f64p), _Opt(_f64p), _f64p, i, i]
+                                 _Opt(_f64p), _Opt(_f64p), _f64p, i, i, _Opt(_u16p), _Opt(_u16p)]
     L.oracle_forward.restype = C.c_int
     L.oracle_quantile_rank.argtypes = [C.c_long, d]
     L.oracle_quantile_rank.restype = C.c_long
     L.oracle_order_statistic.argtypes = [_f64p, C.c_long, d]
     L.oracle_order_statistic.restype = C.c_float
     L.oracle_calibrate.argtypes = [i, i, i, _u16p, _u8p, _f32p, _u8p, _f32p, d, d,
-                                   C.POINTER(C.c_float), C.POINTER(C.c_float), i, i]
+                                   C.POINTER(C.c_float), C.POINTER(C.c_float), i, i,
+                                   _Opt(_u16p), _Opt(_u16p)]
     L.oracle_calibrate.restype = None
     L.oracle_hist_quantile.argtypes = [_f32p, C.c_long, d, C.c_long, i]
     L.oracle_hist_quantile.restype = C.c_float
     L.oracle_calibrate_hist.argtypes = [i, i, i, _u16p, _u8p, _f32p, _u8p, _f32p, d, d,
                                         C.c_long, i, C.POINTER(C.c_float),
-                                        C.POINTER(C.c_float), i, i]
+                                        C.POINTER(C.c_float), i, i, _Opt(_u16p), _Opt(_u16p)]
     L.oracle_calibrate_hist.restype = None
     L.oracle_rmsnorm_bf16.argtypes = [i, _f32p, d, _u16p]
     L.oracle_rmsnorm_bf16.restype = None
@@ -99,16 +100,22 @@ def quantize_proxy(w_cm: np.ndarray):
 ACT_SWIGLU, ACT_GEGLU = 0, 1   # gate activation: SiLU (SwiGLU) or GELU (GeGLU)
 
 
-def stage1(x, tau_x, q_up, s_up, q_gate, s_gate, tau_s, act=ACT_SWIGLU):
-    """Stage 1 for one token. Returns dict mask_x, u, g, s (fp64), mask_s."""
+def stage1(x, tau_x, q_up, s_up, q_gate, s_gate, tau_s, act=ACT_SWIGLU, pw_up=None,
+           pw_gate=None):
+    """Stage 1 for one token. Returns dict mask_x, u, g, s (fp64), mask_s.
+    With pw_up/pw_gate (bf16 [d_ff][d_model]) the proxy is those weights."""
     d_model = x.shape[-1]
     d_ff = q_up.shape[1] * 2
     out = dict(mask_x=np.zeros(d_model, np.uint8), u=np.zeros(d_ff), g=np.zeros(d_ff),
                s=np.zeros(d_ff), mask_s=np.zeros(d_ff, np.uint8))
     lib().oracle_stage1_token(d_model, d_ff, _u16(x), float(tau_x), q_up, s_up, q_gate,
                               s_gate, float(tau_s), out["mask_x"], out["u"], out["g"],
-                              out["s"], out["mask_s"], int(act))
+                              out["s"], out["mask_s"], int(act), _opt16(pw_up), _opt16(pw_gate))
     return out
+
+
+def _opt16(a):
+    return None if a is None else _u16(a)
 
 
 def stage2(x, w_up_cm, w_gate_cm, w_down, mask_s, act=ACT_SWIGLU):
@@ -146,7 +153,8 @@ def forward(x, tau_x, tau_s, layer: dict, proxy: dict, mask_s_in=None, n_threads
         d_model, d_ff, b, x, float(tau_x), float(tau_s), _u16(layer["w_up_cm"]),
         _u16(layer["w_gate_cm"]), _u16(layer["w_down"]), proxy["q_up"], proxy["s_up"],
         proxy["q_gate"], proxy["s_gate"], ms_in, out.get("mask_x"), out.get("mask_s"),
-        out.get("s_proxy"), out.get("s_exact"), out["y"], int(n_threads), int(act))
+        out.get("s_proxy"), out.get("s_exact"), out["y"], int(n_threads), int(act),
+        _opt16(proxy.get("pw_up")), _opt16(proxy.get("pw_gate")))
     return out
 
 
@@ -167,7 +175,8 @@ def calibrate(x_cal, proxy: dict, keep_x: float, keep_s: float, n_threads=0, act
     tx, ts = C.c_float(), C.c_float()
     lib().oracle_calibrate(d_model, d_ff, n, x_cal, proxy["q_up"], proxy["s_up"],
                            proxy["q_gate"], proxy["s_gate"], float(keep_x), float(keep_s),
-                           C.byref(tx), C.byref(ts), int(n_threads), int(act))
+                           C.byref(tx), C.byref(ts), int(n_threads), int(act),
+                           _opt16(proxy.get("pw_up")), _opt16(proxy.get("pw_gate")))
     return tx.value, ts.value
 
 
@@ -192,7 +201,8 @@ def calibrate_hist(x_cal, proxy: dict, keep_x: float, keep_s: float,
     lib().oracle_calibrate_hist(d_model, d_ff, n, x_cal, proxy["q_up"], proxy["s_up"],
                                 proxy["q_gate"], proxy["s_gate"], float(keep_x), float(keep_s),
                                 int(max_samples), int(bins), C.byref(tx), C.byref(ts),
-                                int(n_threads), int(act))
+                                int(n_threads), int(act), _opt16(proxy.get("pw_up")),
+                                _opt16(proxy.get("pw_gate")))
     return tx.value, ts.value
 
 
@@ -214,6 +224,16 @@ def allocate(e: float, alpha: float = 1.0 / 3.0, s1_max: float = 0.7,
 
 def effective_sparsity(s1: float, s2: float, alpha: float = 1.0 / 3.0) -> float:
     return lib().oracle_effective_sparsity(s1, s2, alpha)
+
+
+def make_proxy_bf16(layer: dict) -> dict:
+    """The bf16-proxy ablation: the proxy is the original bf16 weight (the INT4
+    codes and scales below are unused placeholders of the right shapes)."""
+    d_ff, d_model = layer["w_up_cm"].shape
+    z8 = np.zeros((d_model, d_ff // 2), np.uint8)
+    z32 = np.zeros(d_model, np.float32)
+    return {"q_up": z8, "s_up": z32, "q_gate": z8, "s_gate": z32,
+            "pw_up": layer["w_up_cm"], "pw_gate": layer["w_gate_cm"]}
 
 
 def make_proxy(layer: dict) -> dict:

@@ -132,7 +132,10 @@ static double proxy_weight(const uint8_t *q, const float *scale, int d_ff,
  *   u~ = Pi_in(x, W~_up, m_x),  h~ = SiLU(Pi_in(x, W~_gate, m_x))
  *   s~ = u~ (.) h~,             [m_s]_j = 1[|s~_j| >= tau_s]
  * with Pi_in(x, W, m) = x_[I(m)] W_[I(m), :]   [arxiv 2.2].
- * x enters unquantised; only the weights are INT4.
+ * x enters unquantised; only the weights are INT4. With pw_up and pw_gate
+ * given (bf16 [d_ff][d_model], the original weights) the proxy is that bf16
+ * weight instead of the INT4 copy: the FP16/bf16-proxy ablation of the blog's
+ * "Evidence" section (q and scale are then ignored).
  * Outputs: mask_x[d_model], u_proxy/g_proxy/s_proxy[d_ff] (g is the
  * pre-activation proxy gate), mask_s[d_ff]. Any output may be NULL.
  * ---------------------------------------------------------------------- */
@@ -140,7 +143,8 @@ void oracle_stage1_token(int d_model, int d_ff, const uint16_t *x, float tau_x,
                          const uint8_t *q_up, const float *s_up,
                          const uint8_t *q_gate, const float *s_gate,
                          float tau_s, uint8_t *mask_x, double *u_proxy,
-                         double *g_proxy, double *s_proxy, uint8_t *mask_s, int act)
+                         double *g_proxy, double *s_proxy, uint8_t *mask_s, int act,
+                         const uint16_t *pw_up, const uint16_t *pw_gate)
 {
     uint8_t *mx = (uint8_t *)malloc((size_t)d_model);
     for (int i = 0; i < d_model; ++i)
@@ -156,8 +160,10 @@ void oracle_stage1_token(int d_model, int d_ff, const uint16_t *x, float tau_x,
             continue;
         double xi = bf16_value(x[i]);
         for (int j = 0; j < d_ff; ++j) {
-            u[j] += xi * proxy_weight(q_up, s_up, d_ff, i, j);
-            g[j] += xi * proxy_weight(q_gate, s_gate, d_ff, i, j);
+            u[j] += xi * (pw_up ? bf16_value(pw_up[(size_t)j * d_model + i])
+                                : proxy_weight(q_up, s_up, d_ff, i, j));
+            g[j] += xi * (pw_gate ? bf16_value(pw_gate[(size_t)j * d_model + i])
+                                  : proxy_weight(q_gate, s_gate, d_ff, i, j));
         }
     }
     for (int j = 0; j < d_ff; ++j) {
@@ -221,7 +227,8 @@ int oracle_forward(int d_model, int d_ff, int batch, const uint16_t *x,
                    const float *s_up, const uint8_t *q_gate,
                    const float *s_gate, const uint8_t *mask_s_in,
                    uint8_t *mask_x, uint8_t *mask_s, double *s_proxy,
-                   double *s_exact, double *y, int n_threads, int act)
+                   double *s_exact, double *y, int n_threads, int act,
+                   const uint16_t *pw_up, const uint16_t *pw_gate)
 {
     int used = 1;
 #ifdef _OPENMP
@@ -244,7 +251,8 @@ int oracle_forward(int d_model, int d_ff, int batch, const uint16_t *x,
                                 s_gate, tau_s,
                                 mask_x ? mask_x + (size_t)t * d_model : NULL,
                                 NULL, NULL,
-                                s_proxy ? s_proxy + (size_t)t * d_ff : NULL, ms, act);
+                                s_proxy ? s_proxy + (size_t)t * d_ff : NULL, ms, act,
+                                pw_up, pw_gate);
             const uint8_t *use = mask_s_in ? mask_s_in + (size_t)t * d_ff : ms;
             oracle_stage2_token(d_model, d_ff, xt, w_up_cm, w_gate_cm, w_down,
                                 use,
@@ -352,7 +360,8 @@ void oracle_calibrate(int d_model, int d_ff, int n_cal, const uint16_t *x_cal,
                       const uint8_t *q_up, const float *s_up,
                       const uint8_t *q_gate, const float *s_gate,
                       double keep_x, double keep_s, float *tau_x_out,
-                      float *tau_s_out, int n_threads, int act)
+                      float *tau_s_out, int n_threads, int act,
+                      const uint16_t *pw_up, const uint16_t *pw_gate)
 {
     long nx = (long)n_cal * d_model;
     double *ax = (double *)malloc(sizeof(double) * (size_t)nx);
@@ -373,7 +382,7 @@ void oracle_calibrate(int d_model, int d_ff, int n_cal, const uint16_t *x_cal,
     for (int t = 0; t < n_cal; ++t)
         oracle_stage1_token(d_model, d_ff, x_cal + (size_t)t * d_model, tau_x,
                             q_up, s_up, q_gate, s_gate, 0.0f, NULL, NULL, NULL,
-                            sv + (size_t)t * d_ff, NULL, act);
+                            sv + (size_t)t * d_ff, NULL, act, pw_up, pw_gate);
     *tau_s_out = oracle_order_statistic(sv, ns, keep_s);
     *tau_x_out = tau_x;
     free(sv);
@@ -386,7 +395,8 @@ void oracle_calibrate_hist(int d_model, int d_ff, int n_cal, const uint16_t *x_c
                            const uint8_t *q_up, const float *s_up,
                            const uint8_t *q_gate, const float *s_gate,
                            double keep_x, double keep_s, long max_samples, int bins,
-                           float *tau_x_out, float *tau_s_out, int n_threads, int act)
+                           float *tau_x_out, float *tau_s_out, int n_threads, int act,
+                           const uint16_t *pw_up, const uint16_t *pw_gate)
 {
     long nx = (long)n_cal * d_model;
     float *ax = (float *)malloc(sizeof(float) * (size_t)nx);
@@ -407,7 +417,7 @@ void oracle_calibrate_hist(int d_model, int d_ff, int n_cal, const uint16_t *x_c
     for (int t = 0; t < n_cal; ++t)
         oracle_stage1_token(d_model, d_ff, x_cal + (size_t)t * d_model, tau_x,
                             q_up, s_up, q_gate, s_gate, 0.0f, NULL, NULL, NULL,
-                            sv + (size_t)t * d_ff, NULL, act);
+                            sv + (size_t)t * d_ff, NULL, act, pw_up, pw_gate);
     float *sf = (float *)malloc(sizeof(float) * (size_t)ns);
     for (long k = 0; k < ns; ++k)
         sf[k] = (float)sv[k];

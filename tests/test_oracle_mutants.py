@@ -43,6 +43,8 @@ MUTANTS = {
     "rms_sum_not_mean": ("sqrt(ss / (double)d + eps)", "sqrt(ss + eps)"),
     "rms_eps_dropped": ("sqrt(ss / (double)d + eps)", "sqrt(ss / (double)d)"),
     "bf16_truncates": ("nearbyint(fabs(v) / q) * q", "floor(fabs(v) / q) * q"),
+    "bf16_proxy_transposed": ("u[j] += xi * (pw_up ? bf16_value(pw_up[(size_t)j * d_model + i])",
+                              "u[j] += xi * (pw_up ? bf16_value(pw_up[((size_t)i * d_ff + j) % ((size_t)d_ff * d_model)])"),
     "hist_upper_edge": ("    return (float)sel * w;", "    return (float)(sel + 1) * w;"),
     "hist_no_subsample": ("    long k = (n + max_samples - 1) / max_samples;",
                           "    long k = 1;"),

@@ -453,3 +453,32 @@ def test_hist_quantile_brackets_the_order_statistic():
         tx = oracle.order_statistic(v.astype(np.float64), keep)
         w = np.float32(np.abs(v).max()) / np.float32(4096)
         assert th <= tx < th + w * 1.0001, (n, keep, th, tx, w)
+
+
+# ---------------------------------------------------------------------------
+# bf16-proxy ablation (blog, "Evidence", ablation A1: the proxy at full
+# precision instead of INT4): the proxy is the original weight
+# ---------------------------------------------------------------------------
+
+def test_bf16_proxy_at_zero_tau_x_is_the_exact_state():
+    # with every input kept, Stage 1 with the bf16 proxy computes the same
+    # sums in the same order as Stage 2's exact u and g: s~ == s bit for bit
+    L = small_layer(64, 256, seed=2)
+    P = oracle.make_proxy_bf16(L)
+    x = S.make_tokens(3, 64, seed=2)
+    out = oracle.forward(x, 0.0, 0.0, L, P)
+    assert np.array_equal(out["s_proxy"], out["s_exact"])
+
+
+def test_bf16_proxy_masked_state_matches_numpy():
+    # with tau_x > 0 the proxy state is (x (.) m_x) W_up  (.) SiLU((x (.) m_x) W_gate)
+    L = small_layer(64, 256, seed=4)
+    P = oracle.make_proxy_bf16(L)
+    x = S.make_tokens(4, 64, seed=4)
+    tau_x = 0.7
+    out = oracle.forward(x, tau_x, 0.0, L, P)
+    xd = f64(x)
+    xm = np.where(np.abs(xd) >= tau_x, xd, 0.0)
+    u = xm @ f64(L["w_up_cm"]).T
+    g = xm @ f64(L["w_gate_cm"]).T
+    assert rel(out["s_proxy"], u * g * expit(g)) < 1e-12
