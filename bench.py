@@ -59,6 +59,8 @@ def parse():
     ap.add_argument("--effective-sparsity", type=float, default=None,
                     help="target effective sparsity e: keep ratios from the budget split "
                          "(prox_allocate, alpha 1/3, s1 <= 0.7) instead of --keep-x/--keep-s")
+    ap.add_argument("--proxy", choices=["int4", "bf16"], default="int4",
+                    help="proxy kind: the method's INT4 proxy or the bf16-proxy ablation")
     ap.add_argument("--batch", type=int, default=1,
                     help="tokens per forward call (each token keeps its own masks)")
     ap.add_argument("--copies", type=int, default=4, help="rotating weight copies (L2 defeat)")
@@ -235,12 +237,14 @@ def run_ours(args, w, rank, world, local_rank):
     L = S.make_layer(S.LayerSpec(d, f, sigma=w["sigma"], seed=0))
     x_np = S.make_tokens(ntok, d, seed=rank, stream="x_eval", outlier_frac=w["outlier"])
     xc_np = S.make_tokens(w["n_cal"], d, seed=0, stream="x_cal", outlier_frac=w["outlier"])
-    base = P.ProxLayer.from_weights(L["w_up_cm"], L["w_gate_cm"], L["w_down"], device=dev)
+    pk = P.PROXY_BF16 if args.proxy == "bf16" else P.PROXY_INT4
+    base = P.ProxLayer.from_weights(L["w_up_cm"], L["w_gate_cm"], L["w_down"], device=dev,
+                                    proxy_kind=pk)
     tau_x, tau_s = P.calibrate(base, P.as_bf16(xc_np, dev), args.keep_x, args.keep_s)
     R = max(1, args.copies)
-    layers = [base] + [P.ProxLayer(*(t.clone() for t in (
-        base.w_up_cm, base.w_gate_cm, base.w_down, base.q_up, base.q_gate, base.s_up, base.s_gate)))
-        for _ in range(R - 1)]
+    layers = [base] + [P.ProxLayer(*(None if t is None else t.clone() for t in (
+        base.w_up_cm, base.w_gate_cm, base.w_down, base.q_up, base.q_gate, base.s_up, base.s_gate)),
+        proxy_kind=pk) for _ in range(R - 1)]
     structs = [lay.cstruct() for lay in layers]
     x = P.as_bf16(x_np, dev).contiguous()
     y = torch.empty((ntok, d), dtype=torch.float32, device=dev)
@@ -257,7 +261,7 @@ def run_ours(args, w, rank, world, local_rank):
     msu = out.mask_s.view(ngrp, Bt, f).amax(dim=1)
     kx = mxu.sum(dim=1).double().cpu().numpy()          # per call
     ks = msu.sum(dim=1).double().cpu().numpy()
-    touched = np.array([P.touched_bytes(d, f, int(a), int(b)) for a, b in zip(kx, ks)])
+    touched = np.array([P.touched_bytes(d, f, int(a), int(b), pk) for a, b in zip(kx, ks)])
     stage2_bytes = 3 * ks * d * 2
     kx_tok = out.mask_x.sum(dim=1).double().mean().item()
     ks_tok = out.count_s.double().mean().item()
@@ -434,15 +438,16 @@ def run_ours(args, w, rank, world, local_rank):
             "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
             "config": {"workload": args.workload, "d_model": d, "d_ff": f, "batch": Bt,
+                       "proxy": args.proxy,
                        "tokens_per_step": ntok, "keep_x": args.keep_x, "keep_s": args.keep_s,
                        "tau_x": tau_x, "tau_s": tau_s,
-                       "l2": f"{R} rotating weight copies ({R * (3 * d * f * 2 + d * f + 8 * d) / 1e9:.2f} GB > L2)",
+                       "l2": f"{R} rotating weight copies ({R * (3 * d * f * 2 + (d * f + 8 * d if pk == P.PROXY_INT4 else 4 * d * f)) / 1e9:.2f} GB > L2)",
                        "parallelism": f"replicas x{world}"},
             "roofline": {"bound": "hbm", "kernel": "k_stage2 (exact up/gate/down)",
                          "achieved": s2_gbs, "peak": peak, "unit": "GB/s",
-                         "frac": s2_gbs / peak, "traffic": stage2_traffic(args.workload, Bt), "peak_source": peak_src,
+                         "frac": s2_gbs / peak, "traffic": stage2_traffic(args.workload, Bt) if args.proxy == "int4" else None, "peak_source": peak_src,
                          "bytes_per_launch": s2_bytes, "us_per_launch": s2_us},
-            "stage1": {"kernel": "k_stage1 (INT4 proxy + channel mask)", "us_per_launch": s1_us,
+            "stage1": {"kernel": f"k_stage1 ({args.proxy} proxy + channel mask)", "us_per_launch": s1_us,
                        "bytes_per_launch": s1_bytes, "GBps": s1_gbs, "frac": s1_gbs / peak},
             "effective_sparsity": None if args.effective_sparsity is None else {
                 "target": args.effective_sparsity,

@@ -74,6 +74,23 @@ __global__ void __launch_bounds__(256) k_pack(int d, int f, const uint16_t *__re
         make_uint4(out[0], out[1], out[2], out[3]);
 }
 
+// bf16 proxy tiles: q16[(c * d + i) * 256 + k] = w[(256 c + k) * d + i], a
+// tiled transpose through shared memory (32 rows x 256 channels per CTA)
+__global__ void __launch_bounds__(256) k_tile_bf16(int d, const uint16_t *__restrict__ w,
+                                                   uint16_t *__restrict__ q16) {
+    __shared__ uint16_t tile[kQChan][kQRows + 2];
+    const int i0 = blockIdx.x * kQRows, c = blockIdx.y;
+    for (int k = threadIdx.x; k < kQChan * kQRows; k += 256) {
+        const int jj = k / kQRows, ii = k % kQRows;
+        tile[jj][ii] = w[(size_t)(c * kCB + jj) * d + i0 + ii];
+    }
+    __syncthreads();
+    for (int k = threadIdx.x; k < kQChan * kQRows; k += 256) {
+        const int ii = k / kQChan, jj = k % kQChan;
+        q16[((size_t)c * d + i0 + ii) * kCB + jj] = tile[jj][ii];
+    }
+}
+
 __global__ void k_hist_bf16_abs(const uint16_t *__restrict__ v, long n, uint32_t *hist) {
     for (long k = blockIdx.x * (long)blockDim.x + threadIdx.x; k < n;
          k += (long)gridDim.x * blockDim.x)
@@ -185,6 +202,11 @@ __global__ void k_tau_f32(const uint32_t *sel, float *tau) {
 }
 
 }  // namespace
+
+cudaError_t launch_tile_bf16(int d, int f, const uint16_t *w_cm, uint16_t *q16, cudaStream_t s) {
+    k_tile_bf16<<<dim3(d / kQRows, f / kCB), 256, 0, s>>>(d, w_cm, q16);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_quantize(int d, int f, const uint16_t *w_cm, uint8_t *q, float *scale,
                             cudaStream_t s) {

@@ -41,29 +41,37 @@ namespace cg = cooperative_groups;
 namespace prox {
 namespace {
 
+// Proxy kinds (PK): 0 = INT4 codes, two per byte (the method's proxy);
+// 1 = bf16 weights (the FP16/bf16-proxy ablation of the blog's "Evidence").
 // channels per thread: a warp covers whole rows of one row lane
-__host__ __device__ constexpr int s1_cpt(int B, int NB) {
-    return (B <= 2 && NB == 2) ? 32 : (B <= 4 ? 16 : 8);
+__host__ __device__ constexpr int s1_cpt(int B, int NB, int PK = 0) {
+    return PK ? 8 : ((B <= 2 && NB == 2) ? 32 : (B <= 4 ? 16 : 8));
 }
+// bytes of one row a thread moves per copy, and bytes of one row of a block
+__host__ __device__ constexpr int s1_bytes(int B, int NB, int PK) {
+    return PK ? 16 : s1_cpt(B, NB) / 2;
+}
+__host__ __device__ constexpr int s1_gran(int PK) { return PK ? kCB * 2 : kCB / 2; }
 // deepest per-thread ring (rows in flight) and the ring bytes it takes
 __host__ __device__ constexpr int s1_ring_bytes(int B) { return B <= 2 ? 192 : (B == 4 ? 256 : 128); }
-__host__ __device__ constexpr int s1_dmax(int B, int NB) {
-    return s1_ring_bytes(B) / (s1_cpt(B, NB) / 2) < 32 ? s1_ring_bytes(B) / (s1_cpt(B, NB) / 2)
-                                                          : 32;
+__host__ __device__ constexpr int s1_dmax(int B, int NB, int PK = 0) {
+    return s1_ring_bytes(B) / s1_bytes(B, NB, PK) < 32 ? s1_ring_bytes(B) / s1_bytes(B, NB, PK)
+                                                        : 32;
 }
 
-template <int B, int NB>
+template <int B, int NB, int PK = 0>
 struct S1 {
     static constexpr int CW = NB * kCB;                              // channels per CTA
-    static constexpr int CPT = s1_cpt(B, NB);                        // channels per thread
-    static constexpr int BYTES = CPT / 2;                            // bytes per row per thread
+    static constexpr int CPT = s1_cpt(B, NB, PK);                    // channels per thread
+    static constexpr int BYTES = s1_bytes(B, NB, PK);                // bytes per row per thread
+    static constexpr int GRAN = s1_gran(PK);                         // bytes per row per block
     static constexpr int WORDS = BYTES / 4;
     static constexpr int ACC = B * CPT;
     static constexpr int TPRB = kCB / CPT;                           // threads per block per matrix
     static constexpr int TPRM = CW / CPT;                            // threads per row per matrix
     static constexpr int TPR = 2 * TPRM;                             // threads per row
     static constexpr int RL = kS1Threads / TPR;                      // row lanes
-    static constexpr int DMAX = s1_dmax(B, NB);                      // deepest ring (rows)
+    static constexpr int DMAX = s1_dmax(B, NB, PK);                  // deepest ring (rows)
     static constexpr int KMAX = (B == 8 ? 4096 : 8192) / 8 / kS1Threads;  // x chunks per thread
 };
 
@@ -119,6 +127,19 @@ __device__ __forceinline__ void proc_word(uint32_t w0, int wi, const float *xs, 
     }
 }
 
+// bf16 proxy: word wi of a thread's 16-byte chunk holds channels 2 wi (low
+// half) and 2 wi + 1 (high half); acc2[(t * CPT + 2 wi) / 2] gains xs[t] * w
+template <int B, int CPT>
+__device__ __forceinline__ void proc_word_bf16(uint32_t w, int wi, const float *xs, float2 *acc2) {
+    const float2 dw = make_float2(bf16lo(w), bf16hi(w));
+#pragma unroll
+    for (int t = 0; t < B; ++t) {
+        const float2 xx = make_float2(xs[t], xs[t]);
+        float2 *a = acc2 + (t * CPT + wi * 2) / 2;
+        a[0] = __ffma2_rn(xx, dw, a[0]);
+    }
+}
+
 // deterministic block-wide exclusive scan of one int per thread (256 threads)
 __device__ __forceinline__ int block_excl_scan(int v, int *warp_tot, int &total) {
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
@@ -151,12 +172,12 @@ struct S1Smem {
 };
 
 __host__ __device__ inline S1Smem s1_smem(int d, int B, int NB, int unit_cap, int depth_sel,
-                                         int n_r = kS1MaxRowGroups) {
+                                         int n_r = kS1MaxRowGroups, int PK = 0) {
     const int cw = NB * kCB;
-    const int cpt = s1_cpt(B, NB);
+    const int cpt = s1_cpt(B, NB, PK);
     const int rl = kS1Threads / (2 * (cw / cpt));
     const size_t red = (size_t)rl * 2 * B * (cw + cw / cpt) * 4;    // padded row-lane sums
-    const size_t ring = (size_t)kS1Threads * (s1_dmax(B, NB) >> depth_sel) * (cpt / 2);
+    const size_t ring = (size_t)kS1Threads * (s1_dmax(B, NB, PK) >> depth_sel) * s1_bytes(B, NB, PK);
     (void)d;
     S1Smem s;
     size_t o = 0;
@@ -179,11 +200,11 @@ namespace {
 // through a private ring of D shared-memory slots, refilling each slot with
 // the row D positions later as soon as its words are decoded. ssum collects
 // the thread's sum of x_i * scale_i * 2^E (for the +8 code offset).
-template <int B, int NB, int D>
+template <int B, int NB, int PK, int D>
 __device__ __forceinline__ void s1_stream(const uint8_t *qbase, unsigned char *ring,
                                           const int *rowidx, const float *xs, int rl, int m,
                                           int n_rows, float2 *acc2, float *ssum) {
-    using T = S1<B, NB>;
+    using T = S1<B, NB, PK>;
     // slot-major ring (ring[slot][thread]): a warp's accesses to one slot are
     // consecutive words, free of bank conflicts
     unsigned char *myring = ring + (size_t)threadIdx.x * T::BYTES;
@@ -192,7 +213,7 @@ __device__ __forceinline__ void s1_stream(const uint8_t *qbase, unsigned char *r
 #pragma unroll 1
     for (int k = 0; k < D; ++k) {
         if (k < n_rows)
-            cp_async<T::BYTES>(myring + k * SLOT, qbase + (size_t)rowidx[rl + k * T::RL] * (kCB / 2),
+            cp_async<T::BYTES>(myring + k * SLOT, qbase + (size_t)rowidx[rl + k * T::RL] * T::GRAN,
                                pol);
         cp_commit();
     }
@@ -218,25 +239,30 @@ __device__ __forceinline__ void s1_stream(const uint8_t *qbase, unsigned char *r
             ssum[t] += xv[t];
         }
 #pragma unroll
-        for (int q = 0; q < T::WORDS; ++q) proc_word<B, T::CPT>(w[q], q, xv, acc2);
+        for (int q = 0; q < T::WORDS; ++q) {
+            if constexpr (PK == 0)
+                proc_word<B, T::CPT>(w[q], q, xv, acc2);
+            else
+                proc_word_bf16<B, T::CPT>(w[q], q, xv, acc2);
+        }
         const int kn = k + D;
         if (kn < n_rows)
-            cp_async<T::BYTES>(myring + slot * SLOT, qbase + (size_t)rowidx[rl + kn * T::RL] * (kCB / 2),
+            cp_async<T::BYTES>(myring + slot * SLOT, qbase + (size_t)rowidx[rl + kn * T::RL] * T::GRAN,
                                pol);
         cp_commit();
     }
     cp_wait<0>();
 }
 
-template <int B, int NB>
+template <int B, int NB, int PK>
 __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
-    using T = S1<B, NB>;
+    using T = S1<B, NB, PK>;
     extern __shared__ __align__(16) unsigned char smem[];
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     cg::cluster_group cluster = cg::this_cluster();
     const int r = (int)cluster.block_rank();  // row group
     const int c0 = (blockIdx.x / a.n_r) * NB;  // first column block of the group
-    const S1Smem L = s1_smem(a.d, B, NB, a.unit_cap, a.depth_sel);
+    const S1Smem L = s1_smem(a.d, B, NB, a.unit_cap, a.depth_sel, kS1MaxRowGroups, PK);
     unsigned char *ring = smem + L.ring;
     float *red = reinterpret_cast<float *>(smem + L.red);
     int *rowidx = reinterpret_cast<int *>(smem + L.rowidx);          // [unit_cap]
@@ -254,8 +280,8 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
 
     // The proxy scales are layer weights: pull them into L2 while the
     // previous kernel of the stream finishes (a prefetch only warms the
-    // coherent L2 and reads nothing into this CTA).
-    {
+    // coherent L2 and reads nothing into this CTA). A bf16 proxy has none.
+    if (PK == 0) {
         const int lines = a.d * 4 / 128;  // 128-byte lines per scale vector
         const int g = blockIdx.x * kS1Threads + tid;
         if (g < 2 * lines) {
@@ -302,8 +328,9 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
         }
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-            su[k][h] = sg[k][h] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (on) {
+            // a bf16 proxy has no scales: x_i enters as it is
+            su[k][h] = sg[k][h] = PK ? make_float4(1.f, 1.f, 1.f, 1.f) : make_float4(0.f, 0.f, 0.f, 0.f);
+            if (on && PK == 0) {
                 su[k][h] = *reinterpret_cast<const float4 *>(a.s_up + ci * 8 + 4 * h);
                 sg[k][h] = *reinterpret_cast<const float4 *>(a.s_gate + ci * 8 + 4 * h);
             }
@@ -374,7 +401,7 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
         // |x * 2^E| < 2^96: a row sum of (q + 8) * x_i * scale_i * 2^E over
         // <= 8192 rows stays finite for scales below 2^15 and, for scales
         // above 2^-70, partial sums of the subnormal-coded products stay normal
-        E[t] = (mx > 0.f) ? 95 - ilogbf(mx) : 0;
+        E[t] = (PK == 0 && mx > 0.f) ? 95 - ilogbf(mx) : 0;  // bf16 proxy: no pre-scale
     }
     if (woffs < hi && woffs + cnt > lo) {
         float pe1[B], pe2[B];
@@ -416,7 +443,7 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
     const int m = (tid / T::TPRM) & 1;
     const int chunk = tid % T::TPRM;
     const uint8_t *qbase = (m ? a.q_gate : a.q_up) +
-                           (size_t)(c0 + chunk / T::TPRB) * a.d * (kCB / 2) +
+                           (size_t)(c0 + chunk / T::TPRB) * a.d * T::GRAN +
                            (chunk % T::TPRB) * T::BYTES;
     const int n_rows = n_units > rl ? (n_units - rl + T::RL - 1) / T::RL : 0;
     float2 acc2[T::ACC / 2];
@@ -426,11 +453,11 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
 #pragma unroll
     for (int t = 0; t < B; ++t) ssum[t] = 0.f;
     if (a.depth_sel == 0)
-        s1_stream<B, NB, T::DMAX>(qbase, ring, rowidx, xs, rl, m, n_rows, acc2, ssum);
+        s1_stream<B, NB, PK, T::DMAX>(qbase, ring, rowidx, xs, rl, m, n_rows, acc2, ssum);
     else if (a.depth_sel == 1)
-        s1_stream<B, NB, T::DMAX / 2>(qbase, ring, rowidx, xs, rl, m, n_rows, acc2, ssum);
+        s1_stream<B, NB, PK, T::DMAX / 2>(qbase, ring, rowidx, xs, rl, m, n_rows, acc2, ssum);
     else
-        s1_stream<B, NB, T::DMAX / 4>(qbase, ring, rowidx, xs, rl, m, n_rows, acc2, ssum);
+        s1_stream<B, NB, PK, T::DMAX / 4>(qbase, ring, rowidx, xs, rl, m, n_rows, acc2, ssum);
     __syncthreads();  // every thread is done with the ring before it becomes `red`
     if (kPush) asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
 
@@ -465,10 +492,15 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
                 sacc += row[pos];
                 soff += row[T::CPT];
             }
-            const int e1 = E[t] / 2, e2 = E[t] - e1;
-            const float v = (sacc * up1) * up2 - 8.f * soff;  // sum (q + 8 - 8) x s 2^E
-            dst_part[(mm * B + t) * T::CW + ch] =
-                v * __int_as_float((127 - e1) << 23) * __int_as_float((127 - e2) << 23);
+            if constexpr (PK == 0) {
+                const int e1 = E[t] / 2, e2 = E[t] - e1;
+                const float v = (sacc * up1) * up2 - 8.f * soff;  // sum (q + 8 - 8) x s 2^E
+                dst_part[(mm * B + t) * T::CW + ch] =
+                    v * __int_as_float((127 - e1) << 23) * __int_as_float((127 - e2) << 23);
+            } else {
+                (void)up1, (void)up2, (void)soff;
+                dst_part[(mm * B + t) * T::CW + ch] = sacc;  // plain x_i * w_ij sums
+            }
         }
     }
     cluster.sync();  // all partials of the block are in their CTAs' shared memory
@@ -558,15 +590,16 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
 }
 
 // deepest ring that fits next to `unit_cap` rows (2 = the shallowest), or -1
-int s1_depth_sel(int d, int B, int NB, int unit_cap) {
+int s1_depth_sel(int d, int B, int NB, int unit_cap, int PK = 0) {
     for (int sel = 0; sel <= 2; ++sel)
-        if (s1_smem(d, B, NB, unit_cap, sel).total <= (size_t)kS2SmemBudget) return sel;
+        if (s1_smem(d, B, NB, unit_cap, sel, kS1MaxRowGroups, PK).total <= (size_t)kS2SmemBudget)
+            return sel;
     return -1;
 }
 
-template <int B, int NB>
+template <int B, int NB, int PK>
 cudaError_t launch1(Stage1Args a, const Stage1Plan &p0, cudaStream_t s) {
-    auto k = k_stage1<B, NB>;
+    auto k = k_stage1<B, NB, PK>;
     const int groups = a.C / NB;  // clusters
     // Cluster size (row groups per block): every cluster of the grid must be
     // resident at once, or the last clusters run as a second wave. Start from
@@ -585,14 +618,15 @@ cudaError_t launch1(Stage1Args a, const Stage1Plan &p0, cudaStream_t s) {
     } else {
         // fewest row groups whose rows fit in one CTA's shared memory
         int n_min = 1;
-        while (n_min < kS1MaxRowGroups && s1_depth_sel(a.d, B, NB, (a.d + n_min - 1) / n_min) < 0)
+        while (n_min < kS1MaxRowGroups &&
+               s1_depth_sel(a.d, B, NB, (a.d + n_min - 1) / n_min, PK) < 0)
             ++n_min;
         if (p.n_r < n_min) p.n_r = n_min;
         for (;;) {
             p.unit_cap = (a.d + p.n_r - 1) / p.n_r;
-            p.depth_sel = s1_depth_sel(a.d, B, NB, p.unit_cap);
+            p.depth_sel = s1_depth_sel(a.d, B, NB, p.unit_cap, PK);
             if (p.depth_sel < 0) return cudaErrorInvalidConfiguration;
-            p.smem = s1_smem(a.d, B, NB, p.unit_cap, p.depth_sel).total;
+            p.smem = s1_smem(a.d, B, NB, p.unit_cap, p.depth_sel, kS1MaxRowGroups, PK).total;
             cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  (int)p.smem);
             if (e != cudaSuccess) return e;
@@ -644,8 +678,9 @@ cudaError_t launch1(Stage1Args a, const Stage1Plan &p0, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_stage1(int B, const Stage1Args &a, const Stage1Plan &p, cudaStream_t s) {
-#define PROX_S1(BB, NN) \
-    if (B == BB && p.nb_blocks == NN) return launch1<BB, NN>(a, p, s);
+#define PROX_S1(BB, NN)                                                          \
+    if (B == BB && p.nb_blocks == NN)                                            \
+        return a.pk ? launch1<BB, NN, 1>(a, p, s) : launch1<BB, NN, 0>(a, p, s);
     PROX_S1(1, 1) PROX_S1(1, 2) PROX_S1(2, 1) PROX_S1(2, 2)
     PROX_S1(4, 1) PROX_S1(4, 2) PROX_S1(8, 1) PROX_S1(8, 2)
 #undef PROX_S1

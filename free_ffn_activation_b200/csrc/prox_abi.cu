@@ -145,9 +145,10 @@ static bool shape_ok(int d, int f) {
 static prox_status check_layer(const prox_layer *L, bool need_exact) {
     if (!L || !shape_ok(L->d_model, L->d_ff)) return PROX_EINVAL;
     if (L->activation != PROX_ACT_SWIGLU && L->activation != PROX_ACT_GEGLU) return PROX_EINVAL;
-    if (!L->q_up || !L->q_gate || !L->s_up || !L->s_gate) return PROX_EINVAL;
-    if (!aligned16(L->q_up) || !aligned16(L->q_gate) || !aligned16(L->s_up) ||
-        !aligned16(L->s_gate))
+    if (L->proxy_kind != PROX_PROXY_INT4 && L->proxy_kind != PROX_PROXY_BF16) return PROX_EINVAL;
+    if (!L->q_up || !L->q_gate || !aligned16(L->q_up) || !aligned16(L->q_gate)) return PROX_EINVAL;
+    if (L->proxy_kind == PROX_PROXY_INT4 &&
+        (!L->s_up || !L->s_gate || !aligned16(L->s_up) || !aligned16(L->s_gate)))
         return PROX_EINVAL;
     if (need_exact) {
         if (!L->w_up_cm || !L->w_gate_cm || !L->w_down) return PROX_EINVAL;
@@ -194,6 +195,7 @@ static prox_status pass_stage1(const prox_layer *L, const uint16_t *x, int nb, f
     a.s_out = s_out;
     a.build_lists = lists ? 1 : 0;
     a.act = L->activation;
+    a.pk = L->proxy_kind;
     a.wait_us = g_spin_limit;
     a.status = reinterpret_cast<uint32_t *>(w + W.status);
     a.ucount = reinterpret_cast<int32_t *>(w + W.ucount);
@@ -286,6 +288,18 @@ PROX_API prox_status prox_quantize_proxy(int d_model, int d_ff, const uint16_t *
         cudaSuccess)
         return PROX_ECUDA;
     return PROX_OK;
+}
+
+PROX_API prox_status prox_bf16_proxy(int d_model, int d_ff, const uint16_t *w_cm,
+                                     uint16_t *q16_out, void *stream) {
+    if (!w_cm || !q16_out || !shape_ok(d_model, d_ff)) return PROX_EINVAL;
+    if (!aligned16(w_cm) || !aligned16(q16_out)) return PROX_EINVAL;
+    int sms = 0;
+    prox_status ps = current_device(&sms);
+    if (ps != PROX_OK) return ps;
+    return launch_tile_bf16(d_model, d_ff, w_cm, q16_out, (cudaStream_t)stream) == cudaSuccess
+               ? PROX_OK
+               : PROX_ECUDA;
 }
 
 PROX_API size_t prox_workspace_bytes(int d_model, int d_ff, int batch) {

@@ -78,6 +78,7 @@ struct Stage1Args {
     float *s_out;                // [nb][f] or null
     int build_lists;             // write ulist/tlist/counts for Stage 2
     int act;                     // gate activation (PROX_ACT_*)
+    int pk;                      // proxy kind (PROX_PROXY_*): q_up/q_gate INT4 or bf16 tiles
     uint32_t wait_us;            // wall-clock bound of each wait, microseconds
     // workspace
     uint32_t *status;
@@ -121,6 +122,8 @@ cudaError_t launch_hist_quantile_f32(const float *v, long n, long k, long rank, 
                                      cudaStream_t s);
 cudaError_t launch_quantize(int d, int f, const uint16_t *w_cm, uint8_t *q,
                             float *scale, cudaStream_t s);
+// bf16 proxy: block-tiled copy [f/256][d][256] of a channel-major [f][d] weight
+cudaError_t launch_tile_bf16(int d, int f, const uint16_t *w_cm, uint16_t *q16, cudaStream_t s);
 // exact order statistic of |values| (bf16 or fp32 bit patterns) on device;
 // writes the selected magnitude's fp32 value to *tau_dev
 cudaError_t launch_select_bf16_abs(const uint16_t *v, long n, long rank,

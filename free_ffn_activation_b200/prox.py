@@ -37,10 +37,12 @@ class _Layer(C.Structure):
     _fields_ = [("d_model", C.c_int), ("d_ff", C.c_int),
                 ("w_up_cm", C.c_void_p), ("w_gate_cm", C.c_void_p), ("w_down", C.c_void_p),
                 ("q_up", C.c_void_p), ("q_gate", C.c_void_p),
-                ("s_up", C.c_void_p), ("s_gate", C.c_void_p), ("activation", C.c_int)]
+                ("s_up", C.c_void_p), ("s_gate", C.c_void_p), ("activation", C.c_int),
+                ("proxy_kind", C.c_int)]
 
 
 ACT_SWIGLU, ACT_GEGLU = 0, 1   # PROX_ACT_SWIGLU, PROX_ACT_GEGLU
+PROXY_INT4, PROXY_BF16 = 0, 1  # PROX_PROXY_INT4, PROX_PROXY_BF16
 
 
 _lib = None
@@ -62,6 +64,7 @@ def lib() -> C.CDLL:
         L.prox_ffn_forward_static.argtypes = [C.POINTER(_Layer), vp, i, f, f, vp, vp, vp, vp,
                                                vp, vp]
         L.prox_rmsnorm_bf16.argtypes = [i, i, vp, f, vp, vp]
+        L.prox_bf16_proxy.argtypes = [i, i, vp, vp, vp]
         L.prox_ffn_block.argtypes = [C.POINTER(_Layer), vp, i, f, f, f, vp, vp, vp, vp, vp, vp,
                                      vp, sz, vp]
         L.prox_proxy_state.argtypes = [C.POINTER(_Layer), vp, i, f, vp, vp, vp, sz, vp]
@@ -84,6 +87,7 @@ def lib() -> C.CDLL:
         L.prox_test_set_wait.restype = None
         for name in ("prox_quantize_proxy", "prox_ffn_forward", "prox_ffn_forward_static",
                      "prox_rmsnorm_bf16", "prox_ffn_block", "prox_calibrate_histogram",
+                     "prox_bf16_proxy",
                      "prox_proxy_state",
                      "prox_ffn_stage1", "prox_ffn_stage2",
                      "prox_calibrate", "prox_allocate", "prox_last_device_status"):
@@ -145,6 +149,8 @@ class ProxLayer:
     s_up: torch.Tensor         # fp32 [d_model]
     s_gate: torch.Tensor
     activation: int = 0        # ACT_SWIGLU (SiLU gate) or ACT_GEGLU (GELU gate)
+    proxy_kind: int = 0        # PROXY_INT4, or PROXY_BF16: q_* are bf16 tiles
+                               # uint16 [d_ff/256][d_model][256], s_* unused (None)
 
     @property
     def d_model(self) -> int:
@@ -156,24 +162,43 @@ class ProxLayer:
 
     def cstruct(self) -> _Layer:
         d, f = self.d_model, self.d_ff
+        if self.proxy_kind == PROXY_BF16:
+            checks = (("q_up", torch.int16, (f // 256, d, 256)),
+                      ("q_gate", torch.int16, (f // 256, d, 256)))
+        else:
+            checks = (("q_up", torch.uint8, (f // 256, d, 128)),
+                      ("q_gate", torch.uint8, (f // 256, d, 128)), ("s_up", torch.float32, (d,)),
+                      ("s_gate", torch.float32, (d,)))
         for name, dt, shp in (("w_up_cm", torch.bfloat16, (f, d)), ("w_gate_cm", torch.bfloat16, (f, d)),
-                              ("w_down", torch.bfloat16, (f, d)),
-                              ("q_up", torch.uint8, (f // 256, d, 128)),
-                              ("q_gate", torch.uint8, (f // 256, d, 128)), ("s_up", torch.float32, (d,)),
-                              ("s_gate", torch.float32, (d,))):
+                              ("w_down", torch.bfloat16, (f, d))) + checks:
             _need(getattr(self, name), dt, shp, name)
         return _Layer(d, f, _ptr(self.w_up_cm), _ptr(self.w_gate_cm), _ptr(self.w_down),
                       _ptr(self.q_up), _ptr(self.q_gate), _ptr(self.s_up), _ptr(self.s_gate),
-                      int(self.activation))
+                      int(self.activation), int(self.proxy_kind))
 
     @staticmethod
     def from_weights(w_up_cm, w_gate_cm, w_down, device="cuda",
-                     activation: int = ACT_SWIGLU) -> "ProxLayer":
-        """Upload bf16 weights and build their INT4 proxies on the device."""
+                     activation: int = ACT_SWIGLU, proxy_kind: int = PROXY_INT4) -> "ProxLayer":
+        """Upload bf16 weights and build their proxies (INT4, or the bf16
+        ablation's tiled copies) on the device."""
         up, gate, down = (as_bf16(w, device).contiguous() for w in (w_up_cm, w_gate_cm, w_down))
+        if proxy_kind == PROXY_BF16:
+            return ProxLayer(up, gate, down, bf16_proxy(up), bf16_proxy(gate), None, None,
+                             int(activation), PROXY_BF16)
         q_up, s_up = quantize_proxy(up)
         q_gate, s_gate = quantize_proxy(gate)
         return ProxLayer(up, gate, down, q_up, q_gate, s_up, s_gate, int(activation))
+
+
+def bf16_proxy(w_cm: torch.Tensor) -> torch.Tensor:
+    """prox_bf16_proxy: block-tiled copy [d_ff/256][d_model][256] (int16 view of
+    bf16) of a channel-major bf16 weight [d_ff][d_model]."""
+    f, d = w_cm.shape
+    _need(w_cm, torch.bfloat16, (f, d), "w_cm")
+    q = torch.empty((f // 256, d, 256), dtype=torch.int16, device=w_cm.device)
+    _check(lib().prox_bf16_proxy(d, f, _ptr(w_cm), _ptr(q), _stream(w_cm.device)),
+           "prox_bf16_proxy")
+    return q
 
 
 def quantize_proxy(w_cm: torch.Tensor):
@@ -434,15 +459,17 @@ def untile_proxy(q):
     return q.transpose(1, 0, 2).reshape(d, C * 128) ^ 0x88
 
 
-def touched_bytes(d_model: int, d_ff: int, k_x: int, k_s: int) -> int:
-    """Weight bytes one token's forward reads: the kept rows of both INT4
-    proxies with their scales, and three bf16 rows per kept channel."""
-    return 2 * k_x * (d_ff // 2) + 2 * k_x * 4 + 3 * k_s * d_model * 2
+def touched_bytes(d_model: int, d_ff: int, k_x: int, k_s: int,
+                  proxy_kind: int = PROXY_INT4) -> int:
+    """Weight bytes one token's forward reads: the kept rows of both proxies
+    (INT4 with their scales, or bf16) and three bf16 rows per kept channel."""
+    proxy = 2 * k_x * d_ff * 2 if proxy_kind == PROXY_BF16 else 2 * k_x * (d_ff // 2) + 2 * k_x * 4
+    return proxy + 3 * k_s * d_model * 2
 
 
 __all__ = ["ProxLayer", "ProxError", "quantize_proxy", "workspace", "workspace_bytes",
            "ffn_forward", "ffn_forward_static", "STATIC_WORKSPACE_BYTES", "ffn_forward_raw",
            "ffn_stage1_raw", "ffn_stage2_raw", "rmsnorm_bf16", "ffn_block", "ffn_block_raw",
-           "calibrate_histogram",
+           "calibrate_histogram", "bf16_proxy", "PROXY_INT4", "PROXY_BF16",
            "max_batch_per_pass", "proxy_state", "calibrate", "allocate",
            "last_device_status", "touched_bytes", "untile_proxy", "as_bf16"]

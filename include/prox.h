@@ -76,7 +76,16 @@ typedef struct prox_layer {
        PROX_ACT_GEGLU (GELU(z) = z Phi(z), exact erf form: the GeGLU-style
        models of the blog's "Evidence" section); anything else is PROX_EINVAL */
     int activation;
+    /* proxy kind: PROX_PROXY_INT4 (the method: q_up/q_gate INT4 tiles from
+       prox_quantize_proxy, s_up/s_gate their scales) or PROX_PROXY_BF16 (the
+       FP16/bf16-proxy ablation of the blog's "Evidence" section: q_up/q_gate
+       are bf16 tiles [d_ff/256][d_model][256] from prox_bf16_proxy, the
+       original weights; s_up/s_gate are unused and may be NULL) */
+    int proxy_kind;
 } prox_layer;
+
+#define PROX_PROXY_INT4 0
+#define PROX_PROXY_BF16 1
 
 #define PROX_ACT_SWIGLU 0
 #define PROX_ACT_GEGLU 1
@@ -103,6 +112,17 @@ typedef struct prox_layer {
  */
 prox_status prox_quantize_proxy(int d_model, int d_ff, const uint16_t *w_cm,
                                 uint8_t *q_out, float *scale_out, void *stream);
+
+/*
+ * prox_bf16_proxy -- the bf16-proxy ablation's proxy: the weight itself,
+ * block-tiled like the INT4 proxy so that a rejected input coordinate skips
+ * one contiguous 512-byte granule per 256-channel block:
+ *   q16_out[c][i][k] = w_cm[256c + k][i]   (uint16 bf16, [d_ff/256][d_model][256]).
+ *   w_cm : device, bf16 [d_ff][d_model] (channel-major).
+ * Errors: PROX_EINVAL on a null or misaligned pointer or a bad shape.
+ */
+prox_status prox_bf16_proxy(int d_model, int d_ff, const uint16_t *w_cm, uint16_t *q16_out,
+                            void *stream);
 
 /*
  * prox_workspace_bytes -- bytes of device workspace prox_ffn_forward and

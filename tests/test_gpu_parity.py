@@ -33,14 +33,17 @@ class Case:
     """One layer with its oracle proxies, device layer and thresholds."""
 
     def __init__(self, d, f, n_tok, n_cal, sigma=0.02, seed=0, outlier=0.0, layer=0,
-                 keep_x=0.5, keep_s=0.3, dev="cuda", act=oracle.ACT_SWIGLU):
+                 keep_x=0.5, keep_s=0.3, dev="cuda", act=oracle.ACT_SWIGLU,
+                 proxy_kind=P.PROXY_INT4):
         self.spec = S.LayerSpec(d, f, sigma=sigma, seed=seed, layer=layer)
         self.L = S.make_layer(self.spec)
-        self.Por = oracle.make_proxy(self.L)
+        self.Por = (oracle.make_proxy_bf16(self.L) if proxy_kind == P.PROXY_BF16
+                    else oracle.make_proxy(self.L))
         self.dev = dev
         self.act = act
         self.layer = P.ProxLayer.from_weights(self.L["w_up_cm"], self.L["w_gate_cm"],
-                                              self.L["w_down"], device=dev, activation=act)
+                                              self.L["w_down"], device=dev, activation=act,
+                                              proxy_kind=proxy_kind)
         self.x = S.make_tokens(n_tok, d, seed=seed, stream="x_eval", outlier_frac=outlier)
         self.x_cal = S.make_tokens(n_cal, d, seed=seed, stream="x_cal", outlier_frac=outlier)
         self.keep_x, self.keep_s = keep_x, keep_s
@@ -72,6 +75,18 @@ def c4(gpu):
     # case tests: 2-CTA clusters, two coordinate chunks per thread, a 3-stage
     # Stage-2 ring, passes of 4 tokens)
     return Case(8192, 28672, 32, 64, sigma=0.015)
+
+
+@pytest.fixture(scope="module")
+def c1b(gpu):
+    # the tiny layer with the bf16-proxy ablation (the proxy is the weight itself)
+    return Case(256, 768, 64, 256, proxy_kind=P.PROXY_BF16)
+
+
+@pytest.fixture(scope="module")
+def c2b(gpu):
+    # the 4096 x 12288 layer with the bf16 proxy
+    return Case(4096, 12288, 16, 128, outlier=0.001, proxy_kind=P.PROXY_BF16)
 
 
 @pytest.fixture(scope="module")
@@ -162,7 +177,8 @@ def _proxy_check(case, rows):
     s_gpu = s_gpu.cpu().numpy().astype(np.float64)
     ref = np.stack([oracle.stage1(case.x[t], case.tau_x, case.Por["q_up"], case.Por["s_up"],
                                   case.Por["q_gate"], case.Por["s_gate"], case.tau_s,
-                                  act=case.act)["s"]
+                                  act=case.act, pw_up=case.Por.get("pw_up"),
+                                  pw_gate=case.Por.get("pw_gate"))["s"]
                     for t in rows])
     assert np.array_equal(mx.cpu().numpy(),
                           (np.abs(S.bf16_to_f32(case.x[rows])) >= np.float32(case.tau_x)).astype(np.uint8))
@@ -219,6 +235,38 @@ def test_calibrate_histogram_c1(c1):
 def test_calibrate_histogram_c2(c2):
     # 512 x 12288 s~ values: 6.3 M pooled, sampled every 32nd (196,608 samples)
     _check_hist_calibration(c2)
+
+
+def test_bf16_proxy_tiles(c1b):
+    w = c1b.layer.w_up_cm
+    ref = w.view(torch.int16).view(768 // 256, 256, 256).permute(0, 2, 1).contiguous()
+    assert torch.equal(c1b.layer.q_up, ref)
+
+
+def test_bf16_proxy_state_c1(c1b):
+    _proxy_check(c1b, list(range(16)))
+
+
+@pytest.mark.parametrize("b", [1, 3, 64])
+def test_bf16_proxy_forward_c1(c1b, b):
+    rows = list(range(b))
+    out = P.ffn_forward(c1b.layer, c1b.xdev(rows), c1b.tau_x, c1b.tau_s)
+    check_forward(c1b, rows, out, f" c1 bf16-proxy b={b}")
+
+
+def test_bf16_proxy_calibrate_c1(c1b):
+    tx, ts = P.calibrate(c1b.layer, to_dev_bf16(c1b.x_cal, "cuda"), c1b.keep_x, c1b.keep_s)
+    assert np.float32(tx) == np.float32(c1b.tau_x)
+    assert abs(ts - c1b.tau_s) <= 1e-5 * c1b.tau_s, (ts, c1b.tau_s)
+
+
+def test_bf16_proxy_forward_c2_sampled(c2b):
+    ws = P.workspace(4096, 12288, 1)
+    rows = [0, 5, 15]
+    outs = [P.ffn_forward(c2b.layer, c2b.xdev([t]), c2b.tau_x, c2b.tau_s, ws) for t in rows]
+    merged = P.ForwardOut(*(torch.cat([getattr(o, k) for o in outs]) for k in
+                            ("y", "mask_x", "mask_s", "idx_s", "count_s")))
+    check_forward(c2b, rows, merged, " c2 bf16-proxy b=1")
 
 
 def test_geglu_proxy_state_c1(c1g):
