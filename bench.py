@@ -63,11 +63,28 @@ def parse():
                     help="proxy kind: the method's INT4 proxy or the bf16-proxy ablation")
     ap.add_argument("--batch", type=int, default=1,
                     help="tokens per forward call (each token keeps its own masks)")
+    ap.add_argument("--engine", choices=["auto", "simt", "tc"], default="auto",
+                    help="Stage-2 engine: automatic, CUDA cores, or the tensor-core union GEMM "
+                         "(passes of >= 4 tokens)")
     ap.add_argument("--copies", type=int, default=4, help="rotating weight copies (L2 defeat)")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense cuBLAS reference")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     return ap.parse_args()
+
+
+def launches_per_call(args, d, batch):
+    """Kernels one forward call of `batch` tokens launches: per pass, Stage 1
+    and one Stage-2 kernel (CUDA cores) or two (tensor-core union engine:
+    passes of 8 tokens by default, of >= 4 when forced)."""
+    from free_ffn_activation_b200 import prox as P
+    per_pass = P.max_batch_per_pass(d)
+    passes = -(-batch // per_pass)
+    tb = 1
+    while tb < min(batch, per_pass):
+        tb *= 2
+    tc = tb >= 8 if args.engine == "auto" else (args.engine == "tc" and tb >= 4)
+    return passes * (3 if tc else 2)
 
 
 def stage2_traffic(workload, batch):
@@ -438,7 +455,7 @@ def run_ours(args, w, rank, world, local_rank):
             "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
             "config": {"workload": args.workload, "d_model": d, "d_ff": f, "batch": Bt,
-                       "proxy": args.proxy,
+                       "proxy": args.proxy, "engine": args.engine,
                        "tokens_per_step": ntok, "keep_x": args.keep_x, "keep_s": args.keep_s,
                        "tau_x": tau_x, "tau_s": tau_s,
                        "l2": f"{R} rotating weight copies ({R * (3 * d * f * 2 + (d * f + 8 * d if pk == P.PROXY_INT4 else 4 * d * f)) / 1e9:.2f} GB > L2)",
@@ -461,7 +478,7 @@ def run_ours(args, w, rank, world, local_rank):
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_us, "unit": "us/token/layer",
                     "h2d_bytes_per_step": ntok * d * 2, "d2h_bytes_per_step": ntok * d * 4},
-            "gpu_launches": 2 * ntok * args.steps,
+            "gpu_launches": launches_per_call(args, d, Bt) * (ntok // Bt) * args.steps,
             "clocks": clk.summary(),
         }
         print(json.dumps(line), flush=True)
@@ -659,6 +676,8 @@ def main():
             return
         run_reference(args, w, rank, world)
         return
+    from free_ffn_activation_b200 import prox as P
+    P.set_stage2_engine({"auto": P.ENGINE_AUTO, "simt": P.ENGINE_SIMT, "tc": P.ENGINE_TC}[args.engine])
     if world > 1:
         import datetime
 

@@ -305,6 +305,11 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
         for (int k = blockIdx.x * kS1Threads + tid; k < n4; k += gridDim.x * kS1Threads)
             y4[k] = i4 ? i4[k] : make_float4(0.f, 0.f, 0.f, 0.f);
     }
+    // the tensor-core Stage 2 sums split partials and counts arrivals with
+    // atomics: clear them too
+    if (a.z_clear)
+        for (int k = blockIdx.x * kS1Threads + tid; k < a.z_n16; k += gridDim.x * kS1Threads)
+            a.z_clear[k] = make_uint4(0u, 0u, 0u, 0u);
 
     // (2) input masks m_x = 1[|x_i| >= tau_x] per token. Thread tid owns the K
     // adjacent 8-coordinate chunks [tid * K, tid * K + K) (K = 1, or 2 when

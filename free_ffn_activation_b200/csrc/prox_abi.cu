@@ -9,6 +9,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #define PROX_API extern "C" __attribute__((visibility("default")))
@@ -99,6 +100,19 @@ WsLayout ws_layout(int d, int f, int B) {
     o = align_up(o + C * kCB * 4, 256);
     L.tlist = o;
     o = align_up(o + (size_t)B * f * 4, 256);
+    L.ug = L.tile_cnt = L.sb = L.pos_ch = o;
+    L.clear_bytes = 0;
+    if (B >= 4) {  // tensor-core Stage 2 (see k_stage2_umma.cu)
+        L.ug = o;
+        o += (size_t)f * 2 * B * 4;
+        L.tile_cnt = o;
+        o = align_up(o + (size_t)(f / 128) * 4, 256);
+        L.clear_bytes = o - L.ug;
+        L.sb = o;
+        o = align_up(o + (size_t)(f / 64) * 2048, 256);
+        L.pos_ch = o;
+        o = align_up(o + (size_t)f * 4, 256);
+    }
     L.total = o;
     return L;
 }
@@ -164,6 +178,17 @@ static bool tau_ok(float t) { return std::isfinite(t) && t >= 0.f; }
 static uint32_t g_spin_limit = kDefaultWaitUs;
 static int g_debug_skip = -1;
 
+// Stage-2 engine (prox_set_stage2_engine)
+static std::atomic<int> g_engine{PROX_ENGINE_AUTO};
+
+// Whether a pass of B tokens runs the tensor-core Stage 2 (and its plan)
+static bool use_tc(int d, int f, int B, int sms, Stage2UPlan *p) {
+    const int e = g_engine.load();
+    if (e == PROX_ENGINE_SIMT || B < 4) return false;
+    if (e == PROX_ENGINE_AUTO && B < kTcMinBatch) return false;
+    return stage2u_plan(d, f, sms, p);
+}
+
 // One pass (nb <= tokens_per_pass tokens) of Stage 1: masks, kept-channel
 // lists in the workspace, s~ when s_out is given, and y cleared when given.
 static prox_status pass_stage1(const prox_layer *L, const uint16_t *x, int nb, float tau_x,
@@ -196,6 +221,11 @@ static prox_status pass_stage1(const prox_layer *L, const uint16_t *x, int nb, f
     a.build_lists = lists ? 1 : 0;
     a.act = L->activation;
     a.pk = L->proxy_kind;
+    Stage2UPlan pu;
+    if (lists && use_tc(d, f, B, sms, &pu)) {
+        a.z_clear = reinterpret_cast<uint4 *>(w + W.ug);
+        a.z_n16 = (int)(W.clear_bytes / 16);
+    }
     a.wait_us = g_spin_limit;
     a.status = reinterpret_cast<uint32_t *>(w + W.status);
     a.ucount = reinterpret_cast<int32_t *>(w + W.ucount);
@@ -213,6 +243,38 @@ static prox_status pass_stage2(const prox_layer *L, const uint16_t *x, int nb, f
     const int B = pow2_ceil(nb);
     const WsLayout W = ws_layout(d, f, B);
     const int C = f / kCB;
+    Stage2UPlan pu;
+    if (use_tc(d, f, B, sms, &pu)) {
+        Stage2UArgs u{};
+        u.d = d;
+        u.f = f;
+        u.nb = nb;
+        u.C = C;
+        u.x = x;
+        u.w_up = L->w_up_cm;
+        u.w_gate = L->w_gate_cm;
+        u.w_down = L->w_down;
+        u.y = y;
+        u.idx_s = idx_s;
+        u.count_s = count_s;
+        u.act = L->activation;
+        u.ucount = reinterpret_cast<int32_t *>(w + W.ucount);
+        u.tcount = reinterpret_cast<int32_t *>(w + W.tcount);
+        u.ulist = reinterpret_cast<uint32_t *>(w + W.ulist);
+        u.tlist = reinterpret_cast<int32_t *>(w + W.tlist);
+        u.status = reinterpret_cast<uint32_t *>(w + W.status);
+        u.wait_us = g_spin_limit;
+        u.ks = pu.ks;
+        u.span = pu.span;
+        u.nstage = pu.nstage;
+        u.span_dn = pu.span_dn;
+        u.nstage_dn = pu.nstage_dn;
+        u.ug = reinterpret_cast<float *>(w + W.ug);
+        u.tile_cnt = reinterpret_cast<int32_t *>(w + W.tile_cnt);
+        u.sb = reinterpret_cast<uint16_t *>(w + W.sb);
+        u.pos_ch = reinterpret_cast<uint32_t *>(w + W.pos_ch);
+        return launch_stage2_umma(B, u, sms, st) == cudaSuccess ? PROX_OK : PROX_ECUDA;
+    }
     const int max_ch = (f + sms - 1) / sms + 1;
     const Stage2Plan p2 = stage2_plan(d, B, C, max_ch);
     if (p2.nstage < 2) return PROX_EINVAL;
@@ -409,6 +471,12 @@ PROX_API prox_status prox_ffn_block(const prox_layer *layer, const float *h_in, 
 }
 
 PROX_API int prox_max_batch_per_pass(int d_model) { return max_tokens_per_pass(d_model); }
+
+PROX_API int prox_set_stage2_engine(int engine) {
+    if (engine != PROX_ENGINE_AUTO && engine != PROX_ENGINE_SIMT && engine != PROX_ENGINE_TC)
+        return -1;
+    return g_engine.exchange(engine);
+}
 
 PROX_API prox_status prox_ffn_stage1(const prox_layer *layer, const uint16_t *x, int batch,
                                      float tau_x, float tau_s, float *y_clear, uint8_t *mask_x,

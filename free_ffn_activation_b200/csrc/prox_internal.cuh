@@ -26,6 +26,12 @@ constexpr uint32_t kStTimeoutEmpty = 1u << 1;  // producer waited for a free slo
 constexpr uint32_t kStTimeoutRed = 1u << 2;    // consumers waited for partials
 constexpr uint32_t kStTimeoutDrain = 1u << 3;  // producer waited for its copies
 constexpr uint32_t kStTimeoutRing = 1u << 4;   // Stage 1 waited for a ring slot
+constexpr uint32_t kStTimeoutMma = 1u << 5;    // tensor-core Stage 2 waited for its MMAs
+
+// tensor-core Stage 2: union positions per down-projection unit, and the
+// smallest pass (tokens) the automatic engine choice sends to it
+constexpr int kUnitPos = 512;
+constexpr int kTcMinBatch = 8;
 
 // default wall-clock bound of a device-side wait, in microseconds
 constexpr uint32_t kDefaultWaitUs = 2000000u;
@@ -55,9 +61,23 @@ int tokens_per_pass(int d_model, int batch);   // 1, 2, 4 or 8
 Stage1Plan stage1_plan(int d_model, int d_ff, int B, int num_sms);
 Stage2Plan stage2_plan(int d_model, int B, int C, int max_ch);
 
-// Workspace layout of one forward pass (B tokens). Offsets in bytes.
+// Launch plan of the tensor-core (union GEMM) Stage 2
+struct Stage2UPlan {
+    int ks;         // K slices of the up/gate GEMM
+    int span;       // union tiles one up/gate CTA may touch
+    int span_dn;    // position ranges one down CTA may touch
+    int nstage;     // up/gate ring stages
+    int nstage_dn;  // down ring stages
+};
+bool stage2u_plan(int d_model, int d_ff, int num_sms, Stage2UPlan *p);
+
+// Workspace layout of one forward pass (B tokens). Offsets in bytes. The
+// tensor-core Stage 2 (B >= 4) adds fp32 partial sums of u and g per union
+// position with the split counters right after them (one region Stage 1
+// clears), the s tiles and the channel of every union position.
 struct WsLayout {
-    size_t status, ucount, tcount, ulist, tlist, total;
+    size_t status, ucount, tcount, ulist, tlist, ug, tile_cnt, sb, pos_ch, total;
+    size_t clear_bytes;  // ug .. tile_cnt end
 };
 WsLayout ws_layout(int d_model, int d_ff, int B);
 
@@ -79,6 +99,8 @@ struct Stage1Args {
     int build_lists;             // write ulist/tlist/counts for Stage 2
     int act;                     // gate activation (PROX_ACT_*)
     int pk;                      // proxy kind (PROX_PROXY_*): q_up/q_gate INT4 or bf16 tiles
+    uint4 *z_clear;              // region cleared for the tensor-core Stage 2, or null
+    int z_n16;                   // its size in 16-byte words
     uint32_t wait_us;            // wall-clock bound of each wait, microseconds
     // workspace
     uint32_t *status;
@@ -106,6 +128,29 @@ struct Stage2Args {
     int nstage;
     int max_ch;                  // capacity of the per-CTA channel list
 };
+
+struct Stage2UArgs {
+    int d, f, nb, C;
+    const uint16_t *x;           // [nb][d]
+    const uint16_t *w_up, *w_gate, *w_down;
+    float *y;                    // [nb][d], cleared (or seeded) by Stage 1
+    int32_t *idx_s;              // [nb][f] or null
+    int32_t *count_s;            // [nb] or null
+    int act;                     // gate activation (PROX_ACT_*)
+    const int32_t *ucount, *tcount;
+    const uint32_t *ulist;
+    const int32_t *tlist;
+    uint32_t *status;
+    uint32_t wait_us;            // wall-clock bound of each wait, microseconds
+    int ks, span, nstage;        // up/gate plan
+    int span_dn, nstage_dn;      // down plan
+    float *ug;                   // [f][2][B] partial u, g per union position (cleared)
+    int32_t *tile_cnt;           // [f / 128] slices summed per tile (cleared)
+    uint16_t *sb;                // [f / 64][2][8][64] s hi / lo tiles, 128-byte swizzled
+    uint32_t *pos_ch;            // [f] union entry per position
+};
+
+cudaError_t launch_stage2_umma(int B, const Stage2UArgs &a, int grid, cudaStream_t s);
 
 cudaError_t launch_stage1(int B, const Stage1Args &a, const Stage1Plan &p,
                           cudaStream_t s);

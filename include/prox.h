@@ -226,6 +226,28 @@ prox_status prox_ffn_block(const prox_layer *layer, const float *h_in, int batch
 int prox_max_batch_per_pass(int d_model);
 
 /*
+ * prox_set_stage2_engine -- which kernels run Stage 2 (process-wide; takes
+ * effect at the next forward call, returns the previous setting, or -1 for
+ * an unknown value, which changes nothing).
+ *   PROX_ENGINE_AUTO (default): the tensor-core union engine for passes of 8
+ *     tokens, the CUDA-core engine below that;
+ *   PROX_ENGINE_SIMT: the CUDA-core engine always: per channel of the union,
+ *     dot products of the kept rows with x on the CUDA cores;
+ *   PROX_ENGINE_TC: the tensor-core engine for every pass of 4 or more
+ *     tokens: the union's up/gate rows and the W_down rows are dense UMMA
+ *     GEMMs over the pass's tokens (tcgen05, fp32 accumulators), each
+ *     token's own channel mask applied to s, s carried as a bf16 hi + lo
+ *     pair (relative error about 2^-16) into the down GEMM.
+ * The pages give no kernel for batches beyond one token (blog, section
+ * "Limitations"); both engines compute the per-token Stage 2 of the blog's
+ * section "Stage 2" and differ only in summation order.
+ */
+#define PROX_ENGINE_AUTO 0
+#define PROX_ENGINE_SIMT 1
+#define PROX_ENGINE_TC 2
+int prox_set_stage2_engine(int engine);
+
+/*
  * prox_ffn_stage1 / prox_ffn_stage2 -- the two phases of prox_ffn_forward,
  * callable separately (for instance to time or inspect Stage 1 alone).
  * prox_ffn_forward(..) with batch <= prox_max_batch_per_pass(d_model) is

@@ -177,3 +177,25 @@ def test_calibrate_histogram_validates():
     assert call(200000, 4000) == P.PROX_EINVAL     # bins not a multiple of 1024
     assert call(200000, 131072) == P.PROX_EINVAL   # too many bins
     assert call(200000, 4096, wsb - 1) == P.PROX_ENOMEM
+
+
+def test_stage2_engine_switch():
+    prev = P.set_stage2_engine(P.ENGINE_SIMT)
+    try:
+        assert P.set_stage2_engine(P.ENGINE_TC) == P.ENGINE_SIMT
+        assert P.lib().prox_set_stage2_engine(7) == -1          # unknown: nothing changes
+        assert P.set_stage2_engine(P.ENGINE_AUTO) == P.ENGINE_TC
+        with P.stage2_engine(P.ENGINE_SIMT):
+            assert P.set_stage2_engine(P.ENGINE_SIMT) == P.ENGINE_SIMT
+        assert P.set_stage2_engine(P.ENGINE_AUTO) == P.ENGINE_AUTO
+    finally:
+        P.set_stage2_engine(prev)
+
+
+def test_workspace_holds_tensor_core_buffers():
+    # passes of >= 4 tokens add partial sums, split counters, s tiles and
+    # union positions: f*2*B*4 + (f/128)*4 + (f/64)*2048 + f*4 bytes (rounded)
+    d, f = 4096, 12288
+    extra = P.workspace_bytes(d, f, 8) - (P.workspace_bytes(d, f, 2) + 6 * f * 4 + 6 * 48 * 4)
+    assert extra >= f * 2 * 8 * 4 + (f // 128) * 4 + (f // 64) * 2048 + f * 4
+    assert P.workspace_bytes(d, f, 1000) <= P.STATIC_WORKSPACE_BYTES

@@ -433,3 +433,94 @@ def test_split_stages_equal_forward(c2):
     with pytest.raises(P.ProxError):
         P.ffn_stage1_raw(cl, x.data_ptr(), 9, c2.tau_x, c2.tau_s, None, ws.data_ptr(),
                          ws.numel(), st)
+
+
+# ---------------------------------------------------------------------------
+# tensor-core Stage 2 (union GEMM engine), passes of 4 and 8 tokens
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("b", [4, 5, 8, 13, 64])
+def test_tc_forward_c1(c1, b):
+    rows = list(range(b))
+    with P.stage2_engine(P.ENGINE_TC):
+        out = P.ffn_forward(c1.layer, c1.xdev(rows), c1.tau_x, c1.tau_s)
+    check_forward(c1, rows, out, f" c1 tc b={b}")
+
+
+@pytest.mark.parametrize("b", [4, 8])
+def test_tc_forward_c2(c2, b):
+    rows = list(range(20, 20 + b))
+    with P.stage2_engine(P.ENGINE_TC):
+        out = P.ffn_forward(c2.layer, c2.xdev(rows), c2.tau_x, c2.tau_s)
+    check_forward(c2, rows, out, f" c2 tc b={b}")
+
+
+def test_tc_matches_simt_c2(c2):
+    # both engines take the same masks and lists; y differs by summation order
+    # (and the bf16 hi + lo split of s, about 2^-16 relative)
+    rows = list(range(40, 48))
+    x = c2.xdev(rows)
+    with P.stage2_engine(P.ENGINE_SIMT):
+        a = P.ffn_forward(c2.layer, x, c2.tau_x, c2.tau_s)
+    with P.stage2_engine(P.ENGINE_TC):
+        b = P.ffn_forward(c2.layer, x, c2.tau_x, c2.tau_s)
+    torch.cuda.synchronize()
+    assert torch.equal(a.mask_x, b.mask_x) and torch.equal(a.mask_s, b.mask_s)
+    assert torch.equal(a.count_s, b.count_s)
+    for t in range(len(rows)):
+        n = int(a.count_s[t])
+        assert torch.equal(a.idx_s[t, :n], b.idx_s[t, :n])
+    rel = (torch.linalg.norm(a.y - b.y, dim=1) / torch.linalg.norm(a.y, dim=1)).max().item()
+    print(f"[tc vs simt c2 b=8] y rel max {rel:.2e}")
+    assert rel < 1e-4
+
+
+def test_tc_forward_c4_b16(c4):
+    # d_model 8192: passes of 4 tokens, 16 K slices per up/gate tile
+    rows = list(range(16))
+    with P.stage2_engine(P.ENGINE_TC):
+        out = P.ffn_forward(c4.layer, c4.xdev(rows), c4.tau_x, c4.tau_s)
+    check_forward(c4, rows, out, " c4 tc b=16")
+
+
+def test_tc_geglu_c1(c1g):
+    rows = list(range(8))
+    with P.stage2_engine(P.ENGINE_TC):
+        out = P.ffn_forward(c1g.layer, c1g.xdev(rows), c1g.tau_x, c1g.tau_s)
+    check_forward(c1g, rows, out, " c1 geglu tc b=8")
+
+
+def test_tc_dense_and_empty_c1(c1):
+    rows = list(range(8))
+    x = c1.xdev(rows)
+    with P.stage2_engine(P.ENGINE_TC):
+        dense = P.ffn_forward(c1.layer, x, 0.0, 0.0)         # every channel kept
+        empty = P.ffn_forward(c1.layer, x, c1.tau_x, 1e30)   # no channel kept
+    torch.cuda.synchronize()
+    ref = oracle.forward(c1.x[rows], 0.0, 0.0, c1.L, c1.Por, want=())["y"]
+    rel = np.linalg.norm(dense.y.cpu().numpy() - ref, axis=1) / np.linalg.norm(ref, axis=1)
+    assert rel.max() <= Y_TOL
+    assert int(empty.count_s.sum()) == 0 and not bool(empty.y.any())
+
+
+def test_tc_split_stages_equal_forward(c2):
+    # prox_ffn_stage1 clears the tensor-core buffers when the next Stage 2 uses them
+    rows = list(range(60, 68))
+    x = c2.xdev(rows)
+    st = torch.cuda.current_stream().cuda_stream
+    ws = P.workspace(4096, 12288, 8)
+    cl = c2.layer.cstruct()
+    y = torch.empty((8, 4096), dtype=torch.float32, device="cuda")
+    cnt = torch.empty((8,), dtype=torch.int32, device="cuda")
+    with P.stage2_engine(P.ENGINE_TC):
+        for _ in range(2):  # the second pass reuses the workspace the first one left
+            P.ffn_stage1_raw(cl, x.data_ptr(), 8, c2.tau_x, c2.tau_s, y.data_ptr(), ws.data_ptr(),
+                             ws.numel(), st)
+            P.ffn_stage2_raw(cl, x.data_ptr(), 8, y.data_ptr(), ws.data_ptr(), ws.numel(), st,
+                             count_s=cnt.data_ptr())
+        ref = P.ffn_forward(c2.layer, x, c2.tau_x, c2.tau_s)
+    torch.cuda.synchronize()
+    assert torch.equal(cnt, ref.count_s)
+    rel = (torch.linalg.norm(y - ref.y, dim=1) / torch.linalg.norm(ref.y, dim=1)).max().item()
+    assert rel < 1e-5
+    assert P.last_device_status(ws)[0] == P.PROX_OK
