@@ -10,24 +10,31 @@
 // the plain reading: a channel kept by any token is read once per pass.
 //
 // Two kernels, chained with programmatic dependent launch after Stage 1:
-//   k_s2u_updown: U = W_up[union] x^T and G = W_gate[union] x^T over the full
-//     x, M = 128 union channels per tile, K = d_model split into ks slices.
-//     A CTA takes a contiguous range of (tile, slice) units and accumulates
-//     consecutive slices of one tile in TMEM; partial tiles are summed in
-//     global fp32 with vector atomics, and the CTA that completes a tile forms
-//     s = u * act(g) (zero where the token did not keep the channel), splits it
-//     into bf16 hi + lo (s = hi + lo to about 2^-16) and stores it as ready
-//     128-byte-swizzled B tiles.
-//   k_s2u_down: y^T += W_down[union]^T s^T, M = 128 d_model coordinates, K =
-//     union positions (W_down is row-major, so the A tile is MN-major), N =
-//     tokens; the hi and lo halves of s are two MMAs into one accumulator.
-//     Units (position range, coordinate tile) go to CTAs in contiguous ranges;
-//     each unit adds its 128 x nb block to y with fp32 atomics.
+//   k_s2u_updown: one MMA tile is 64 union channels: A rows 0..63 are their
+//     W_up rows and rows 64..127 their W_gate rows (K-major), B = x over the
+//     full d_model (K-major), so D holds u (lanes 0..63) and g (lanes 64..127).
+//     The (tile, 64-wide K block) steps are split evenly among the CTAs as
+//     contiguous ranges (stream-K); a CTA accumulates in TMEM while its steps
+//     stay in one tile. A tile split between CTAs is summed in global fp32
+//     with vector atomics, and the CTA that completes it forms s = u * act(g)
+//     (zero where the token did not keep the channel), splits it into bf16 hi
+//     + lo (s = hi + lo to about 2^-16) and stores it as ready 128-byte-
+//     swizzled B tiles (one 64-position K block per tile).
+//   k_s2u_down: y^T += W_down[union]^T s^T. A stage holds 32 union positions
+//     x 512 (or 256) output coordinates of W_down (row-major, so each position
+//     is one 1 KB run; an MN-major A operand) and the s tiles of those
+//     positions; four (two) M = 128 MMAs per 16 positions, hi and lo of s into
+//     one accumulator each. Steps (coordinate tile, 32 positions) are split
+//     evenly among CTAs; each CTA adds its accumulated block to y with fp32
+//     atomics whenever its range leaves a coordinate tile.
 // Both kernels: 256 threads, one CTA per SM; every thread moves 16-byte
 // pieces of the gathered rows with cp.async (L2 evict-first) straight into
 // the swizzled layout the MMA reads, one thread issues the MMAs, and
-// tcgen05.commit on a per-stage mbarrier frees a stage for reuse. All waits
-// are bounded; TMEM (32 columns) is freed before exit.
+// tcgen05.commit on a per-stage mbarrier frees a stage for reuse. The up/gate
+// ring is refilled in batches of half its depth, so each gathered row is
+// requested in runs of several consecutive 128-byte pieces (a run per stage
+// would scatter single 128-byte requests over the rows and leave DRAM far
+// from its streaming rate). All waits are bounded; TMEM is freed before exit.
 #include "prox_internal.cuh"
 
 #include <cuda_bf16.h>
@@ -38,17 +45,18 @@ namespace prox {
 
 namespace {
 
-constexpr int kUT = 256;              // threads per CTA
 constexpr int kUM = 128;              // UMMA M
 constexpr int kUN = 16;               // UMMA N: token slots (the pass's tokens, rest zero)
-constexpr int kUK = 64;               // K elements per stage: one 128-byte swizzle row of bf16
+constexpr int kUK = 64;               // K elements per up/gate stage: one 128-byte swizzle row
+constexpr int kTile = 64;             // union channels per up/gate tile (= positions per s tile)
+constexpr int kDnPos = 32;            // union positions per down stage
 constexpr uint32_t kAtom = 1024;      // 8 rows x 128 bytes
 constexpr uint32_t kInvalid = 0xFFFFFFFFu;
-constexpr int kTmemCols = 32;
 
 // ring stage sizes (bytes, multiples of the 1024-byte swizzle atom)
-constexpr uint32_t kUgStage = 2 * 16384 + 2 * kAtom;   // A_up | A_gate | x (16 rows)
-constexpr uint32_t kDnStage = 16384 + 4 * kAtom;       // A_down | s hi (16 rows) | s lo (16 rows)
+constexpr uint32_t kUgStage = 16384 + 2 * kAtom;   // A (64 up + 64 gate rows) | x (16 rows)
+__host__ __device__ constexpr uint32_t dn_a_bytes(int cw) { return (uint32_t)kDnPos * cw * 2; }
+__host__ __device__ constexpr uint32_t dn_stage(int cw) { return dn_a_bytes(cw) + 4 * kAtom; }
 
 // ---------------------------------------------------------------------------
 // tcgen05 / UMMA helpers
@@ -93,8 +101,8 @@ __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// generic-proxy writes to shared memory (cp.async, st.shared) made visible to
-// the tensor core's async-proxy reads
+// generic-proxy writes to shared memory (st.shared) made visible to the
+// tensor core's async-proxy reads
 __device__ __forceinline__ void fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -120,17 +128,18 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
     v[7] = __uint_as_float(r7);
 }
 
-// TMEM allocation by one whole warp; the address lands in *slot
-__device__ __forceinline__ void tmem_alloc(uint32_t *slot) {
+// TMEM allocation (a power of two >= 32 columns) by one whole warp; the
+// address lands in *slot
+__device__ __forceinline__ void tmem_alloc(uint32_t *slot, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_addr(slot)),
-                 "r"(kTmemCols)
+                 "r"(ncols)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
 }
-__device__ __forceinline__ void tmem_free(uint32_t taddr) {
+__device__ __forceinline__ void tmem_free(uint32_t taddr, uint32_t ncols) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr),
-                 "r"(kTmemCols)
+                 "r"(ncols)
                  : "memory");
 }
 
@@ -145,27 +154,6 @@ __device__ __forceinline__ void cp16_pol(uint32_t dst, const void *src, uint32_t
 __device__ __forceinline__ void cp16(uint32_t dst, const void *src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
-__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-__device__ __forceinline__ void cp_wait_dyn(int n) {
-    // the ring depth is a launch parameter; wait_group takes an immediate
-    switch (n) {
-        case 0: cp_wait<0>(); break;
-        case 1: cp_wait<1>(); break;
-        case 2: cp_wait<2>(); break;
-        case 3: cp_wait<3>(); break;
-        case 4: cp_wait<4>(); break;
-        case 5: cp_wait<5>(); break;
-        case 6: cp_wait<6>(); break;
-        case 7: cp_wait<7>(); break;
-        case 8: cp_wait<8>(); break;
-        default: cp_wait<9>(); break;
-    }
-}
-
 // byte offset of 16-byte chunk `c` of row `r` in a K-major 128-byte-swizzled
 // tile (8-row atoms, 1024 bytes apart)
 __device__ __forceinline__ uint32_t kmaj_off(int r, int c) {
@@ -211,7 +199,7 @@ __device__ int warp_scan_inplace(int *v, int n, int lane) {
 // shared-memory carve-up (offsets from a 1024-byte aligned base)
 // ---------------------------------------------------------------------------
 struct UgSmem {
-    uint32_t ring, bars, misc, uscan, rows, total;
+    uint32_t ring, bars, misc, xg, uscan, rows, total;
 };
 __host__ __device__ inline UgSmem ug_smem(int nstage, int C, int span) {
     UgSmem s;
@@ -219,14 +207,16 @@ __host__ __device__ inline UgSmem ug_smem(int nstage, int C, int span) {
     s.ring = o;
     o += (uint32_t)nstage * kUgStage;
     s.bars = o;
-    o += (uint32_t)(nstage + 1) * 8;
+    o += (uint32_t)(2 * nstage + 4) * 8;
     s.misc = o;
     o += 16;
+    s.xg = o;                                      // g of a tile, handed to the u warps
+    o += (uint32_t)kTile * 8 * 4;
     s.uscan = o;
     o += (uint32_t)(C + 1 > 8 ? C + 1 : 8) * 4;  // also per-token offsets at the end
     o = (o + 15) & ~15u;
     s.rows = o;
-    o += (uint32_t)span * kUM * 4;
+    o += (uint32_t)span * kTile * 4;
     s.total = o + 1024;  // alignment slack of the dynamic shared memory base
     return s;
 }
@@ -234,57 +224,100 @@ __host__ __device__ inline UgSmem ug_smem(int nstage, int C, int span) {
 struct DnSmem {
     uint32_t ring, bars, misc, rows, total;
 };
-__host__ __device__ inline DnSmem dn_smem(int nstage, int span) {
+__host__ __device__ inline DnSmem dn_smem(int nstage, int cw, int rows_cap) {
     DnSmem s;
     uint32_t o = 0;
     s.ring = o;
-    o += (uint32_t)nstage * kDnStage;
+    o += (uint32_t)nstage * dn_stage(cw);
     s.bars = o;
-    o += (uint32_t)(nstage + 1) * 8;
+    o += (uint32_t)(2 * nstage + 4) * 8;
     s.misc = o;
     o += 16;
     s.rows = o;
-    o += (uint32_t)span * kUnitPos * 4;
+    o += (uint32_t)rows_cap * 4;
     s.total = o + 1024;
     return s;
 }
 
+// This CTA's share [s0, s1) of n steps split evenly over the grid
+__device__ __forceinline__ void even_range(int n, int &s0, int &s1) {
+    s0 = (int)((long long)n * blockIdx.x / gridDim.x);
+    s1 = (int)((long long)n * (blockIdx.x + 1) / gridDim.x);
+}
+
+// Roles (both kernels): warps 0..7 load (every thread issues its share of a
+// stage's 16-byte copies, then cp.async.mbarrier.arrive.noinc on the stage's
+// "full" barrier, so no thread ever waits for its own copies and the whole
+// ring stays in flight); warp 8 issues the MMAs (one lane) and frees stages
+// with tcgen05.commit on their "empty" barriers; warps 9..12 (one per TMEM
+// lane quadrant) run the epilogues from two alternating accumulators.
+constexpr int kLoadWarps = 8;
+constexpr int kMmaWarp = 8;
+constexpr int kEpiWarp0 = 9;
+constexpr int kThreads = (kEpiWarp0 + 4) * 32;
+
+__device__ __forceinline__ void cp_arrive_noinc(uint64_t *bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void cp_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// barriers of a kernel: full[NST], empty[NST], acc_full[2], acc_empty[2]
+struct Bars {
+    uint64_t *full, *empty, *acc_full, *acc_empty;
+};
+__device__ __forceinline__ Bars carve_bars(unsigned char *p, int nst) {
+    uint64_t *b = reinterpret_cast<uint64_t *>(p);
+    return Bars{b, b + nst, b + 2 * nst, b + 2 * nst + 2};
+}
+__device__ __forceinline__ void init_bars(const Bars &b, int nst) {
+    for (int s = 0; s < nst; ++s) {
+        mbar_init(&b.full[s], kLoadWarps * 32);
+        mbar_init(&b.empty[s], 1);
+    }
+    for (int k = 0; k < 2; ++k) {
+        mbar_init(&b.acc_full[k], 1);
+        mbar_init(&b.acc_empty[k], 128);
+    }
+    mbar_fence_init();
+}
+
 // ---------------------------------------------------------------------------
-// up/gate over the union: U, G (TMEM) -> s tiles
+// up/gate over the union: u, g (TMEM) -> s tiles
 // ---------------------------------------------------------------------------
 template <int B>
-__global__ void __launch_bounds__(kUT, 1) k_s2u_updown(const Stage2UArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) k_s2u_updown(const Stage2UArgs a) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    const int d = a.d, C = a.C, KS = a.ks, NST = a.nstage;
+    const int d = a.d, C = a.C, NST = a.nstage;
     const uint32_t sbase = (smem_addr(smem_raw) + 1023u) & ~1023u;
     unsigned char *smem = smem_raw + (sbase - smem_addr(smem_raw));
     const UgSmem L = ug_smem(NST, C, a.span);
-    uint64_t *bar_free = reinterpret_cast<uint64_t *>(smem + L.bars);
-    uint64_t *bar_acc = bar_free + NST;
+    const Bars bar = carve_bars(smem + L.bars, NST);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L.misc);
     volatile int *fail = reinterpret_cast<volatile int *>(smem + L.misc + 4);
     volatile int *last = reinterpret_cast<volatile int *>(smem + L.misc + 8);
+    float *xg = reinterpret_cast<float *>(smem + L.xg);
     int *uscan = reinterpret_cast<int *>(smem + L.uscan);
     uint32_t *rows = reinterpret_cast<uint32_t *>(smem + L.rows);
 
-    // the x tiles' unused token rows stay zero for the whole kernel
+    // token rows of the x tiles that no copy fills stay zero
     for (int s = 0; s < NST; ++s) {
-        uint4 *xz = reinterpret_cast<uint4 *>(smem + L.ring + s * kUgStage + 2 * 16384);
-        for (int k = tid; k < (int)(2 * kAtom / 16); k += kUT) xz[k] = make_uint4(0, 0, 0, 0);
+        uint4 *xz = reinterpret_cast<uint4 *>(smem + L.ring + s * kUgStage + 16384);
+        for (int k = tid; k < (int)(2 * kAtom / 16); k += kThreads) xz[k] = make_uint4(0, 0, 0, 0);
     }
+    fence_async_smem();
     if (tid == 0) {
-        for (int s = 0; s <= NST; ++s) mbar_init(&bar_free[s], 1);
+        init_bars(bar, NST);
         *fail = 0;
-        mbar_fence_init();
     }
-    if (wid == 0) tmem_alloc(tmem_slot);
+    if (wid == kMmaWarp) tmem_alloc(tmem_slot, 32);
 
     // Stage 1's lists (and its clearing of the partial sums) are complete
     // once it has finished
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;");
-    for (int c = tid; c < C; c += kUT) uscan[c] = a.ucount[c];
+    for (int c = tid; c < C; c += kThreads) uscan[c] = a.ucount[c];
     __syncthreads();
     if (wid == 0) {
         const int tot = warp_scan_inplace(uscan, C, lane);
@@ -292,168 +325,175 @@ __global__ void __launch_bounds__(kUT, 1) k_s2u_updown(const Stage2UArgs a) {
     }
     __syncthreads();
     const int nU = uscan[C] < a.f ? uscan[C] : a.f;
-    const int ntiles = (nU + kUM - 1) / kUM;
-    const int nunits = ntiles * KS;
-    const int G = gridDim.x, g = blockIdx.x;
-    const int u0 = (int)((long long)nunits * g / G), u1 = (int)((long long)nunits * (g + 1) / G);
-    const int t_lo = u0 / KS;
+    const int NKB = d / kUK;                      // K blocks per tile
+    const int ntiles = (nU + kTile - 1) / kTile;
+    int S0, S1;
+    even_range(ntiles * NKB, S0, S1);
+    const int nsteps = S1 - S0;
+    const int t_lo = S0 / NKB;
+    const int t_hi = nsteps > 0 ? (S1 - 1) / NKB : t_lo - 1;
     // union entries (channel | token bits << 24) of this CTA's tiles
-    if (u1 > u0) {
-        const int t_hi = (u1 - 1) / KS;
-        for (int k = tid; k < (t_hi - t_lo + 1) * kUM; k += kUT) {
-            const int tile = t_lo + k / kUM, p = tile * kUM + k % kUM;
-            uint32_t e = kInvalid;
-            if (p < nU) {
-                int lo = 0, hi = C - 1;  // block c with uscan[c] <= p < uscan[c + 1]
-                while (lo < hi) {
-                    const int mid = (lo + hi + 1) >> 1;
-                    if (uscan[mid] <= p) lo = mid; else hi = mid - 1;
-                }
-                e = a.ulist[(size_t)lo * kCB + (p - uscan[lo])];
-                if ((int)(e & 0xFFFFFFu) >= a.f) e = kInvalid;  // never read outside W
-                // the CTA holding the tile's first slice publishes the positions
-                if (tile * KS >= u0) a.pos_ch[p] = e;
+    for (int k = tid; k < (t_hi - t_lo + 1) * kTile; k += kThreads) {
+        const int tile = t_lo + k / kTile, p = tile * kTile + k % kTile;
+        uint32_t e = kInvalid;
+        if (p < nU) {
+            int lo = 0, hi = C - 1;  // block c with uscan[c] <= p < uscan[c + 1]
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (uscan[mid] <= p) lo = mid; else hi = mid - 1;
             }
-            rows[k] = e;
+            e = a.ulist[(size_t)lo * kCB + (p - uscan[lo])];
+            if ((int)(e & 0xFFFFFFu) >= a.f) e = kInvalid;  // never read outside W
+            // the CTA holding the tile's first K block publishes the positions
+            if (tile * NKB >= S0) a.pos_ch[p] = e;
         }
+        rows[k] = e;
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-
-    const int kbpu = d / kUK / KS;  // K blocks per unit
-    const int nsteps = (u1 - u0) * kbpu;
-    const uint64_t pol = l2_evict_first();
     const uint32_t ring = sbase + L.ring;
-    constexpr uint32_t idesc = bf16_idesc(false);
 
-    // issue the copies of step ls into its ring stage
-    auto load = [&](int ls) {
-        const int u = u0 + ls / kbpu;
-        const int tile = u / KS, kb = (u % KS) * kbpu + ls % kbpu;
-        const uint32_t st = ring + (uint32_t)(ls % NST) * kUgStage;
-        const uint32_t *er = rows + (tile - t_lo) * kUM;
+    if (wid < kLoadWarps) {
+        // ---------------- loaders ----------------
+        const uint64_t pol = l2_evict_first();
         const int c = tid & 7;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int r = (tid >> 3) + 32 * (j & 3);
-            const uint32_t e = er[r];
-            if (e == kInvalid) continue;  // rows past the union: never read back
-            const uint16_t *w = (j < 4) ? a.w_up : a.w_gate;
-            cp16_pol(st + (uint32_t)(j >> 2) * 16384u + kmaj_off(r, c),
-                     w + (size_t)(e & 0xFFFFFFu) * d + kb * kUK + c * 8, 16, pol);
-        }
-        if (tid < B * 8) {
-            const int t = tid >> 3;
-            if (t < a.nb) cp16(st + 2 * 16384u + kmaj_off(t, c), a.x + (size_t)t * d + kb * kUK + c * 8);
-        }
-    };
-
-    for (int ls = 0; ls < NST - 1; ++ls) {
-        if (ls < nsteps) load(ls);
-        cp_commit();
-    }
-    int nseg = 0;
-    for (int s = 0; s < nsteps; ++s) {
-        const int u = u0 + s / kbpu, j = s % kbpu;
-        const int tile = u / KS;
-        const bool seg_first = (s == 0) || (j == 0 && (u % KS) == 0);
-        const bool seg_last = (s == nsteps - 1) || (j == kbpu - 1 && ((u + 1) % KS) == 0);
-        const int stg = s % NST;
-        cp_wait_dyn(NST - 2);
-        fence_async_smem();
-        __syncthreads();
-        if (tid == 0 && !*fail) {
-            tc_fence_after();
+        for (int ls = 0; ls < nsteps; ++ls) {
+            const int stg = ls % NST;
+            if (ls >= NST) cta_wait(&bar.empty[stg], ((ls / NST) - 1) & 1, a, fail);
+            const int step = S0 + ls;
+            const int tile = step / NKB, kb = step % NKB;
             const uint32_t st = ring + (uint32_t)stg * kUgStage;
+            const uint32_t *er = rows + (tile - t_lo) * kTile;
+            // 64 up rows, then the same channels' gate rows, 128 bytes each
 #pragma unroll
-            for (int kk = 0; kk < kUK / 16; ++kk) {
-                const uint64_t db = sw128_desc(st + 2 * 16384u + kk * 32, 16, kAtom);
-                const uint32_t acc = (seg_first && kk == 0) ? 0u : 1u;
-                umma(tmem, sw128_desc(st + kk * 32, 16, kAtom), db, idesc, acc);
-                umma(tmem + 16, sw128_desc(st + 16384u + kk * 32, 16, kAtom), db, idesc, acc);
+            for (int j = 0; j < 4; ++j) {
+                const int r = (tid >> 3) + 32 * j;
+                const uint32_t e = er[r & (kTile - 1)];
+                if (e == kInvalid) continue;  // rows past the union: never read back
+                const uint16_t *w = (r < kTile) ? a.w_up : a.w_gate;
+                cp16_pol(st + kmaj_off(r, c), w + (size_t)(e & 0xFFFFFFu) * d + kb * kUK + c * 8,
+                         16, pol);
             }
-            umma_commit(&bar_free[stg]);
-            if (seg_last) umma_commit(bar_acc);
-        }
-        // refill the stage step s - 1 used, once its MMAs are done
-        if (s >= 1) cta_wait(&bar_free[(s - 1) % NST], ((s - 1) / NST) & 1, a, fail);
-        if (s + NST - 1 < nsteps) load(s + NST - 1);
-        cp_commit();
-
-        if (!seg_last) continue;
-        // ---- epilogue of a tile segment: slices [ks_lo, ks_hi) of `tile`
-        const int ks_lo = (tile * KS > u0 ? tile * KS : u0) - tile * KS;
-        const int ks_hi = u + 1 - tile * KS;
-        const bool whole = (ks_lo == 0 && ks_hi == KS);
-        cta_wait(bar_acc, nseg & 1, a, fail);
-        ++nseg;
-        tc_fence_after();
-        const int r = (wid & 3) * 32 + lane;
-        const int p = tile * kUM + r;
-        float U[8], Gt[8];
-        if (wid < 4) {
-            const uint32_t ta = tmem + ((uint32_t)(wid * 32) << 16);
-            tmem_ld8(ta, U);
-            tmem_ld8(ta + 16, Gt);
-            if (!whole && p < nU) {
-                float *dst = a.ug + (size_t)p * 2 * B;
-                red_add_v4(dst, U[0], U[1], U[2], U[3]);
-                if (B == 8) red_add_v4(dst + 4, U[4], U[5], U[6], U[7]);
-                red_add_v4(dst + B, Gt[0], Gt[1], Gt[2], Gt[3]);
-                if (B == 8) red_add_v4(dst + B + 4, Gt[4], Gt[5], Gt[6], Gt[7]);
-                __threadfence();
+            if (tid < B * 8) {
+                const int t = tid >> 3;
+                if (t < a.nb)
+                    cp16(st + 16384u + kmaj_off(t, c), a.x + (size_t)t * d + kb * kUK + c * 8);
             }
+            cp_arrive_noinc(&bar.full[stg]);
         }
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
-            int l = 1;
-            if (!whole) {
-                const int n = ks_hi - ks_lo;
-                l = (atomicAdd(a.tile_cnt + tile, n) + n == KS);
-            }
-            *last = l;
-        }
-        __syncthreads();
-        if (*last && wid < 4) {
-            // this CTA completes the tile: s = u * act(g) per kept (token,
-            // channel), as bf16 hi + lo in the down GEMM's swizzled B layout
-            if (!whole) {
-                __threadfence();
-                if (p < nU) {
-                    const float4 *src = reinterpret_cast<const float4 *>(a.ug + (size_t)p * 2 * B);
-                    float4 v = __ldcg(src);
-                    U[0] = v.x; U[1] = v.y; U[2] = v.z; U[3] = v.w;
-                    if (B == 8) { v = __ldcg(src + 1); U[4] = v.x; U[5] = v.y; U[6] = v.z; U[7] = v.w; }
-                    v = __ldcg(src + B / 4);
-                    Gt[0] = v.x; Gt[1] = v.y; Gt[2] = v.z; Gt[3] = v.w;
-                    if (B == 8) { v = __ldcg(src + B / 4 + 1); Gt[4] = v.x; Gt[5] = v.y; Gt[6] = v.z; Gt[7] = v.w; }
+        cp_wait_all();
+    } else if (wid == kMmaWarp) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            constexpr uint32_t idesc = bf16_idesc(false);
+            int seg = 0;
+            for (int s = 0; s < nsteps; ++s) {
+                const int stg = s % NST;
+                const int kb = (S0 + s) % NKB;
+                const bool seg_first = (s == 0) || kb == 0;
+                const bool seg_last = (s == nsteps - 1) || kb == NKB - 1;
+                const uint32_t acc = tmem + (uint32_t)(seg & 1) * kUN;
+                if (seg_first && seg >= 2) cta_wait(&bar.acc_empty[seg & 1], ((seg >> 1) - 1) & 1, a, fail);
+                cta_wait(&bar.full[stg], (s / NST) & 1, a, fail);
+                tc_fence_after();
+                if (!*fail) {
+                    const uint32_t st = ring + (uint32_t)stg * kUgStage;
+#pragma unroll
+                    for (int kk = 0; kk < kUK / 16; ++kk)
+                        umma(acc, sw128_desc(st + kk * 32, 16, kAtom),
+                             sw128_desc(st + 16384u + kk * 32, 16, kAtom), idesc,
+                             (seg_first && kk == 0) ? 0u : 1u);
+                }
+                umma_commit(&bar.empty[stg]);
+                if (seg_last) {
+                    umma_commit(&bar.acc_full[seg & 1]);
+                    ++seg;
                 }
             }
-            const uint32_t e = rows[(tile - t_lo) * kUM + r];
-            const uint32_t bits = (p < nU) ? (e >> 24) : 0u;
-            unsigned char *tb = reinterpret_cast<unsigned char *>(a.sb) + (size_t)(p >> 6) * 2 * kAtom;
-            const int kk = p & 63;
+        }
+        __syncwarp();
+    } else {
+        // ---------------- epilogue: one segment per tile this CTA touches ----
+        const int q = wid & 3;                       // TMEM lane quadrant
+        const int r = q * 32 + lane;                 // A row: u (r < 64) or g
+        const int et = tid - kEpiWarp0 * 32;         // 0..127
+        for (int tile = t_lo, seg = 0; tile <= t_hi; ++tile, ++seg) {
+            const int kb0 = (tile * NKB > S0 ? tile * NKB : S0) - tile * NKB;
+            const int kb1 = ((tile + 1) * NKB < S1 ? (tile + 1) * NKB : S1) - tile * NKB;
+            const bool whole = (kb0 == 0 && kb1 == NKB);
+            const int p = tile * kTile + (r & (kTile - 1));
+            cta_wait(&bar.acc_full[seg & 1], (seg >> 1) & 1, a, fail);
+            tc_fence_after();
+            float v[8];
+            tmem_ld8(tmem + (uint32_t)(seg & 1) * kUN + ((uint32_t)(q * 32) << 16), v);
+            tc_fence_before();
+            mbar_arrive(&bar.acc_empty[seg & 1]);
+            if (!whole) {
+                if (p < nU) {
+                    float *dst = a.ug + (size_t)p * 2 * B + (r < kTile ? 0 : B);
+                    red_add_v4(dst, v[0], v[1], v[2], v[3]);
+                    if (B == 8) red_add_v4(dst + 4, v[4], v[5], v[6], v[7]);
+                    __threadfence();
+                }
+            } else if (r >= kTile) {
 #pragma unroll
-            for (int t = 0; t < 8; ++t) {
-                float sv = 0.f;
-                if (t < B && t < a.nb && ((bits >> t) & 1u)) sv = U[t] * gate_act(Gt[t], a.act);
-                const __nv_bfloat16 hi = __float2bfloat16_rn(sv);
-                const __nv_bfloat16 lo = __float2bfloat16_rn(sv - __bfloat162float(hi));
-                const uint32_t off = (uint32_t)t * 128u + ((uint32_t)((kk >> 3) ^ t) << 4) + (kk & 7) * 2;
-                *reinterpret_cast<__nv_bfloat16 *>(tb + off) = hi;
-                *reinterpret_cast<__nv_bfloat16 *>(tb + kAtom + off) = lo;
+                for (int t = 0; t < 8; ++t) xg[(r - kTile) * 8 + t] = v[t];
             }
+            named_bar_sync(1, 128);
+            if (et == 0) {
+                int l = 1;
+                if (!whole) {
+                    const int n = kb1 - kb0;
+                    l = (atomicAdd(a.tile_cnt + tile, n) + n == NKB);
+                }
+                *last = l;
+            }
+            named_bar_sync(1, 128);
+            if (*last && r < kTile) {
+                // this CTA completes the tile: s = u * act(g) per kept (token,
+                // channel), as bf16 hi + lo in the down GEMM's swizzled B layout
+                float g[8];
+                if (whole) {
+#pragma unroll
+                    for (int t = 0; t < 8; ++t) g[t] = xg[r * 8 + t];
+                } else {
+                    __threadfence();
+                    if (p < nU) {
+                        const float4 *src = reinterpret_cast<const float4 *>(a.ug + (size_t)p * 2 * B);
+                        float4 w4 = __ldcg(src);
+                        v[0] = w4.x; v[1] = w4.y; v[2] = w4.z; v[3] = w4.w;
+                        if (B == 8) { w4 = __ldcg(src + 1); v[4] = w4.x; v[5] = w4.y; v[6] = w4.z; v[7] = w4.w; }
+                        w4 = __ldcg(src + B / 4);
+                        g[0] = w4.x; g[1] = w4.y; g[2] = w4.z; g[3] = w4.w;
+                        if (B == 8) { w4 = __ldcg(src + B / 4 + 1); g[4] = w4.x; g[5] = w4.y; g[6] = w4.z; g[7] = w4.w; }
+                    }
+                }
+                const uint32_t e = rows[(tile - t_lo) * kTile + r];
+                const uint32_t bits = (p < nU) ? (e >> 24) : 0u;
+                unsigned char *tb = reinterpret_cast<unsigned char *>(a.sb) + (size_t)tile * 2 * kAtom;
+#pragma unroll
+                for (int t = 0; t < 8; ++t) {
+                    float sv = 0.f;
+                    if (t < B && t < a.nb && ((bits >> t) & 1u)) sv = v[t] * gate_act(g[t], a.act);
+                    const __nv_bfloat16 hi = __float2bfloat16_rn(sv);
+                    const __nv_bfloat16 lo = __float2bfloat16_rn(sv - __bfloat162float(hi));
+                    const uint32_t off = (uint32_t)t * 128u + ((uint32_t)((r >> 3) ^ t) << 4) + (r & 7) * 2;
+                    *reinterpret_cast<__nv_bfloat16 *>(tb + off) = hi;
+                    *reinterpret_cast<__nv_bfloat16 *>(tb + kAtom + off) = lo;
+                }
+            }
+            named_bar_sync(1, 128);  // xg and *last are reused by the next tile
         }
     }
-    cp_wait<0>();
 
     // per-token ascending kept-channel lists and counts (blocks c = g, g + G, ...)
+    __syncthreads();
+    const int G = gridDim.x, gi = blockIdx.x;
     if (a.idx_s || a.count_s) {
         int *tbase = uscan;  // reused: [B] per-token offsets of block c
-        for (int c = g; c < C; c += G) {
+        for (int c = gi; c < C; c += G) {
             __syncthreads();
             if (wid < a.nb) {
                 int sum = 0;
@@ -466,11 +506,11 @@ __global__ void __launch_bounds__(kUT, 1) k_s2u_updown(const Stage2UArgs a) {
             if (a.idx_s)
                 for (int t = 0; t < a.nb; ++t) {
                     const int nk = a.tcount[c * B + t];
-                    for (int k = tid; k < nk; k += kUT)
+                    for (int k = tid; k < nk; k += kThreads)
                         a.idx_s[(size_t)t * a.f + tbase[t] + k] = a.tlist[(size_t)t * a.f + c * kCB + k];
                 }
         }
-        if (g == 0 && a.count_s && wid < a.nb) {
+        if (gi == 0 && a.count_s && wid < a.nb) {
             int sum = 0;
             for (int k = lane; k < C; k += 32) sum += a.tcount[k * B + wid];
 #pragma unroll
@@ -480,44 +520,49 @@ __global__ void __launch_bounds__(kUT, 1) k_s2u_updown(const Stage2UArgs a) {
     }
     tc_fence_before();
     __syncthreads();
-    if (wid == 0) {
+    if (wid == kMmaWarp) {
         tc_fence_after();
-        tmem_free(tmem);
+        tmem_free(tmem, 32);
     }
 }
 
 // ---------------------------------------------------------------------------
 // down over the union: y^T += W_down[union]^T (s_hi + s_lo)^T
 // ---------------------------------------------------------------------------
-template <int B>
-__global__ void __launch_bounds__(kUT, 1) k_s2u_down(const Stage2UArgs a) {
+template <int B, int NM>  // NM: 128-coordinate M tiles per stage (coordinate tile = 128 NM)
+__global__ void __launch_bounds__(kThreads, 1) k_s2u_down(const Stage2UArgs a) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
+    constexpr int CW = NM * kUM;                 // output coordinates per stage
+    constexpr uint32_t ABYTES = dn_a_bytes(CW);
+    constexpr uint32_t STG = dn_stage(CW);
+    constexpr uint32_t LBO = (kDnPos / 8) * kAtom;  // stride of 64-coordinate atoms
+    constexpr uint32_t ACOLS = NM * kUN;           // columns of one accumulator
+    constexpr uint32_t TCOLS = 2 * ACOLS < 32 ? 32 : 2 * ACOLS;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int d = a.d, C = a.C, NST = a.nstage_dn;
     const uint32_t sbase = (smem_addr(smem_raw) + 1023u) & ~1023u;
     unsigned char *smem = smem_raw + (sbase - smem_addr(smem_raw));
-    const DnSmem L = dn_smem(NST, a.span_dn);
-    uint64_t *bar_free = reinterpret_cast<uint64_t *>(smem + L.bars);
-    uint64_t *bar_acc = bar_free + NST;
+    const DnSmem L = dn_smem(NST, CW, a.rows_dn);
+    const Bars bar = carve_bars(smem + L.bars, NST);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L.misc);
     volatile int *fail = reinterpret_cast<volatile int *>(smem + L.misc + 4);
     int *ntot = reinterpret_cast<int *>(smem + L.misc + 8);
     uint32_t *rows = reinterpret_cast<uint32_t *>(smem + L.rows);
 
-    // the s tiles' token rows 8..15 stay zero for the whole kernel
+    // token rows 8..15 of the s tiles stay zero for the whole kernel
     for (int s = 0; s < NST; ++s) {
-        unsigned char *bz = smem + L.ring + s * kDnStage + 16384;
-        for (int k = tid; k < (int)(2 * kAtom / 16); k += kUT) {
+        unsigned char *bz = smem + L.ring + s * STG + ABYTES;
+        for (int k = tid; k < (int)(2 * kAtom / 16); k += kThreads) {
             const int h = k / (kAtom / 16), q = k % (kAtom / 16);
             reinterpret_cast<uint4 *>(bz + h * 2 * kAtom + kAtom)[q] = make_uint4(0, 0, 0, 0);
         }
     }
+    fence_async_smem();
     if (tid == 0) {
-        for (int s = 0; s <= NST; ++s) mbar_init(&bar_free[s], 1);
+        init_bars(bar, NST);
         *fail = 0;
-        mbar_fence_init();
     }
-    if (wid == 0) tmem_alloc(tmem_slot);
+    if (wid == kMmaWarp) tmem_alloc(tmem_slot, TCOLS);
 
     // the up/gate kernel's s tiles and positions are complete once it has finished
     asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -531,118 +576,124 @@ __global__ void __launch_bounds__(kUT, 1) k_s2u_down(const Stage2UArgs a) {
     }
     __syncthreads();
     const int nU = *ntot < a.f ? *ntot : a.f;
-    const int MT = d / kUM;
-    constexpr int KPB = kUnitPos / kUK;             // K blocks per unit
-    const int nkb_all = (nU + kUK - 1) / kUK;       // K blocks holding union positions
-    const int NKR = (nU + kUnitPos - 1) / kUnitPos;
-    const int nunits = NKR * MT;
-    const int G = gridDim.x, g = blockIdx.x;
-    const int u0 = (int)((long long)nunits * g / G), u1 = (int)((long long)nunits * (g + 1) / G);
-    const int kr_lo = u0 / MT;
-    if (u1 > u0) {
-        const int kr_hi = (u1 - 1) / MT;
-        for (int k = tid; k < (kr_hi - kr_lo + 1) * kUnitPos; k += kUT) {
-            const int p = kr_lo * kUnitPos + k;
-            rows[k] = p < nU ? __ldcg(a.pos_ch + p) : kInvalid;
-        }
+    const int NPB = (nU + kDnPos - 1) / kDnPos;   // position blocks
+    int S0, S1;
+    even_range((d / CW) * NPB, S0, S1);
+    const int nsteps = S1 - S0;
+    for (int k = tid; k < nsteps * kDnPos; k += kThreads) {
+        const int p = ((S0 + k / kDnPos) % NPB) * kDnPos + k % kDnPos;
+        rows[k] = p < nU ? __ldcg(a.pos_ch + p) : kInvalid;
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint64_t pol = l2_evict_first();
     const uint32_t ring = sbase + L.ring;
-    constexpr uint32_t idesc = bf16_idesc(true);
-    const unsigned char *sbg = reinterpret_cast<const unsigned char *>(a.sb);
 
-    auto nkb = [&](int u) {
-        const int r = nkb_all - (u / MT) * KPB;
-        return r < KPB ? r : KPB;
-    };
-    // issue the copies of (unit u, K block j) into ring stage stg
-    auto load = [&](int u, int j, int stg) {
-        const int kr = u / MT, mt = u % MT;
-        const int kb = kr * KPB + j;
-        const uint32_t st = ring + (uint32_t)stg * kDnStage;
-        const uint32_t *er = rows + (kr - kr_lo) * kUnitPos + j * kUK;
-        const int c = tid & 15;
+    if (wid < kLoadWarps) {
+        // ---------------- loaders ----------------
+        const uint64_t pol = l2_evict_first();
+        const unsigned char *sbg = reinterpret_cast<const unsigned char *>(a.sb);
+        constexpr int CPR = CW / 8;               // 16-byte pieces per position
+        for (int ls = 0; ls < nsteps; ++ls) {
+            const int stg = ls % NST;
+            if (ls >= NST) cta_wait(&bar.empty[stg], ((ls / NST) - 1) & 1, a, fail);
+            const int step = S0 + ls;
+            const int mt = step / NPB, pb = step % NPB;
+            const uint32_t st = ring + (uint32_t)stg * STG;
+            const uint32_t *er = rows + ls * kDnPos;
+            // 32 positions x CW coordinates of W_down: each position one
+            // contiguous 2 CW-byte run; MN-major, 64 coordinates per 128-byte
+            // row, 8 positions per atom
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int row = (tid >> 4) + 16 * i;  // union position within the block (K)
-            const uint32_t e = er[row];
-            const bool ok = e != kInvalid && (int)(e & 0xFFFFFFu) < a.f;
-            const uint16_t *src = ok ? a.w_down + (size_t)(e & 0xFFFFFFu) * d + mt * kUM + c * 8 : a.w_down;
-            // MN-major: 64 coordinates per 128-byte row, 8 positions per atom
-            const uint32_t off = (uint32_t)(c >> 3) * (8 * kAtom) + (uint32_t)(row >> 3) * kAtom +
-                                 (uint32_t)(row & 7) * 128u + ((uint32_t)((c & 7) ^ (row & 7)) << 4);
-            cp16_pol(st + off, src, ok ? 16u : 0u, pol);
-        }
-        if (tid < 128) {  // s hi and lo atoms (token rows 0..7), stored pre-swizzled
-            const int h = tid >> 6, q = tid & 63;
-            cp16(st + 16384u + (uint32_t)h * 2 * kAtom + q * 16,
-                 sbg + (size_t)kb * 2 * kAtom + h * kAtom + q * 16);
-        }
-    };
-
-    // loader cursor runs NST - 1 steps ahead of the consumer cursor
-    int lu = u0, lj = 0, ln = 0;
-    auto load_next = [&]() {
-        if (lu < u1) {
-            load(lu, lj, ln % NST);
-            if (++lj == nkb(lu)) { ++lu; lj = 0; }
-            ++ln;
-        }
-        cp_commit();
-    };
-    for (int k = 0; k < NST - 1; ++k) load_next();
-    int cu = u0, cj = 0, n = 0, nseg = 0;
-    while (cu < u1) {
-        const int stg = n % NST;
-        const bool unit_last = (cj + 1 == nkb(cu));
-        cp_wait_dyn(NST - 2);
-        fence_async_smem();
-        __syncthreads();
-        if (tid == 0 && !*fail) {
-            tc_fence_after();
-            const uint32_t st = ring + (uint32_t)stg * kDnStage;
-#pragma unroll
-            for (int kk = 0; kk < kUK / 16; ++kk) {
-                const uint64_t da = sw128_desc(st + kk * 2 * kAtom, 8 * kAtom, kAtom);
-                umma(tmem, da, sw128_desc(st + 16384u + kk * 32, 16, kAtom), idesc,
-                     (cj == 0 && kk == 0) ? 0u : 1u);
-                umma(tmem, da, sw128_desc(st + 16384u + 2 * kAtom + kk * 32, 16, kAtom), idesc, 1u);
+            for (int i = 0; i < kDnPos * CPR / (kLoadWarps * 32); ++i) {
+                const int qq = tid + kLoadWarps * 32 * i;
+                const int row = qq / CPR, c = qq % CPR;
+                const uint32_t e = er[row];
+                const bool ok = e != kInvalid && (int)(e & 0xFFFFFFu) < a.f;
+                const uint16_t *src =
+                    ok ? a.w_down + (size_t)(e & 0xFFFFFFu) * d + mt * CW + c * 8 : a.w_down;
+                const uint32_t off = (uint32_t)(c >> 3) * LBO + (uint32_t)(row >> 3) * kAtom +
+                                     (uint32_t)(row & 7) * 128u + ((uint32_t)((c & 7) ^ (row & 7)) << 4);
+                cp16_pol(st + off, src, ok ? 16u : 0u, pol);
             }
-            umma_commit(&bar_free[stg]);
-            if (unit_last) umma_commit(bar_acc);
+            if (tid < 128) {  // s hi and lo atoms (token rows 0..7) of the 64-position block
+                const int h = tid >> 6, qq = tid & 63;
+                cp16(st + ABYTES + (uint32_t)h * 2 * kAtom + qq * 16,
+                     sbg + (size_t)(pb >> 1) * 2 * kAtom + h * kAtom + qq * 16);
+            }
+            cp_arrive_noinc(&bar.full[stg]);
         }
-        if (n >= 1) cta_wait(&bar_free[(n - 1) % NST], ((n - 1) / NST) & 1, a, fail);
-        load_next();
-        if (unit_last) {
-            cta_wait(bar_acc, nseg & 1, a, fail);
-            ++nseg;
+        cp_wait_all();
+    } else if (wid == kMmaWarp) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            constexpr uint32_t idesc = bf16_idesc(true);
+            int seg = 0;
+            for (int s = 0; s < nsteps; ++s) {
+                const int stg = s % NST;
+                const int pb = (S0 + s) % NPB;
+                const bool seg_first = (s == 0) || pb == 0;
+                const bool seg_last = (s == nsteps - 1) || pb == NPB - 1;
+                const uint32_t acc = tmem + (uint32_t)(seg & 1) * ACOLS;
+                if (seg_first && seg >= 2) cta_wait(&bar.acc_empty[seg & 1], ((seg >> 1) - 1) & 1, a, fail);
+                cta_wait(&bar.full[stg], (s / NST) & 1, a, fail);
+                tc_fence_after();
+                if (!*fail) {
+                    const uint32_t st = ring + (uint32_t)stg * STG;
+#pragma unroll
+                    for (int kk = 0; kk < kDnPos / 16; ++kk) {
+                        const uint32_t bo = st + ABYTES + (uint32_t)((pb & 1) * 2 + kk) * 32;
+                        const uint64_t dbh = sw128_desc(bo, 16, kAtom);
+                        const uint64_t dbl = sw128_desc(bo + 2 * kAtom, 16, kAtom);
+#pragma unroll
+                        for (int mi = 0; mi < NM; ++mi) {
+                            const uint64_t da = sw128_desc(st + mi * 2 * LBO + kk * 2 * kAtom, LBO, kAtom);
+                            umma(acc + mi * kUN, da, dbh, idesc, (seg_first && kk == 0) ? 0u : 1u);
+                            umma(acc + mi * kUN, da, dbl, idesc, 1u);
+                        }
+                    }
+                }
+                umma_commit(&bar.empty[stg]);
+                if (seg_last) {
+                    umma_commit(&bar.acc_full[seg & 1]);
+                    ++seg;
+                }
+            }
+        }
+        __syncwarp();
+    } else {
+        // ---------------- epilogue: y += one coordinate tile's block ----------
+        const int q = wid & 3;
+        int seg = 0;
+        for (int s = 0; s < nsteps; ++s) {
+            const int step = S0 + s;
+            const int pb = step % NPB;
+            if (!(s == nsteps - 1 || pb == NPB - 1)) continue;
+            const int mt = step / NPB;
+            cta_wait(&bar.acc_full[seg & 1], (seg >> 1) & 1, a, fail);
             tc_fence_after();
-            if (wid < 4) {
-                float D[8];
-                tmem_ld8(tmem + ((uint32_t)(wid * 32) << 16), D);
-                const int m = (cu % MT) * kUM + wid * 32 + lane;
+            float D[NM][8];
+#pragma unroll
+            for (int mi = 0; mi < NM; ++mi)
+                tmem_ld8(tmem + (uint32_t)(seg & 1) * ACOLS + mi * kUN + ((uint32_t)(q * 32) << 16), D[mi]);
+            tc_fence_before();
+            mbar_arrive(&bar.acc_empty[seg & 1]);
+#pragma unroll
+            for (int mi = 0; mi < NM; ++mi) {
+                const int m = mt * CW + mi * kUM + q * 32 + lane;
 #pragma unroll
                 for (int t = 0; t < B; ++t)
-                    if (t < a.nb) atomicAdd(a.y + (size_t)t * d + m, D[t]);
+                    if (t < a.nb) atomicAdd(a.y + (size_t)t * d + m, D[mi][t]);
             }
-            tc_fence_before();
-            ++cu;
-            cj = 0;
-        } else {
-            ++cj;
+            ++seg;
         }
-        ++n;
     }
-    cp_wait<0>();
     tc_fence_before();
     __syncthreads();
-    if (wid == 0) {
+    if (wid == kMmaWarp) {
         tc_fence_after();
-        tmem_free(tmem);
+        tmem_free(tmem, TCOLS);
     }
 }
 
@@ -656,15 +707,15 @@ cudaError_t set_smem(K k, size_t smem, size_t &configured) {
     return cudaSuccess;
 }
 
-template <int B>
+template <int B, int NM>
 cudaError_t launch_u(const Stage2UArgs &a, int grid, cudaStream_t s) {
     static size_t cfg_ug = 0, cfg_dn = 0;
     const size_t sm_ug = ug_smem(a.nstage, a.C, a.span).total;
-    const size_t sm_dn = dn_smem(a.nstage_dn, a.span_dn).total;
+    const size_t sm_dn = dn_smem(a.nstage_dn, NM * kUM, a.rows_dn).total;
     cudaError_t e = set_smem(k_s2u_updown<B>, sm_ug, cfg_ug);
-    if (e == cudaSuccess) e = set_smem(k_s2u_down<B>, sm_dn, cfg_dn);
-    if (e == cudaSuccess) e = launch_pdl(k_s2u_updown<B>, dim3(grid), dim3(kUT), sm_ug, s, a);
-    if (e == cudaSuccess) e = launch_pdl(k_s2u_down<B>, dim3(grid), dim3(kUT), sm_dn, s, a);
+    if (e == cudaSuccess) e = set_smem(k_s2u_down<B, NM>, sm_dn, cfg_dn);
+    if (e == cudaSuccess) e = launch_pdl(k_s2u_updown<B>, dim3(grid), dim3(kThreads), sm_ug, s, a);
+    if (e == cudaSuccess) e = launch_pdl(k_s2u_down<B, NM>, dim3(grid), dim3(kThreads), sm_dn, s, a);
     return e;
 }
 
@@ -672,32 +723,32 @@ cudaError_t launch_u(const Stage2UArgs &a, int grid, cudaStream_t s) {
 
 // Launch plan of the tensor-core Stage 2; false if the shape is outside it
 bool stage2u_plan(int d, int f, int num_sms, Stage2UPlan *p) {
-    const int kblocks = d / kUK;
-    int ks = 8;
-    while (ks > 1 && kblocks % ks) ks >>= 1;
     const int C = f / kCB;
-    const int ntiles_max = f / kUM;
-    const int lenA = (ntiles_max * ks + num_sms - 1) / num_sms;  // units per CTA, at most
-    p->ks = ks;
-    p->span = (lenA + ks - 1) / ks + 1;
-    const int MT = d / kUM;
-    const int nkr_max = (f + kUnitPos - 1) / kUnitPos;
-    const int lenB = (nkr_max * MT + num_sms - 1) / num_sms;
-    p->span_dn = (lenB + MT - 1) / MT + 1;
+    const int nkb = d / kUK;
+    const int stepsA = (f / kTile) * nkb;                       // at most
+    const int lenA = (stepsA + num_sms - 1) / num_sms;
+    p->span = (lenA + nkb - 1) / nkb + 1;
+    p->cw = (d % 512 == 0) ? 512 : 256;
+    const int stepsB = (d / p->cw) * ((f + kDnPos - 1) / kDnPos);
+    p->rows_dn = (stepsB + num_sms - 1) / num_sms * kDnPos;
     const size_t budget = (size_t)kS2SmemBudget;
-    const size_t fixA = ug_smem(0, C, p->span).total, fixB = dn_smem(0, p->span_dn).total;
-    if (fixA >= budget || fixB >= budget) return false;
-    int na = (int)((budget - fixA) / kUgStage), nb = (int)((budget - fixB) / kDnStage);
-    if (na > 8) na = 8;
-    if (nb > 10) nb = 10;
+    int na = 12, nb = 8;
+    while (na > 0 && ug_smem(na, C, p->span).total > budget) --na;
+    while (nb > 0 && dn_smem(nb, p->cw, p->rows_dn).total > budget) --nb;
     p->nstage = na;
+    p->refill = 0;
     p->nstage_dn = nb;
-    return na >= 3 && nb >= 3;
+    return na >= 4 && nb >= 3;
 }
 
 cudaError_t launch_stage2_umma(int B, const Stage2UArgs &a, int grid, cudaStream_t s) {
-    if (B == 4) return launch_u<4>(a, grid, s);
-    if (B == 8) return launch_u<8>(a, grid, s);
+    if (a.cw == 512) {
+        if (B == 4) return launch_u<4, 4>(a, grid, s);
+        if (B == 8) return launch_u<8, 4>(a, grid, s);
+    } else if (a.cw == 256) {
+        if (B == 4) return launch_u<4, 2>(a, grid, s);
+        if (B == 8) return launch_u<8, 2>(a, grid, s);
+    }
     return cudaErrorInvalidValue;
 }
 

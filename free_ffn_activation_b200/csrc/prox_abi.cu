@@ -106,7 +106,7 @@ WsLayout ws_layout(int d, int f, int B) {
         L.ug = o;
         o += (size_t)f * 2 * B * 4;
         L.tile_cnt = o;
-        o = align_up(o + (size_t)(f / 128) * 4, 256);
+        o = align_up(o + (size_t)(f / 64) * 4, 256);
         L.clear_bytes = o - L.ug;
         L.sb = o;
         o = align_up(o + (size_t)(f / 64) * 2048, 256);
@@ -264,10 +264,11 @@ static prox_status pass_stage2(const prox_layer *L, const uint16_t *x, int nb, f
         u.tlist = reinterpret_cast<int32_t *>(w + W.tlist);
         u.status = reinterpret_cast<uint32_t *>(w + W.status);
         u.wait_us = g_spin_limit;
-        u.ks = pu.ks;
         u.span = pu.span;
         u.nstage = pu.nstage;
-        u.span_dn = pu.span_dn;
+        u.refill = pu.refill;
+        u.cw = pu.cw;
+        u.rows_dn = pu.rows_dn;
         u.nstage_dn = pu.nstage_dn;
         u.ug = reinterpret_cast<float *>(w + W.ug);
         u.tile_cnt = reinterpret_cast<int32_t *>(w + W.tile_cnt);

@@ -63,10 +63,11 @@ Stage2Plan stage2_plan(int d_model, int B, int C, int max_ch);
 
 // Launch plan of the tensor-core (union GEMM) Stage 2
 struct Stage2UPlan {
-    int ks;         // K slices of the up/gate GEMM
     int span;       // union tiles one up/gate CTA may touch
-    int span_dn;    // position ranges one down CTA may touch
     int nstage;     // up/gate ring stages
+    int refill;     // up/gate stages refilled together
+    int cw;         // output coordinates per down stage (512 or 256)
+    int rows_dn;    // union positions one down CTA may touch
     int nstage_dn;  // down ring stages
 };
 bool stage2u_plan(int d_model, int d_ff, int num_sms, Stage2UPlan *p);
@@ -142,10 +143,10 @@ struct Stage2UArgs {
     const int32_t *tlist;
     uint32_t *status;
     uint32_t wait_us;            // wall-clock bound of each wait, microseconds
-    int ks, span, nstage;        // up/gate plan
-    int span_dn, nstage_dn;      // down plan
+    int span, nstage, refill;    // up/gate plan
+    int cw, rows_dn, nstage_dn;  // down plan
     float *ug;                   // [f][2][B] partial u, g per union position (cleared)
-    int32_t *tile_cnt;           // [f / 128] slices summed per tile (cleared)
+    int32_t *tile_cnt;           // [f / 64] K blocks summed per tile (cleared)
     uint16_t *sb;                // [f / 64][2][8][64] s hi / lo tiles, 128-byte swizzled
     uint32_t *pos_ch;            // [f] union entry per position
 };
