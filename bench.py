@@ -76,14 +76,15 @@ def parse():
 def launches_per_call(args, d, batch):
     """Kernels one forward call of `batch` tokens launches: per pass, Stage 1
     and one Stage-2 kernel (CUDA cores) or two (tensor-core union engine:
-    passes of 8 tokens by default, of >= 4 when forced)."""
+    by default passes of 8 tokens, or of 4 when d_model >= 8192; of >= 4
+    when forced)."""
     from free_ffn_activation_b200 import prox as P
     per_pass = P.max_batch_per_pass(d)
     passes = -(-batch // per_pass)
     tb = 1
     while tb < min(batch, per_pass):
         tb *= 2
-    tc = tb >= 8 if args.engine == "auto" else (args.engine == "tc" and tb >= 4)
+    tc = (tb >= 8 or (tb >= 4 and d >= 8192)) if args.engine == "auto" else (args.engine == "tc" and tb >= 4)
     return passes * (3 if tc else 2)
 
 

@@ -185,7 +185,9 @@ static std::atomic<int> g_engine{PROX_ENGINE_AUTO};
 static bool use_tc(int d, int f, int B, int sms, Stage2UPlan *p) {
     const int e = g_engine.load();
     if (e == PROX_ENGINE_SIMT || B < 4) return false;
-    if (e == PROX_ENGINE_AUTO && B < kTcMinBatch) return false;
+    // automatic: passes of 8 tokens, or of 4 on layers of d_model >= 8192
+    // (whose passes hold at most 4 tokens); measured faster there
+    if (e == PROX_ENGINE_AUTO && B < kTcMinBatch && !(B >= 4 && d >= 8192)) return false;
     return stage2u_plan(d, f, sms, p);
 }
 

@@ -230,7 +230,8 @@ int prox_max_batch_per_pass(int d_model);
  * effect at the next forward call, returns the previous setting, or -1 for
  * an unknown value, which changes nothing).
  *   PROX_ENGINE_AUTO (default): the tensor-core union engine for passes of 8
- *     tokens, the CUDA-core engine below that;
+ *     tokens and, on layers of d_model >= 8192, of 4 tokens; the CUDA-core
+ *     engine otherwise;
  *   PROX_ENGINE_SIMT: the CUDA-core engine always: per channel of the union,
  *     dot products of the kept rows with x on the CUDA cores;
  *   PROX_ENGINE_TC: the tensor-core engine for every pass of 4 or more
