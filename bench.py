@@ -88,10 +88,10 @@ def launches_per_call(args, d, batch):
     return passes * (3 if tc else 2)
 
 
-def stage2_traffic(workload, batch):
+def stage2_traffic(workload, batch, mean_bytes=None):
     """DRAM bytes per launch of the Stage-2 kernel from the committed ncu summary,
     if it covers this workload and was captured from the current kernel source
-    (else None)."""
+    (else None), scaled from the captured token to `mean_bytes` algorithmic bytes."""
     if workload != "qwen3-8b-ffn" or batch != 1:
         return None
     import hashlib
@@ -108,9 +108,13 @@ def stage2_traffic(workload, batch):
     if fields.get("k_stage2.cu sha256") != digest:
         return None
     try:
-        return float(fields["dram bytes per launch (read + write)"])
-    except (KeyError, ValueError):
+        traffic = float(fields["dram bytes per launch (read + write)"])
+        captured = float(fields["algorithmic bytes of the captured launch"].split()[0])
+    except (KeyError, ValueError, IndexError):
         return None
+    # the captured launch is one token; scale to the mean token's algorithmic
+    # bytes (traffic grows with the kept channels) so it compares with `achieved`
+    return traffic * mean_bytes / captured if mean_bytes else traffic
 
 
 def max_over_ranks(x, world, dev):
@@ -463,7 +467,7 @@ def run_ours(args, w, rank, world, local_rank):
                        "parallelism": f"replicas x{world}"},
             "roofline": {"bound": "hbm", "kernel": "k_stage2 (exact up/gate/down)",
                          "achieved": s2_gbs, "peak": peak, "unit": "GB/s",
-                         "frac": s2_gbs / peak, "traffic": stage2_traffic(args.workload, Bt) if args.proxy == "int4" else None, "peak_source": peak_src,
+                         "frac": s2_gbs / peak, "traffic": stage2_traffic(args.workload, Bt, s2_bytes) if args.proxy == "int4" else None, "peak_source": peak_src,
                          "bytes_per_launch": s2_bytes, "us_per_launch": s2_us},
             "stage1": {"kernel": f"k_stage1 ({args.proxy} proxy + channel mask)", "us_per_launch": s1_us,
                        "bytes_per_launch": s1_bytes, "GBps": s1_gbs, "frac": s1_gbs / peak},

@@ -35,6 +35,7 @@
 #include <cooperative_groups.h>
 #include <cuda_runtime.h>
 #include <cstdint>
+#include <mutex>
 
 namespace cg = cooperative_groups;
 
@@ -609,11 +610,17 @@ cudaError_t launch1(Stage1Args a, const Stage1Plan &p0, cudaStream_t s) {
     // Cluster size (row groups per block): every cluster of the grid must be
     // resident at once, or the last clusters run as a second wave. Start from
     // the plan's choice and shrink until the occupancy calculator agrees.
+    // (per device: the shared-memory attribute and the occupancy are per device)
     struct Cache {
         int d = 0, C = 0, n_r = 0, cap = 0, sel = 0;
         size_t smem = 0;
     };
-    static Cache cache;
+    static Cache caches[64];
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::unique_lock<std::mutex> lk(mu);
+    Cache &cache = caches[dev];
     Stage1Plan p = p0;
     if (cache.d == a.d && cache.C == a.C) {
         p.n_r = cache.n_r;
@@ -660,6 +667,7 @@ cudaError_t launch1(Stage1Args a, const Stage1Plan &p0, cudaStream_t s) {
         cache.sel = p.depth_sel;
         cache.smem = p.smem;
     }
+    lk.unlock();
     a.n_r = p.n_r;
     a.unit_cap = p.unit_cap;
     a.depth_sel = p.depth_sel;

@@ -430,13 +430,8 @@ __global__ void __launch_bounds__(s2_threads(B), 1) k_stage2(const Stage2Args a)
 template <int B, int NCHD>
 cudaError_t launch2(const Stage2Args &a, int grid, size_t smem, cudaStream_t s) {
     auto k = k_stage2<B, NCHD>;
-    static size_t configured = 0;  // dynamic smem limit already set for this kernel
-    if (smem > configured) {
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
-        if (e != cudaSuccess) return e;
-        configured = smem;
-    }
+    cudaError_t e = set_max_dynamic_smem((const void *)k, smem);
+    if (e != cudaSuccess) return e;
     return launch_pdl(k, dim3(grid), dim3(s2_threads(B)), smem, s, a);
 }
 

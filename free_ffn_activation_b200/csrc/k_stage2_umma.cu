@@ -697,23 +697,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_s2u_down(const Stage2UArgs a) {
     }
 }
 
-template <typename K>
-cudaError_t set_smem(K k, size_t smem, size_t &configured) {
-    if (smem > configured) {
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        configured = smem;
-    }
-    return cudaSuccess;
-}
-
 template <int B, int NM>
 cudaError_t launch_u(const Stage2UArgs &a, int grid, cudaStream_t s) {
-    static size_t cfg_ug = 0, cfg_dn = 0;
     const size_t sm_ug = ug_smem(a.nstage, a.C, a.span).total;
     const size_t sm_dn = dn_smem(a.nstage_dn, NM * kUM, a.rows_dn).total;
-    cudaError_t e = set_smem(k_s2u_updown<B>, sm_ug, cfg_ug);
-    if (e == cudaSuccess) e = set_smem(k_s2u_down<B, NM>, sm_dn, cfg_dn);
+    cudaError_t e = set_max_dynamic_smem((const void *)k_s2u_updown<B>, sm_ug);
+    if (e == cudaSuccess) e = set_max_dynamic_smem((const void *)k_s2u_down<B, NM>, sm_dn);
     if (e == cudaSuccess) e = launch_pdl(k_s2u_updown<B>, dim3(grid), dim3(kThreads), sm_ug, s, a);
     if (e == cudaSuccess) e = launch_pdl(k_s2u_down<B, NM>, dim3(grid), dim3(kThreads), sm_dn, s, a);
     return e;

@@ -10,7 +10,9 @@
 #include <cstdint>
 #include <cstring>
 #include <atomic>
+#include <map>
 #include <mutex>
+#include <utility>
 
 #define PROX_API extern "C" __attribute__((visibility("default")))
 
@@ -146,6 +148,20 @@ static prox_status current_device(int *sms) {
     if (!di.ok) return PROX_EDEVICE;
     *sms = di.sms;
     return PROX_OK;
+}
+
+cudaError_t set_max_dynamic_smem(const void *kern, size_t smem) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    static std::mutex mu;
+    static std::map<std::pair<int, const void *>, size_t> done;
+    std::lock_guard<std::mutex> lk(mu);
+    size_t &cur = done[{dev, kern}];
+    if (smem <= cur) return cudaSuccess;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess) cur = smem;
+    return e;
 }
 
 // NULL counts as aligned: optional outputs are checked only when given

@@ -179,6 +179,11 @@ cudaError_t launch_select_f32_abs(const float *v, long n, long rank,
                                   uint32_t *hist, uint32_t *scratch,
                                   float *tau_dev, cudaStream_t s);
 
+// Raise a kernel's dynamic shared-memory limit to at least `smem` bytes on the
+// current device (the attribute is per device; set once per device and kernel,
+// thread-safe)
+cudaError_t set_max_dynamic_smem(const void *kern, size_t smem);
+
 // Launch with programmatic stream serialization (PDL): the kernel may start
 // while the previous kernel in the stream finishes; it must execute
 // griddepcontrol.wait before touching anything that kernel writes.

@@ -524,3 +524,15 @@ def test_tc_split_stages_equal_forward(c2):
     rel = (torch.linalg.norm(y - ref.y, dim=1) / torch.linalg.norm(ref.y, dim=1)).max().item()
     assert rel < 1e-5
     assert P.last_device_status(ws)[0] == P.PROX_OK
+
+
+def test_tc_shapes_interleaved(c1, c2, c4):
+    # the up/gate kernel is shared by the 256- and 512-coordinate down variants
+    # and its shared-memory size depends on the shape: calls that alternate
+    # shapes must each raise the kernel's limit as far as they need it
+    with P.stage2_engine(P.ENGINE_TC):
+        for case, b in ((c4, 4), (c1, 4), (c2, 4), (c1, 8), (c4, 4), (c2, 4)):
+            rows = list(range(b))
+            out = P.ffn_forward(case.layer, case.xdev(rows), case.tau_x, case.tau_s)
+            torch.cuda.synchronize()
+            assert out.count_s.shape[0] == b
