@@ -27,14 +27,11 @@
 //     one accumulator each. Steps (coordinate tile, 32 positions) are split
 //     evenly among CTAs; each CTA adds its accumulated block to y with fp32
 //     atomics whenever its range leaves a coordinate tile.
-// Both kernels: 256 threads, one CTA per SM; every thread moves 16-byte
-// pieces of the gathered rows with cp.async (L2 evict-first) straight into
-// the swizzled layout the MMA reads, one thread issues the MMAs, and
-// tcgen05.commit on a per-stage mbarrier frees a stage for reuse. The up/gate
-// ring is refilled in batches of half its depth, so each gathered row is
-// requested in runs of several consecutive 128-byte pieces (a run per stage
-// would scatter single 128-byte requests over the rows and leave DRAM far
-// from its streaming rate). All waits are bounded; TMEM is freed before exit.
+// Both kernels: one CTA per SM, warp-specialised (roles below); the loader
+// threads move 16-byte pieces of the gathered rows with cp.async (L2
+// evict-first) straight into the swizzled layout the MMA reads, one thread
+// issues the MMAs, and tcgen05.commit on a per-stage mbarrier frees a stage
+// for reuse. All waits are bounded; TMEM is freed before exit.
 #include "prox_internal.cuh"
 
 #include <cuda_bf16.h>
@@ -725,7 +722,6 @@ bool stage2u_plan(int d, int f, int num_sms, Stage2UPlan *p) {
     while (na > 0 && ug_smem(na, C, p->span).total > budget) --na;
     while (nb > 0 && dn_smem(nb, p->cw, p->rows_dn).total > budget) --nb;
     p->nstage = na;
-    p->refill = 0;
     p->nstage_dn = nb;
     return na >= 4 && nb >= 3;
 }

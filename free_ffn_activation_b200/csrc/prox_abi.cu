@@ -284,7 +284,6 @@ static prox_status pass_stage2(const prox_layer *L, const uint16_t *x, int nb, f
         u.wait_us = g_spin_limit;
         u.span = pu.span;
         u.nstage = pu.nstage;
-        u.refill = pu.refill;
         u.cw = pu.cw;
         u.rows_dn = pu.rows_dn;
         u.nstage_dn = pu.nstage_dn;

@@ -28,9 +28,8 @@ constexpr uint32_t kStTimeoutDrain = 1u << 3;  // producer waited for its copies
 constexpr uint32_t kStTimeoutRing = 1u << 4;   // Stage 1 waited for a ring slot
 constexpr uint32_t kStTimeoutMma = 1u << 5;    // tensor-core Stage 2 waited for its MMAs
 
-// tensor-core Stage 2: union positions per down-projection unit, and the
-// smallest pass (tokens) the automatic engine choice sends to it
-constexpr int kUnitPos = 512;
+// smallest pass (tokens) the automatic engine choice sends to the
+// tensor-core Stage 2 (4 on layers of d_model >= 8192)
 constexpr int kTcMinBatch = 8;
 
 // default wall-clock bound of a device-side wait, in microseconds
@@ -65,7 +64,6 @@ Stage2Plan stage2_plan(int d_model, int B, int C, int max_ch);
 struct Stage2UPlan {
     int span;       // union tiles one up/gate CTA may touch
     int nstage;     // up/gate ring stages
-    int refill;     // up/gate stages refilled together
     int cw;         // output coordinates per down stage (512 or 256)
     int rows_dn;    // union positions one down CTA may touch
     int nstage_dn;  // down ring stages
@@ -143,7 +141,7 @@ struct Stage2UArgs {
     const int32_t *tlist;
     uint32_t *status;
     uint32_t wait_us;            // wall-clock bound of each wait, microseconds
-    int span, nstage, refill;    // up/gate plan
+    int span, nstage;            // up/gate plan
     int cw, rows_dn, nstage_dn;  // down plan
     float *ug;                   // [f][2][B] partial u, g per union position (cleared)
     int32_t *tile_cnt;           // [f / 64] K blocks summed per tile (cleared)
