@@ -31,6 +31,7 @@
 // down by 12 bits (to positions 2..4). Subnormal operands need FMA without
 // flush-to-zero, which is the default without fast-math.
 #include "prox_internal.cuh"
+#include "umma.cuh"
 
 #include <cooperative_groups.h>
 #include <cuda_runtime.h>
@@ -165,6 +166,17 @@ __device__ __forceinline__ int block_excl_scan(int v, int *warp_tot, int &total)
 
 }  // namespace
 
+// Tensor-core proxy products (passes of 4 or 8 tokens, INT4 proxy): shared
+// memory of the stream, which replaces the copy ring and row-lane reduction
+// area: two K steps of decoded codes for both matrices and the digits of x.
+constexpr int kTcKStep = 32;   // proxy rows per K step (the K of one kind::i8 MMA)
+constexpr int kTcPre = 6;      // K steps of codes each thread keeps in flight (registers)
+__host__ __device__ inline size_t s1tc_bytes(int B, int NB, int unit_cap) {
+    const size_t a = (size_t)2 * 2 * kTcKStep * NB * kCB;                  // 2 buffers x 2 matrices
+    const size_t b = (size_t)2 * ((unit_cap + 127) / 128) * (4 * B / 8) * 1024;  // digits
+    return 1024 + a + b;                                                   // + alignment slack
+}
+
 // shared-memory carve-up of one Stage-1 CTA (kept next to the kernel). The
 // copy ring (depth DMAX >> depth_sel rows per thread) and the row-lane
 // reduction area are used one after the other and share one region.
@@ -173,7 +185,7 @@ struct S1Smem {
 };
 
 __host__ __device__ inline S1Smem s1_smem(int d, int B, int NB, int unit_cap, int depth_sel,
-                                         int n_r = kS1MaxRowGroups, int PK = 0) {
+                                         int n_r = kS1MaxRowGroups, int PK = 0, int TC = 0) {
     const int cw = NB * kCB;
     const int cpt = s1_cpt(B, NB, PK);
     const int rl = kS1Threads / (2 * (cw / cpt));
@@ -183,7 +195,9 @@ __host__ __device__ inline S1Smem s1_smem(int d, int B, int NB, int unit_cap, in
     S1Smem s;
     size_t o = 0;
     s.ring = s.red = o;
-    o += ring > red ? ring : red;
+    size_t region = ring > red ? ring : red;
+    if (TC && s1tc_bytes(B, NB, unit_cap) > region) region = s1tc_bytes(B, NB, unit_cap);
+    o += region;
     s.rowidx = o;
     o += ((size_t)unit_cap * 4 + 15) / 16 * 16;
     s.xs = o;
@@ -255,7 +269,225 @@ __device__ __forceinline__ void s1_stream(const uint8_t *qbase, unsigned char *r
     cp_wait<0>();
 }
 
-template <int B, int NB, int PK>
+// global -> registers, 16 bytes, read-only path, under L2 policy pol
+__device__ __forceinline__ uint4 ldg16_pol(const void *src, uint64_t pol) {
+    uint4 v;
+    asm volatile("ld.global.nc.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(src), "l"(pol));
+    return v;
+}
+
+// (5'), passes of 4 or 8 tokens with the INT4 proxy: the CTA's proxy rows are
+// the K dimension of kind::i8 UMMAs. A = the offset-binary codes q + 8 of one
+// matrix as unsigned bytes (MN-major, 128 channels per 128-byte row, 32 rows
+// per K step; decoded in registers with two ANDs, a shift and two byte
+// permutes per 8 codes). B = x_i * scale_i * 2^E per (matrix, token) as a
+// 27-bit fixed-point value v = round(xs * 2^F) split into four signed 8-bit
+// digits (v = d0 + 2^7 d1 + 2^14 d2 + 2^21 d3); the digits are the N rows, so
+// each code tile is read once for all tokens. D is int32 in TMEM and exact;
+// the epilogue removes the +8 offset (8 * the digit sums, exact in int64) and
+// undoes 2^F and 2^E: this CTA's partial sums sum_i q_ij x_i scale_i, in the
+// same place the CUDA-core stream leaves them. One thread issues the MMAs; the
+// decoded tiles are double-buffered and each thread keeps kTcPre K steps of
+// codes in flight in registers. Waits are bounded.
+template <int B, int NB>
+__device__ void s1_tc_stream(const Stage1Args &a, unsigned char *region, const int *rowidx,
+                             const float *xs, int n_units, const int (&E)[B], int c0,
+                             float *part) {
+    constexpr int CW = NB * kCB;
+    constexpr int N = 4 * B;                          // digit rows
+    constexpr int MT = CW / 128;                      // 128-channel M tiles per matrix
+    constexpr uint32_t ABUF = 2u * CW * kTcKStep;     // one K step of both matrices
+    constexpr uint32_t LBO = (kTcKStep / 8) * 1024u;  // stride of 128-channel atoms
+    constexpr uint32_t TCOLS = 2 * MT * N;            // a power of two >= 32
+    constexpr uint32_t IDESC = (2u << 4) | (0u << 7) | (1u << 10) | (1u << 15) |
+                               ((uint32_t)(N >> 3) << 17) | (8u << 24);  // u8 x s8 -> s32, M 128
+    __shared__ float s_mx[2][kMaxB];
+    __shared__ int s_F[2][kMaxB];
+    __shared__ int s_S[2][kMaxB][4];
+    __shared__ uint32_t s_tmem;
+    __shared__ __align__(8) uint64_t s_done[2];
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const uint32_t rb = (smem_addr(region) + 1023u) & ~1023u;
+    unsigned char *abuf = region + (rb - smem_addr(region));
+    unsigned char *bdig = abuf + 2 * ABUF;
+    const uint32_t aaddr = rb, baddr = rb + 2 * ABUF;
+    const uint32_t BM = (uint32_t)((a.unit_cap + 127) / 128) * (N / 8) * 1024u;  // one matrix
+    const int nks = (n_units + kTcKStep - 1) / kTcKStep;
+
+    if (tid < 2 * kMaxB) (&s_mx[0][0])[tid] = 0.f;
+    if (tid < 2 * kMaxB * 4) (&s_S[0][0][0])[tid] = 0;
+    if (tid == 0) {
+        mbar_init(&s_done[0], 1);
+        mbar_init(&s_done[1], 1);
+        mbar_fence_init();
+    }
+    if (wid == 0) tmem_alloc(&s_tmem, TCOLS);
+    __syncthreads();
+    // fixed-point exponent per (matrix, token): max |xs| * 2^F < 2^27
+    {
+        float mx[2][B];
+#pragma unroll
+        for (int mm = 0; mm < 2; ++mm)
+#pragma unroll
+            for (int t = 0; t < B; ++t) mx[mm][t] = 0.f;
+        for (int u = tid; u < n_units; u += kS1Threads)
+#pragma unroll
+            for (int mm = 0; mm < 2; ++mm)
+#pragma unroll
+                for (int t = 0; t < B; ++t) mx[mm][t] = fmaxf(mx[mm][t], fabsf(xs[(u * 2 + mm) * B + t]));
+#pragma unroll
+        for (int mm = 0; mm < 2; ++mm)
+#pragma unroll
+            for (int t = 0; t < B; ++t) {
+                float v = mx[mm][t];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+                // non-negative floats order like their bit patterns
+                if (lane == 0) atomicMax(reinterpret_cast<int *>(&s_mx[mm][t]), __float_as_int(v));
+            }
+    }
+    __syncthreads();
+    if (tid < 2 * B) {
+        const float v = s_mx[tid / B][tid % B];
+        s_F[tid / B][tid % B] = v > 0.f ? 26 - ilogbf(v) : 0;
+    }
+    __syncthreads();
+    // the digits (B operand, K-major, 128-byte swizzle: 8 digit rows x 128
+    // proxy rows per atom); rows past the CTA's units up to the last K step are 0
+    for (int u = tid; u < nks * kTcKStep; u += kS1Threads) {
+        const int kblk = u >> 7, kin = u & 127;
+#pragma unroll
+        for (int mm = 0; mm < 2; ++mm)
+#pragma unroll
+            for (int t = 0; t < B; ++t) {
+                int v = 0;
+                if (u < n_units) {
+                    const int F = s_F[mm][t], f1 = F / 2, f2 = F - f1;
+                    v = __float2int_rn(xs[(u * 2 + mm) * B + t] * __int_as_float((127 + f1) << 23) *
+                                       __int_as_float((127 + f2) << 23));
+                }
+                const int d3 = v >> 21;
+                const int r = v - d3 * (1 << 21);
+                const int dg[4] = {r & 127, (r >> 7) & 127, r >> 14, d3};
+#pragma unroll
+                for (int l = 0; l < 4; ++l) {
+                    const int n = t * 4 + l;
+                    bdig[mm * BM + (uint32_t)kblk * (N / 8) * 1024u + (n >> 3) * 1024u + (n & 7) * 128u +
+                         ((uint32_t)((kin >> 4) ^ (n & 7)) << 4) + (kin & 15)] = (unsigned char)dg[l];
+                    if (dg[l]) atomicAdd(&s_S[mm][t][l], dg[l]);
+                }
+            }
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_tmem;
+
+    // stream: thread tid owns pieces q = tid + 512 j (j < NB) of each K step:
+    // 16 bytes (32 channels) of proxy row k of block b of matrix m
+    const uint64_t pol = l2_evict_first();
+    auto fetch = [&](int ks, uint4 (&dst)[NB]) {
+#pragma unroll
+        for (int j = 0; j < NB; ++j) {
+            const int qq = tid + kS1Threads * j;
+            const int piece = qq & 7, k = (qq >> 3) & 31, bm = qq >> 8;
+            const int mm = bm & 1, b = bm >> 1;
+            const int u = ks * kTcKStep + k;
+            dst[j] = make_uint4(0u, 0u, 0u, 0u);
+            if (ks < nks && u < n_units)
+                dst[j] = ldg16_pol((mm ? a.q_gate : a.q_up) +
+                                       ((size_t)(c0 + b) * a.d + rowidx[u]) * (kCB / 2) + piece * 16,
+                                   pol);
+        }
+    };
+    uint4 pre[kTcPre][NB];
+#pragma unroll
+    for (int p = 0; p < kTcPre; ++p) fetch(p, pre[p]);
+    bool ok = true;
+    for (int ks0 = 0; ks0 < nks; ks0 += kTcPre) {
+#pragma unroll
+        for (int p = 0; p < kTcPre; ++p) {
+            const int ks = ks0 + p;
+            if (ks >= nks) break;  // uniform across the CTA
+            const int bb = ks & 1;
+            // the buffer's previous MMAs (K step ks - 2) are done
+            if (ks >= 2 && ok) ok = mbar_wait(&s_done[bb], ((ks - 2) >> 1) & 1, a.wait_us);
+#pragma unroll
+            for (int j = 0; j < NB; ++j) {
+                const int qq = tid + kS1Threads * j;
+                const int piece = qq & 7, k = (qq >> 3) & 31, bm = qq >> 8;
+                const int mm = bm & 1, b = bm >> 1;
+                if (ks * kTcKStep + k >= n_units) continue;  // its digits are 0
+                const uint32_t w[4] = {pre[p][j].x, pre[p][j].y, pre[p][j].z, pre[p][j].w};
+                uint32_t o[8];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint32_t lo = w[i] & 0x0F0F0F0Fu, hi = (w[i] >> 4) & 0x0F0F0F0Fu;
+                    o[2 * i] = __byte_perm(lo, hi, 0x5140);      // codes of channels 8i .. 8i+3
+                    o[2 * i + 1] = __byte_perm(lo, hi, 0x7362);  // channels 8i+4 .. 8i+7
+                }
+                const int ma = b * 2 + (piece >> 2), cc = (piece & 3) * 2;
+                unsigned char *row = abuf + bb * ABUF + mm * (CW * kTcKStep) + ma * LBO +
+                                     (k >> 3) * 1024 + (k & 7) * 128;
+                *reinterpret_cast<uint4 *>(row + (((cc) ^ (k & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+                *reinterpret_cast<uint4 *>(row + (((cc + 1) ^ (k & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+            }
+            fetch(ks + kTcPre, pre[p]);
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncthreads();
+            if (tid == 0) {
+                tc_fence_after();
+                const uint32_t kb_off = (uint32_t)(ks >> 2) * (N / 8) * 1024u + (uint32_t)(ks & 3) * 32u;
+#pragma unroll
+                for (int mm = 0; mm < 2; ++mm) {
+                    const uint64_t db = sw128_desc(baddr + mm * BM + kb_off, 16, 1024);
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt)
+                        umma_i8(tmem + (mm * MT + mt) * N,
+                                sw128_desc(aaddr + bb * ABUF + mm * (CW * kTcKStep) + mt * LBO, LBO, 1024),
+                                db, IDESC, ks > 0 ? 1u : 0u);
+                }
+                umma_commit(&s_done[bb]);
+            }
+        }
+    }
+    if (nks > 0 && ok) ok = mbar_wait(&s_done[(nks - 1) & 1], ((nks - 1) >> 1) & 1, a.wait_us);
+    if (!ok) atomicOr(a.status, kStTimeoutMma);
+    tc_fence_after();
+    // epilogue: warp quadrant q reads TMEM lanes 32q..32q+31 (channels of an M
+    // tile); the four groups of four warps take the (matrix, M tile) pairs
+    const int q = wid & 3;
+    for (int pi = wid >> 2; pi < 2 * MT; pi += kS1Threads / 128) {
+        const int mm = pi / MT, mt = pi % MT;
+        uint32_t D[N];
+        if (nks > 0) {
+            if constexpr (N == 32) tmem_ld32(tmem + pi * N + ((uint32_t)(q * 32) << 16), D);
+            else tmem_ld16(tmem + pi * N + ((uint32_t)(q * 32) << 16), D);
+        }
+        const int ch = mt * 128 + q * 32 + lane;
+#pragma unroll
+        for (int t = 0; t < B; ++t) {
+            long long V = 0;
+            if (nks > 0) {
+#pragma unroll
+                for (int l = 0; l < 4; ++l)
+                    V += ((long long)(int)D[t * 4 + l] - 8ll * s_S[mm][t][l]) * (1ll << (7 * l));
+            }
+            part[(mm * B + t) * CW + ch] = (float)ldexp((double)V, -(s_F[mm][t] + E[t]));
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (wid == 0) {
+        tc_fence_after();
+        tmem_free(tmem, TCOLS);
+    }
+}
+
+template <int B, int NB, int PK, int TC = 0>
 __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
     using T = S1<B, NB, PK>;
     extern __shared__ __align__(16) unsigned char smem[];
@@ -263,7 +495,7 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
     cg::cluster_group cluster = cg::this_cluster();
     const int r = (int)cluster.block_rank();  // row group
     const int c0 = (blockIdx.x / a.n_r) * NB;  // first column block of the group
-    const S1Smem L = s1_smem(a.d, B, NB, a.unit_cap, a.depth_sel, kS1MaxRowGroups, PK);
+    const S1Smem L = s1_smem(a.d, B, NB, a.unit_cap, a.depth_sel, kS1MaxRowGroups, PK, TC);
     unsigned char *ring = smem + L.ring;
     float *red = reinterpret_cast<float *>(smem + L.red);
     int *rowidx = reinterpret_cast<int *>(smem + L.rowidx);          // [unit_cap]
@@ -445,67 +677,71 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
     }
     __syncthreads();
 
-    const int rl = tid / T::TPR;
-    const int m = (tid / T::TPRM) & 1;
-    const int chunk = tid % T::TPRM;
-    const uint8_t *qbase = (m ? a.q_gate : a.q_up) +
-                           (size_t)(c0 + chunk / T::TPRB) * a.d * T::GRAN +
-                           (chunk % T::TPRB) * T::BYTES;
-    const int n_rows = n_units > rl ? (n_units - rl + T::RL - 1) / T::RL : 0;
-    float2 acc2[T::ACC / 2];
-#pragma unroll
-    for (int k = 0; k < T::ACC / 2; ++k) acc2[k] = make_float2(0.f, 0.f);
-    float ssum[B];
-#pragma unroll
-    for (int t = 0; t < B; ++t) ssum[t] = 0.f;
-    if (a.depth_sel == 0)
-        s1_stream<B, NB, PK, T::DMAX>(qbase, ring, rowidx, xs, rl, m, n_rows, acc2, ssum);
-    else if (a.depth_sel == 1)
-        s1_stream<B, NB, PK, T::DMAX / 2>(qbase, ring, rowidx, xs, rl, m, n_rows, acc2, ssum);
-    else
-        s1_stream<B, NB, PK, T::DMAX / 4>(qbase, ring, rowidx, xs, rl, m, n_rows, acc2, ssum);
-    __syncthreads();  // every thread is done with the ring before it becomes `red`
-    if (kPush) asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+    if constexpr (TC) {
+        s1_tc_stream<B, NB>(a, ring, rowidx, xs, n_units, E, c0, dst_part);
+    } else {
+        const int rl = tid / T::TPR;
+        const int m = (tid / T::TPRM) & 1;
+        const int chunk = tid % T::TPRM;
+        const uint8_t *qbase = (m ? a.q_gate : a.q_up) +
+                               (size_t)(c0 + chunk / T::TPRB) * a.d * T::GRAN +
+                               (chunk % T::TPRB) * T::BYTES;
+        const int n_rows = n_units > rl ? (n_units - rl + T::RL - 1) / T::RL : 0;
+        float2 acc2[T::ACC / 2];
+    #pragma unroll
+        for (int k = 0; k < T::ACC / 2; ++k) acc2[k] = make_float2(0.f, 0.f);
+        float ssum[B];
+    #pragma unroll
+        for (int t = 0; t < B; ++t) ssum[t] = 0.f;
+        if (a.depth_sel == 0)
+            s1_stream<B, NB, PK, T::DMAX>(qbase, ring, rowidx, xs, rl, m, n_rows, acc2, ssum);
+        else if (a.depth_sel == 1)
+            s1_stream<B, NB, PK, T::DMAX / 2>(qbase, ring, rowidx, xs, rl, m, n_rows, acc2, ssum);
+        else
+            s1_stream<B, NB, PK, T::DMAX / 4>(qbase, ring, rowidx, xs, rl, m, n_rows, acc2, ssum);
+        __syncthreads();  // every thread is done with the ring before it becomes `red`
+        if (kPush) asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
 
-    // (6) reduce row lanes (padded rows: conflict-free both ways), undo the
-    // pre-scale and the +8 code offset: this CTA's partial sums in `part`.
-    // The pad word after chunk 0's channels carries the row lane's offset sum.
-    constexpr int PAD = T::CW + T::TPRM;  // one extra word per chunk row
-#pragma unroll
-    for (int t = 0; t < B; ++t) {
-        float *row = red + ((rl * 2 + m) * B + t) * PAD;
-#pragma unroll
-        for (int k = 0; k < T::CPT; k += 2) {
-            row[chunk * (T::CPT + 1) + k] = acc2[(t * T::CPT + k) / 2].x;
-            row[chunk * (T::CPT + 1) + k + 1] = acc2[(t * T::CPT + k) / 2].y;
-        }
-        if (chunk == 0) row[T::CPT] = ssum[t];
-    }
-    __syncthreads();
-    for (int o = tid; o < 2 * T::CW; o += kS1Threads) {
-        // (matrix, channel within the CTA's columns)
-        const int mm = o / T::CW, ch = o % T::CW;
-        const int p = nib_pos(ch % 8);
-        const int pos = (ch / T::CPT) * (T::CPT + 1) + ch % T::CPT;
-        // 2^(149 - 4p) and 2^-E as products of normal floats
-        const float up1 = __int_as_float((127 + 75) << 23);
-        const float up2 = __int_as_float((127 + 74 - 4 * p) << 23);
-#pragma unroll
+        // (6) reduce row lanes (padded rows: conflict-free both ways), undo the
+        // pre-scale and the +8 code offset: this CTA's partial sums in `part`.
+        // The pad word after chunk 0's channels carries the row lane's offset sum.
+        constexpr int PAD = T::CW + T::TPRM;  // one extra word per chunk row
+    #pragma unroll
         for (int t = 0; t < B; ++t) {
-            float sacc = 0.f, soff = 0.f;
-            for (int q = 0; q < T::RL; ++q) {
-                const float *row = red + ((q * 2 + mm) * B + t) * PAD;
-                sacc += row[pos];
-                soff += row[T::CPT];
+            float *row = red + ((rl * 2 + m) * B + t) * PAD;
+    #pragma unroll
+            for (int k = 0; k < T::CPT; k += 2) {
+                row[chunk * (T::CPT + 1) + k] = acc2[(t * T::CPT + k) / 2].x;
+                row[chunk * (T::CPT + 1) + k + 1] = acc2[(t * T::CPT + k) / 2].y;
             }
-            if constexpr (PK == 0) {
-                const int e1 = E[t] / 2, e2 = E[t] - e1;
-                const float v = (sacc * up1) * up2 - 8.f * soff;  // sum (q + 8 - 8) x s 2^E
-                dst_part[(mm * B + t) * T::CW + ch] =
-                    v * __int_as_float((127 - e1) << 23) * __int_as_float((127 - e2) << 23);
-            } else {
-                (void)up1, (void)up2, (void)soff;
-                dst_part[(mm * B + t) * T::CW + ch] = sacc;  // plain x_i * w_ij sums
+            if (chunk == 0) row[T::CPT] = ssum[t];
+        }
+        __syncthreads();
+        for (int o = tid; o < 2 * T::CW; o += kS1Threads) {
+            // (matrix, channel within the CTA's columns)
+            const int mm = o / T::CW, ch = o % T::CW;
+            const int p = nib_pos(ch % 8);
+            const int pos = (ch / T::CPT) * (T::CPT + 1) + ch % T::CPT;
+            // 2^(149 - 4p) and 2^-E as products of normal floats
+            const float up1 = __int_as_float((127 + 75) << 23);
+            const float up2 = __int_as_float((127 + 74 - 4 * p) << 23);
+    #pragma unroll
+            for (int t = 0; t < B; ++t) {
+                float sacc = 0.f, soff = 0.f;
+                for (int q = 0; q < T::RL; ++q) {
+                    const float *row = red + ((q * 2 + mm) * B + t) * PAD;
+                    sacc += row[pos];
+                    soff += row[T::CPT];
+                }
+                if constexpr (PK == 0) {
+                    const int e1 = E[t] / 2, e2 = E[t] - e1;
+                    const float v = (sacc * up1) * up2 - 8.f * soff;  // sum (q + 8 - 8) x s 2^E
+                    dst_part[(mm * B + t) * T::CW + ch] =
+                        v * __int_as_float((127 - e1) << 23) * __int_as_float((127 - e2) << 23);
+                } else {
+                    (void)up1, (void)up2, (void)soff;
+                    dst_part[(mm * B + t) * T::CW + ch] = sacc;  // plain x_i * w_ij sums
+                }
             }
         }
     }
@@ -596,16 +832,16 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
 }
 
 // deepest ring that fits next to `unit_cap` rows (2 = the shallowest), or -1
-int s1_depth_sel(int d, int B, int NB, int unit_cap, int PK = 0) {
+int s1_depth_sel(int d, int B, int NB, int unit_cap, int PK = 0, int TC = 0) {
     for (int sel = 0; sel <= 2; ++sel)
-        if (s1_smem(d, B, NB, unit_cap, sel, kS1MaxRowGroups, PK).total <= (size_t)kS2SmemBudget)
+        if (s1_smem(d, B, NB, unit_cap, sel, kS1MaxRowGroups, PK, TC).total <= (size_t)kS2SmemBudget)
             return sel;
     return -1;
 }
 
-template <int B, int NB, int PK>
+template <int B, int NB, int PK, int TC = 0>
 cudaError_t launch1(Stage1Args a, const Stage1Plan &p0, cudaStream_t s) {
-    auto k = k_stage1<B, NB, PK>;
+    auto k = k_stage1<B, NB, PK, TC>;
     const int groups = a.C / NB;  // clusters
     // Cluster size (row groups per block): every cluster of the grid must be
     // resident at once, or the last clusters run as a second wave. Start from
@@ -631,14 +867,14 @@ cudaError_t launch1(Stage1Args a, const Stage1Plan &p0, cudaStream_t s) {
         // fewest row groups whose rows fit in one CTA's shared memory
         int n_min = 1;
         while (n_min < kS1MaxRowGroups &&
-               s1_depth_sel(a.d, B, NB, (a.d + n_min - 1) / n_min, PK) < 0)
+               s1_depth_sel(a.d, B, NB, (a.d + n_min - 1) / n_min, PK, TC) < 0)
             ++n_min;
         if (p.n_r < n_min) p.n_r = n_min;
         for (;;) {
             p.unit_cap = (a.d + p.n_r - 1) / p.n_r;
-            p.depth_sel = s1_depth_sel(a.d, B, NB, p.unit_cap, PK);
+            p.depth_sel = s1_depth_sel(a.d, B, NB, p.unit_cap, PK, TC);
             if (p.depth_sel < 0) return cudaErrorInvalidConfiguration;
-            p.smem = s1_smem(a.d, B, NB, p.unit_cap, p.depth_sel, kS1MaxRowGroups, PK).total;
+            p.smem = s1_smem(a.d, B, NB, p.unit_cap, p.depth_sel, kS1MaxRowGroups, PK, TC).total;
             cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  (int)p.smem);
             if (e != cudaSuccess) return e;
@@ -694,6 +930,11 @@ cudaError_t launch_stage1(int B, const Stage1Args &a, const Stage1Plan &p, cudaS
 #define PROX_S1(BB, NN)                                                          \
     if (B == BB && p.nb_blocks == NN)                                            \
         return a.pk ? launch1<BB, NN, 1>(a, p, s) : launch1<BB, NN, 0>(a, p, s);
+    // the tensor-core stream: passes of 4 or 8 tokens, INT4 proxy
+    if (a.tc && a.pk == 0 && (B == 4 || B == 8)) {
+        if (B == 4) return p.nb_blocks == 2 ? launch1<4, 2, 0, 1>(a, p, s) : launch1<4, 1, 0, 1>(a, p, s);
+        return p.nb_blocks == 2 ? launch1<8, 2, 0, 1>(a, p, s) : launch1<8, 1, 0, 1>(a, p, s);
+    }
     PROX_S1(1, 1) PROX_S1(1, 2) PROX_S1(2, 1) PROX_S1(2, 2)
     PROX_S1(4, 1) PROX_S1(4, 2) PROX_S1(8, 1) PROX_S1(8, 2)
 #undef PROX_S1

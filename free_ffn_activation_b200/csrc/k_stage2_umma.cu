@@ -33,6 +33,7 @@
 // issues the MMAs, and tcgen05.commit on a per-stage mbarrier frees a stage
 // for reuse. All waits are bounded; TMEM is freed before exit.
 #include "prox_internal.cuh"
+#include "umma.cuh"
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -55,89 +56,11 @@ constexpr uint32_t kUgStage = 16384 + 2 * kAtom;   // A (64 up + 64 gate rows) |
 __host__ __device__ constexpr uint32_t dn_a_bytes(int cw) { return (uint32_t)kDnPos * cw * 2; }
 __host__ __device__ constexpr uint32_t dn_stage(int cw) { return dn_a_bytes(cw) + 4 * kAtom; }
 
-// ---------------------------------------------------------------------------
-// tcgen05 / UMMA helpers
-// ---------------------------------------------------------------------------
-// shared-memory matrix descriptor of a 128-byte-swizzled tile: start address,
-// leading and stride byte offsets in 16-byte units, descriptor version 1,
-// layout type 2 (128-byte swizzle)
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
-}
-
 // instruction descriptor of kind::f16: bf16 A and B, fp32 D, M = 128,
 // N = 16, B K-major, A K-major or MN-major
 __host__ __device__ constexpr uint32_t bf16_idesc(bool a_mn) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) |
            ((uint32_t)(kUN >> 3) << 17) | ((uint32_t)(kUM >> 4) << 24);
-}
-
-__device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t da, uint64_t db, uint32_t idesc,
-                                     uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(da), "l"(db), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// arrive on `bar` once every MMA this thread issued so far has completed
-__device__ __forceinline__ void umma_commit(uint64_t *bar) {
-    asm volatile(
-        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-            smem_addr(bar))
-        : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() {
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-
-// generic-proxy writes to shared memory (st.shared) made visible to the
-// tensor core's async-proxy reads
-__device__ __forceinline__ void fence_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-// 8 consecutive fp32 columns of this thread's TMEM lane (warp w reads lanes
-// 32 (w % 4) .. + 31); load and wait in one statement so no use of the
-// registers can be scheduled before the wait
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
-    uint32_t r0, r1, r2, r3, r4, r5, r6, r7;
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
-        : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3), "=r"(r4), "=r"(r5), "=r"(r6), "=r"(r7)
-        : "r"(taddr)
-        : "memory");
-    v[0] = __uint_as_float(r0);
-    v[1] = __uint_as_float(r1);
-    v[2] = __uint_as_float(r2);
-    v[3] = __uint_as_float(r3);
-    v[4] = __uint_as_float(r4);
-    v[5] = __uint_as_float(r5);
-    v[6] = __uint_as_float(r6);
-    v[7] = __uint_as_float(r7);
-}
-
-// TMEM allocation (a power of two >= 32 columns) by one whole warp; the
-// address lands in *slot
-__device__ __forceinline__ void tmem_alloc(uint32_t *slot, uint32_t ncols) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_addr(slot)),
-                 "r"(ncols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_free(uint32_t taddr, uint32_t ncols) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr),
-                 "r"(ncols)
-                 : "memory");
 }
 
 // 16-byte cp.async with an L2 policy; src_bytes 0 fills the 16 bytes with

@@ -194,8 +194,15 @@ static bool tau_ok(float t) { return std::isfinite(t) && t >= 0.f; }
 static uint32_t g_spin_limit = kDefaultWaitUs;
 static int g_debug_skip = -1;
 
-// Stage-2 engine (prox_set_stage2_engine)
+// Stage-2 and Stage-1 engines (prox_set_stage2_engine, prox_set_stage1_engine)
 static std::atomic<int> g_engine{PROX_ENGINE_AUTO};
+static std::atomic<int> g_engine1{PROX_ENGINE_AUTO};
+
+// Whether a Stage-1 pass of B tokens takes the tensor-core proxy products
+// (passes of 4 or 8 tokens with the INT4 proxy; automatic there)
+static bool use_tc1(int B, int proxy_kind) {
+    return g_engine1.load() != PROX_ENGINE_SIMT && B >= 4 && proxy_kind == PROX_PROXY_INT4;
+}
 
 // Whether a pass of B tokens runs the tensor-core Stage 2 (and its plan)
 static bool use_tc(int d, int f, int B, int sms, Stage2UPlan *p) {
@@ -239,6 +246,7 @@ static prox_status pass_stage1(const prox_layer *L, const uint16_t *x, int nb, f
     a.build_lists = lists ? 1 : 0;
     a.act = L->activation;
     a.pk = L->proxy_kind;
+    a.tc = use_tc1(B, L->proxy_kind) ? 1 : 0;
     Stage2UPlan pu;
     if (lists && use_tc(d, f, B, sms, &pu)) {
         a.z_clear = reinterpret_cast<uint4 *>(w + W.ug);
@@ -489,6 +497,12 @@ PROX_API prox_status prox_ffn_block(const prox_layer *layer, const float *h_in, 
 }
 
 PROX_API int prox_max_batch_per_pass(int d_model) { return max_tokens_per_pass(d_model); }
+
+PROX_API int prox_set_stage1_engine(int engine) {
+    if (engine != PROX_ENGINE_AUTO && engine != PROX_ENGINE_SIMT && engine != PROX_ENGINE_TC)
+        return -1;
+    return g_engine1.exchange(engine);
+}
 
 PROX_API int prox_set_stage2_engine(int engine) {
     if (engine != PROX_ENGINE_AUTO && engine != PROX_ENGINE_SIMT && engine != PROX_ENGINE_TC)

@@ -98,6 +98,7 @@ struct Stage1Args {
     int build_lists;             // write ulist/tlist/counts for Stage 2
     int act;                     // gate activation (PROX_ACT_*)
     int pk;                      // proxy kind (PROX_PROXY_*): q_up/q_gate INT4 or bf16 tiles
+    int tc;                      // tensor-core proxy products (B 4 or 8, INT4 proxy)
     uint4 *z_clear;              // region cleared for the tensor-core Stage 2, or null
     int z_n16;                   // its size in 16-byte words
     uint32_t wait_us;            // wall-clock bound of each wait, microseconds

@@ -24,6 +24,7 @@ ABI_FUNCTIONS = (
     "prox_max_batch_per_pass", "prox_ffn_stage1", "prox_ffn_stage2",
     "prox_calibrate_workspace_bytes", "prox_calibrate", "prox_allocate",
     "prox_last_device_status", "prox_status_str", "prox_set_stage2_engine",
+    "prox_set_stage1_engine",
 )
 
 # Stage-2 engines (prox_set_stage2_engine)
@@ -84,6 +85,8 @@ def lib() -> C.CDLL:
         L.prox_status_str.restype = C.c_char_p
         L.prox_set_stage2_engine.argtypes = [i]
         L.prox_set_stage2_engine.restype = C.c_int
+        L.prox_set_stage1_engine.argtypes = [i]
+        L.prox_set_stage1_engine.restype = C.c_int
         L.prox_max_batch_per_pass.argtypes = [i]
         L.prox_max_batch_per_pass.restype = C.c_int
         L.prox_ffn_stage1.argtypes = [C.POINTER(_Layer), vp, i, f, f, vp, vp, vp, vp, sz, vp]
@@ -371,6 +374,30 @@ def set_stage2_engine(engine: int) -> int:
     return prev
 
 
+def set_stage1_engine(engine: int) -> int:
+    """Select the Stage-1 engine (ENGINE_AUTO, ENGINE_SIMT, ENGINE_TC) for
+    later calls in this process; returns the previous one."""
+    prev = int(lib().prox_set_stage1_engine(int(engine)))
+    if prev < 0:
+        raise ProxError(PROX_EINVAL, f"prox_set_stage1_engine({engine})")
+    return prev
+
+
+class stage1_engine:
+    """Context manager: run the enclosed calls with one Stage-1 engine."""
+
+    def __init__(self, engine: int):
+        self.engine = engine
+
+    def __enter__(self):
+        self.prev = set_stage1_engine(self.engine)
+        return self
+
+    def __exit__(self, *exc):
+        set_stage1_engine(self.prev)
+        return False
+
+
 class stage2_engine:
     """Context manager: run the enclosed calls with one Stage-2 engine."""
 
@@ -500,6 +527,7 @@ __all__ = ["ProxLayer", "ProxError", "quantize_proxy", "workspace", "workspace_b
            "ffn_forward", "ffn_forward_static", "STATIC_WORKSPACE_BYTES", "ffn_forward_raw",
            "ffn_stage1_raw", "ffn_stage2_raw", "rmsnorm_bf16", "ffn_block", "ffn_block_raw",
            "calibrate_histogram", "bf16_proxy", "PROXY_INT4", "PROXY_BF16",
-           "max_batch_per_pass", "set_stage2_engine", "stage2_engine", "ENGINE_AUTO",
+           "max_batch_per_pass", "set_stage2_engine", "stage2_engine", "set_stage1_engine",
+           "stage1_engine", "ENGINE_AUTO",
            "ENGINE_SIMT", "ENGINE_TC", "proxy_state", "calibrate", "allocate",
            "last_device_status", "touched_bytes", "untile_proxy", "as_bf16"]

@@ -249,6 +249,20 @@ int prox_max_batch_per_pass(int d_model);
 int prox_set_stage2_engine(int engine);
 
 /*
+ * prox_set_stage1_engine -- which kernels form the INT4 proxy products of
+ * Stage 1 (process-wide, same values and return as prox_set_stage2_engine).
+ *   PROX_ENGINE_AUTO (default) and PROX_ENGINE_TC: passes of 4 or 8 tokens
+ *     with the INT4 proxy run the proxy products on the tensor cores
+ *     (tcgen05 kind::i8: the codes as unsigned bytes, x_i * scale_i per token
+ *     as a 27-bit fixed-point value in four signed 8-bit digits, int32
+ *     accumulation, so the CTA's sums are exact up to that fixed point);
+ *     smaller passes and the bf16 proxy use the CUDA cores;
+ *   PROX_ENGINE_SIMT: the CUDA cores always.
+ * Masks, lists and the proxy state are formed the same way after either.
+ */
+int prox_set_stage1_engine(int engine);
+
+/*
  * prox_ffn_stage1 / prox_ffn_stage2 -- the two phases of prox_ffn_forward,
  * callable separately (for instance to time or inspect Stage 1 alone).
  * prox_ffn_forward(..) with batch <= prox_max_batch_per_pass(d_model) is

@@ -179,6 +179,18 @@ def test_calibrate_histogram_validates():
     assert call(200000, 4096, wsb - 1) == P.PROX_ENOMEM
 
 
+def test_stage1_engine_switch():
+    prev = P.set_stage1_engine(P.ENGINE_SIMT)
+    try:
+        assert P.set_stage1_engine(P.ENGINE_TC) == P.ENGINE_SIMT
+        assert P.lib().prox_set_stage1_engine(-3) == -1          # unknown: nothing changes
+        with P.stage1_engine(P.ENGINE_AUTO):
+            assert P.set_stage1_engine(P.ENGINE_AUTO) == P.ENGINE_AUTO
+        assert P.set_stage1_engine(P.ENGINE_AUTO) == P.ENGINE_TC
+    finally:
+        P.set_stage1_engine(prev)
+
+
 def test_stage2_engine_switch():
     prev = P.set_stage2_engine(P.ENGINE_SIMT)
     try:

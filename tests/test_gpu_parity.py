@@ -536,3 +536,51 @@ def test_tc_shapes_interleaved(c1, c2, c4):
             out = P.ffn_forward(case.layer, case.xdev(rows), case.tau_x, case.tau_s)
             torch.cuda.synchronize()
             assert out.count_s.shape[0] == b
+
+
+# ---------------------------------------------------------------------------
+# tensor-core proxy products in Stage 1 (kind::i8), passes of 4 and 8 tokens
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("engine", [P.ENGINE_TC, P.ENGINE_SIMT])
+def test_stage1_engines_proxy_state_c2(c2, engine):
+    # s~ of 8 tokens (one pass) against the oracle, with either Stage-1 engine
+    with P.stage1_engine(engine):
+        _proxy_check(c2, list(range(100, 108)))
+
+
+@pytest.mark.parametrize("b", [4, 8, 13, 64])
+def test_tc1_forward_c1(c1, b):
+    rows = list(range(b))
+    with P.stage1_engine(P.ENGINE_TC):
+        out = P.ffn_forward(c1.layer, c1.xdev(rows), c1.tau_x, c1.tau_s)
+    check_forward(c1, rows, out, f" c1 tc1 b={b}")
+
+
+def test_tc1_forward_c2_b8(c2):
+    rows = list(range(200, 208))
+    with P.stage1_engine(P.ENGINE_TC):
+        out = P.ffn_forward(c2.layer, c2.xdev(rows), c2.tau_x, c2.tau_s)
+    check_forward(c2, rows, out, " c2 tc1 b=8")
+
+
+def test_tc1_forward_c4_b16(c4):
+    rows = list(range(16))
+    with P.stage1_engine(P.ENGINE_TC):
+        out = P.ffn_forward(c4.layer, c4.xdev(rows), c4.tau_x, c4.tau_s)
+    check_forward(c4, rows, out, " c4 tc1 b=16")
+
+
+def test_tc1_matches_simt_c2(c2):
+    # the two Stage-1 engines sum in different orders (the tensor-core one
+    # exactly, up to its 27-bit fixed point): s~ agrees far inside the mask band
+    x = c2.xdev(list(range(300, 308)))
+    with P.stage1_engine(P.ENGINE_SIMT):
+        s_a, mx_a = P.proxy_state(c2.layer, x, c2.tau_x)
+    with P.stage1_engine(P.ENGINE_TC):
+        s_b, mx_b = P.proxy_state(c2.layer, x, c2.tau_x)
+    torch.cuda.synchronize()
+    assert torch.equal(mx_a, mx_b)
+    err = (s_a - s_b).abs().max().item() / c2.tau_s
+    print(f"[tc1 vs simt c2 b=8] max |ds~| / tau_s = {err:.2e}")
+    assert err < 1e-4
