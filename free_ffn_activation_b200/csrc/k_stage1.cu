@@ -170,9 +170,10 @@ __device__ __forceinline__ int block_excl_scan(int v, int *warp_tot, int &total)
 // memory of the stream, which replaces the copy ring and row-lane reduction
 // area: two K steps of decoded codes for both matrices and the digits of x.
 constexpr int kTcKStep = 32;   // proxy rows per K step (the K of one kind::i8 MMA)
-constexpr int kTcPre = 6;      // K steps of codes each thread keeps in flight (registers)
+// K steps decoded per group (one group of codes in flight per thread)
+__host__ __device__ constexpr int s1tc_group(int NB) { return NB == 2 ? 2 : 3; }
 __host__ __device__ inline size_t s1tc_bytes(int B, int NB, int unit_cap) {
-    const size_t a = (size_t)2 * 2 * kTcKStep * NB * kCB;                  // 2 buffers x 2 matrices
+    const size_t a = (size_t)s1tc_group(NB) * 2 * kTcKStep * NB * kCB;     // group x 2 matrices
     const size_t b = (size_t)2 * ((unit_cap + 127) / 128) * (4 * B / 8) * 1024;  // digits
     return 1024 + a + b;                                                   // + alignment slack
 }
@@ -288,9 +289,12 @@ __device__ __forceinline__ uint4 ldg16_pol(const void *src, uint64_t pol) {
 // each code tile is read once for all tokens. D is int32 in TMEM and exact;
 // the epilogue removes the +8 offset (8 * the digit sums, exact in int64) and
 // undoes 2^F and 2^E: this CTA's partial sums sum_i q_ij x_i scale_i, in the
-// same place the CUDA-core stream leaves them. One thread issues the MMAs; the
-// decoded tiles are double-buffered and each thread keeps kTcPre K steps of
-// codes in flight in registers. Waits are bounded.
+// same place the CUDA-core stream leaves them. The K steps go in groups of G:
+// each thread decodes its codes of the whole group into G tile buffers, makes
+// them visible to the tensor core (fence.proxy.async), and only then issues
+// the loads of the next group into registers, so no load is outstanding at a
+// fence (a fence would wait for it); one CTA barrier and one thread's MMAs
+// per group. Waits are bounded.
 template <int B, int NB>
 __device__ void s1_tc_stream(const Stage1Args &a, unsigned char *region, const int *rowidx,
                              const float *xs, int n_units, const int (&E)[B], int c0,
@@ -307,12 +311,13 @@ __device__ void s1_tc_stream(const Stage1Args &a, unsigned char *region, const i
     __shared__ int s_F[2][kMaxB];
     __shared__ int s_S[2][kMaxB][4];
     __shared__ uint32_t s_tmem;
-    __shared__ __align__(8) uint64_t s_done[2];
+    __shared__ __align__(8) uint64_t s_done[1];
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const uint32_t rb = (smem_addr(region) + 1023u) & ~1023u;
+    constexpr int GR = s1tc_group(NB);                // tile buffers (one group)
     unsigned char *abuf = region + (rb - smem_addr(region));
-    unsigned char *bdig = abuf + 2 * ABUF;
-    const uint32_t aaddr = rb, baddr = rb + 2 * ABUF;
+    unsigned char *bdig = abuf + GR * ABUF;
+    const uint32_t aaddr = rb, baddr = rb + GR * ABUF;
     const uint32_t BM = (uint32_t)((a.unit_cap + 127) / 128) * (N / 8) * 1024u;  // one matrix
     const int nks = (n_units + kTcKStep - 1) / kTcKStep;
 
@@ -320,7 +325,6 @@ __device__ void s1_tc_stream(const Stage1Args &a, unsigned char *region, const i
     if (tid < 2 * kMaxB * 4) (&s_S[0][0][0])[tid] = 0;
     if (tid == 0) {
         mbar_init(&s_done[0], 1);
-        mbar_init(&s_done[1], 1);
         mbar_fence_init();
     }
     if (wid == 0) tmem_alloc(&s_tmem, TCOLS);
@@ -388,6 +392,7 @@ __device__ void s1_tc_stream(const Stage1Args &a, unsigned char *region, const i
 
     // stream: thread tid owns pieces q = tid + 512 j (j < NB) of each K step:
     // 16 bytes (32 channels) of proxy row k of block b of matrix m
+    constexpr int G = GR;
     const uint64_t pol = l2_evict_first();
     auto fetch = [&](int ks, uint4 (&dst)[NB]) {
 #pragma unroll
@@ -403,24 +408,23 @@ __device__ void s1_tc_stream(const Stage1Args &a, unsigned char *region, const i
                                    pol);
         }
     };
-    uint4 pre[kTcPre][NB];
+    uint4 pre[G][NB];
 #pragma unroll
-    for (int p = 0; p < kTcPre; ++p) fetch(p, pre[p]);
+    for (int p = 0; p < G; ++p) fetch(p, pre[p]);
     bool ok = true;
-    for (int ks0 = 0; ks0 < nks; ks0 += kTcPre) {
+    const int ngrp = (nks + G - 1) / G;
+    for (int g = 0; g < ngrp; ++g) {
+        // the group's tile buffers are free once the previous group's MMAs are done
+        if (g >= 1 && ok) ok = mbar_wait(&s_done[0], (g - 1) & 1, a.wait_us);
 #pragma unroll
-        for (int p = 0; p < kTcPre; ++p) {
-            const int ks = ks0 + p;
-            if (ks >= nks) break;  // uniform across the CTA
-            const int bb = ks & 1;
-            // the buffer's previous MMAs (K step ks - 2) are done
-            if (ks >= 2 && ok) ok = mbar_wait(&s_done[bb], ((ks - 2) >> 1) & 1, a.wait_us);
+        for (int p = 0; p < G; ++p) {
+            const int ks = g * G + p;
 #pragma unroll
             for (int j = 0; j < NB; ++j) {
                 const int qq = tid + kS1Threads * j;
                 const int piece = qq & 7, k = (qq >> 3) & 31, bm = qq >> 8;
                 const int mm = bm & 1, b = bm >> 1;
-                if (ks * kTcKStep + k >= n_units) continue;  // its digits are 0
+                if (ks >= nks || ks * kTcKStep + k >= n_units) continue;  // digits 0 there
                 const uint32_t w[4] = {pre[p][j].x, pre[p][j].y, pre[p][j].z, pre[p][j].w};
                 uint32_t o[8];
 #pragma unroll
@@ -430,16 +434,22 @@ __device__ void s1_tc_stream(const Stage1Args &a, unsigned char *region, const i
                     o[2 * i + 1] = __byte_perm(lo, hi, 0x7362);  // channels 8i+4 .. 8i+7
                 }
                 const int ma = b * 2 + (piece >> 2), cc = (piece & 3) * 2;
-                unsigned char *row = abuf + bb * ABUF + mm * (CW * kTcKStep) + ma * LBO +
+                unsigned char *row = abuf + p * ABUF + mm * (CW * kTcKStep) + ma * LBO +
                                      (k >> 3) * 1024 + (k & 7) * 128;
                 *reinterpret_cast<uint4 *>(row + (((cc) ^ (k & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
                 *reinterpret_cast<uint4 *>(row + (((cc + 1) ^ (k & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
             }
-            fetch(ks + kTcPre, pre[p]);
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            __syncthreads();
-            if (tid == 0) {
-                tc_fence_after();
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+#pragma unroll
+        for (int p = 0; p < G; ++p) fetch((g + 1) * G + p, pre[p]);
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int p = 0; p < G; ++p) {
+                const int ks = g * G + p;
+                if (ks >= nks) break;
                 const uint32_t kb_off = (uint32_t)(ks >> 2) * (N / 8) * 1024u + (uint32_t)(ks & 3) * 32u;
 #pragma unroll
                 for (int mm = 0; mm < 2; ++mm) {
@@ -447,14 +457,14 @@ __device__ void s1_tc_stream(const Stage1Args &a, unsigned char *region, const i
 #pragma unroll
                     for (int mt = 0; mt < MT; ++mt)
                         umma_i8(tmem + (mm * MT + mt) * N,
-                                sw128_desc(aaddr + bb * ABUF + mm * (CW * kTcKStep) + mt * LBO, LBO, 1024),
+                                sw128_desc(aaddr + p * ABUF + mm * (CW * kTcKStep) + mt * LBO, LBO, 1024),
                                 db, IDESC, ks > 0 ? 1u : 0u);
                 }
-                umma_commit(&s_done[bb]);
             }
+            umma_commit(&s_done[0]);
         }
     }
-    if (nks > 0 && ok) ok = mbar_wait(&s_done[(nks - 1) & 1], ((nks - 1) >> 1) & 1, a.wait_us);
+    if (ngrp > 0 && ok) ok = mbar_wait(&s_done[0], (ngrp - 1) & 1, a.wait_us);
     if (!ok) atomicOr(a.status, kStTimeoutMma);
     tc_fence_after();
     // epilogue: warp quadrant q reads TMEM lanes 32q..32q+31 (channels of an M
