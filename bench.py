@@ -66,6 +66,9 @@ def parse():
     ap.add_argument("--engine", choices=["auto", "simt", "tc"], default="auto",
                     help="Stage-2 engine: automatic, CUDA cores, or the tensor-core union GEMM "
                          "(passes of >= 4 tokens)")
+    ap.add_argument("--stage1-engine", choices=["auto", "simt", "tc"], default="auto",
+                    help="Stage-1 proxy products: automatic, CUDA cores, or tensor cores "
+                         "(passes of >= 4 tokens, INT4 proxy)")
     ap.add_argument("--copies", type=int, default=4, help="rotating weight copies (L2 defeat)")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense cuBLAS reference")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
@@ -461,6 +464,7 @@ def run_ours(args, w, rank, world, local_rank):
             "dtype": "bf16", "data": "synthetic",
             "config": {"workload": args.workload, "d_model": d, "d_ff": f, "batch": Bt,
                        "proxy": args.proxy, "engine": args.engine,
+                       "stage1_engine": args.stage1_engine,
                        "tokens_per_step": ntok, "keep_x": args.keep_x, "keep_s": args.keep_s,
                        "tau_x": tau_x, "tau_s": tau_s,
                        "l2": f"{R} rotating weight copies ({R * (3 * d * f * 2 + (d * f + 8 * d if pk == P.PROXY_INT4 else 4 * d * f)) / 1e9:.2f} GB > L2)",
@@ -682,7 +686,9 @@ def main():
         run_reference(args, w, rank, world)
         return
     from free_ffn_activation_b200 import prox as P
-    P.set_stage2_engine({"auto": P.ENGINE_AUTO, "simt": P.ENGINE_SIMT, "tc": P.ENGINE_TC}[args.engine])
+    engines = {"auto": P.ENGINE_AUTO, "simt": P.ENGINE_SIMT, "tc": P.ENGINE_TC}
+    P.set_stage2_engine(engines[args.engine])
+    P.set_stage1_engine(engines[args.stage1_engine])
     if world > 1:
         import datetime
 

@@ -30,6 +30,11 @@
 // 8 * sum(x_i * scale_i) is removed. Nibbles 5..7 of a word are first shifted
 // down by 12 bits (to positions 2..4). Subnormal operands need FMA without
 // flush-to-zero, which is the default without fast-math.
+//
+// Passes of 4 or 8 tokens with the INT4 proxy can form the proxy products on
+// the tensor cores instead (s1_tc_stream below: tcgen05 kind::i8 over the
+// codes as bytes and fixed-point digits of x, exact int32 accumulation); the
+// prologue, the cluster reduction and the lists are shared.
 #include "prox_internal.cuh"
 #include "umma.cuh"
 
