@@ -71,3 +71,41 @@ def test_reference_arm_other_ranks_exit_quietly():
     r = _run_reference(1, 2)
     assert r.returncode == 0, r.stderr[-2000:]
     assert not [l for l in r.stdout.splitlines() if l.startswith("{")]
+
+
+def test_launches_per_call_counts_kernels_per_pass():
+    # per pass: Stage 1 and one Stage-2 kernel (CUDA cores) or two (tensor-core
+    # union engine: automatic for 8-token passes, and for 4-token passes when
+    # d_model >= 8192, whose passes hold at most 4 tokens)
+    sys.path.insert(0, ROOT)
+    import argparse
+
+    import bench
+
+    def n(engine, d, batch):
+        return bench.launches_per_call(argparse.Namespace(engine=engine), d, batch)
+
+    assert n("auto", 4096, 1) == 2 and n("auto", 4096, 2) == 2 and n("auto", 4096, 4) == 2
+    assert n("auto", 4096, 8) == 3 and n("auto", 4096, 5) == 3      # one pass of 8 slots
+    assert n("simt", 4096, 8) == 2 and n("tc", 4096, 4) == 3 and n("tc", 4096, 2) == 2
+    assert n("auto", 8192, 4) == 3 and n("auto", 8192, 16) == 4 * 3  # passes of 4
+    assert n("simt", 8192, 16) == 4 * 2
+
+
+def test_stage2_traffic_scaled_to_the_mean_token():
+    # the committed Stage-2 summary holds one token's traffic and algorithmic
+    # bytes; the bench reports it scaled to the mean token's bytes, and only
+    # for the workload and batch the capture covers
+    sys.path.insert(0, ROOT)
+    import bench
+    fields = {}
+    for line in open(os.path.join(ROOT, "profiles", "k_stage2_qwen3-8b-ffn_b1.md")):
+        if line.startswith("- ") and ":" in line:
+            k, v = line[2:].split(":", 1)
+            fields[k.strip()] = v.strip()
+    traffic = float(fields["dram bytes per launch (read + write)"])
+    captured = float(fields["algorithmic bytes of the captured launch"].split()[0])
+    got = bench.stage2_traffic("qwen3-8b-ffn", 1, 90537600.0)
+    assert got is not None and abs(got - traffic * 90537600.0 / captured) < 1.0
+    assert bench.stage2_traffic("qwen3-8b-ffn", 8, 1.0) is None
+    assert bench.stage2_traffic("large-ffn", 1, 1.0) is None
