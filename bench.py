@@ -218,8 +218,13 @@ def cpu_oracle_time(w, keep_x, keep_s, seconds):
         t_used += time.perf_counter() - t0
         threads = out["threads"]
         done += n
+    # the same path on one thread, over the first two tokens of the sample
+    t0 = time.perf_counter()
+    oracle.forward(x[0:2], tau_x, tau_s, L, Por, n_threads=1, want=())
+    us_one = (time.perf_counter() - t0) / 2 * 1e6
     sample = (f"{done} of {w['tokens']} tokens of the {w['d']}x{w['f']} layer "
-              f"(thresholds from {x_cal.shape[0]} calibration vectors), all stages, fp64")
+              f"(thresholds from {x_cal.shape[0]} calibration vectors), all stages, fp64, "
+              f"{threads} threads (one thread, 2 tokens: {us_one:.0f} us/token)")
     return t_used / done * 1e6, threads, sample
 
 
