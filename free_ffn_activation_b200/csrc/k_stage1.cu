@@ -364,30 +364,40 @@ __device__ void s1_tc_stream(const Stage1Args &a, unsigned char *region, const i
     }
     __syncthreads();
     // the digits (B operand, K-major, 128-byte swizzle: 8 digit rows x 128
-    // proxy rows per atom); rows past the CTA's units up to the last K step are 0
-    for (int u = tid; u < nks * kTcKStep; u += kS1Threads) {
-        const int kblk = u >> 7, kin = u & 127;
+    // proxy rows per atom); rows past the CTA's units up to the last K step are
+    // 0. Thread tid owns the (matrix, token) pair tid % (2B) over every
+    // (512 / 2B)-th row and sums its digits in registers; the lanes of a warp
+    // that share a pair are reduced with shuffles, so each warp adds 4 counts
+    // per pair (integers: the order does not change the sums)
+    {
+        constexpr int NP = 2 * B;                 // (matrix, token) pairs: 8 or 16
+        constexpr int NS = kS1Threads / NP;       // row stripes
+        const int pair = tid & (NP - 1), stripe = tid / NP;
+        const int mm = pair / B, t = pair % B;
+        const int F = s_F[mm][t], f1 = F / 2, f2 = F - f1;
+        const float sc1 = __int_as_float((127 + f1) << 23), sc2 = __int_as_float((127 + f2) << 23);
+        int dsum[4] = {0, 0, 0, 0};
+        for (int u = stripe; u < nks * kTcKStep; u += NS) {
+            const int kblk = u >> 7, kin = u & 127;
+            int v = 0;
+            if (u < n_units) v = __float2int_rn(xs[(u * 2 + mm) * B + t] * sc1 * sc2);
+            const int d3 = v >> 21;
+            const int r = v - d3 * (1 << 21);
+            const int dg[4] = {r & 127, (r >> 7) & 127, r >> 14, d3};
 #pragma unroll
-        for (int mm = 0; mm < 2; ++mm)
-#pragma unroll
-            for (int t = 0; t < B; ++t) {
-                int v = 0;
-                if (u < n_units) {
-                    const int F = s_F[mm][t], f1 = F / 2, f2 = F - f1;
-                    v = __float2int_rn(xs[(u * 2 + mm) * B + t] * __int_as_float((127 + f1) << 23) *
-                                       __int_as_float((127 + f2) << 23));
-                }
-                const int d3 = v >> 21;
-                const int r = v - d3 * (1 << 21);
-                const int dg[4] = {r & 127, (r >> 7) & 127, r >> 14, d3};
-#pragma unroll
-                for (int l = 0; l < 4; ++l) {
-                    const int n = t * 4 + l;
-                    bdig[mm * BM + (uint32_t)kblk * (N / 8) * 1024u + (n >> 3) * 1024u + (n & 7) * 128u +
-                         ((uint32_t)((kin >> 4) ^ (n & 7)) << 4) + (kin & 15)] = (unsigned char)dg[l];
-                    if (dg[l]) atomicAdd(&s_S[mm][t][l], dg[l]);
-                }
+            for (int l = 0; l < 4; ++l) {
+                const int n = t * 4 + l;
+                bdig[mm * BM + (uint32_t)kblk * (N / 8) * 1024u + (n >> 3) * 1024u + (n & 7) * 128u +
+                     ((uint32_t)((kin >> 4) ^ (n & 7)) << 4) + (kin & 15)] = (unsigned char)dg[l];
+                dsum[l] += dg[l];
             }
+        }
+#pragma unroll
+        for (int l = 0; l < 4; ++l) {
+#pragma unroll
+            for (int o = NP; o < 32; o <<= 1) dsum[l] += __shfl_xor_sync(0xffffffffu, dsum[l], o);
+            if (lane < NP) atomicAdd(&s_S[mm][t][l], dsum[l]);
+        }
     }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     tc_fence_before();
