@@ -91,6 +91,28 @@ def launches_per_call(args, d, batch):
     return passes * (3 if tc else 2)
 
 
+def summary_fields(path):
+    """'- key: value' lines of a profiles/ summary as a dict."""
+    fields = {}
+    for line in open(path):
+        if ":" in line and line.startswith("- "):
+            k, v = line[2:].split(":", 1)
+            fields[k.strip()] = v.strip().strip("`")
+    return fields
+
+
+def traffic_from_summary(fields, mean_bytes=None):
+    """DRAM bytes per launch from a summary's fields, scaled from the captured
+    launch's algorithmic bytes to `mean_bytes` (traffic grows with the kept
+    rows); None if the fields are missing."""
+    try:
+        traffic = float(fields["dram bytes per launch (read + write)"])
+        captured = float(fields["algorithmic bytes of the captured launch"].split()[0])
+    except (KeyError, ValueError, IndexError):
+        return None
+    return traffic * mean_bytes / captured if mean_bytes else traffic
+
+
 def stage2_traffic(workload, batch, mean_bytes=None):
     """DRAM bytes per launch of the Stage-2 kernel from the committed ncu summary,
     if it covers this workload and was captured from the current kernel source
@@ -103,21 +125,54 @@ def stage2_traffic(workload, batch, mean_bytes=None):
     if not os.path.exists(summ):
         return None
     digest = hashlib.sha256(open(src, "rb").read()).hexdigest()
-    fields = {}
-    for line in open(summ):
-        if ":" in line and line.startswith("- "):
-            k, v = line[2:].split(":", 1)
-            fields[k.strip()] = v.strip().strip("`")
+    fields = summary_fields(summ)
     if fields.get("k_stage2.cu sha256") != digest:
         return None
-    try:
-        traffic = float(fields["dram bytes per launch (read + write)"])
-        captured = float(fields["algorithmic bytes of the captured launch"].split()[0])
-    except (KeyError, ValueError, IndexError):
-        return None
-    # the captured launch is one token; scale to the mean token's algorithmic
-    # bytes (traffic grows with the kept channels) so it compares with `achieved`
-    return traffic * mean_bytes / captured if mean_bytes else traffic
+    return traffic_from_summary(fields, mean_bytes)
+
+
+def stamp_phases(st, sampled, slot):
+    """Mean phase durations (us) over the sampled calls from their
+    %globaltimer stamps (slot names in prox_internal.cuh's StampSlot).
+    stage1 + stage2 is the time from one call's Stage 1 passing its wait for
+    the previous kernel to the next call's: Stage 1 runs until Stage 2 passes
+    its wait, Stage 2 until the next Stage 1 does."""
+    import numpy as np
+    st = st.astype(np.uint64)
+    NONE = np.uint64(0xFFFFFFFFFFFFFFFF)
+
+    def us(a, b):
+        return (float(b) - float(a)) / 1e3
+
+    rows = {k: [] for k in ("stage1", "stage2", "s1_wait_spread", "s1_prologue", "s1_stream",
+                            "s1_reduce", "s1_lists", "s1_exit_to_s2_go", "s2_go_spread",
+                            "s2_list", "s2_first_data", "s2_stream_window", "s2_tail",
+                            "s2_exit_to_next_s1_go", "call")}
+    for c in sampled:
+        if c + 1 not in slot:
+            continue
+        a, b = st[slot[c]], st[slot[c + 1]]
+        if a[1] == NONE or a[9] == NONE or b[1] == NONE:
+            continue
+        rows["stage1"].append(us(a[1], a[9]))
+        rows["stage2"].append(us(a[9], b[1]))
+        rows["call"].append(us(a[1], b[1]))
+        rows["s1_wait_spread"].append(us(a[1], a[2]))
+        rows["s1_prologue"].append(us(a[1], a[3]))
+        rows["s1_stream"].append(us(a[3], a[4]))
+        rows["s1_reduce"].append(us(a[4], a[5]))
+        rows["s1_lists"].append(us(a[5], a[6]))
+        rows["s1_exit_to_s2_go"].append(us(a[6], a[9]))
+        rows["s2_go_spread"].append(us(a[9], a[10]))
+        rows["s2_exit_to_next_s1_go"].append(us(a[15], b[1]))
+        if a[11] != 0 and a[12] != NONE:
+            rows["s2_list"].append(us(a[9], a[11]))
+            rows["s2_first_data"].append(us(a[11], a[13]))
+            rows["s2_stream_window"].append(us(a[12], a[14]))
+            rows["s2_tail"].append(us(a[14], a[15]))
+    out = {k: (float(np.mean(v)) if v else None) for k, v in rows.items()}
+    out["pairs"] = len(rows["call"])
+    return out
 
 
 def max_over_ranks(x, world, dev):
@@ -301,37 +356,32 @@ def run_ours(args, w, rank, world, local_rank):
     xrow = d * 2
     yrow = d * 4
     xp, yp, wp = x.data_ptr(), y.data_ptr(), ws.data_ptr()
-    sample_every = 8
-    sampled = list(range(0, ngrp, sample_every))        # call indices
-    ev_s = {t: torch.cuda.Event(enable_timing=True, external=True) for t in sampled}
-    ev_a = {t: torch.cuda.Event(enable_timing=True, external=True) for t in sampled}
-    ev_b = {t: torch.cuda.Event(enable_timing=True, external=True) for t in sampled}
+    # phase stamps (%globaltimer, prox_test_set_stamps) on pairs of adjacent
+    # calls, every 8th pair: the second call of a pair gives the time from
+    # the first call's Stage 2 to the next call's Stage 1
+    sampled = sorted({c for c0 in range(0, ngrp, 8) for c in (c0, c0 + 1) if c < ngrp})
+    slot = {c: k for k, c in enumerate(sampled)}
+    stamps = P.stamp_buffer(len(sampled), dev)
 
-    def one_step(record):
-        # the public forward is Stage 1 then Stage 2; the split entry points
-        # let the instrumented copy put events between the two kernels
+    def one_step():
+        # the timed step: the public forward per call; the sampled calls are
+        # captured with the stamp hook set, so the timed graph is the one
+        # whose phases are read below
         for c in range(ngrp):
             t = c * Bt
-            Ls = structs[c % R]
-            rec = record and c in ev_a
-            if rec:
-                ev_s[c].record(stream)
-            P.ffn_stage1_raw(Ls, xp + t * xrow, Bt, tau_x, tau_s, yp + t * yrow, wp, wsb, sp)
-            if rec:
-                ev_a[c].record(stream)
-            P.ffn_stage2_raw(Ls, xp + t * xrow, Bt, yp + t * yrow, wp, wsb, sp)
-            if rec:
-                ev_b[c].record(stream)
+            if c in slot:
+                P.test_set_stamps(stamps[slot[c]].data_ptr())
+            P.ffn_forward_raw(structs[c % R], xp + t * xrow, Bt, tau_x, tau_s, yp + t * yrow,
+                              wp, wsb, sp)
+            if c in slot:
+                P.test_set_stamps(0)
 
     with torch.cuda.stream(stream):
-        one_step(False)
+        one_step()
     torch.cuda.synchronize(dev)
-    g = torch.cuda.CUDAGraph()          # the timed step: no events inside
+    g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream):
-        one_step(False)
-    gi = torch.cuda.CUDAGraph()         # instrumented copy for per-kernel times
-    with torch.cuda.graph(gi, stream=stream):
-        one_step(True)
+        one_step()
     # parity spot-check of the graph's output against direct calls with the same
     # tokens per call (calls of another batch size sum the proxy in another
     # order, so a channel within rounding of tau_s may legitimately differ)
@@ -352,7 +402,6 @@ def run_ours(args, w, rank, world, local_rank):
     barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    s2_ms = []
     with ClockSampler(local_rank) as clk:
         e0.record(stream)
         for _ in range(args.steps):
@@ -361,15 +410,13 @@ def run_ours(args, w, rank, world, local_rank):
             torch.cuda.current_stream(dev).wait_stream(stream)
         e1.record(stream)
         barrier()
-        # per-kernel durations: events around each kernel of every 8th token,
-        # from instrumented replays run right after the timed ones
-        s1_ms, s2_ms = [], []
-        for _ in range(max(1, min(args.steps, 5))):
-            with torch.cuda.stream(stream):
-                gi.replay()
-            torch.cuda.synchronize(dev)
-            s1_ms += [ev_s[t].elapsed_time(ev_a[t]) for t in sampled]
-            s2_ms += [ev_a[t].elapsed_time(ev_b[t]) for t in sampled]
+        # one more replay of the same graph with the stamp slots reset
+        P.reset_stamps(stamps)
+        torch.cuda.synchronize(dev)
+        with torch.cuda.stream(stream):
+            g.replay()
+        torch.cuda.synchronize(dev)
+    status = P.last_device_status(ws)[1]
     ms_total = e0.elapsed_time(e1)
     ms_total = max_over_ranks(ms_total, world, dev)
     ms_step = ms_total / args.steps
@@ -377,13 +424,17 @@ def run_ours(args, w, rank, world, local_rank):
     us_tok_rank = ms_step * 1e3 / ntok
 
     peak, peak_src = load_peaks()
-    s2_us = statistics.mean(s2_ms) * 1e3
-    s1_us = statistics.mean(s1_ms) * 1e3
-    s2_bytes = float(np.mean(stage2_bytes[sampled]))
+    ph = stamp_phases(stamps.cpu().numpy(), sampled, slot)
+    pair = [c for c in sampled if c + 1 in slot]
+    s1_us, s2_us = ph["stage1"], ph["stage2"]
+    s2_bytes = float(np.mean(stage2_bytes[pair]))
     s2_gbs = s2_bytes / (s2_us * 1e-6) / 1e9
-    s1_bytes = float(np.mean((touched - stage2_bytes)[sampled]))
+    s1_bytes = float(np.mean((touched - stage2_bytes)[pair]))
     s1_gbs = s1_bytes / (s1_us * 1e-6) / 1e9
     path_gbs = float(np.mean(touched)) / (us_tok_rank * Bt * 1e-6) / 1e9  # per call
+    s2_stream_gbs = None
+    if ph.get("s2_stream_window"):
+        s2_stream_gbs = s2_bytes / (ph["s2_stream_window"] * 1e-6) / 1e9
 
     # e2e through the public API with host buffers: pinned x in, y out
     x_host = x.cpu().pin_memory()
@@ -477,9 +528,14 @@ def run_ours(args, w, rank, world, local_rank):
             "roofline": {"bound": "hbm", "kernel": "k_stage2 (exact up/gate/down)",
                          "achieved": s2_gbs, "peak": peak, "unit": "GB/s",
                          "frac": s2_gbs / peak, "traffic": stage2_traffic(args.workload, Bt, s2_bytes) if args.proxy == "int4" else None, "peak_source": peak_src,
-                         "bytes_per_launch": s2_bytes, "us_per_launch": s2_us},
+                         "bytes_per_launch": s2_bytes, "us_per_launch": s2_us,
+                         "timing": "in the timed graph: from Stage 2 passing its wait for Stage 1 "
+                                   "to the next call's Stage 1 passing its wait (globaltimer stamps)",
+                         "stream_GBps": s2_stream_gbs},
             "stage1": {"kernel": f"k_stage1 ({args.proxy} proxy + channel mask)", "us_per_launch": s1_us,
                        "bytes_per_launch": s1_bytes, "GBps": s1_gbs, "frac": s1_gbs / peak},
+            "phases_us": ph,
+            "device_status": status,
             "effective_sparsity": None if args.effective_sparsity is None else {
                 "target": args.effective_sparsity,
                 "realised": (1.0 - ks_tok / f) - 2.0 / 3.0 * (kx_tok / d) / 3.0,
@@ -496,7 +552,7 @@ def run_ours(args, w, rank, world, local_rank):
             "clocks": clk.summary(),
         }
         print(json.dumps(line), flush=True)
-    del g, gi
+    del g
 
 
 def run_stack(args, w, rank, world, local_rank):

@@ -535,6 +535,7 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
     // every CTA of the cluster has started once this phase completes: only
     // then may ranks store into CTA 0's shared memory (waited for before (6))
     if (kPush) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+    if (tid == 0) stamp_min(a.stamps, kS1Entry);
 
     // The proxy scales are layer weights: pull them into L2 while the
     // previous kernel of the stream finishes (a prefetch only warms the
@@ -553,6 +554,10 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
     // (Stage 2) start its own prologue.
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;");
+    if (tid == 0) {
+        stamp_min(a.stamps, kS1Go);
+        stamp_max(a.stamps, kS1GoMax);
+    }
 
     // (1) Stage 2 accumulates y with atomics: clear it here (or start it
     // from y_init, the residual stream of a layer stack).
@@ -701,9 +706,11 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
         }
     }
     __syncthreads();
+    if (tid == 0) stamp_max(a.stamps, kS1Pro);
 
     if constexpr (TC) {
         s1_tc_stream<B, NB>(a, ring, rowidx, xs, n_units, E, c0, dst_part);
+        if (tid == 0) stamp_max(a.stamps, kS1Stream);
     } else {
         const int rl = tid / T::TPR;
         const int m = (tid / T::TPRM) & 1;
@@ -725,6 +732,7 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
         else
             s1_stream<B, NB, PK, T::DMAX / 4>(qbase, ring, rowidx, xs, rl, m, n_rows, acc2, ssum);
         __syncthreads();  // every thread is done with the ring before it becomes `red`
+        if (tid == 0) stamp_max(a.stamps, kS1Stream);
         if (kPush) asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
 
         // (6) reduce row lanes (padded rows: conflict-free both ways), undo the
@@ -771,6 +779,7 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
         }
     }
     cluster.sync();  // all partials of the block are in their CTAs' shared memory
+    if (r == 0 && tid == 0) stamp_max(a.stamps, kS1Red);
 
     if (r == 0) {
         // (7) CTA 0 of the cluster: gather the cluster's partials (in rank
@@ -853,6 +862,10 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
         // peers keep their shared memory until CTA 0 has gathered it
         asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
         asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+    }
+    if (a.stamps) {  // uniform over the grid
+        __syncthreads();
+        if (tid == 0) stamp_max(a.stamps, kS1End);
     }
 }
 

@@ -108,6 +108,7 @@ __global__ void __launch_bounds__(s2_threads(B), 1) k_stage2(const Stage2Args a)
     const int nch16 = d / 8;  // 16-byte chunks per row
 
     if (tid == 0) {
+        stamp_min(a.stamps, kS2Entry);
         for (int s = 0; s < NST; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1 + NDOWN);
@@ -139,6 +140,10 @@ __global__ void __launch_bounds__(s2_threads(B), 1) k_stage2(const Stage2Args a)
     // the per-block counts and the list blocks this CTA most likely owns
     // (those around block g * C / G).
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (tid == 0) {
+        stamp_min(a.stamps, kS2Go);
+        stamp_max(a.stamps, kS2GoMax);
+    }
     // (G is one CTA per SM, so every product below fits in 32 bits)
     const int G = gridDim.x, g = blockIdx.x;
     const int npf = C < kS2Prefetch ? C : kS2Prefetch;
@@ -250,6 +255,7 @@ __global__ void __launch_bounds__(s2_threads(B), 1) k_stage2(const Stage2Args a)
         }
     }
     __syncthreads();
+    if (tid == 0) stamp_max(a.stamps, kS2List);
     const unsigned U = (unsigned)uscan[C];
     const int n_ch = (int)(U * (g + 1) / G) - (int)(U * g / G);
     asm volatile("griddepcontrol.launch_dependents;");
@@ -301,6 +307,10 @@ __global__ void __launch_bounds__(s2_threads(B), 1) k_stage2(const Stage2Args a)
             if (!__all_sync(0xffffffffu, mbar_wait(&full[s], k & 1, a.spin_limit))) {
                 if (lane == 0) atomicOr(a.status, kStTimeoutFull);
                 break;
+            }
+            if (n == 0 && lane == 0) {
+                stamp_min(a.stamps, kS2First);
+                stamp_max(a.stamps, kS2FirstMax);
             }
             const uint32_t bits = (B == 1) ? 1u : (meta[s] >> 24);
             const uint16_t *up = stages + (size_t)s * 3 * d;
@@ -410,6 +420,7 @@ __global__ void __launch_bounds__(s2_threads(B), 1) k_stage2(const Stage2Args a)
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
     }
+    if (lane == 0) stamp_max(a.stamps, kS2Stream);
 
     if (n_ch == 0) return;
 #pragma unroll
@@ -425,6 +436,7 @@ __global__ void __launch_bounds__(s2_threads(B), 1) k_stage2(const Stage2Args a)
             }
         }
     }
+    if (lane == 0) stamp_max(a.stamps, kS2End);
 }
 
 template <int B, int NCHD>

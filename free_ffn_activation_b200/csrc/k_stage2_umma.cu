@@ -235,8 +235,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_s2u_updown(const Stage2UArgs a)
 
     // Stage 1's lists (and its clearing of the partial sums) are complete
     // once it has finished
+    if (tid == 0) stamp_min(a.stamps, kS2Entry);
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;");
+    if (tid == 0) {
+        stamp_min(a.stamps, kS2Go);
+        stamp_max(a.stamps, kS2GoMax);
+    }
     for (int c = tid; c < C; c += kThreads) uscan[c] = a.ucount[c];
     __syncthreads();
     if (wid == 0) {
@@ -615,6 +620,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_s2u_down(const Stage2UArgs a) {
         tc_fence_after();
         tmem_free(tmem, TCOLS);
     }
+    if (tid == 0) stamp_max(a.stamps, kS2End);
 }
 
 template <int B, int NM>

@@ -115,6 +115,13 @@ WsLayout ws_layout(int d, int f, int B) {
         L.pos_ch = o;
         o = align_up(o + (size_t)f * 4, 256);
     }
+    L.acc = L.blk_cnt = o;
+    if (B <= 4) {  // tensor-core Stage 1 (see k_stage1_tc.cu)
+        L.acc = o;
+        o = align_up(o + (size_t)2 * B * f * 8, 256);
+        L.blk_cnt = o;
+        o = align_up(o + C * 4, 256);
+    }
     L.total = o;
     return L;
 }
@@ -193,15 +200,31 @@ static bool tau_ok(float t) { return std::isfinite(t) && t >= 0.f; }
 // test hooks (set by prox_debug_set through the binding's test helpers only)
 static uint32_t g_spin_limit = kDefaultWaitUs;
 static int g_debug_skip = -1;
+// measurement hook (prox_test_set_stamps): phase stamps of the next passes
+static unsigned long long *g_stamps = nullptr;
 
 // Stage-2 and Stage-1 engines (prox_set_stage2_engine, prox_set_stage1_engine)
 static std::atomic<int> g_engine{PROX_ENGINE_AUTO};
 static std::atomic<int> g_engine1{PROX_ENGINE_AUTO};
 
 // Whether a Stage-1 pass of B tokens takes the tensor-core proxy products
-// (passes of 4 or 8 tokens with the INT4 proxy; automatic there)
+// of k_stage1.cu (passes of 8 tokens, or of 4 on shapes the tensor-core
+// Stage 1 of k_stage1_tc.cu does not take; INT4 proxy; automatic there)
 static bool use_tc1(int B, int proxy_kind) {
     return g_engine1.load() != PROX_ENGINE_SIMT && B >= 4 && proxy_kind == PROX_PROXY_INT4;
+}
+
+// Whether a Stage-1 pass of B tokens runs k_stage1_tc (passes of <= 4
+// tokens, INT4 proxy, d_model <= 4096, when the tensor-core Stage-1 engine
+// is selected) and its plan. The automatic choice keeps the CUDA-core
+// kernel there: it streams the gathered proxy rows faster (each thread's
+// copies progress on their own; a tensor-core K step waits for all of its
+// 512 pieces).
+static bool use_tc1_small(int d, int f, int B, int proxy_kind, int sms, int *n_r, int *cap,
+                          size_t *smem) {
+    if (g_engine1.load() != PROX_ENGINE_TC || proxy_kind != PROX_PROXY_INT4 || B > 4)
+        return false;
+    return stage1_tc_plan(d, f, B, sms, n_r, cap, smem);
 }
 
 // Whether a pass of B tokens runs the tensor-core Stage 2 (and its plan)
@@ -253,11 +276,22 @@ static prox_status pass_stage1(const prox_layer *L, const uint16_t *x, int nb, f
         a.z_n16 = (int)(W.clear_bytes / 16);
     }
     a.wait_us = g_spin_limit;
+    a.stamps = g_stamps;
     a.status = reinterpret_cast<uint32_t *>(w + W.status);
     a.ucount = reinterpret_cast<int32_t *>(w + W.ucount);
     a.tcount = reinterpret_cast<int32_t *>(w + W.tcount);
     a.ulist = reinterpret_cast<uint32_t *>(w + W.ulist);
     a.tlist = reinterpret_cast<int32_t *>(w + W.tlist);
+    int nr = 0, cap = 0;
+    size_t smem = 0;
+    if (use_tc1_small(d, f, B, L->proxy_kind, sms, &nr, &cap, &smem)) {
+        a.n_r = nr;
+        a.unit_cap = cap;
+        a.tc = 1;
+        a.acc = reinterpret_cast<long long *>(w + W.acc);
+        a.blk_cnt = reinterpret_cast<int32_t *>(w + W.blk_cnt);
+        return launch_stage1_tc(B, a, smem, st) == cudaSuccess ? PROX_OK : PROX_ECUDA;
+    }
     return launch_stage1(B, a, p1, st) == cudaSuccess ? PROX_OK : PROX_ECUDA;
 }
 
@@ -299,6 +333,7 @@ static prox_status pass_stage2(const prox_layer *L, const uint16_t *x, int nb, f
         u.tile_cnt = reinterpret_cast<int32_t *>(w + W.tile_cnt);
         u.sb = reinterpret_cast<uint16_t *>(w + W.sb);
         u.pos_ch = reinterpret_cast<uint32_t *>(w + W.pos_ch);
+        u.stamps = g_stamps;
         return launch_stage2_umma(B, u, sms, st) == cudaSuccess ? PROX_OK : PROX_ECUDA;
     }
     const int max_ch = (f + sms - 1) / sms + 1;
@@ -326,6 +361,7 @@ static prox_status pass_stage2(const prox_layer *L, const uint16_t *x, int nb, f
     b.debug_skip = g_debug_skip;
     b.nstage = p2.nstage;
     b.max_ch = max_ch;
+    b.stamps = g_stamps;
     return launch_stage2(B, p2.nchunk, b, sms, p2.smem, st) == cudaSuccess ? PROX_OK : PROX_ECUDA;
 }
 
@@ -741,3 +777,7 @@ PROX_API void prox_test_set_wait(uint32_t spin_limit, int skip_position) {
     prox::g_spin_limit = spin_limit ? spin_limit : kDefaultWaitUs;
     prox::g_debug_skip = skip_position;
 }
+
+// Measurement hook, not part of prox.h: passes launched while `slots` is set
+// record %globaltimer phase stamps (prox::StampSlot) into it.
+PROX_API void prox_test_set_stamps(unsigned long long *slots) { prox::g_stamps = slots; }

@@ -35,6 +35,27 @@ constexpr int kTcMinBatch = 8;
 // default wall-clock bound of a device-side wait, in microseconds
 constexpr uint32_t kDefaultWaitUs = 2000000u;
 
+// Phase stamps (measurement hook prox_test_set_stamps): %globaltimer values
+// of one forward pass, each the minimum or maximum over the kernel's CTAs
+enum StampSlot : int {
+    kS1Entry = 0,    // min: a Stage-1 CTA starts
+    kS1Go = 1,       // min: past griddepcontrol.wait (the previous kernel is done)
+    kS1GoMax = 2,    // max: the same
+    kS1Pro = 3,      // max: masks, ranks and scaled x ready (stream starts)
+    kS1Stream = 4,   // max: the CTA's proxy products are done
+    kS1Red = 5,      // max: the cluster's partials are summed (CTA 0)
+    kS1End = 6,      // max: a Stage-1 CTA is done (lists written)
+    kS2Entry = 8,    // min: a Stage-2 CTA starts
+    kS2Go = 9,       // min: past griddepcontrol.wait (Stage 1 is done)
+    kS2GoMax = 10,   // max: the same
+    kS2List = 11,    // max: the CTA's channel list is ready
+    kS2First = 12,   // min: first ring stage full
+    kS2FirstMax = 13,  // max: the same
+    kS2Stream = 14,  // max: the last channel of a CTA is accumulated
+    kS2End = 15,     // max: a CTA's y reductions are issued
+    kStampSlots = 16
+};
+
 // ---------------------------------------------------------------------------
 // Host-side plans
 // ---------------------------------------------------------------------------
@@ -75,7 +96,7 @@ bool stage2u_plan(int d_model, int d_ff, int num_sms, Stage2UPlan *p);
 // position with the split counters right after them (one region Stage 1
 // clears), the s tiles and the channel of every union position.
 struct WsLayout {
-    size_t status, ucount, tcount, ulist, tlist, ug, tile_cnt, sb, pos_ch, total;
+    size_t status, ucount, tcount, ulist, tlist, ug, tile_cnt, sb, pos_ch, acc, blk_cnt, total;
     size_t clear_bytes;  // ug .. tile_cnt end
 };
 WsLayout ws_layout(int d_model, int d_ff, int B);
@@ -102,8 +123,12 @@ struct Stage1Args {
     uint4 *z_clear;              // region cleared for the tensor-core Stage 2, or null
     int z_n16;                   // its size in 16-byte words
     uint32_t wait_us;            // wall-clock bound of each wait, microseconds
+    unsigned long long *stamps;  // phase stamps (StampSlot) or null
     // workspace
     uint32_t *status;
+    long long *acc;              // tensor-core Stage 1 (<= 4 tokens): [2][B][f] exact
+                                 // int64 proxy sums, zero between passes
+    int32_t *blk_cnt;            // [C] CTAs done per column block, zero between passes
     int32_t *ucount;             // [C]
     int32_t *tcount;             // [C][B]
     uint32_t *ulist;             // [C][kCB]  channel | token bits << 24
@@ -127,6 +152,7 @@ struct Stage2Args {
                                  // channel position of CTA 0 (-1: off)
     int nstage;
     int max_ch;                  // capacity of the per-CTA channel list
+    unsigned long long *stamps;  // phase stamps (StampSlot) or null
 };
 
 struct Stage2UArgs {
@@ -148,12 +174,18 @@ struct Stage2UArgs {
     int32_t *tile_cnt;           // [f / 64] K blocks summed per tile (cleared)
     uint16_t *sb;                // [f / 64][2][8][64] s hi / lo tiles, 128-byte swizzled
     uint32_t *pos_ch;            // [f] union entry per position
+    unsigned long long *stamps;  // phase stamps (StampSlot: entry, go, end) or null
 };
 
 cudaError_t launch_stage2_umma(int B, const Stage2UArgs &a, int grid, cudaStream_t s);
 
 cudaError_t launch_stage1(int B, const Stage1Args &a, const Stage1Plan &p,
                           cudaStream_t s);
+// tensor-core Stage 1 for passes of <= 4 tokens (k_stage1_tc.cu): its plan
+// (false if the shape is outside it) and launch (grid a.C * a.n_r)
+bool stage1_tc_plan(int d_model, int d_ff, int B, int num_sms, int *n_r, int *unit_cap,
+                    size_t *smem);
+cudaError_t launch_stage1_tc(int B, const Stage1Args &a, size_t smem, cudaStream_t s);
 cudaError_t launch_stage2(int B, int nchunk, const Stage2Args &a, int grid,
                           size_t smem, cudaStream_t s);
 cudaError_t launch_rmsnorm(int d, int nb, const float *h, float eps, uint16_t *x,
@@ -252,6 +284,14 @@ __device__ __forceinline__ uint64_t global_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
+}
+
+// phase stamps: no-ops unless the pass was launched with a stamp buffer
+__device__ __forceinline__ void stamp_min(unsigned long long *st, int k) {
+    if (st) atomicMin(st + k, (unsigned long long)global_ns());
+}
+__device__ __forceinline__ void stamp_max(unsigned long long *st, int k) {
+    if (st) atomicMax(st + k, (unsigned long long)global_ns());
 }
 
 // Bounded wait on the phase of `bar` with the given parity: gives up and

@@ -93,6 +93,8 @@ def lib() -> C.CDLL:
         L.prox_ffn_stage2.argtypes = [C.POINTER(_Layer), vp, i, vp, vp, vp, vp, sz, vp]
         L.prox_test_set_wait.argtypes = [C.c_uint32, i]
         L.prox_test_set_wait.restype = None
+        L.prox_test_set_stamps.argtypes = [vp]
+        L.prox_test_set_stamps.restype = None
         for name in ("prox_quantize_proxy", "prox_ffn_forward", "prox_ffn_forward_static",
                      "prox_rmsnorm_bf16", "prox_ffn_block", "prox_calibrate_histogram",
                      "prox_bf16_proxy",
@@ -502,6 +504,28 @@ def last_device_status(ws: torch.Tensor) -> tuple[int, int]:
 def test_set_wait(wait_us: int = 0, skip_position: int = -1) -> None:
     """Test hook (prox_testing.h): shorter bounded waits / one unfilled stage."""
     lib().prox_test_set_wait(int(wait_us), int(skip_position))
+
+
+STAMP_SLOTS = 16
+# stamp slots that hold a minimum over CTAs (all others hold a maximum)
+STAMP_MIN_SLOTS = (0, 1, 8, 9, 12)
+
+
+def stamp_buffer(n_passes: int, device) -> torch.Tensor:
+    """Zeroed int64 [n_passes][16] buffer for prox_test_set_stamps."""
+    return torch.zeros((n_passes, STAMP_SLOTS), dtype=torch.int64, device=device)
+
+
+def reset_stamps(buf: torch.Tensor) -> None:
+    """Minimum slots to all ones (as unsigned), maximum slots to zero."""
+    buf.zero_()
+    buf[:, list(STAMP_MIN_SLOTS)] = -1
+
+
+def test_set_stamps(ptr: int) -> None:
+    """Measurement hook (prox_testing.h): passes launched while ptr != 0
+    record phase stamps at that device address (16 uint64 slots)."""
+    lib().prox_test_set_stamps(C.c_void_p(int(ptr)) if ptr else None)
 
 
 def untile_proxy(q):

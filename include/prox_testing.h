@@ -21,6 +21,22 @@ extern "C" {
 
 void prox_test_set_wait(uint32_t wait_us, int skip_position);
 
+/*
+ * prox_test_set_stamps: measurement hook. While `slots` is non-NULL, every
+ * CUDA-core forward pass launched (or captured into a CUDA graph) records
+ * %globaltimer phase stamps of its two kernels into slots[0..15], device
+ * memory owned by the caller: each slot is the minimum or the maximum over
+ * the kernel's CTAs of the time one phase began or ended (Stage 1: entry,
+ * past the wait for the previous kernel, stream start, stream end, partials
+ * summed, end; Stage 2: entry, past the wait for Stage 1, channel list
+ * ready, first stage full, last channel accumulated, end). The caller sets
+ * the minimum slots (0, 1, 8, 9, 12) to all ones and the others to zero
+ * before the pass runs. NULL turns stamping off. The stamps are a few
+ * atomics per CTA; the results of the pass are unchanged. Host-side state,
+ * affects launches made after the call; not thread-safe.
+ */
+void prox_test_set_stamps(unsigned long long *slots);
+
 #ifdef __cplusplus
 }
 #endif

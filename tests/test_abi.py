@@ -205,9 +205,26 @@ def test_stage2_engine_switch():
 
 
 def test_workspace_holds_tensor_core_buffers():
-    # passes of >= 4 tokens add partial sums, split counters, s tiles and
-    # union positions: f*2*B*4 + (f/128)*4 + (f/64)*2048 + f*4 bytes (rounded)
+    # every pass: status word, per-block counts, union list and per-token lists;
+    # passes of <= 4 tokens add the tensor-core Stage 1's int64 proxy sums and
+    # block counters (2*B*f*8 + C*4 bytes); passes of >= 4 tokens the
+    # tensor-core Stage 2's partial sums, split counters, s tiles and union
+    # positions (f*2*B*4 + (f/64)*4 + (f/64)*2048 + f*4 bytes)
     d, f = 4096, 12288
-    extra = P.workspace_bytes(d, f, 8) - (P.workspace_bytes(d, f, 2) + 6 * f * 4 + 6 * 48 * 4)
-    assert extra >= f * 2 * 8 * 4 + (f // 128) * 4 + (f // 64) * 2048 + f * 4
+    C = f // 256
+
+    def lists(B):
+        return 256 + C * 4 + C * B * 4 + C * 256 * 4 + B * f * 4
+
+    def s1_tc(B):
+        return 2 * B * f * 8 + C * 4
+
+    def s2_tc(B):
+        return f * 2 * B * 4 + (f // 64) * 4 + (f // 64) * 2048 + f * 4
+
+    assert P.workspace_bytes(d, f, 1) >= lists(1) + s1_tc(1)
+    assert P.workspace_bytes(d, f, 2) >= lists(2) + s1_tc(2)
+    assert P.workspace_bytes(d, f, 4) >= lists(4) + s1_tc(4) + s2_tc(4)
+    assert P.workspace_bytes(d, f, 8) >= lists(8) + s2_tc(8)
     assert P.workspace_bytes(d, f, 1000) <= P.STATIC_WORKSPACE_BYTES
+    assert P.workspace_bytes(d, f, 4) <= P.STATIC_WORKSPACE_BYTES

@@ -98,14 +98,43 @@ def test_stage2_traffic_scaled_to_the_mean_token():
     # for the workload and batch the capture covers
     sys.path.insert(0, ROOT)
     import bench
-    fields = {}
-    for line in open(os.path.join(ROOT, "profiles", "k_stage2_qwen3-8b-ffn_b1.md")):
-        if line.startswith("- ") and ":" in line:
-            k, v = line[2:].split(":", 1)
-            fields[k.strip()] = v.strip()
+    fields = bench.summary_fields(os.path.join(ROOT, "profiles", "k_stage2_qwen3-8b-ffn_b1.md"))
     traffic = float(fields["dram bytes per launch (read + write)"])
     captured = float(fields["algorithmic bytes of the captured launch"].split()[0])
-    got = bench.stage2_traffic("qwen3-8b-ffn", 1, 90537600.0)
+    got = bench.traffic_from_summary(fields, 90537600.0)
     assert got is not None and abs(got - traffic * 90537600.0 / captured) < 1.0
+    assert bench.traffic_from_summary({}, 1.0) is None
     assert bench.stage2_traffic("qwen3-8b-ffn", 8, 1.0) is None
     assert bench.stage2_traffic("large-ffn", 1, 1.0) is None
+
+
+def test_stamp_phases_add_up_to_the_call():
+    # two adjacent calls' stamps (ns): stage1 + stage2 is the call, and each
+    # sub-phase is the difference of its slots
+    sys.path.insert(0, ROOT)
+    import numpy as np
+
+    import bench
+    NONE = -1
+    a = np.zeros(16, dtype=np.int64)
+    b = np.zeros(16, dtype=np.int64)
+    base = 10_000_000
+    a[[0, 1, 2, 3, 4, 5, 6]] = base + np.array([0, 1000, 1200, 2000, 6000, 6500, 7500])
+    a[[8, 9, 10, 11, 12, 13, 14, 15]] = base + np.array([500, 8000, 8100, 8900, 9500, 9800,
+                                                         24000, 25000])
+    b[[0, 1]] = base + np.array([24500, 26000])
+    b[8] = b[9] = b[12] = NONE
+    st = np.stack([a, b])
+    ph = bench.stamp_phases(st, [0, 1], {0: 0, 1: 1})
+    assert ph["pairs"] == 1
+    assert abs(ph["stage1"] - 7.0) < 1e-9 and abs(ph["stage2"] - 18.0) < 1e-9
+    assert abs(ph["call"] - (ph["stage1"] + ph["stage2"])) < 1e-9
+    assert abs(ph["s1_prologue"] - 1.0) < 1e-9 and abs(ph["s1_stream"] - 4.0) < 1e-9
+    assert abs(ph["s1_exit_to_s2_go"] - 0.5) < 1e-9
+    assert abs(ph["s2_list"] - 0.9) < 1e-9 and abs(ph["s2_first_data"] - 0.9) < 1e-9
+    assert abs(ph["s2_stream_window"] - 14.5) < 1e-9 and abs(ph["s2_tail"] - 1.0) < 1e-9
+    assert abs(ph["s2_exit_to_next_s1_go"] - 1.0) < 1e-9
+    # a call whose Stage 2 left no stamps (slots still at their reset values) is skipped
+    st2 = st.copy()
+    st2[0, 9] = NONE
+    assert bench.stamp_phases(st2, [0, 1], {0: 0, 1: 1})["pairs"] == 0

@@ -585,3 +585,89 @@ def test_tc1_matches_simt_c2(c2):
     err = (s_a - s_b).abs().max().item() / c2.tau_s
     print(f"[tc1 vs simt c2 b=8] max |ds~| / tau_s = {err:.2e}")
     assert err < 3e-4
+
+
+# ---------------------------------------------------------------------------
+# tensor-core Stage 1 for passes of 1, 2 and 4 tokens (k_stage1_tc: exact
+# int64 proxy sums over 27-bit fixed-point digits of x * scale, summed across
+# the CTAs of a column block in global memory)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("engine", [P.ENGINE_TC, P.ENGINE_SIMT])
+@pytest.mark.parametrize("b", [1, 2, 3, 4])
+def test_stage1_small_engines_proxy_state_c2(c2, engine, b):
+    # s~ of one pass of b tokens against the oracle with either Stage-1 engine
+    with P.stage1_engine(engine):
+        _proxy_check(c2, list(range(40, 40 + b)))
+
+
+@pytest.mark.parametrize("b", [1, 2, 3, 4, 7])
+def test_tc1s_forward_c1(c1, b):
+    rows = list(range(10, 10 + b))
+    with P.stage1_engine(P.ENGINE_TC):
+        out = P.ffn_forward(c1.layer, c1.xdev(rows), c1.tau_x, c1.tau_s)
+    check_forward(c1, rows, out, f" c1 tc1s b={b}")
+
+
+@pytest.mark.parametrize("b", [1, 2, 4])
+def test_tc1s_forward_c2(c2, b):
+    # four calls of b tokens on one workspace
+    rows = list(range(64, 64 + 4 * b))
+    ws = P.workspace(4096, 12288, b)
+    with P.stage1_engine(P.ENGINE_TC):
+        outs = [P.ffn_forward(c2.layer, c2.xdev(rows[k:k + b]), c2.tau_x, c2.tau_s, ws)
+                for k in range(0, len(rows), b)]
+    merged = P.ForwardOut(*(torch.cat([getattr(o, k) for o in outs]) for k in
+                            ("y", "mask_x", "mask_s", "idx_s", "count_s")))
+    check_forward(c2, rows, merged, f" c2 tc1s b={b}")
+
+
+def test_tc1s_exact_across_splits_and_repeats(c2):
+    # the proxy sums are exact integers on one fixed-point grid: the same
+    # token gives bit-identical s~ alone, as the first or the last token of a
+    # 4-token pass, and on every repeat (the accumulators and block counters
+    # are left at zero by each pass)
+    x = c2.xdev(list(range(120, 124)))
+    ws = P.workspace(c2.layer.d_model, c2.layer.d_ff, 4, "cuda")
+    with P.stage1_engine(P.ENGINE_TC):
+        s1, _ = P.proxy_state(c2.layer, x[:1], c2.tau_x, ws=ws)
+        s4a, _ = P.proxy_state(c2.layer, x, c2.tau_x, ws=ws)
+        s4b, _ = P.proxy_state(c2.layer, x, c2.tau_x, ws=ws)
+        s1b, _ = P.proxy_state(c2.layer, x[:1], c2.tau_x, ws=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(s4a, s4b)
+    assert torch.equal(s1, s1b)
+    # the fixed-point exponent is per token, so a token's sums do not depend
+    # on the other tokens of its pass
+    assert torch.equal(s1[0], s4a[0])
+    st, flags = P.last_device_status(ws)
+    assert st == P.PROX_OK and flags == 0
+
+
+def test_tc1s_matches_simt_c2(c2):
+    x = c2.xdev(list(range(300, 304)))
+    with P.stage1_engine(P.ENGINE_SIMT):
+        s_a, mx_a = P.proxy_state(c2.layer, x, c2.tau_x)
+    with P.stage1_engine(P.ENGINE_TC):
+        s_b, mx_b = P.proxy_state(c2.layer, x, c2.tau_x)
+    torch.cuda.synchronize()
+    assert torch.equal(mx_a, mx_b)
+    err = (s_a - s_b).abs().max().item() / c2.tau_s
+    print(f"[tc1s vs simt c2 b=4] max |ds~| / tau_s = {err:.2e}")
+    assert err < 3e-4
+
+
+def test_tc1s_nothing_kept_and_all_kept_c1(c1):
+    rows = [0, 1]
+    with P.stage1_engine(P.ENGINE_TC):
+        out = P.ffn_forward(c1.layer, c1.xdev(rows), 1e30, 1e30)
+        torch.cuda.synchronize()
+        assert int(out.mask_x.sum()) == 0
+        assert float(out.y.abs().max()) == 0.0
+        dense = P.ffn_forward(c1.layer, c1.xdev(rows), 0.0, 0.0)
+    torch.cuda.synchronize()
+    assert int(dense.mask_x.sum()) == 2 * c1.layer.d_model
+    ref = oracle.forward(c1.x[rows], 0.0, 0.0, c1.L, c1.Por, want=())["y"]
+    y = dense.y.cpu().numpy().astype(np.float64)
+    rel = np.linalg.norm(y - ref, axis=1) / np.linalg.norm(ref, axis=1)
+    assert rel.max() <= Y_TOL
