@@ -316,7 +316,7 @@ __device__ void s1_tc_stream(const Stage1Args &a, unsigned char *region, const i
     __shared__ int s_F[2][kMaxB];
     __shared__ int s_S[2][kMaxB][4];
     __shared__ uint32_t s_tmem;
-    __shared__ __align__(8) uint64_t s_done[1];
+    __shared__ __align__(8) uint64_t s_done[2];   // [0]: a group's MMAs, [1]: all MMAs
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const uint32_t rb = (smem_addr(region) + 1023u) & ~1023u;
     constexpr int GR = s1tc_group(NB);                // tile buffers (one group)
@@ -330,6 +330,7 @@ __device__ void s1_tc_stream(const Stage1Args &a, unsigned char *region, const i
     if (tid < 2 * kMaxB * 4) (&s_S[0][0][0])[tid] = 0;
     if (tid == 0) {
         mbar_init(&s_done[0], 1);
+        mbar_init(&s_done[1], 1);
         mbar_fence_init();
     }
     if (wid == 0) tmem_alloc(&s_tmem, TCOLS);
@@ -476,11 +477,16 @@ __device__ void s1_tc_stream(const Stage1Args &a, unsigned char *region, const i
                                 db, IDESC, ks > 0 ? 1u : 0u);
                 }
             }
-            umma_commit(&s_done[0]);
+            // test hook: in CTA 0 this group's completion is never signalled
+            if (!(a.debug_skip == g && blockIdx.x == 0)) umma_commit(&s_done[0]);
         }
     }
     if (ngrp > 0 && ok) ok = mbar_wait(&s_done[0], (ngrp - 1) & 1, a.wait_us);
     if (!ok) atomicOr(a.status, kStTimeoutMma);
+    // tensor memory is read and freed only once every MMA issued has completed
+    // (a wait that gave up may leave MMAs of later groups running)
+    if (tid == 0) umma_commit(&s_done[1]);
+    mbar_wait(&s_done[1], 0, kDefaultWaitUs);
     tc_fence_after();
     // epilogue: warp quadrant q reads TMEM lanes 32q..32q+31 (channels of an M
     // tile); the four groups of four warps take the (matrix, M tile) pairs

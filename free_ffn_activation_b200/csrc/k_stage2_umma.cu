@@ -127,7 +127,7 @@ __host__ __device__ inline UgSmem ug_smem(int nstage, int C, int span) {
     s.ring = o;
     o += (uint32_t)nstage * kUgStage;
     s.bars = o;
-    o += (uint32_t)(2 * nstage + 4) * 8;
+    o += (uint32_t)(2 * nstage + 5) * 8;
     s.misc = o;
     o += 16;
     s.xg = o;                                      // g of a tile, handed to the u warps
@@ -150,7 +150,7 @@ __host__ __device__ inline DnSmem dn_smem(int nstage, int cw, int rows_cap) {
     s.ring = o;
     o += (uint32_t)nstage * dn_stage(cw);
     s.bars = o;
-    o += (uint32_t)(2 * nstage + 4) * 8;
+    o += (uint32_t)(2 * nstage + 5) * 8;
     s.misc = o;
     o += 16;
     s.rows = o;
@@ -182,13 +182,14 @@ __device__ __forceinline__ void cp_arrive_noinc(uint64_t *bar) {
 }
 __device__ __forceinline__ void cp_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-// barriers of a kernel: full[NST], empty[NST], acc_full[2], acc_empty[2]
+// barriers of a kernel: full[NST], empty[NST], acc_full[2], acc_empty[2],
+// fin (every MMA the kernel issued is complete)
 struct Bars {
-    uint64_t *full, *empty, *acc_full, *acc_empty;
+    uint64_t *full, *empty, *acc_full, *acc_empty, *fin;
 };
 __device__ __forceinline__ Bars carve_bars(unsigned char *p, int nst) {
     uint64_t *b = reinterpret_cast<uint64_t *>(p);
-    return Bars{b, b + nst, b + 2 * nst, b + 2 * nst + 2};
+    return Bars{b, b + nst, b + 2 * nst, b + 2 * nst + 2, b + 2 * nst + 4};
 }
 __device__ __forceinline__ void init_bars(const Bars &b, int nst) {
     for (int s = 0; s < nst; ++s) {
@@ -199,6 +200,7 @@ __device__ __forceinline__ void init_bars(const Bars &b, int nst) {
         mbar_init(&b.acc_full[k], 1);
         mbar_init(&b.acc_empty[k], 128);
     }
+    mbar_init(b.fin, 1);
     mbar_fence_init();
 }
 
@@ -306,6 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_s2u_updown(const Stage2UArgs a)
                 if (t < a.nb)
                     cp16(st + 16384u + kmaj_off(t, c), a.x + (size_t)t * d + kb * kUK + c * 8);
             }
+            if (a.debug_skip == ls && blockIdx.x == 0) continue;  // test hook: never filled
             cp_arrive_noinc(&bar.full[stg]);
         }
         cp_wait_all();
@@ -337,6 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_s2u_updown(const Stage2UArgs a)
                     ++seg;
                 }
             }
+            umma_commit(bar.fin);  // also after a failed wait: no MMA is left running
         }
         __syncwarp();
     } else {
@@ -349,7 +353,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_s2u_updown(const Stage2UArgs a)
             const int kb1 = ((tile + 1) * NKB < S1 ? (tile + 1) * NKB : S1) - tile * NKB;
             const bool whole = (kb0 == 0 && kb1 == NKB);
             const int p = tile * kTile + (r & (kTile - 1));
-            cta_wait(&bar.acc_full[seg & 1], (seg >> 1) & 1, a, fail);
+            if (!cta_wait(&bar.acc_full[seg & 1], (seg >> 1) & 1, a, fail))
+                mbar_wait(bar.fin, 0, kDefaultWaitUs);  // no MMA running while TMEM is read
             tc_fence_after();
             float v[8];
             tmem_ld8(tmem + (uint32_t)(seg & 1) * kUN + ((uint32_t)(q * 32) << 16), v);
@@ -443,6 +448,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_s2u_updown(const Stage2UArgs a)
             if (lane == 0) a.count_s[wid] = sum;
         }
     }
+    // tensor memory is read and freed only once every MMA issued has completed
+    // (a bounded wait that gave up leaves MMAs issued before it)
+    mbar_wait(bar.fin, 0, kDefaultWaitUs);
     tc_fence_before();
     __syncthreads();
     if (wid == kMmaWarp) {
@@ -585,6 +593,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_s2u_down(const Stage2UArgs a) {
                     ++seg;
                 }
             }
+            umma_commit(bar.fin);  // also after a failed wait: no MMA is left running
         }
         __syncwarp();
     } else {
@@ -596,7 +605,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_s2u_down(const Stage2UArgs a) {
             const int pb = step % NPB;
             if (!(s == nsteps - 1 || pb == NPB - 1)) continue;
             const int mt = step / NPB;
-            cta_wait(&bar.acc_full[seg & 1], (seg >> 1) & 1, a, fail);
+            if (!cta_wait(&bar.acc_full[seg & 1], (seg >> 1) & 1, a, fail))
+                mbar_wait(bar.fin, 0, kDefaultWaitUs);  // no MMA running while TMEM is read
             tc_fence_after();
             float D[NM][8];
 #pragma unroll
@@ -614,6 +624,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_s2u_down(const Stage2UArgs a) {
             ++seg;
         }
     }
+    mbar_wait(bar.fin, 0, kDefaultWaitUs);
     tc_fence_before();
     __syncthreads();
     if (wid == kMmaWarp) {

@@ -200,6 +200,9 @@ static bool tau_ok(float t) { return std::isfinite(t) && t >= 0.f; }
 // test hooks (set by prox_debug_set through the binding's test helpers only)
 static uint32_t g_spin_limit = kDefaultWaitUs;
 static int g_debug_skip = -1;
+// prox_test_set_skip: which kernel's arrival CTA 0 skips (kSkip*) and where
+static int g_skip_where = 0, g_skip_pos = -1;
+constexpr int kSkipStage1Tc = 1, kSkipStage2Tc = 3;
 // measurement hook (prox_test_set_stamps): phase stamps of the next passes
 static unsigned long long *g_stamps = nullptr;
 
@@ -277,6 +280,7 @@ static prox_status pass_stage1(const prox_layer *L, const uint16_t *x, int nb, f
     }
     a.wait_us = g_spin_limit;
     a.stamps = g_stamps;
+    a.debug_skip = g_skip_where == kSkipStage1Tc ? g_skip_pos : -1;
     a.status = reinterpret_cast<uint32_t *>(w + W.status);
     a.ucount = reinterpret_cast<int32_t *>(w + W.ucount);
     a.tcount = reinterpret_cast<int32_t *>(w + W.tcount);
@@ -290,6 +294,9 @@ static prox_status pass_stage1(const prox_layer *L, const uint16_t *x, int nb, f
         a.tc = 1;
         a.acc = reinterpret_cast<long long *>(w + W.acc);
         a.blk_cnt = reinterpret_cast<int32_t *>(w + W.blk_cnt);
+        // the sums and block counters start from zero (the region also holds
+        // other data when the workspace served another shape or batch)
+        if (cudaMemsetAsync(w + W.acc, 0, W.total - W.acc, st) != cudaSuccess) return PROX_ECUDA;
         return launch_stage1_tc(B, a, smem, st) == cudaSuccess ? PROX_OK : PROX_ECUDA;
     }
     return launch_stage1(B, a, p1, st) == cudaSuccess ? PROX_OK : PROX_ECUDA;
@@ -334,6 +341,7 @@ static prox_status pass_stage2(const prox_layer *L, const uint16_t *x, int nb, f
         u.sb = reinterpret_cast<uint16_t *>(w + W.sb);
         u.pos_ch = reinterpret_cast<uint32_t *>(w + W.pos_ch);
         u.stamps = g_stamps;
+        u.debug_skip = g_skip_where == kSkipStage2Tc ? g_skip_pos : -1;
         return launch_stage2_umma(B, u, sms, st) == cudaSuccess ? PROX_OK : PROX_ECUDA;
     }
     const int max_ch = (f + sms - 1) / sms + 1;
@@ -490,6 +498,19 @@ PROX_API prox_status prox_ffn_forward_static(const prox_layer *layer, const uint
     if (ps != PROX_OK) return ps;
     return run_forward(layer, x, batch, tau_x, tau_s, y, mask_x, mask_s, idx_s, count_s, nullptr,
                        ws, kStaticWsBytes, (cudaStream_t)stream, true);
+}
+
+PROX_API prox_status prox_static_last_device_status(void *stream, uint32_t *flags_out) {
+    void *ws = nullptr;
+    prox_status ps = static_workspace(&ws);
+    if (ps != PROX_OK) return ps;
+    cudaStream_t st = (cudaStream_t)stream;
+    uint32_t v = 0;
+    if (cudaMemcpyAsync(&v, ws, sizeof v, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaMemsetAsync(ws, 0, sizeof v, st) != cudaSuccess || cudaStreamSynchronize(st) != cudaSuccess)
+        return PROX_ECUDA;
+    if (flags_out) *flags_out = v;
+    return v ? PROX_ETIMEOUT : PROX_OK;
 }
 
 static bool eps_ok(float e) { return std::isfinite(e) && e >= 0.f; }
@@ -776,6 +797,13 @@ PROX_API const char *prox_status_str(prox_status s) {
 PROX_API void prox_test_set_wait(uint32_t spin_limit, int skip_position) {
     prox::g_spin_limit = spin_limit ? spin_limit : kDefaultWaitUs;
     prox::g_debug_skip = skip_position;
+}
+
+// Test hook, not part of prox.h: in CTA 0 of the tensor-core kernels, one
+// arrival never happens, so that a bounded wait runs out (see prox_testing.h)
+PROX_API void prox_test_set_skip(int where, int position) {
+    prox::g_skip_where = where;
+    prox::g_skip_pos = position;
 }
 
 // Measurement hook, not part of prox.h: passes launched while `slots` is set

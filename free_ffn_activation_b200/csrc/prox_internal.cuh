@@ -124,11 +124,13 @@ struct Stage1Args {
     int z_n16;                   // its size in 16-byte words
     uint32_t wait_us;            // wall-clock bound of each wait, microseconds
     unsigned long long *stamps;  // phase stamps (StampSlot) or null
+    int debug_skip;              // test hook: in CTA 0 of a tensor-core pass, this K
+                                 // step (group) never completes (-1: off)
     // workspace
     uint32_t *status;
     long long *acc;              // tensor-core Stage 1 (<= 4 tokens): [2][B][f] exact
-                                 // int64 proxy sums, zero between passes
-    int32_t *blk_cnt;            // [C] CTAs done per column block, zero between passes
+                                 // int64 proxy sums, cleared before the pass
+    int32_t *blk_cnt;            // [C] CTAs done per column block, cleared before the pass
     int32_t *ucount;             // [C]
     int32_t *tcount;             // [C][B]
     uint32_t *ulist;             // [C][kCB]  channel | token bits << 24
@@ -175,6 +177,8 @@ struct Stage2UArgs {
     uint16_t *sb;                // [f / 64][2][8][64] s hi / lo tiles, 128-byte swizzled
     uint32_t *pos_ch;            // [f] union entry per position
     unsigned long long *stamps;  // phase stamps (StampSlot: entry, go, end) or null
+    int debug_skip;              // test hook: the up/gate loaders of CTA 0 never
+                                 // complete this step (-1: off)
 };
 
 cudaError_t launch_stage2_umma(int B, const Stage2UArgs &a, int grid, cudaStream_t s);

@@ -91,16 +91,20 @@ def lib() -> C.CDLL:
         L.prox_max_batch_per_pass.restype = C.c_int
         L.prox_ffn_stage1.argtypes = [C.POINTER(_Layer), vp, i, f, f, vp, vp, vp, vp, sz, vp]
         L.prox_ffn_stage2.argtypes = [C.POINTER(_Layer), vp, i, vp, vp, vp, vp, sz, vp]
+        L.prox_static_last_device_status.argtypes = [vp, C.POINTER(C.c_uint32)]
         L.prox_test_set_wait.argtypes = [C.c_uint32, i]
         L.prox_test_set_wait.restype = None
         L.prox_test_set_stamps.argtypes = [vp]
         L.prox_test_set_stamps.restype = None
+        L.prox_test_set_skip.argtypes = [i, i]
+        L.prox_test_set_skip.restype = None
         for name in ("prox_quantize_proxy", "prox_ffn_forward", "prox_ffn_forward_static",
                      "prox_rmsnorm_bf16", "prox_ffn_block", "prox_calibrate_histogram",
                      "prox_bf16_proxy",
                      "prox_proxy_state",
                      "prox_ffn_stage1", "prox_ffn_stage2",
-                     "prox_calibrate", "prox_allocate", "prox_last_device_status"):
+                     "prox_calibrate", "prox_allocate", "prox_last_device_status",
+                     "prox_static_last_device_status"):
             getattr(L, name).restype = C.c_int
         _lib = L
     return _lib
@@ -501,6 +505,24 @@ def last_device_status(ws: torch.Tensor) -> tuple[int, int]:
     return st, flags.value
 
 
+def static_last_device_status(device=None) -> tuple[int, int]:
+    """(status, raw flags) of the static array's status word (the array of
+    ffn_forward_static on the current device); clears it."""
+    flags = C.c_uint32()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    st = lib().prox_static_last_device_status(_stream(dev), C.byref(flags))
+    return st, flags.value
+
+
+SKIP_OFF, SKIP_STAGE1_TC, SKIP_STAGE2_TC = 0, 1, 3
+
+
+def test_set_skip(where: int, position: int = -1) -> None:
+    """Test hook (prox_testing.h): one arrival in CTA 0 of a tensor-core
+    kernel never happens, so that its bounded wait runs out."""
+    lib().prox_test_set_skip(int(where), int(position))
+
+
 def test_set_wait(wait_us: int = 0, skip_position: int = -1) -> None:
     """Test hook (prox_testing.h): shorter bounded waits / one unfilled stage."""
     lib().prox_test_set_wait(int(wait_us), int(skip_position))
@@ -554,4 +576,5 @@ __all__ = ["ProxLayer", "ProxError", "quantize_proxy", "workspace", "workspace_b
            "max_batch_per_pass", "set_stage2_engine", "stage2_engine", "set_stage1_engine",
            "stage1_engine", "ENGINE_AUTO",
            "ENGINE_SIMT", "ENGINE_TC", "proxy_state", "calibrate", "allocate",
-           "last_device_status", "touched_bytes", "untile_proxy", "as_bf16"]
+           "last_device_status", "static_last_device_status", "touched_bytes", "untile_proxy",
+           "as_bf16"]

@@ -178,11 +178,10 @@ prox_status prox_ffn_forward(const prox_layer *layer, const uint16_t *x, int bat
  *   Sharing: every call on a device uses the same array, so calls must not
  *     overlap on the device (one stream, or ordered by the caller); two
  *     overlapping calls race on it.
- *   Zero state: the array starts zero-filled (static device storage). The
- *     only part that must be zero at a call's start is the status word, which
- *     the kernels set only when a bounded wait gives up; such a timeout is not
- *     reported here (use prox_ffn_forward with prox_last_device_status to
- *     observe timeouts).
+ *   Timeouts: the array starts zero-filled (static device storage). When a
+ *     bounded device-side wait gives up, the kernels set a bit of its status
+ *     word and return early, and this call has still returned PROX_OK: read
+ *     (and clear) that word with prox_static_last_device_status.
  * Errors: as prox_ffn_forward; PROX_ENOMEM for a shape over the limit;
  * PROX_ECUDA if the symbol lookup fails.
  */
@@ -191,6 +190,16 @@ prox_status prox_ffn_forward_static(const prox_layer *layer, const uint16_t *x, 
                                     float tau_x, float tau_s, float *y, uint8_t *mask_x,
                                     uint8_t *mask_s, int32_t *idx_s, int32_t *count_s,
                                     void *stream);
+
+/*
+ * prox_static_last_device_status -- prox_last_device_status for the array of
+ * prox_ffn_forward_static on the current device: copies its status word to
+ * *flags_out (if not NULL) and clears it, after the work queued on `stream`
+ * (synchronises `stream`). Returns PROX_ETIMEOUT if a bounded wait gave up
+ * since the last read, else PROX_OK; PROX_ECUDA on a failed copy or lookup.
+ * The first use on a device looks the array up like the forward does.
+ */
+prox_status prox_static_last_device_status(void *stream, uint32_t *flags_out);
 
 /*
  * Layer stacks. The Prox pages define one FFN; a stack of FFN layers (as in

@@ -37,6 +37,23 @@ void prox_test_set_wait(uint32_t wait_us, int skip_position);
  */
 void prox_test_set_stamps(unsigned long long *slots);
 
+/*
+ * prox_test_set_skip: makes one arrival in CTA 0 of a tensor-core kernel
+ * never happen, so that the bounded wait on it runs out (use with a short
+ * bound from prox_test_set_wait). `where`:
+ *   1  Stage 1 on the tensor cores: for passes of 1-4 tokens, warp 0 never
+ *      signals K step `position` ready (status bit 4); for passes of 8 tokens,
+ *      the MMA thread never signals group `position` done (status bit 5);
+ *   3  the tensor-core Stage 2: the up/gate loaders never complete their
+ *      step `position` (status bit 5);
+ *   0  off.
+ * Nothing faults: the kernel records the timeout in the status word, skips
+ * the rest of its MMAs, waits (with the default bound) for those already
+ * issued, frees its tensor memory and returns. Host-side state, affects
+ * launches made after the call; not thread-safe.
+ */
+void prox_test_set_skip(int where, int position);
+
 #ifdef __cplusplus
 }
 #endif

@@ -18,40 +18,9 @@ import torch
 import oracle
 from free_ffn_activation_b200 import prox as P
 from free_ffn_activation_b200 import synth as S
+from parity_helpers import BAND, Y_TOL, Case, check_forward, to_dev_bf16  # noqa: F401
 
 pytestmark = pytest.mark.gpu
-
-BAND = 1e-3
-Y_TOL = 2e-3
-
-
-def to_dev_bf16(a, dev):
-    return P.as_bf16(a, dev).contiguous()
-
-
-class Case:
-    """One layer with its oracle proxies, device layer and thresholds."""
-
-    def __init__(self, d, f, n_tok, n_cal, sigma=0.02, seed=0, outlier=0.0, layer=0,
-                 keep_x=0.5, keep_s=0.3, dev="cuda", act=oracle.ACT_SWIGLU,
-                 proxy_kind=P.PROXY_INT4):
-        self.spec = S.LayerSpec(d, f, sigma=sigma, seed=seed, layer=layer)
-        self.L = S.make_layer(self.spec)
-        self.Por = (oracle.make_proxy_bf16(self.L) if proxy_kind == P.PROXY_BF16
-                    else oracle.make_proxy(self.L))
-        self.dev = dev
-        self.act = act
-        self.layer = P.ProxLayer.from_weights(self.L["w_up_cm"], self.L["w_gate_cm"],
-                                              self.L["w_down"], device=dev, activation=act,
-                                              proxy_kind=proxy_kind)
-        self.x = S.make_tokens(n_tok, d, seed=seed, stream="x_eval", outlier_frac=outlier)
-        self.x_cal = S.make_tokens(n_cal, d, seed=seed, stream="x_cal", outlier_frac=outlier)
-        self.keep_x, self.keep_s = keep_x, keep_s
-        self.tau_x, self.tau_s = oracle.calibrate(self.x_cal, self.Por, keep_x, keep_s, act=act)
-
-    def xdev(self, rows=None):
-        x = self.x if rows is None else self.x[rows]
-        return to_dev_bf16(x, self.dev)
 
 
 @pytest.fixture(scope="module")
@@ -93,39 +62,6 @@ def c2b(gpu):
 def c1g(gpu):
     # the tiny layer with a GeGLU gate (GELU instead of SiLU)
     return Case(256, 768, 64, 256, act=oracle.ACT_GEGLU)
-
-
-def check_forward(case, rows, out, tag=""):
-    """Compare a device ForwardOut for tokens `rows` with the oracle."""
-    x = case.x[rows]
-    ref = oracle.forward(x, case.tau_x, case.tau_s, case.L, case.Por, act=case.act)
-    mx = out.mask_x.cpu().numpy()
-    ms = out.mask_s.cpu().numpy()
-    idx = out.idx_s.cpu().numpy()
-    cnt = out.count_s.cpu().numpy()
-    assert np.array_equal(mx, ref["mask_x"]), f"{tag} mask_x differs"
-    sabs = np.abs(ref["s_proxy"])
-    band = np.abs(sabs - case.tau_s) <= BAND * case.tau_s
-    diff = ms != ref["mask_s"]
-    assert not np.any(diff & ~band), f"{tag} m_s differs outside the band"
-    n_band = int(band.sum())
-    if band.size >= 20000:   # the 0.1% rule is a rate: checked on large samples
-        assert n_band < 1e-3 * band.size, f"{tag} band holds {n_band} of {band.size}"
-    for t in range(len(rows)):
-        kept = np.flatnonzero(ms[t])
-        assert cnt[t] == kept.size
-        assert np.array_equal(idx[t, :cnt[t]], kept), f"{tag} idx_s token {t}"
-    y_ref = oracle.forward(x, case.tau_x, case.tau_s, case.L, case.Por, mask_s_in=ms,
-                           want=(), act=case.act)["y"]
-    y = out.y.cpu().numpy().astype(np.float64)
-    num = np.linalg.norm(y - y_ref, axis=1)
-    den = np.maximum(np.linalg.norm(y_ref, axis=1), 1e-30)
-    worst = float((num / den).max())
-    assert worst <= Y_TOL, f"{tag} y rel err {worst}"
-    print(f"[parity{tag}] tokens={len(rows)} band={n_band}/{band.size} "
-          f"mask_s diffs={int(diff.sum())} y_rel_max={worst:.2e} "
-          f"keep_x={mx.mean():.3f} keep_s={ms.mean():.3f}")
-    return worst
 
 
 # ---------------------------------------------------------------------------
@@ -312,14 +248,16 @@ def test_forward_c1_batched(c1, b):
     check_forward(c1, rows, out, f" c1 b={b}")
 
 
-def test_forward_c2_sampled_b1(c2):
-    # full-size layer in the launch configuration the benchmark times (b = 1)
+def test_forward_c2_all_tokens_b1(c2):
+    # the full-size layer in the launch configuration the benchmark times
+    # (one token per call, one workspace), on all 512 of its tokens
     ws = P.workspace(4096, 12288, 1)
-    rows = [0, 1, 2, 63, 128, 255, 300, 511]
+    rows = list(range(512))
     outs = [P.ffn_forward(c2.layer, c2.xdev([t]), c2.tau_x, c2.tau_s, ws) for t in rows]
     merged = P.ForwardOut(*(torch.cat([getattr(o, k) for o in outs]) for k in
                             ("y", "mask_x", "mask_s", "idx_s", "count_s")))
-    check_forward(c2, rows, merged, " c2 b=1")
+    check_forward(c2, rows, merged, " c2 b=1 all tokens")
+    assert P.last_device_status(ws) == (P.PROX_OK, 0)
 
 
 @pytest.mark.parametrize("b", [2, 4, 8])
@@ -405,6 +343,37 @@ def test_bounded_wait_timeout_reports_status(c1):
     out = P.ffn_forward(c1.layer, c1.xdev([1]), c1.tau_x, c1.tau_s, ws)
     check_forward(c1, [1], out, " after-timeout")
     assert P.last_device_status(ws)[0] == P.PROX_OK
+
+
+@pytest.mark.parametrize("where,n_tok,engine,bit", [
+    (P.SKIP_STAGE1_TC, 1, P.ENGINE_TC, 1 << 4),    # Stage 1 on the tensor cores, 1 token
+    (P.SKIP_STAGE1_TC, 8, P.ENGINE_TC, 1 << 5),    # tensor-core proxy products, 8 tokens
+    (P.SKIP_STAGE2_TC, 8, P.ENGINE_AUTO, 1 << 5),  # tensor-core Stage 2
+])
+def test_tensor_core_wait_timeouts(c2, where, n_tok, engine, bit):
+    # one arrival in CTA 0 never happens (test hook) and the bounded wait on it
+    # runs out (2 ms): the kernel records the timeout, skips its remaining
+    # MMAs, waits for the issued ones, frees tensor memory and returns; the
+    # status reader reports it, and the next call on the workspace is whole
+    rows = list(range(40, 40 + n_tok))
+    ws = P.workspace(4096, 12288, n_tok)
+    x = c2.xdev(rows)
+    assert P.last_device_status(ws) == (P.PROX_OK, 0)
+    try:
+        P.test_set_wait(wait_us=2000, skip_position=-1)
+        P.test_set_skip(where, 1)
+        with P.stage1_engine(engine):
+            P.ffn_forward(c2.layer, x, c2.tau_x, c2.tau_s, ws)
+        torch.cuda.synchronize()
+    finally:
+        P.test_set_skip(P.SKIP_OFF, -1)
+        P.test_set_wait(0, -1)
+    st, flags = P.last_device_status(ws)
+    assert st == P.PROX_ETIMEOUT and (flags & bit), (st, flags)
+    with P.stage1_engine(engine):
+        out = P.ffn_forward(c2.layer, x, c2.tau_x, c2.tau_s, ws)
+    check_forward(c2, rows, out, f" after a timeout (hook {where}, {n_tok} tokens)")
+    assert P.last_device_status(ws) == (P.PROX_OK, 0)
 
 
 def test_split_stages_equal_forward(c2):
