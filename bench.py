@@ -73,6 +73,10 @@ def parse():
     ap.add_argument("--no-dense", action="store_true", help="skip the dense cuBLAS reference")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the compact records of the other workloads (sparsity and "
+                         "batch sweeps, the 8192 x 28672 layer, the 36-layer stack)")
+    ap.add_argument("--sec-steps", type=int, default=3, help="timed steps of each secondary record")
     return ap.parse_args()
 
 
@@ -254,53 +258,242 @@ class ClockSampler:
 # reference arm: the fp64 CPU oracle, timed on the host cores
 # ---------------------------------------------------------------------------
 
-def cpu_oracle_time(w, keep_x, keep_s, seconds):
-    """Time the oracle on a bounded token sample; returns (us/token, cores, sample)."""
+def band_count(s_abs, tau_s, rel=1e-3):
+    """Channels whose |s~| lies within rel * tau_s of tau_s (the mask band)."""
+    import numpy as np
+    return int(np.count_nonzero(np.abs(np.asarray(s_abs, dtype=np.float64) - tau_s) <= rel * tau_s))
+
+
+def cpu_oracle_time(w, x, tau_x, tau_s, seconds):
+    """The fp64 oracle on a bounded sample of the workload's tokens `x`, at the
+    given thresholds (the GPU arm's): returns (us/token, threads, sample string,
+    oracle band count, channels compared, realised keep_x, keep_s)."""
+    import numpy as np
+
     import oracle
     from free_ffn_activation_b200 import synth as S
     L = S.make_layer(S.LayerSpec(w["d"], w["f"], sigma=w["sigma"], seed=0))
     Por = oracle.make_proxy(L)
-    x_cal = S.make_tokens(min(w["n_cal"], 64), w["d"], stream="x_cal", outlier_frac=w["outlier"])
-    tau_x, tau_s = oracle.calibrate(x_cal, Por, keep_x, keep_s)
-    x = S.make_tokens(w["tokens"], w["d"], stream="x_eval", outlier_frac=w["outlier"])
     cores = os.cpu_count() or 1
     done, t_used, threads = 0, 0.0, 1
-    chunk = max(1, cores)
-    while done < w["tokens"] and t_used < seconds:
-        n = min(chunk, w["tokens"] - done)
+    band, kx, ks = 0, 0.0, 0.0
+    while done < x.shape[0] and t_used < seconds:
+        n = min(max(1, cores), x.shape[0] - done)
         t0 = time.perf_counter()
-        out = oracle.forward(x[done:done + n], tau_x, tau_s, L, Por, want=())
+        out = oracle.forward(x[done:done + n], tau_x, tau_s, L, Por, want=("mask_x", "mask_s", "s_proxy"))
         t_used += time.perf_counter() - t0
         threads = out["threads"]
+        band += band_count(np.abs(out["s_proxy"]), tau_s)
+        kx += float(out["mask_x"].sum())
+        ks += float(out["mask_s"].sum())
         done += n
     # the same path on one thread, over the first two tokens of the sample
     t0 = time.perf_counter()
     oracle.forward(x[0:2], tau_x, tau_s, L, Por, n_threads=1, want=())
     us_one = (time.perf_counter() - t0) / 2 * 1e6
-    sample = (f"{done} of {w['tokens']} tokens of the {w['d']}x{w['f']} layer "
-              f"(thresholds from {x_cal.shape[0]} calibration vectors), all stages, fp64, "
-              f"{threads} threads (one thread, 2 tokens: {us_one:.0f} us/token)")
-    return t_used / done * 1e6, threads, sample
+    sample = (f"{done} of {x.shape[0]} tokens of the {w['d']}x{w['f']} layer at the GPU arm's "
+              f"thresholds, all stages, fp64, {threads} threads (one thread, 2 tokens: "
+              f"{us_one:.0f} us/token); realised keep_x {kx / (done * w['d']):.4f}, "
+              f"keep_s {ks / (done * w['f']):.4f}")
+    return t_used / done * 1e6, threads, sample, band, done * w["f"]
 
 
 def run_reference(args, w, rank, world):
+    """The fp64 CPU oracle as the reference arm: thresholds calibrated by the
+    oracle on the same calibration vectors as the GPU arm (n_cal of them), then
+    W untimed and K timed steps, each over a bounded sample of the workload's
+    tokens (the whole workload would take minutes per step)."""
     if rank != 0:
         return
-    us, cores, sample = cpu_oracle_time(w, args.keep_x, args.keep_s, args.cpu_seconds)
-    ms_step = us * w["tokens"] / 1e3
+    import numpy as np
+
+    import oracle
+    from free_ffn_activation_b200 import synth as S
+    L = S.make_layer(S.LayerSpec(w["d"], w["f"], sigma=w["sigma"], seed=0))
+    Por = oracle.make_proxy(L)
+    x_cal = S.make_tokens(w["n_cal"], w["d"], seed=0, stream="x_cal", outlier_frac=w["outlier"])
+    t0 = time.perf_counter()
+    tau_x, tau_s = oracle.calibrate(x_cal, Por, args.keep_x, args.keep_s)
+    cal_s = time.perf_counter() - t0
+    x = S.make_tokens(w["tokens"], w["d"], seed=0, stream="x_eval", outlier_frac=w["outlier"])
+    cores = os.cpu_count() or 1
+    per_step = min(w["tokens"], max(16, cores))
+    times, threads, done = [], 1, 0
+    for it in range(args.warmup + args.steps):
+        rows = [(done + k) % w["tokens"] for k in range(per_step)]
+        done += per_step
+        t0 = time.perf_counter()
+        out = oracle.forward(x[rows], tau_x, tau_s, L, Por, want=())
+        dt = time.perf_counter() - t0
+        threads = out["threads"]
+        if it >= args.warmup:
+            times.append(dt)
+    ms_step = float(np.mean(times)) * 1e3
+    us = ms_step * 1e3 / per_step
+    sample = (f"{per_step} of {w['tokens']} tokens per step (consecutive, wrapping), "
+              f"{args.steps} timed steps after {args.warmup}, all stages, fp64, {threads} threads; "
+              f"thresholds calibrated by the oracle on {w['n_cal']} vectors ({cal_s:.1f} s)")
     line = {
         "impl": "reference", "metric": METRIC, "value": us, "unit": "us/token/layer",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": False, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": args.workload, "d_model": w["d"], "d_ff": w["f"], "batch": 1,
-                   "tokens_per_step": w["tokens"], "keep_x": args.keep_x, "keep_s": args.keep_s},
-        "cpu_baseline": {"value": us, "unit": "us/token/layer", "cores": cores,
+                   "tokens_per_step": per_step, "workload_tokens": w["tokens"],
+                   "n_cal": w["n_cal"], "keep_x": args.keep_x, "keep_s": args.keep_s,
+                   "tau_x": tau_x, "tau_s": tau_s},
+        "cpu_baseline": {"value": us, "unit": "us/token/layer", "cores": threads,
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": us, "unit": "us/token/layer", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# secondary records: the other workloads of the benchmark, in the same run
+# ---------------------------------------------------------------------------
+
+def graph_us_per_token(P, torch, dev, stream, calls, ntok, steps, warmup):
+    """Capture `calls` (a list of zero-argument launch functions, one forward
+    call each) in one CUDA graph and return device us per token over `steps`
+    timed replays after `warmup` (CUDA events on the launching stream)."""
+    def one():
+        for fn in calls:
+            fn()
+    with torch.cuda.stream(stream):
+        one()
+    torch.cuda.synchronize(dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        one()
+    for _ in range(warmup):
+        with torch.cuda.stream(stream):
+            g.replay()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        with torch.cuda.stream(stream):
+            g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    del g
+    return e0.elapsed_time(e1) / steps * 1e3 / ntok
+
+
+def sparse_calls(P, structs, x, y, ws, Bt, tau_x, tau_s, stream):
+    d = x.shape[1]
+    R = len(structs)
+    ntok = x.shape[0]
+    return [(lambda c=c: P.ffn_forward_raw(structs[c % R], x.data_ptr() + c * Bt * d * 2, Bt,
+                                           tau_x, tau_s, y.data_ptr() + c * Bt * d * 4,
+                                           ws.data_ptr(), ws.numel(), stream.cuda_stream))
+            for c in range(ntok // Bt)]
+
+
+def dense_calls(torch, layers, x, Bt):
+    """torch bf16 F.linear x3 + silu*mul (cuBLAS) per call of Bt tokens."""
+    import torch.nn.functional as F
+    wd_t = [lay.w_down.t().contiguous() for lay in layers]
+    yd = torch.empty(x.shape, dtype=torch.bfloat16, device=x.device)
+    R = len(layers)
+
+    def call(c):
+        lay = layers[c % R]
+        xt = x[c * Bt:(c + 1) * Bt]
+        yd[c * Bt:(c + 1) * Bt] = F.linear(F.silu(F.linear(xt, lay.w_gate_cm)) * F.linear(xt, lay.w_up_cm),
+                                           wd_t[c % R])
+    return [(lambda c=c: call(c)) for c in range(x.shape[0] // Bt)], wd_t
+
+
+def touched_per_call(P, base, x, Bt, tau_x, tau_s):
+    """Mean weight bytes one call of Bt tokens touches, and the realised
+    per-token keep ratios (an untimed forward)."""
+    d, f = base.d_model, base.d_ff
+    out = P.ffn_forward(base, x, tau_x, tau_s)
+    n = x.shape[0] // Bt
+    kx = out.mask_x.view(n, Bt, d).amax(dim=1).sum(dim=1).double().cpu().numpy()
+    ks = out.mask_s.view(n, Bt, f).amax(dim=1).sum(dim=1).double().cpu().numpy()
+    tb = sum(P.touched_bytes(d, f, int(a), int(b)) for a, b in zip(kx, ks)) / n
+    return tb, out.mask_x.float().mean().item(), out.mask_s.float().mean().item()
+
+
+def secondary_records(args, dev, base, layers, structs, x, x_cal, dense_b1_us, peak):
+    """Compact records of the sparsity sweep and batch sweep on the same layer,
+    the 8192 x 28672 layer at batch 1 and 16, and the 36-layer stack (fewer
+    timed steps than the primary measurement; same protocol)."""
+    import torch
+
+    from free_ffn_activation_b200 import prox as P
+    from free_ffn_activation_b200 import synth as S
+    out = {"steps": args.sec_steps, "warmup": 2}
+    stream = torch.cuda.Stream(dev)
+    d, f = base.d_model, base.d_ff
+    ntok = x.shape[0]
+    y = torch.empty((ntok, d), dtype=torch.float32, device=dev)
+
+    def sparse_point(tx, ts, Bt):
+        ws = P.workspace(d, f, Bt, dev)
+        us = graph_us_per_token(P, torch, dev, stream, sparse_calls(P, structs, x, y, ws, Bt, tx, ts, stream),
+                                ntok, args.sec_steps, 2)
+        tb, kx, ks = touched_per_call(P, base, x, Bt, tx, ts)
+        return {"us_per_token": us, "keep_x": kx, "keep_s": ks,
+                "path_GBps": tb / (us * Bt * 1e-6) / 1e9}
+
+    # sparsity sweep at batch 1 (input keep fixed at 50%)
+    sweep = []
+    for keep_s in (1.0, 0.7, 0.5, 0.4, 0.3, 0.2, 0.1):
+        tx, ts = P.calibrate(base, x_cal, args.keep_x, keep_s)
+        r = sparse_point(tx, ts, 1)
+        r.update({"channel_sparsity": round(1.0 - keep_s, 3), "dense_us_per_token": dense_b1_us,
+                  "speedup": dense_b1_us / r["us_per_token"]})
+        sweep.append(r)
+    out["qwen3-8b-ffn sparsity sweep, batch 1"] = sweep
+    # batch sweep at 70% channel sparsity (each token its own masks)
+    tx, ts = P.calibrate(base, x_cal, args.keep_x, args.keep_s)
+    bsw = []
+    for Bt in (1, 2, 4, 8):
+        r = sparse_point(tx, ts, Bt)
+        calls, _ = dense_calls(torch, layers, x, Bt)
+        du = graph_us_per_token(P, torch, dev, stream, calls, ntok, args.sec_steps, 2)
+        r.update({"batch": Bt, "dense_us_per_token": du, "speedup": du / r["us_per_token"]})
+        bsw.append(r)
+    out["qwen3-8b-ffn batch sweep, 70% channel sparsity"] = bsw
+    del y
+    torch.cuda.empty_cache()
+
+    # the 8192 x 28672 layer (1.41 GB of bf16 weights: larger than L2 as it is)
+    wl = WORKLOADS["large-ffn"]
+    Ll = S.make_layer(S.LayerSpec(wl["d"], wl["f"], sigma=wl["sigma"], seed=0))
+    big = P.ProxLayer.from_weights(Ll["w_up_cm"], Ll["w_gate_cm"], Ll["w_down"], device=dev)
+    del Ll
+    xl = P.as_bf16(S.make_tokens(wl["tokens"], wl["d"], seed=0, stream="x_eval"), dev).contiguous()
+    xlc = P.as_bf16(S.make_tokens(wl["n_cal"], wl["d"], seed=0, stream="x_cal"), dev)
+    txl, tsl = P.calibrate(big, xlc, args.keep_x, args.keep_s)
+    yl = torch.empty((wl["tokens"], wl["d"]), dtype=torch.float32, device=dev)
+    bl = []
+    for Bt in (1, 16):
+        ws = P.workspace(wl["d"], wl["f"], Bt, dev)
+        us = graph_us_per_token(P, torch, dev, stream,
+                                sparse_calls(P, [big.cstruct()], xl, yl, ws, Bt, txl, tsl, stream),
+                                wl["tokens"], args.sec_steps, 2)
+        tb, kx, ks = touched_per_call(P, big, xl, Bt, txl, tsl)
+        calls, _ = dense_calls(torch, [big], xl, Bt)
+        du = graph_us_per_token(P, torch, dev, stream, calls, wl["tokens"], args.sec_steps, 2)
+        bl.append({"batch": Bt, "us_per_token": us, "dense_us_per_token": du,
+                   "speedup": du / us, "keep_x": kx, "keep_s": ks,
+                   "path_GBps": tb / (us * Bt * 1e-6) / 1e9, "path_frac": tb / (us * Bt * 1e-6) / 1e9 / peak})
+    out["large-ffn 8192x28672, 70% channel sparsity"] = bl
+    del big, xl, yl
+    torch.cuda.empty_cache()
+
+    # the 36-layer stack (per token, every layer; 128 decode tokens)
+    ws_ = WORKLOADS["qwen3-8b-stack36"]
+    out["qwen3-8b-stack36, 70% channel sparsity per layer, batch 1"] = stack_measure(
+        args, ws_, dev, 1, 0, steps=args.sec_steps, warmup=1, e2e=False)
+    return out
 
 
 # ---------------------------------------------------------------------------
@@ -325,7 +518,8 @@ def run_ours(args, w, rank, world, local_rank):
     pk = P.PROXY_BF16 if args.proxy == "bf16" else P.PROXY_INT4
     base = P.ProxLayer.from_weights(L["w_up_cm"], L["w_gate_cm"], L["w_down"], device=dev,
                                     proxy_kind=pk)
-    tau_x, tau_s = P.calibrate(base, P.as_bf16(xc_np, dev), args.keep_x, args.keep_s)
+    xc = P.as_bf16(xc_np, dev)
+    tau_x, tau_s = P.calibrate(base, xc, args.keep_x, args.keep_s)
     R = max(1, args.copies)
     layers = [base] + [P.ProxLayer(*(None if t is None else t.clone() for t in (
         base.w_up_cm, base.w_gate_cm, base.w_down, base.q_up, base.q_gate, base.s_up, base.s_gate)),
@@ -350,6 +544,14 @@ def run_ours(args, w, rank, world, local_rank):
     stage2_bytes = 3 * ks * d * 2
     kx_tok = out.mask_x.sum(dim=1).double().mean().item()
     ks_tok = out.count_s.double().mean().item()
+    # the mask band (channels whose |s~| lies within 1e-3 tau_s of tau_s) on the
+    # benchmark's own tokens, from the device's proxy state (untimed)
+    nband = 0
+    for c in range(ngrp):
+        s_dev, _ = P.proxy_state(base, x[c * Bt:(c + 1) * Bt], tau_x)
+        nband += int(((s_dev.abs() - tau_s).abs() <= 1e-3 * tau_s).sum().item())
+    band = {"rel": 1e-3, "device_band": nband, "channels": ntok * f,
+            "device_band_frac": nband / (ntok * f)}
 
     stream = torch.cuda.Stream(dev)
     sp = stream.cuda_stream
@@ -506,11 +708,25 @@ def run_ours(args, w, rank, world, local_rank):
                  "kind": "torch F.linear x3 + silu*mul (cuBLAS), bf16, same graph/L2 protocol"}
         del gd
 
+    secondary = None
+    if world == 1 and not args.no_secondary and args.workload == "qwen3-8b-ffn" and Bt == 1 \
+            and args.proxy == "int4" and dense is not None:
+        t_sec = time.perf_counter()
+        try:
+            secondary = secondary_records(args, dev, base, layers, structs, x, xc,
+                                          dense["us_per_token"], peak)
+        except Exception as exc:  # a secondary record never voids the primary one
+            secondary = {"error": f"{type(exc).__name__}: {exc}"}
+        secondary["wall_s"] = time.perf_counter() - t_sec
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
-        us_cpu, cores, sample = cpu_oracle_time(w, args.keep_x, args.keep_s, args.cpu_seconds)
+        us_cpu, cores, sample, oband, ochan = cpu_oracle_time(w, x_np, tau_x, tau_s, args.cpu_seconds)
         cpu = {"value": us_cpu, "unit": "us/token/layer", "cores": cores, "kind": "oracle",
                "sample": sample}
+        band["oracle_band"] = oband
+        band["oracle_channels"] = ochan
+        band["oracle_band_frac"] = oband / max(1, ochan)
 
     if rank == 0:
         line = {
@@ -536,6 +752,7 @@ def run_ours(args, w, rank, world, local_rank):
                        "bytes_per_launch": s1_bytes, "GBps": s1_gbs, "frac": s1_gbs / peak},
             "phases_us": ph,
             "device_status": status,
+            "band": band,
             "effective_sparsity": None if args.effective_sparsity is None else {
                 "target": args.effective_sparsity,
                 "realised": (1.0 - ks_tok / f) - 2.0 / 3.0 * (kx_tok / d) / 3.0,
@@ -550,24 +767,23 @@ def run_ours(args, w, rank, world, local_rank):
                     "h2d_bytes_per_step": ntok * d * 2, "d2h_bytes_per_step": ntok * d * 4},
             "gpu_launches": launches_per_call(args, d, Bt) * (ntok // Bt) * args.steps,
             "clocks": clk.summary(),
+            "secondary": secondary,
         }
         print(json.dumps(line), flush=True)
     del g
 
 
-def run_stack(args, w, rank, world, local_rank):
-    """A step is `tokens` decode tokens, each through all layers of the stack
-    (prox_ffn_block per layer: pre-norm, Prox FFN, residual add). The whole
-    stack is far larger than L2, so every layer streams from HBM."""
-    import numpy as np
+def stack_measure(args, w, dev, world, rank, steps, warmup, e2e=True, dense=True, clk=None):
+    """The layer stack: a step is `tokens` decode tokens, each through all
+    layers (prox_ffn_block per layer: pre-norm, Prox FFN, residual add). The
+    whole stack is far larger than L2, so every layer streams from HBM.
+    Returns a dict of the measurements (max over ranks)."""
     import torch
     import torch.distributed as dist
 
     from free_ffn_activation_b200 import prox as P
     from free_ffn_activation_b200 import synth as S
 
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
     d, f, ntok, nl = w["d"], w["f"], w["tokens"], w["layers"]
     eps = 1e-6
     layers = []
@@ -610,7 +826,7 @@ def run_stack(args, w, rank, world, local_rank):
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream):
         one_step()
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         with torch.cuda.stream(stream):
             g.replay()
     torch.cuda.synchronize(dev)
@@ -618,18 +834,19 @@ def run_stack(args, w, rank, world, local_rank):
         dist.barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local_rank) as clk:
+    with (clk if clk is not None else _Null()):
         e0.record(stream)
-        for _ in range(args.steps):
+        for _ in range(steps):
             with torch.cuda.stream(stream):
                 g.replay()
         e1.record(stream)
         torch.cuda.synchronize(dev)
-    ms_total = e0.elapsed_time(e1)
-    ms_total = max_over_ranks(ms_total, world, dev)
-    ms_step = ms_total / args.steps
+    ms_total = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    ms_step = ms_total / steps
     us_tok = ms_step * 1e3 / ntok                     # all layers, per token (per rank)
-    # touched bytes: realised keep ratios of the last step's tokens, layer by layer
+    status = P.last_device_status(ws)[1]
+    del g
+    # touched bytes: realised keep ratios of the step's tokens, layer by layer
     hh = h0.clone()
     touched = 0.0
     for ell, lay in enumerate(layers):
@@ -638,34 +855,40 @@ def run_stack(args, w, rank, world, local_rank):
         ks = out.count_s.double().mean().item()
         touched += P.touched_bytes(d, f, int(round(kx)), int(round(ks)))
     peak, peak_src = load_peaks()
-    path_gbs = touched / (us_tok * 1e-6) / 1e9
+    res = {"ms_per_step": ms_step, "us_per_token": us_tok, "us_per_layer": us_tok / nl,
+           "layers": nl, "tokens_per_step": ntok, "steps": steps, "warmup": warmup,
+           "device_status": status,
+           "path": {"touched_MB_per_token": touched / 1e6,
+                    "GBps": touched / (us_tok * 1e-6) / 1e9,
+                    "frac_of_peak": touched / (us_tok * 1e-6) / 1e9 / peak,
+                    "peak_source": peak_src}}
 
-    # e2e: host h in, host h out, the public call per layer
-    h_host = h0.cpu().pin_memory()
-    out_host = torch.empty((ntok, d), dtype=torch.float32).pin_memory()
+    if e2e:
+        # host h in, host h out, the public call per layer
+        h_host = h0.cpu().pin_memory()
+        out_host = torch.empty((ntok, d), dtype=torch.float32).pin_memory()
 
-    def e2e_step():
-        with torch.cuda.stream(stream):
-            h.copy_(h_host, non_blocking=True)
-            for t in range(ntok):
-                hp, xp = h.data_ptr() + t * hrow, xbuf.data_ptr() + t * xrow
-                for ell in range(nl):
-                    P.ffn_block_raw(structs[ell], hp, 1, taus[ell][0], taus[ell][1], eps, hp,
-                                    xp, wp, wsb, sp)
-            out_host.copy_(h, non_blocking=True)
+        def e2e_step():
+            with torch.cuda.stream(stream):
+                h.copy_(h_host, non_blocking=True)
+                for t in range(ntok):
+                    hp, xp = h.data_ptr() + t * hrow, xbuf.data_ptr() + t * xrow
+                    for ell in range(nl):
+                        P.ffn_block_raw(structs[ell], hp, 1, taus[ell][0], taus[ell][1], eps, hp,
+                                        xp, wp, wsb, sp)
+                out_host.copy_(h, non_blocking=True)
 
-    e2e_step()
-    torch.cuda.synchronize(dev)
-    f0 = torch.cuda.Event(enable_timing=True)
-    f1 = torch.cuda.Event(enable_timing=True)
-    f0.record(stream)
-    e2e_step()
-    f1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_us = f0.elapsed_time(f1) * 1e3 / ntok
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        f0 = torch.cuda.Event(enable_timing=True)
+        f1 = torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        e2e_step()
+        f1.record(stream)
+        torch.cuda.synchronize(dev)
+        res["e2e_us_per_token"] = max_over_ranks(f0.elapsed_time(f1), world, dev) * 1e3 / ntok
 
-    dense = None
-    if not args.no_dense:
+    if dense:
         import torch.nn.functional as F
         wd_t = [lay.w_down.t().contiguous() for lay in layers]
         hd = torch.empty_like(h0)
@@ -686,41 +909,61 @@ def run_stack(args, w, rank, world, local_rank):
         gd = torch.cuda.CUDAGraph()
         with torch.cuda.graph(gd, stream=stream):
             dense_step()
-        for _ in range(args.warmup):
+        for _ in range(warmup):
             with torch.cuda.stream(stream):
                 gd.replay()
         torch.cuda.synchronize(dev)
         d0 = torch.cuda.Event(enable_timing=True)
         d1 = torch.cuda.Event(enable_timing=True)
         d0.record(stream)
-        for _ in range(args.steps):
+        for _ in range(steps):
             with torch.cuda.stream(stream):
                 gd.replay()
         d1.record(stream)
         torch.cuda.synchronize(dev)
-        dense_us = d0.elapsed_time(d1) / args.steps * 1e3 / ntok
-        dense = {"us_per_token": dense_us, "speedup_of_sparse": dense_us / us_tok,
-                 "kind": "torch RMSNorm + F.linear x3 + silu*mul (cuBLAS), bf16, same protocol"}
-        del gd
+        dense_us = max_over_ranks(d0.elapsed_time(d1), world, dev) / steps * 1e3 / ntok
+        res["dense_ref"] = {"us_per_token": dense_us, "speedup_of_sparse": dense_us / us_tok,
+                            "kind": "torch RMSNorm + F.linear x3 + silu*mul (cuBLAS), bf16, same protocol"}
+        del gd, wd_t
+    del layers, structs
+    torch.cuda.empty_cache()
+    return res
 
+
+class _Null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        return False
+
+
+def run_stack(args, w, rank, world, local_rank):
+    import torch
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    with ClockSampler(local_rank) as clk:
+        r = stack_measure(args, w, dev, world, rank, args.steps, args.warmup, clk=clk)
     if rank == 0:
+        d, f, ntok, nl = w["d"], w["f"], w["tokens"], w["layers"]
         line = {
             "metric": "sparse SwiGLU FFN stack µs/token (all layers) @70% sparsity",
-            "value": ms_step * 1e3 / (ntok * world),
+            "value": r["us_per_token"] / world,
             "unit": "us/token", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": ms_step, "higher_is_better": False, "scaling": "weak",
+            "ms_per_step": r["ms_per_step"], "higher_is_better": False, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": args.workload, "layers": nl, "d_model": d, "d_ff": f,
                        "batch": 1, "tokens_per_step": ntok, "keep_x": args.keep_x,
-                       "keep_s": args.keep_s, "rmsnorm_eps": eps,
+                       "keep_s": args.keep_s, "rmsnorm_eps": 1e-6,
                        "l2": f"{nl} distinct layers ({nl * (3 * d * f * 2 + d * f + 8 * d) / 1e9:.1f} GB > L2)",
                        "parallelism": f"replicas x{world}"},
-            "us_per_layer": us_tok / nl,
-            "path": {"touched_MB_per_token": touched / 1e6, "GBps": path_gbs,
-                     "frac_of_peak": path_gbs / peak, "peak_source": peak_src},
-            "dense_ref": dense,
-            "e2e": {"value": e2e_us, "unit": "us/token", "h2d_bytes_per_step": ntok * d * 4,
-                    "d2h_bytes_per_step": ntok * d * 4},
+            "us_per_layer": r["us_per_layer"],
+            "path": r["path"],
+            "dense_ref": r.get("dense_ref"),
+            "device_status": r["device_status"],
+            "e2e": {"value": r["e2e_us_per_token"] / world, "unit": "us/token",
+                    "h2d_bytes_per_step": ntok * d * 4, "d2h_bytes_per_step": ntok * d * 4},
             "gpu_launches": 3 * nl * ntok * args.steps,
             "clocks": clk.summary(),
         }

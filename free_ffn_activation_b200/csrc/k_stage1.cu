@@ -919,8 +919,7 @@ cudaError_t launch1(Stage1Args a, const Stage1Plan &p0, cudaStream_t s) {
             p.depth_sel = s1_depth_sel(a.d, B, NB, p.unit_cap, PK, TC);
             if (p.depth_sel < 0) return cudaErrorInvalidConfiguration;
             p.smem = s1_smem(a.d, B, NB, p.unit_cap, p.depth_sel, kS1MaxRowGroups, PK, TC).total;
-            cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 (int)p.smem);
+            cudaError_t e = set_max_dynamic_smem((const void *)k, p.smem);
             if (e != cudaSuccess) return e;
             if (p.n_r <= n_min) break;
             cudaLaunchConfig_t q = {};
