@@ -27,7 +27,7 @@ ABI_FUNCTIONS = (
     "prox_set_stage1_engine",
 )
 
-# Stage-2 engines (prox_set_stage2_engine)
+# Stage-2 and Stage-1 engines (prox_set_stage2_engine, prox_set_stage1_engine)
 ENGINE_AUTO, ENGINE_SIMT, ENGINE_TC = 0, 1, 2
 
 

@@ -108,8 +108,8 @@ def test_quantize_bit_exact_c2(c2):
 # Stage 1 values, calibration
 # ---------------------------------------------------------------------------
 
-def _proxy_check(case, rows):
-    s_gpu, mx = P.proxy_state(case.layer, case.xdev(rows), case.tau_x)
+def _proxy_check(case, rows, ws=None):
+    s_gpu, mx = P.proxy_state(case.layer, case.xdev(rows), case.tau_x, ws=ws)
     s_gpu = s_gpu.cpu().numpy().astype(np.float64)
     ref = np.stack([oracle.stage1(case.x[t], case.tau_x, case.Por["q_up"], case.Por["s_up"],
                                   case.Por["q_gate"], case.Por["s_gate"], case.tau_s,
@@ -566,8 +566,11 @@ def test_tc1_matches_simt_c2(c2):
 @pytest.mark.parametrize("b", [1, 2, 3, 4])
 def test_stage1_small_engines_proxy_state_c2(c2, engine, b):
     # s~ of one pass of b tokens against the oracle with either Stage-1 engine
+    ws = P.workspace(c2.layer.d_model, c2.layer.d_ff, b, "cuda")
     with P.stage1_engine(engine):
-        _proxy_check(c2, list(range(40, 40 + b)))
+        _proxy_check(c2, list(range(40, 40 + b)), ws=ws)
+    st, flags = P.last_device_status(ws)
+    assert st == P.PROX_OK and flags == 0
 
 
 @pytest.mark.parametrize("b", [1, 2, 3, 4, 7])
