@@ -229,35 +229,38 @@ __device__ __forceinline__ void s1_stream(const uint8_t *qbase, unsigned char *r
     using T = S1<B, NB, PK>;
     // slot-major ring (ring[slot][thread]): a warp's accesses to one slot are
     // consecutive words, free of bank conflicts
-    unsigned char *myring = ring + (size_t)threadIdx.x * T::BYTES;
+    unsigned char *const myring = ring + (size_t)threadIdx.x * T::BYTES;
     constexpr int SLOT = kS1Threads * T::BYTES;  // bytes between a thread's slots
+    unsigned char *const ring_end = myring + D * SLOT;
     const uint64_t pol = l2_evict_first();      // each granule is read once per pass
+    // walking pointers: the next row to copy, the slot and x of the row to use
+    const int *rp = rowidx + rl;
+    const float *xp = xs + (rl * 2 + m) * B;
+    unsigned char *sp = myring;
+    // one copy per loop iteration (no unrolled run of hinted copies)
 #pragma unroll 1
     for (int k = 0; k < D; ++k) {
-        if (k < n_rows)
-            cp_async<T::BYTES>(myring + k * SLOT, qbase + (size_t)rowidx[rl + k * T::RL] * T::GRAN,
-                               pol);
+        if (k < n_rows) {
+            cp_async<T::BYTES>(myring + k * SLOT, qbase + (size_t)*rp * T::GRAN, pol);
+            rp += T::RL;
+        }
         cp_commit();
     }
-#pragma unroll 1
-    for (int k = 0; k < n_rows; ++k) {
-        cp_wait<D - 1>();
-        const int u = rl + k * T::RL;
-        const int slot = k % D;
+    auto use = [&]() {
         uint32_t w[T::WORDS];
         if constexpr (T::WORDS == 4) {
-            const uint4 v = *reinterpret_cast<const uint4 *>(myring + slot * SLOT);
+            const uint4 v = *reinterpret_cast<const uint4 *>(sp);
             w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
         } else if constexpr (T::WORDS == 2) {
-            const uint2 v = *reinterpret_cast<const uint2 *>(myring + slot * SLOT);
+            const uint2 v = *reinterpret_cast<const uint2 *>(sp);
             w[0] = v.x; w[1] = v.y;
         } else {
-            w[0] = *reinterpret_cast<const uint32_t *>(myring + slot * SLOT);
+            w[0] = *reinterpret_cast<const uint32_t *>(sp);
         }
         float xv[B];
 #pragma unroll
         for (int t = 0; t < B; ++t) {
-            xv[t] = xs[(u * 2 + m) * B + t];
+            xv[t] = xp[t];
             ssum[t] += xv[t];
         }
 #pragma unroll
@@ -267,11 +270,29 @@ __device__ __forceinline__ void s1_stream(const uint8_t *qbase, unsigned char *r
             else
                 proc_word_bf16<B, T::CPT>(w[q], q, xv, acc2);
         }
-        const int kn = k + D;
-        if (kn < n_rows)
-            cp_async<T::BYTES>(myring + slot * SLOT, qbase + (size_t)rowidx[rl + kn * T::RL] * T::GRAN,
-                               pol);
+    };
+    // rows 0 .. n_rows - D - 1: each refills its slot with the row D later
+    int k = 0;
+#pragma unroll 1
+    for (; k < n_rows - D; ++k) {
+        cp_wait<D - 1>();
+        use();
+        cp_async<T::BYTES>(sp, qbase + (size_t)*rp * T::GRAN, pol);
+        rp += T::RL;
         cp_commit();
+        xp += T::RL * 2 * B;
+        sp += SLOT;
+        if (sp == ring_end) sp = myring;
+    }
+    // the last D rows (empty groups keep the wait count)
+#pragma unroll 1
+    for (; k < n_rows; ++k) {
+        cp_wait<D - 1>();
+        use();
+        cp_commit();
+        xp += T::RL * 2 * B;
+        sp += SLOT;
+        if (sp == ring_end) sp = myring;
     }
     cp_wait<0>();
 }
