@@ -67,6 +67,7 @@ __host__ __device__ inline S2Smem s2_smem(int d, int B, int nstage, int C, int m
     o += (size_t)B * (C + 1) * 4;
     s.chan = o;
     o += (size_t)max_ch * 4;
+    o = (o + 15) & ~(size_t)15;  // 16-byte copies of the list blocks
     s.chanpf = o;
     o += (size_t)kS2Prefetch * kCB * 4;
     s.total = (o + 127) & ~(size_t)127;
@@ -136,6 +137,8 @@ __global__ void __launch_bounds__(s2_threads(B), 1) k_stage2(const Stage2Args a)
             *reinterpret_cast<uint4 *>(xh + (size_t)t * d + ci * 8) = v;
         }
     }
+    // x and the barriers are in place before Stage 1 has finished
+    __syncthreads();
     // Stage 1's lists are ready once it has completed. One round trip brings
     // the per-block counts and the list blocks this CTA most likely owns
     // (those around block g * C / G).
@@ -144,6 +147,7 @@ __global__ void __launch_bounds__(s2_threads(B), 1) k_stage2(const Stage2Args a)
         stamp_min(a.stamps, kS2Go);
         stamp_max(a.stamps, kS2GoMax);
     }
+    asm volatile("griddepcontrol.launch_dependents;");
     // (G is one CTA per SM, so every product below fits in 32 bits)
     const int G = gridDim.x, g = blockIdx.x;
     const int npf = C < kS2Prefetch ? C : kS2Prefetch;
@@ -151,114 +155,174 @@ __global__ void __launch_bounds__(s2_threads(B), 1) k_stage2(const Stage2Args a)
     cpf = cpf < 0 ? 0 : (cpf > C - npf ? C - npf : cpf);
     // per-token counts only when per-token lists or counts are requested
     const bool tok = a.idx_s != nullptr || a.count_s != nullptr;
-    constexpr int NT = s2_threads(B);
-    // Warp 0 takes the union counts into registers (4 per lane covers
-    // C <= 128 column blocks; more go through shared memory), every thread a
-    // share of the likely list blocks and, when asked for, of the per-token
-    // counts: all loads of this round trip are issued before any is used.
-    constexpr int PER = 4;
-    const bool creg = C <= 32 * PER;
-    int cnt[PER];
+    int n_ch;
+    if (!tok && C <= 32 * 4) {
+        // Every warp reads the union counts itself (lane l owns blocks 4 l ..
+        // 4 l + 3) and derives this CTA's share [U g / G, U (g + 1) / G); the
+        // producer warp also takes the likely list blocks in the same round
+        // trip, scans the counts into shared memory and builds its channel
+        // list, so its first copies go out with no CTA-wide barrier.
+        const bool prod = wid == kNDot + NDOWN;
+        int cnt[4];
 #pragma unroll
-    for (int k = 0; k < PER; ++k) cnt[k] = 0;
-    if (wid == 0 && creg) {
+        for (int k = 0; k < 4; ++k) cnt[k] = lane * 4 + k < C ? a.ucount[lane * 4 + k] : 0;
+        uint4 pf[kS2Prefetch * kCB / 4 / 32];
+        if (prod) {
 #pragma unroll
-        for (int k = 0; k < PER; ++k)
-            if (lane * PER + k < C) cnt[k] = a.ucount[lane * PER + k];
-    }
-    {
-        const int nuc = creg ? 0 : C;          // union counts via shared memory
-        const int ntc = tok ? C * B : 0;       // per-token counts
-        const int total = nuc + ntc + npf * kCB;
-        for (int base = tid; base < total; base += 4 * NT) {
-            uint32_t v[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int k = base + q * NT;
-                v[q] = 0;
-                if (k < nuc) v[q] = (uint32_t)a.ucount[k];
-                else if (k < nuc + ntc) v[q] = (uint32_t)a.tcount[k - nuc];
-                else if (k < total) v[q] = a.ulist[(size_t)cpf * kCB + (k - nuc - ntc)];
+            for (int q = 0; q < kS2Prefetch * kCB / 4 / 32; ++q) {
+                const int e = (q * 32 + lane) * 4;  // first of 4 list entries
+                pf[q] = e < npf * kCB
+                            ? *reinterpret_cast<const uint4 *>(a.ulist + (size_t)cpf * kCB + e)
+                            : make_uint4(0u, 0u, 0u, 0u);
             }
+        }
+        const int loc = cnt[0] + cnt[1] + cnt[2] + cnt[3];
+        int inc = loc;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int k = base + q * NT;
-                if (k < nuc) {
-                    uscan[k] = (int)v[q];
-                } else if (k < nuc + ntc) {
-                    const int c = (k - nuc) / B, t = (k - nuc) % B;
-                    tscan[t * (C + 1) + c] = (int)v[q];
-                } else if (k < total) {
-                    chanpf[k - nuc - ntc] = v[q];
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += v;
+        }
+        const unsigned U = (unsigned)__shfl_sync(0xffffffffu, inc, 31);
+        const int p0 = (int)(U * g / G);
+        n_ch = (int)(U * (g + 1) / G) - p0;
+        if (prod) {
+            int run = inc - loc;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                if (lane * 4 + k < C) uscan[lane * 4 + k] = run;
+                run += cnt[k];
+            }
+            if (lane == 31) uscan[C] = inc;
+#pragma unroll
+            for (int q = 0; q < kS2Prefetch * kCB / 4 / 32; ++q) {
+                const int e = (q * 32 + lane) * 4;
+                if (e < npf * kCB) *reinterpret_cast<uint4 *>(chanpf + e) = pf[q];
+            }
+            __syncwarp();
+            for (int n = lane; n < n_ch; n += 32) {
+                const int pp = p0 + n;
+                int lo = 0, hi = C - 1;  // block cb with uscan[cb] <= pp < uscan[cb + 1]
+                while (lo < hi) {
+                    const int mid = (lo + hi + 1) >> 1;
+                    if (uscan[mid] <= pp) lo = mid; else hi = mid - 1;
+                }
+                const int off = pp - uscan[lo];
+                chan[n] = (lo >= cpf && lo < cpf + npf) ? chanpf[(lo - cpf) * kCB + off]
+                                                        : a.ulist[(size_t)lo * kCB + off];
+            }
+            __syncwarp();
+            if (lane == 0) stamp_max(a.stamps, kS2List);
+        }
+    } else {
+        constexpr int NT = s2_threads(B);
+        // Warp 0 takes the union counts into registers (4 per lane covers
+        // C <= 128 column blocks; more go through shared memory), every thread a
+        // share of the likely list blocks and, when asked for, of the per-token
+        // counts: all loads of this round trip are issued before any is used.
+        constexpr int PER = 4;
+        const bool creg = C <= 32 * PER;
+        int cnt[PER];
+#pragma unroll
+        for (int k = 0; k < PER; ++k) cnt[k] = 0;
+        if (wid == 0 && creg) {
+#pragma unroll
+            for (int k = 0; k < PER; ++k)
+                if (lane * PER + k < C) cnt[k] = a.ucount[lane * PER + k];
+        }
+        {
+            const int nuc = creg ? 0 : C;          // union counts via shared memory
+            const int ntc = tok ? C * B : 0;       // per-token counts
+            const int total = nuc + ntc + npf * kCB;
+            for (int base = tid; base < total; base += 4 * NT) {
+                uint32_t v[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int k = base + q * NT;
+                    v[q] = 0;
+                    if (k < nuc) v[q] = (uint32_t)a.ucount[k];
+                    else if (k < nuc + ntc) v[q] = (uint32_t)a.tcount[k - nuc];
+                    else if (k < total) v[q] = a.ulist[(size_t)cpf * kCB + (k - nuc - ntc)];
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int k = base + q * NT;
+                    if (k < nuc) {
+                        uscan[k] = (int)v[q];
+                    } else if (k < nuc + ntc) {
+                        const int c = (k - nuc) / B, t = (k - nuc) % B;
+                        tscan[t * (C + 1) + c] = (int)v[q];
+                    } else if (k < total) {
+                        chanpf[k - nuc - ntc] = v[q];
+                    }
                 }
             }
         }
-    }
-    __syncthreads();
-    // Exclusive scans of the per-block counts: warp 0 the union counts (in
-    // registers), warp 1 + t those of token t (in place). A lane owns
-    // contiguous counts, so one shuffle scan suffices.
-    if (wid == 0 && creg) {
-        int loc = 0;
+        __syncthreads();
+        // Exclusive scans of the per-block counts: warp 0 the union counts (in
+        // registers), warp 1 + t those of token t (in place). A lane owns
+        // contiguous counts, so one shuffle scan suffices.
+        if (wid == 0 && creg) {
+            int loc = 0;
 #pragma unroll
-        for (int k = 0; k < PER; ++k) loc += cnt[k];
-        int inc = loc;
+            for (int k = 0; k < PER; ++k) loc += cnt[k];
+            int inc = loc;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int n = __shfl_up_sync(0xffffffffu, inc, o);
-            if (lane >= o) inc += n;
-        }
-        int run = inc - loc;
-#pragma unroll
-        for (int k = 0; k < PER; ++k) {
-            if (lane * PER + k < C) uscan[lane * PER + k] = run;
-            run += cnt[k];
-        }
-        if (lane == 31) uscan[C] = inc;
-    } else if (wid == 0 || (tok && wid <= B)) {
-        int *dst = (wid == 0) ? uscan : tscan + (wid - 1) * (C + 1);
-        const int per = (C + 31) / 32;
-        const int c0 = lane * per;
-        int loc = 0;
-        for (int k = 0; k < per; ++k)
-            if (c0 + k < C) loc += dst[c0 + k];
-        int inc = loc;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int n = __shfl_up_sync(0xffffffffu, inc, o);
-            if (lane >= o) inc += n;
-        }
-        int run = inc - loc;
-        for (int k = 0; k < per; ++k)
-            if (c0 + k < C) {
-                const int v = dst[c0 + k];
-                dst[c0 + k] = run;
-                run += v;
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(0xffffffffu, inc, o);
+                if (lane >= o) inc += n;
             }
-        if (lane == 31) dst[C] = inc;
-    }
-    // warp 0: this CTA's share of the ascending kept-channel list
-    if (wid == 0) {
-        __syncwarp();
-        const unsigned U = (unsigned)uscan[C];  // <= 2^18 kept channels
-        const int p0 = (int)(U * g / G), p1 = (int)(U * (g + 1) / G);
-        for (int n = lane; n < p1 - p0; n += 32) {
-            const int p = p0 + n;
-            int lo = 0, hi = C - 1;  // block cb with uscan[cb] <= p < uscan[cb + 1]
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if (uscan[mid] <= p) lo = mid; else hi = mid - 1;
+            int run = inc - loc;
+#pragma unroll
+            for (int k = 0; k < PER; ++k) {
+                if (lane * PER + k < C) uscan[lane * PER + k] = run;
+                run += cnt[k];
             }
-            const int off = p - uscan[lo];
-            chan[n] = (lo >= cpf && lo < cpf + npf) ? chanpf[(lo - cpf) * kCB + off]
-                                                    : a.ulist[(size_t)lo * kCB + off];
+            if (lane == 31) uscan[C] = inc;
+        } else if (wid == 0 || (tok && wid <= B)) {
+            int *dst = (wid == 0) ? uscan : tscan + (wid - 1) * (C + 1);
+            const int per = (C + 31) / 32;
+            const int c0 = lane * per;
+            int loc = 0;
+            for (int k = 0; k < per; ++k)
+                if (c0 + k < C) loc += dst[c0 + k];
+            int inc = loc;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(0xffffffffu, inc, o);
+                if (lane >= o) inc += n;
+            }
+            int run = inc - loc;
+            for (int k = 0; k < per; ++k)
+                if (c0 + k < C) {
+                    const int v = dst[c0 + k];
+                    dst[c0 + k] = run;
+                    run += v;
+                }
+            if (lane == 31) dst[C] = inc;
         }
+        // warp 0: this CTA's share of the ascending kept-channel list
+        if (wid == 0) {
+            __syncwarp();
+            const unsigned U = (unsigned)uscan[C];  // <= 2^18 kept channels
+            const int p0 = (int)(U * g / G), p1 = (int)(U * (g + 1) / G);
+            for (int n = lane; n < p1 - p0; n += 32) {
+                const int p = p0 + n;
+                int lo = 0, hi = C - 1;  // block cb with uscan[cb] <= p < uscan[cb + 1]
+                while (lo < hi) {
+                    const int mid = (lo + hi + 1) >> 1;
+                    if (uscan[mid] <= p) lo = mid; else hi = mid - 1;
+                }
+                const int off = p - uscan[lo];
+                chan[n] = (lo >= cpf && lo < cpf + npf) ? chanpf[(lo - cpf) * kCB + off]
+                                                        : a.ulist[(size_t)lo * kCB + off];
+            }
+        }
+        __syncthreads();
+        if (tid == 0) stamp_max(a.stamps, kS2List);
+        const unsigned U = (unsigned)uscan[C];
+        n_ch = (int)(U * (g + 1) / G) - (int)(U * g / G);
     }
-    __syncthreads();
-    if (tid == 0) stamp_max(a.stamps, kS2List);
-    const unsigned U = (unsigned)uscan[C];
-    const int n_ch = (int)(U * (g + 1) / G) - (int)(U * g / G);
-    asm volatile("griddepcontrol.launch_dependents;");
 
     if (wid == kNDot + NDOWN) {
         // ---------------- producer ----------------

@@ -643,3 +643,46 @@ def test_tc1s_nothing_kept_and_all_kept_c1(c1):
     y = dense.y.cpu().numpy().astype(np.float64)
     rel = np.linalg.norm(y - ref, axis=1) / np.linalg.norm(ref, axis=1)
     assert rel.max() <= Y_TOL
+
+
+# ---------------------------------------------------------------------------
+# y only (no mask or list outputs): Stage 2 takes its list without a CTA-wide
+# barrier. y is checked against the oracle under the masks of the same call
+# with outputs (masks are deterministic).
+# ---------------------------------------------------------------------------
+
+def _y_only_check(case, rows, b, ws=None):
+    xs = [case.xdev(rows[k:k + b]) for k in range(0, len(rows), b)]
+    full = [P.ffn_forward(case.layer, x, case.tau_x, case.tau_s, ws) for x in xs]
+    bare = [P.ffn_forward(case.layer, x, case.tau_x, case.tau_s, ws, want_masks=False)
+            for x in xs]
+    ms = torch.cat([o.mask_s for o in full]).cpu().numpy()
+    y = torch.cat([o.y for o in bare]).cpu().numpy().astype(np.float64)
+    y_full = torch.cat([o.y for o in full]).cpu().numpy().astype(np.float64)
+    y_ref = oracle.forward(case.x[rows], case.tau_x, case.tau_s, case.L, case.Por, mask_s_in=ms,
+                           want=(), act=case.act)["y"]
+    num = np.linalg.norm(y - y_ref, axis=1)
+    den = np.maximum(np.linalg.norm(y_ref, axis=1), 1e-30)
+    worst = float((num / den).max())
+    print(f"[y-only {len(rows)} tokens b={b}] y_rel_max={worst:.2e}")
+    assert worst <= Y_TOL
+    # the two entry modes differ only in summation order
+    assert np.allclose(y, y_full, rtol=1e-4, atol=1e-6 * np.abs(y_full).max())
+    if ws is not None:
+        st, flags = P.last_device_status(ws)
+        assert st == P.PROX_OK and flags == 0
+
+
+@pytest.mark.parametrize("b", [1, 2, 3])
+def test_forward_y_only_c1(c1, b):
+    _y_only_check(c1, list(range(30, 30 + 3 * b)), b)
+
+
+@pytest.mark.parametrize("b", [1, 2, 4])
+def test_forward_y_only_c2(c2, b):
+    ws = P.workspace(4096, 12288, b)
+    _y_only_check(c2, list(range(400, 400 + 4 * b)), b, ws)
+
+
+def test_forward_y_only_c4_b1(c4):
+    _y_only_check(c4, [5, 20], 1)
