@@ -33,7 +33,7 @@ constexpr int kNDot = 8;
 // warps and shared x precision per tokens-per-pass
 __host__ __device__ constexpr int s2_ndown(int B) { return B <= 2 ? 8 : 16; }
 __host__ __device__ constexpr int s2_threads(int B) { return (kNDot + s2_ndown(B) + 1) * 32; }
-__host__ __device__ constexpr int s2_xbytes(int B) { return B <= 2 ? 4 : 2; }
+__host__ __device__ constexpr int s2_xbytes(int B) { return (void)B, 2; }  // x as bf16
 
 // shared-memory carve-up, shared by the kernel and the host plan
 constexpr int kS2Prefetch = 4;  // channel-list blocks fetched with the counts
@@ -80,6 +80,16 @@ __device__ __forceinline__ uint4 lds128(const void *p) {
     return *reinterpret_cast<const uint4 *>(p);
 }
 
+// acc.x += w.lo * x.lo, acc.y += w.hi * x.hi for a word of two bf16 weights
+// and two bf16 inputs: the products are exact in fp32 (8-bit significands),
+// so this equals an fp32 FMA of the widened values, without widening them
+__device__ __forceinline__ void fma_bf16_pair(float2 &acc, uint32_t w, uint32_t x) {
+    asm("{\n\t.reg .b16 wl, wh, xl, xh;\n\tmov.b32 {wl, wh}, %2;\n\tmov.b32 {xl, xh}, %3;\n\t"
+        "fma.rn.f32.bf16 %0, wl, xl, %0;\n\tfma.rn.f32.bf16 %1, wh, xh, %1;\n\t}"
+        : "+f"(acc.x), "+f"(acc.y)
+        : "r"(w), "r"(x));
+}
+
 __device__ __forceinline__ void bf16x8_to_f2(const uint4 &w, float2 (&o)[4]) {
     const uint32_t a[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
@@ -89,14 +99,12 @@ __device__ __forceinline__ void bf16x8_to_f2(const uint4 &w, float2 (&o)[4]) {
 template <int B, int NCHD>
 __global__ void __launch_bounds__(s2_threads(B), 1) k_stage2(const Stage2Args a) {
     constexpr int NDOWN = s2_ndown(B);
-    constexpr bool XF32 = (B <= 2);
     extern __shared__ __align__(128) unsigned char smem[];
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int d = a.d, C = a.C, NST = a.nstage;
     const S2Smem L = s2_smem(d, B, NST, C, a.max_ch);
     uint16_t *stages = reinterpret_cast<uint16_t *>(smem + L.stages);
-    float *xf = reinterpret_cast<float *>(smem + L.xs);        // XF32: [B][2][d/2]
-    uint16_t *xh = reinterpret_cast<uint16_t *>(smem + L.xs);  // else: [B][d]
+    uint16_t *xh = reinterpret_cast<uint16_t *>(smem + L.xs);  // x, bf16 [B][d]
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.full);
     uint64_t *empty = reinterpret_cast<uint64_t *>(smem + L.empty);
     uint64_t *sready = reinterpret_cast<uint64_t *>(smem + L.sready);
@@ -117,25 +125,15 @@ __global__ void __launch_bounds__(s2_threads(B), 1) k_stage2(const Stage2Args a)
         }
         mbar_fence_init();
     }
-    // x into shared memory (fp32, split in halves so that a lane's two
-    // 16-byte reads of a chunk fall in different bank groups; or bf16).
-    // Stage 1, the kernel this one may overlap, only triggers this launch
-    // after its own griddepcontrol.wait, so x (written before Stage 1 ran)
-    // is complete.
+    // x into shared memory as it is (bf16; the dot warps multiply bf16 pairs
+    // into fp32 sums). Stage 1, the kernel this one may overlap, only
+    // triggers this launch after its own griddepcontrol.wait, so x (written
+    // before Stage 1 ran) is complete.
     for (int k = tid; k < B * nch16; k += s2_threads(B)) {
         const int t = k / nch16, ci = k % nch16;
         uint4 v = make_uint4(0, 0, 0, 0);
         if (t < a.nb) v = *reinterpret_cast<const uint4 *>(a.x + (size_t)t * d + ci * 8);
-        if constexpr (XF32) {
-            float2 f[4];
-            bf16x8_to_f2(v, f);
-            float *base = xf + (size_t)t * d;
-            *reinterpret_cast<float4 *>(base + ci * 4) = make_float4(f[0].x, f[0].y, f[1].x, f[1].y);
-            *reinterpret_cast<float4 *>(base + d / 2 + ci * 4) =
-                make_float4(f[2].x, f[2].y, f[3].x, f[3].y);
-        } else {
-            *reinterpret_cast<uint4 *>(xh + (size_t)t * d + ci * 8) = v;
-        }
+        *reinterpret_cast<uint4 *>(xh + (size_t)t * d + ci * 8) = v;
     }
     // x and the barriers are in place before Stage 1 has finished
     __syncthreads();
@@ -383,29 +381,19 @@ __global__ void __launch_bounds__(s2_threads(B), 1) k_stage2(const Stage2Args a)
 #pragma unroll
             for (int t = 0; t < B; ++t) u2[t] = g2[t] = make_float2(0.f, 0.f);
             for (int ci = lane; ci < nch16; ci += 32) {
-                float2 wu[4], wg[4];
-                bf16x8_to_f2(lds128(up + ci * 8), wu);
-                bf16x8_to_f2(lds128(gt + ci * 8), wg);
+                const uint4 wu = lds128(up + ci * 8), wg = lds128(gt + ci * 8);
 #pragma unroll
                 for (int t = 0; t < B; ++t) {
                     if (B > 1 && !((bits >> t) & 1u)) continue;
-                    float2 xv[4];
-                    if constexpr (XF32) {
-                        const float4 xa = *reinterpret_cast<const float4 *>(xf + (size_t)t * d + ci * 4);
-                        const float4 xb =
-                            *reinterpret_cast<const float4 *>(xf + (size_t)t * d + d / 2 + ci * 4);
-                        xv[0] = make_float2(xa.x, xa.y);
-                        xv[1] = make_float2(xa.z, xa.w);
-                        xv[2] = make_float2(xb.x, xb.y);
-                        xv[3] = make_float2(xb.z, xb.w);
-                    } else {
-                        bf16x8_to_f2(lds128(xh + (size_t)t * d + ci * 8), xv);
-                    }
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        u2[t] = __ffma2_rn(xv[q], wu[q], u2[t]);
-                        g2[t] = __ffma2_rn(xv[q], wg[q], g2[t]);
-                    }
+                    const uint4 xq = lds128(xh + (size_t)t * d + ci * 8);
+                    fma_bf16_pair(u2[t], wu.x, xq.x);
+                    fma_bf16_pair(u2[t], wu.y, xq.y);
+                    fma_bf16_pair(u2[t], wu.z, xq.z);
+                    fma_bf16_pair(u2[t], wu.w, xq.w);
+                    fma_bf16_pair(g2[t], wg.x, xq.x);
+                    fma_bf16_pair(g2[t], wg.y, xq.y);
+                    fma_bf16_pair(g2[t], wg.z, xq.z);
+                    fma_bf16_pair(g2[t], wg.w, xq.w);
                 }
             }
             float sv[B];
