@@ -984,15 +984,21 @@ cudaError_t launch1(Stage1Args a, const Stage1Plan &p0, cudaStream_t s) {
     cfg.blockDim = dim3(kS1Threads);
     cfg.dynamicSmemBytes = p.smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[2];
+    // Load-balancing cluster placement: with the default policy the clusters
+    // of some processes are placed late while the previous kernel's CTAs
+    // leave their SMs, and the first and last CTA pass the grid wait about
+    // 1 us apart (0.06 us with this policy, every run measured).
+    cudaLaunchAttribute attr[3];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     attr[1].id = cudaLaunchAttributeClusterDimension;
     attr[1].val.clusterDim.x = a.n_r;
     attr[1].val.clusterDim.y = 1;
     attr[1].val.clusterDim.z = 1;
+    attr[2].id = cudaLaunchAttributeClusterSchedulingPolicyPreference;
+    attr[2].val.clusterSchedulingPolicyPreference = cudaClusterSchedulingPolicyLoadBalancing;
     cfg.attrs = attr;
-    cfg.numAttrs = 2;
+    cfg.numAttrs = 3;
     return cudaLaunchKernelEx(&cfg, k, a);
 }
 
