@@ -19,8 +19,8 @@
 // A stage is refilled once its dot warp and every down warp have released it
 // (mbarrier "empty"). Channels never wait on each other through a CTA-wide
 // barrier, so several channels are in flight at once, and every wait is
-// bounded. At the end each CTA adds its partial y to global memory with
-// 16-byte vector reductions.
+// bounded. At the end each CTA adds its partial y to global memory with one
+// bulk reduction of the copy engine.
 #include "prox_internal.cuh"
 
 #include <cuda_runtime.h>
@@ -475,6 +475,13 @@ __global__ void __launch_bounds__(s2_threads(B), 1) k_stage2(const Stage2Args a)
     if (lane == 0) stamp_max(a.stamps, kS2Stream);
 
     if (n_ch == 0) return;
+    // The CTA's partial y goes to global memory as one bulk reduction (the
+    // copy engine adds a shared-memory copy of it into y), not as one 16-byte
+    // atomic per thread and chunk. Every down warp is past its last stage, and
+    // the dot warps and the producer are done with theirs, so the ring is free
+    // for that copy once all down warps are here.
+    named_bar_sync(1, NDOWN * 32);
+    float *ys = reinterpret_cast<float *>(stages);  // [nb][d]
 #pragma unroll
     for (int t = 0; t < B; ++t) {
         if (t >= a.nb) break;
@@ -482,13 +489,18 @@ __global__ void __launch_bounds__(s2_threads(B), 1) k_stage2(const Stage2Args a)
         for (int m = 0; m < NCHD; ++m) {
             const int ci = dt + m * NDOWN * 32;
             if (ci < nch16) {
-                float *dst = a.y + (size_t)t * d + ci * 8;
-                red_add_v4(dst, acc[t][m][0].x, acc[t][m][0].y, acc[t][m][1].x, acc[t][m][1].y);
-                red_add_v4(dst + 4, acc[t][m][2].x, acc[t][m][2].y, acc[t][m][3].x, acc[t][m][3].y);
+                float4 *dst = reinterpret_cast<float4 *>(ys + (size_t)t * d + ci * 8);
+                dst[0] = make_float4(acc[t][m][0].x, acc[t][m][0].y, acc[t][m][1].x, acc[t][m][1].y);
+                dst[1] = make_float4(acc[t][m][2].x, acc[t][m][2].y, acc[t][m][3].x, acc[t][m][3].y);
             }
         }
     }
-    if (lane == 0) stamp_max(a.stamps, kS2End);
+    fence_proxy_async_smem();  // the copy engine reads what these threads wrote
+    named_bar_sync(1, NDOWN * 32);
+    if (dt == 0) {
+        bulk_reduce_add_f32(a.y, ys, (uint32_t)(a.nb * d * 4));
+        stamp_max(a.stamps, kS2End);
+    }
 }
 
 template <int B, int NCHD>

@@ -329,6 +329,24 @@ __device__ __forceinline__ uint64_t l2_evict_first() {
 }
 
 // bulk_g2s with an L2 cache policy
+// dst[i] += src[i] (fp32) for bytes / 4 elements: a bulk reduction from
+// shared to global memory by the copy engine (16-byte aligned, size a
+// multiple of 16). The calling thread waits until the reduction has been
+// performed, so the CTA may exit and the grid completes with y final.
+__device__ __forceinline__ void bulk_reduce_add_f32(float *dst, const float *src, uint32_t bytes) {
+    asm volatile(
+        "cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(dst),
+        "r"(smem_addr(src)), "r"(bytes)
+        : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+// generic-proxy writes to shared memory made visible to the async proxy
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ __forceinline__ void bulk_g2s_hint(void *dst, const void *src, uint32_t bytes,
                                               uint64_t *bar, uint64_t pol) {
     asm volatile(
