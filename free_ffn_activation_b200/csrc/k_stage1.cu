@@ -196,7 +196,9 @@ __host__ __device__ inline S1Smem s1_smem(int d, int B, int NB, int unit_cap, in
     const int cw = NB * kCB;
     const int cpt = s1_cpt(B, NB, PK);
     const int rl = kS1Threads / (2 * (cw / cpt));
-    const size_t red = (size_t)rl * 2 * B * (cw + cw / cpt) * 4;    // padded row-lane sums
+    // row-lane sums: 32-channel chunks swizzled in 16-byte units, narrower
+    // chunks padded by one word
+    const size_t red = (size_t)rl * 2 * B * (cpt == 32 ? cw : cw + cw / cpt) * 4;
     const size_t ring = (size_t)kS1Threads * (s1_dmax(B, NB, PK) >> depth_sel) * s1_bytes(B, NB, PK);
     (void)d;
     S1Smem s;
@@ -560,6 +562,7 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
     __shared__ int s_warp[kS1Threads / 32];
     __shared__ __align__(16) float s_red[kS1Threads / 32][kMaxB];
     __shared__ int s_cnt[kS1Threads / 32][kMaxB + 1];
+    __shared__ float s_off[T::CPT == 32 ? T::RL : 1][2][T::CPT == 32 ? B : 1];  // row-lane offset sums
     // every CTA of the cluster has started once this phase completes: only
     // then may ranks store into CTA 0's shared memory (waited for before (6))
     if (kPush) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
@@ -770,9 +773,60 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
         if (tid == 0) stamp_max(a.stamps, kS1Stream);
         if (kPush) asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
 
-        // (6) reduce row lanes (padded rows: conflict-free both ways), undo the
-        // pre-scale and the +8 code offset: this CTA's partial sums in `part`.
-        // The pad word after chunk 0's channels carries the row lane's offset sum.
+        // (6) reduce row lanes, undo the pre-scale and the +8 code offset:
+        // this CTA's partial sums in `part`
+        if constexpr (T::CPT == 32) {
+            // 32-channel chunks: 16-byte unit i of chunk c sits at unit
+            // i ^ (c % 8) of the chunk (conflict-free 16-byte stores and
+            // loads); each thread then sums four adjacent channels over the
+            // row lanes with 16-byte loads and pushes them with one store.
+            // The row lanes' offset sums go to s_off.
+    #pragma unroll
+            for (int t = 0; t < B; ++t) {
+                float *row = red + ((size_t)((rl * 2 + m) * B + t) * T::CW) + chunk * 32;
+    #pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    *reinterpret_cast<float4 *>(row + 4 * (i ^ (chunk & 7))) =
+                        make_float4(acc2[(t * 32 + 4 * i) / 2].x, acc2[(t * 32 + 4 * i) / 2].y,
+                                    acc2[(t * 32 + 4 * i) / 2 + 1].x, acc2[(t * 32 + 4 * i) / 2 + 1].y);
+                if (chunk == 0) s_off[rl][m][t] = ssum[t];
+            }
+            __syncthreads();
+            for (int o = tid; o < 2 * T::CW / 4; o += kS1Threads) {
+                const int mm = o / (T::CW / 4), ch0 = (o % (T::CW / 4)) * 4;
+                const int c = ch0 / 32, j = (ch0 % 32) / 4;
+                const int pos = c * 32 + 4 * (j ^ (c & 7));
+    #pragma unroll
+                for (int t = 0; t < B; ++t) {
+                    float4 sacc = make_float4(0.f, 0.f, 0.f, 0.f);
+                    float soff = 0.f;
+    #pragma unroll
+                    for (int q = 0; q < T::RL; ++q) {
+                        const float4 v = *reinterpret_cast<const float4 *>(
+                            red + (size_t)((q * 2 + mm) * B + t) * T::CW + pos);
+                        sacc.x += v.x; sacc.y += v.y; sacc.z += v.z; sacc.w += v.w;
+                        soff += s_off[q][mm][t];
+                    }
+                    const int e1 = E[t] / 2, e2 = E[t] - e1;
+                    const float pe = __int_as_float((127 - e1) << 23), pf = __int_as_float((127 - e2) << 23);
+                    const float sv[4] = {sacc.x, sacc.y, sacc.z, sacc.w};
+                    float ov[4];
+    #pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        // 2^(149 - 4p) as a product of normal floats, p the nibble position
+                        const int p = nib_pos((ch0 + e) % 8);
+                        const float v = (sv[e] * __int_as_float((127 + 75) << 23)) *
+                                            __int_as_float((127 + 74 - 4 * p) << 23) -
+                                        8.f * soff;  // sum (q + 8 - 8) x s 2^E
+                        ov[e] = v * pe * pf;
+                    }
+                    *reinterpret_cast<float4 *>(dst_part + (mm * B + t) * T::CW + ch0) =
+                        make_float4(ov[0], ov[1], ov[2], ov[3]);
+                }
+            }
+        } else {
+        // padded rows (conflict-free both ways); the pad word after chunk 0's
+        // channels carries the row lane's offset sum
         constexpr int PAD = T::CW + T::TPRM;  // one extra word per chunk row
     #pragma unroll
         for (int t = 0; t < B; ++t) {
@@ -811,6 +865,7 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
                     dst_part[(mm * B + t) * T::CW + ch] = sacc;  // plain x_i * w_ij sums
                 }
             }
+        }
         }
     }
     cluster.sync();  // all partials of the block are in their CTAs' shared memory
