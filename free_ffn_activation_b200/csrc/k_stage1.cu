@@ -147,7 +147,8 @@ __device__ __forceinline__ void proc_word_bf16(uint32_t w, int wi, const float *
     }
 }
 
-// deterministic block-wide exclusive scan of one int per thread (256 threads)
+// deterministic block-wide exclusive scan of one int per thread (one
+// barrier; warp_tot is written once per kernel, so it needs no second one)
 __device__ __forceinline__ int block_excl_scan(int v, int *warp_tot, int &total) {
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     int inc = v;
@@ -164,7 +165,6 @@ __device__ __forceinline__ int block_excl_scan(int v, int *warp_tot, int &total)
         if (w < wid) base += warp_tot[w];
         tot += warp_tot[w];
     }
-    __syncthreads();
     total = tot;
     return base + inc - v;
 }
@@ -914,10 +914,13 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
             bits |= (keep ? 1u : 0u) << t;
         }
         if (a.build_lists) {
-            // warp ballots and per-warp counts (token t in column t, union in column B)
+            // warp ballots and per-warp counts (token t in column t, union in
+            // column B). A one-token pass writes only the union list and
+            // count: they are the token's (Stage 2 reads them for both).
+            constexpr int T0 = B == 1 ? 1 : 0;
             uint32_t bal[kMaxB + 1];
 #pragma unroll
-            for (int t = 0; t <= B; ++t) {
+            for (int t = T0; t <= B; ++t) {
                 const bool k = (t < B) ? ((bits >> t) & 1u) : (bits != 0u);
                 bal[t] = __ballot_sync(0xffffffffu, k);
                 if (lane == 0) s_cnt[wid][t] = __popc(bal[t]);
@@ -928,7 +931,7 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
             if (blk < NB) {
                 const int cb = c0 + blk;
 #pragma unroll
-                for (int t = 0; t <= B; ++t) {
+                for (int t = T0; t <= B; ++t) {
                     int base = 0, tot = 0;
                     for (int w = blk * WPB; w < (blk + 1) * WPB; ++w) {
                         if (w < wid) base += s_cnt[w][t];

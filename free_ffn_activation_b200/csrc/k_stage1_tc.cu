@@ -483,10 +483,13 @@ __global__ void __launch_bounds__(kT, 1) k_stage1_tc(const Stage1Args a) {
             }
         }
         if (a.build_lists) {
-            // warp ballots and per-warp counts (token t in column t, union in column B)
+            // warp ballots and per-warp counts (token t in column t, union in
+            // column B). A one-token pass writes only the union list and
+            // count: they are the token's (Stage 2 reads them for both).
+            constexpr int T0 = B == 1 ? 1 : 0;
             uint32_t bal[B + 1];
 #pragma unroll
-            for (int t = 0; t <= B; ++t) {
+            for (int t = T0; t <= B; ++t) {
                 const bool k = (t < B) ? ((bits >> t) & 1u) : (bits != 0u);
                 bal[t] = __ballot_sync(0xffffffffu, k);
                 if (lane == 0) s_cnt[wid][t] = __popc(bal[t]);
@@ -496,7 +499,7 @@ __global__ void __launch_bounds__(kT, 1) k_stage1_tc(const Stage1Args a) {
             constexpr int WPB = kCB / 32;
             if (wid < WPB) {
 #pragma unroll
-                for (int t = 0; t <= B; ++t) {
+                for (int t = T0; t <= B; ++t) {
                     int bse = 0, tot = 0;
                     for (int w = 0; w < WPB; ++w) {
                         if (w < wid) bse += s_cnt[w][t];

@@ -239,7 +239,8 @@ __global__ void __launch_bounds__(s2_threads(B), 1) k_stage2(const Stage2Args a)
                     const int k = base + q * NT;
                     v[q] = 0;
                     if (k < nuc) v[q] = (uint32_t)a.ucount[k];
-                    else if (k < nuc + ntc) v[q] = (uint32_t)a.tcount[k - nuc];
+                    else if (k < nuc + ntc)  // one token: the union's counts are its own
+                        v[q] = (uint32_t)(B == 1 ? a.ucount[k - nuc] : a.tcount[k - nuc]);
                     else if (k < total) v[q] = a.ulist[(size_t)cpf * kCB + (k - nuc - ntc)];
                 }
 #pragma unroll
@@ -419,11 +420,12 @@ __global__ void __launch_bounds__(s2_threads(B), 1) k_stage2(const Stage2Args a)
         if (a.idx_s) {
             for (int c = g; c < C; c += G) {
                 for (int t = 0; t < a.nb; ++t) {
-                    const int nk = a.tcount[c * B + t];
+                    const int nk = B == 1 ? a.ucount[c] : a.tcount[c * B + t];
                     const int base = tscan[t * (C + 1) + c];
                     for (int k = tid; k < nk; k += kNDot * 32)
                         a.idx_s[(size_t)t * a.f + base + k] =
-                            a.tlist[(size_t)t * a.f + c * kCB + k];
+                            B == 1 ? (int32_t)(a.ulist[(size_t)c * kCB + k] & 0xFFFFFFu)
+                                   : a.tlist[(size_t)t * a.f + c * kCB + k];
                 }
             }
         }
