@@ -204,8 +204,9 @@ __host__ __device__ inline S1Smem s1_smem(int d, int B, int NB, int unit_cap, in
     S1Smem s;
     size_t o = 0;
     s.ring = s.red = o;
-    size_t region = ring > red ? ring : red;
-    if (TC && s1tc_bytes(B, NB, unit_cap) > region) region = s1tc_bytes(B, NB, unit_cap);
+    // the tensor-core stream uses neither the copy ring nor the row-lane
+    // area, only its own tiles
+    const size_t region = TC ? s1tc_bytes(B, NB, unit_cap) : (ring > red ? ring : red);
     o += region;
     s.rowidx = o;
     o += ((size_t)unit_cap * 4 + 15) / 16 * 16;
