@@ -881,26 +881,33 @@ __global__ void __launch_bounds__(kS1Threads, 1) k_stage1(const Stage1Args a) {
         const int j = c0 * kCB + ch;         // channel index
         const int blk = wid / (kCB / 32);    // block of this warp's channels
         float uu[B], gg[B];
-#pragma unroll(B > 2 ? 1 : B)
-        for (int t = 0; t < B; ++t) {
-            uu[t] = gg[t] = 0.f;
-            if (t >= a.nb || ch >= T::CW) continue;
-            // all remote loads first, then the sums in rank order
-            float pu[kS1MaxRowGroups], pg[kS1MaxRowGroups];
+        // tokens in groups of up to 4: all (remote) loads of a group first,
+        // then its sums in rank order
+        constexpr int TG = B > 4 ? 4 : B;
+#pragma unroll
+        for (int t0 = 0; t0 < B; t0 += TG) {
+            float pu[kS1MaxRowGroups][TG], pg[kS1MaxRowGroups][TG];
 #pragma unroll
             for (int q = 0; q < kS1MaxRowGroups; ++q) {
-                pu[q] = pg[q] = 0.f;
-                if (q < a.n_r) {
-                    const float *pq = kPush ? part + (size_t)q * 2 * B * T::CW
-                                            : cluster.map_shared_rank(part, q);
-                    pu[q] = pq[(0 * B + t) * T::CW + ch];
-                    pg[q] = pq[(1 * B + t) * T::CW + ch];
+                const float *pq = kPush ? part + (size_t)q * 2 * B * T::CW
+                                        : cluster.map_shared_rank(part, q < a.n_r ? q : 0);
+#pragma unroll
+                for (int tt = 0; tt < TG; ++tt) {
+                    pu[q][tt] = pg[q][tt] = 0.f;
+                    if (q < a.n_r && t0 + tt < a.nb && ch < T::CW) {
+                        pu[q][tt] = pq[(0 * B + t0 + tt) * T::CW + ch];
+                        pg[q][tt] = pq[(1 * B + t0 + tt) * T::CW + ch];
+                    }
                 }
             }
 #pragma unroll
-            for (int q = 0; q < kS1MaxRowGroups; ++q) {
-                uu[t] += pu[q];
-                gg[t] += pg[q];
+            for (int tt = 0; tt < TG; ++tt) {
+                uu[t0 + tt] = gg[t0 + tt] = 0.f;
+#pragma unroll
+                for (int q = 0; q < kS1MaxRowGroups; ++q) {
+                    uu[t0 + tt] += pu[q][tt];
+                    gg[t0 + tt] += pg[q][tt];
+                }
             }
         }
         if (!kPush) asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
