@@ -68,8 +68,16 @@ __host__ __device__ inline S2Smem s2_smem(int d, int B, int nstage, int C, int m
     s.chan = o;
     o += (size_t)max_ch * 4;
     o = (o + 15) & ~(size_t)15;  // 16-byte copies of the list blocks
-    s.chanpf = o;
-    o += (size_t)kS2Prefetch * kCB * 4;
+    // The list blocks are read only while the channel list is built, before
+    // the producer's first copy into the ring's last slot: they share that
+    // slot when they fit in it.
+    const size_t pf = (size_t)kS2Prefetch * kCB * 4;
+    if (nstage >= 2 && pf <= (size_t)3 * d * 2) {
+        s.chanpf = (size_t)(nstage - 1) * 3 * d * 2;
+    } else {
+        s.chanpf = o;
+        o += pf;
+    }
     s.total = (o + 127) & ~(size_t)127;
     return s;
 }

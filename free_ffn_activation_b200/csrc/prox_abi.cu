@@ -76,10 +76,15 @@ Stage1Plan stage1_plan(int d, int f, int B, int num_sms) {
 Stage2Plan stage2_plan(int d, int B, int C, int max_ch) {
     Stage2Plan p;
     p.nchunk = stage2_nchd(d, B);
+    // The deepest ring within the 227 KB of dynamic shared memory an sm_100
+    // CTA may opt into, of at most 16 slots and 192 KB of rows (a ninth 24 KB
+    // slot on the 4096-wide layer measured slower)
+    constexpr size_t kSmemMax = 227 * 1024, kRingMax = 192 * 1024;
     const size_t stage = (size_t)6 * d;
-    const size_t fixed = stage2_smem_bytes(d, B, 0, C, max_ch);
-    int ns = fixed < (size_t)kS2SmemBudget ? (int)((kS2SmemBudget - fixed) / stage) : 0;
-    if (ns > 16) ns = 16;
+    int ns = 16;
+    while (ns > 0 && ((size_t)ns * stage > kRingMax ||
+                      stage2_smem_bytes(d, B, ns, C, max_ch) > kSmemMax))
+        --ns;
     p.nstage = ns;
     p.smem = stage2_smem_bytes(d, B, ns, C, max_ch);
     return p;
